@@ -1,0 +1,466 @@
+/*
+ * oracle.c -- plain, slow, obviously-correct CPU reference for the
+ * DeepSeek-V4 hybrid compressed attention hot path (CSA + HCA).
+ *
+ * TEST INFRASTRUCTURE ONLY.  The tests, the smoke check and the benchmark's
+ * CPU-baseline leg load this file's shared library; the GPU product path
+ * never does, and nothing here is shared with the CUDA sources.
+ *
+ * Sources (page titles and sections):
+ *   [N8]  "DeepSeek V4: Towards Highly Efficient Million Token Context
+ *         Intelligence" (papers.chlience.com reading note), section 8 "HCA":
+ *         C = H W^KV, Z = H W^Z, S = Softmax_row(Z_block + B),
+ *         C^Comp_i = sum_j S_j (.) C_j  (per-channel softmax over a block).
+ *   [N7]  same note, section 7 "CSA": m = 4, lightning indexer
+ *         I_{t,s} = sum_h w^I_{t,h} ReLU(q^I_{t,h} . K^IComp_s), Top-k
+ *         selection, shared key-value MQA core attention, sliding window.
+ *   [N9]  same note, section 9 "CSA/HCA other details": RoPE dims in BF16,
+ *         the rest of the KV in FP8; indexer in FP4; 128-token window.
+ *   [HF]  "DeepSeek-V4: a million-token context that agents can actually
+ *         use" (Hugging Face blog), section "Hybrid attention: CSA and HCA".
+ *
+ * Where the pages leave the arithmetic open, the reading taken is written
+ * next to the code.  Two places must be bit-exact with the GPU, so both
+ * sides take their floating-point decisions in the same fp32 sequence:
+ *   (1) pooling + FP8 quantisation (codes and scales),
+ *   (2) index scores (which decide the top-k sets).
+ * Everything else (attention) is computed in fp64.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fPIC -shared -lm.
+ * -ffp-contract=off matters: every a*b+c below is two roundings unless it is
+ * written as fmaf().
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------ */
+/* Scalar format helpers                                               */
+/* ------------------------------------------------------------------ */
+
+static float f32_from_bits(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+static uint32_t bits_from_f32(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
+
+/* bf16 -> fp32 is exact: bf16 is the top half of an fp32. */
+float oracle_bf16_to_f32(uint16_t h) { return f32_from_bits((uint32_t)h << 16); }
+
+/* fp32 -> bf16, round to nearest, ties to even (finite inputs). */
+uint16_t oracle_f32_to_bf16(float f)
+{
+    uint32_t u = bits_from_f32(f);
+    if ((u & 0x7F800000u) == 0x7F800000u)           /* inf / nan: truncate */
+        return (uint16_t)((u >> 16) | ((u & 0xFFFFu) ? 0x40u : 0u));
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7FFFu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+void oracle_f32_to_bf16_array(const float* x, uint16_t* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_f32_to_bf16(x[i]);
+}
+
+/* FP8 e4m3fn: 1 sign, 4 exponent (bias 7), 3 mantissa bits; no infinities,
+ * 0x7F/0xFF are NaN, so the largest finite magnitude is 0x7E = 448.  The
+ * "/448" in the scale rule fixes this variant. */
+double oracle_e4m3_value(uint8_t code)
+{
+    int e = (code >> 3) & 0xF, f = code & 7;
+    double mag = (e == 0) ? ldexp((double)f, -9) : ldexp(1.0 + f / 8.0, e - 7);
+    return (code & 0x80) ? -mag : mag;
+}
+
+/* fp32 -> e4m3fn, round to nearest with ties to the even code, saturating
+ * to +-448 (the "satfinite" rule).  Plain search over the 127 non-negative
+ * finite codes, whose values increase with the code; the sign is copied, so
+ * a value that rounds to zero keeps its sign (-0 -> 0x80). */
+uint8_t oracle_f32_to_e4m3(float v)
+{
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs((double)v);
+    if (a >= 448.0) return sign | 0x7E;
+    int lo = 0;                                  /* largest code with value <= a */
+    while (lo + 1 <= 0x7E && oracle_e4m3_value((uint8_t)(lo + 1)) <= a) lo++;
+    double vlo = oracle_e4m3_value((uint8_t)lo);
+    if (vlo == a) return sign | (uint8_t)lo;
+    double vhi = oracle_e4m3_value((uint8_t)(lo + 1));
+    double dlo = a - vlo, dhi = vhi - a;
+    int pick;
+    if (dlo < dhi) pick = lo;
+    else if (dhi < dlo) pick = lo + 1;
+    else pick = (lo & 1) ? lo + 1 : lo;          /* tie: even mantissa */
+    return sign | (uint8_t)pick;
+}
+
+void oracle_f32_to_e4m3_array(const float* x, uint8_t* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_f32_to_e4m3(x[i]);
+}
+
+void oracle_exp_neg_array(const float* z, float* out, int64_t n);
+
+/* FP4 e2m1 (OCP microscaling formats): 1 sign bit, 2 exponent bits (bias 1),
+ * 1 mantissa bit.  Magnitudes of codes 0..7: 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
+double oracle_e2m1_value(int nib)
+{
+    static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    return (nib & 8) ? -mag[nib & 7] : mag[nib & 7];
+}
+
+/* ue8m0 scale byte u -> 2^(u-127) (exponent-only scale of the MX formats). */
+double oracle_ue8m0_value(uint8_t u) { return ldexp(1.0, (int)u - 127); }
+
+/* ------------------------------------------------------------------ */
+/* (1) Softmax-gated pooling  [N8] and [HF] "softmax-gated pooling with a */
+/*     learned positional bias"                                        */
+/* ------------------------------------------------------------------ */
+
+/* The pages give the pooling formula but no precision or exp.  Reading:
+ * fp32 arithmetic in a fixed order, with exp evaluated by one named method
+ * so that a GPU kernel can reproduce the bits:
+ *   Cody & Waite argument reduction (Cody & Waite, "Software Manual for the
+ *   Elementary Functions", 1980): n = rint(z*log2(e)), r = z - n*ln2 with
+ *   ln2 split into a short head (trailing mantissa bits zero, so n*LN2_HI
+ *   is exact) and a tail; then the Taylor series of e^r to degree 7 in
+ *   Horner form with fused multiply-adds; then the scale 2^n.
+ * Constants are the correctly rounded fp32 values of their definitions. */
+static const uint32_t K_L2E    = 0x3FB8AA3Bu;  /* RN(1/ln 2)                         */
+static const uint32_t K_LN2_HI = 0x3F317200u;  /* RN(ln 2) with 9 low mantissa bits 0 */
+static const uint32_t K_LN2_LO = 0x35BFBE8Eu;  /* RN(ln 2 - LN2_HI)                   */
+static const uint32_t K_INV_FACT[8] = {        /* RN(1/k!), k = 0..7                 */
+    0x3F800000u, 0x3F800000u, 0x3F000000u, 0x3E2AAAABu,
+    0x3D2AAAABu, 0x3C088889u, 0x3AB60B61u, 0x39500D01u};
+
+float oracle_const(int which)  /* exposed so a test can check each constant */
+{
+    if (which == 0) return f32_from_bits(K_L2E);
+    if (which == 1) return f32_from_bits(K_LN2_HI);
+    if (which == 2) return f32_from_bits(K_LN2_LO);
+    if (which >= 10 && which < 18) return f32_from_bits(K_INV_FACT[which - 10]);
+    return NAN;
+}
+
+/* E(z) ~= e^z for z <= 0 (the pooling only ever needs z - max <= 0). */
+float oracle_exp_neg(float z)
+{
+    if (!(z >= -87.0f)) return 0.0f;                 /* e^-87 ~ 1.6e-38: flush */
+    float t  = z * f32_from_bits(K_L2E);
+    float nf = nearbyintf(t);                        /* ties to even           */
+    float r  = fmaf(-nf, f32_from_bits(K_LN2_HI), z);
+    r        = fmaf(-nf, f32_from_bits(K_LN2_LO), r);
+    float p  = f32_from_bits(K_INV_FACT[7]);
+    for (int k = 6; k >= 0; --k) p = fmaf(p, r, f32_from_bits(K_INV_FACT[k]));
+    int n = (int)nf;                                 /* -126 <= n <= 0         */
+    return p * f32_from_bits((uint32_t)(n + 127) << 23);
+}
+
+void oracle_exp_neg_array(const float* z, float* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_exp_neg(z[i]);
+}
+
+/* Pool one block of m tokens into one entry of d channels.
+ *   x, gate : [m][d] bf16 rows of the block (token jm+i is row i)
+ *   bias    : [m][d] fp32 learned positional bias, row i = position i in block
+ * Per channel c (the softmax runs over the block's tokens, per channel, as
+ * the (.) product in [N8] implies):
+ *   z_i = fp32(gate_i) + b_i          (fp32 add)
+ *   zmax = max_i z_i
+ *   e_i = E(z_i - zmax)
+ *   S   = e_0 + e_1 + ... (fp32, ascending i)
+ *   N   = e_0*x_0 + e_1*x_1 + ... (each product rounded, ascending i)
+ *   y   = N / S  (one IEEE division)
+ * y64 (optional) gets the same pooled value in fp64 with libm exp(), as an
+ * independent cross-check of the fp32 sequence, and mag64 (optional) the
+ * fp64 sum of p_i |x_i|, the natural scale of the pooled value's error. */
+void oracle_pool_block(const uint16_t* x, const uint16_t* gate, const float* bias,
+                       int m, int d, float* y, double* y64, double* mag64)
+{
+    for (int c = 0; c < d; ++c) {
+        float zmax = -INFINITY;
+        for (int i = 0; i < m; ++i) {
+            float z = oracle_bf16_to_f32(gate[(size_t)i * d + c]) + bias[(size_t)i * d + c];
+            if (z > zmax) zmax = z;
+        }
+        float S = 0.0f, N = 0.0f;
+        for (int i = 0; i < m; ++i) {
+            float z = oracle_bf16_to_f32(gate[(size_t)i * d + c]) + bias[(size_t)i * d + c];
+            float e = oracle_exp_neg(z - zmax);
+            float xv = oracle_bf16_to_f32(x[(size_t)i * d + c]);
+            S = S + e;
+            float prod = e * xv;
+            N = N + prod;
+        }
+        y[c] = N / S;
+        if (y64) {
+            double zm = -INFINITY, s = 0.0, n = 0.0, a = 0.0;
+            for (int i = 0; i < m; ++i) {
+                double z = (double)oracle_bf16_to_f32(gate[(size_t)i * d + c]) + (double)bias[(size_t)i * d + c];
+                if (z > zm) zm = z;
+            }
+            for (int i = 0; i < m; ++i) {
+                double z = (double)oracle_bf16_to_f32(gate[(size_t)i * d + c]) + (double)bias[(size_t)i * d + c];
+                double e = exp(z - zm);
+                s += e;
+                n += e * (double)oracle_bf16_to_f32(x[(size_t)i * d + c]);
+                a += e * fabs((double)oracle_bf16_to_f32(x[(size_t)i * d + c]));
+            }
+            y64[c] = n / s;
+            if (mag64) mag64[c] = a / s;
+        }
+    }
+}
+
+/* Storage of one pooled entry ([N9]: RoPE dims BF16, the rest FP8; the
+ * scale rule is amax/448 per group of g channels):
+ *   channels [0, d - d_rope)  : per group, amax = max |y|, scale = amax/448
+ *                               (fp32 division); amax == 0 -> scale 0 and
+ *                               codes 0x00; else code = e4m3(y / scale)
+ *                               (fp32 division, then RN-even, satfinite)
+ *   channels [d - d_rope, d)  : bf16 RN of y. */
+void oracle_quant_entry(const float* y, int d, int d_rope, int g,
+                        uint8_t* codes, float* scales, uint16_t* rope)
+{
+    int dn = d - d_rope;
+    for (int G = 0; G < dn / g; ++G) {
+        float amax = 0.0f;
+        for (int c = G * g; c < (G + 1) * g; ++c) {
+            float a = fabsf(y[c]);
+            if (a > amax) amax = a;
+        }
+        float scale = amax / 448.0f;
+        scales[G] = scale;
+        for (int c = G * g; c < (G + 1) * g; ++c)
+            codes[c] = (amax == 0.0f) ? 0x00 : oracle_f32_to_e4m3(y[c] / scale);
+    }
+    for (int c = dn; c < d; ++c) rope[c - dn] = oracle_f32_to_bf16(y[c]);
+}
+
+/* Pool and store n_blocks entries for each of B sequences.
+ *   x, gate : [B][x_seq_stride][d] bf16; x points at the first token of
+ *             block entry_begin, so block entry_begin+jj is rows jj*m..jj*m+m-1
+ *   out     : codes [B][cap][d-d_rope], scales [B][cap][(d-d_rope)/g],
+ *             rope [B][cap][d_rope]; entry entry_begin+jj is written.
+ * Returns the largest |y32 - y64| / sum_i p_i |x_i| seen (the fp64
+ * cross-check of the defined fp32 sequence). */
+double oracle_compress(const uint16_t* x, const uint16_t* gate, int64_t x_seq_stride,
+                       const float* bias, int m, int B, int64_t n_blocks,
+                       int d, int d_rope, int g,
+                       uint8_t* codes, float* scales, uint16_t* rope,
+                       int64_t cap, int64_t entry_begin)
+{
+    int dn = d - d_rope, ng = dn / g;
+    float*  y   = (float*)malloc(sizeof(float) * d);
+    double* y64 = (double*)malloc(sizeof(double) * d);
+    double* mag = (double*)malloc(sizeof(double) * d);
+    double worst = 0.0;
+    for (int b = 0; b < B; ++b) {
+        for (int64_t jj = 0; jj < n_blocks; ++jj) {
+            const size_t row = (size_t)b * x_seq_stride + (size_t)jj * m;
+            oracle_pool_block(x + row * d, gate + row * d, bias, m, d, y, y64, mag);
+            for (int c = 0; c < d; ++c) {
+                double den = mag[c] > 1e-30 ? mag[c] : 1e-30;
+                double dev = fabs((double)y[c] - y64[c]) / den;
+                if (dev > worst) worst = dev;
+            }
+            int64_t e = entry_begin + jj;
+            oracle_quant_entry(y, d, d_rope, g,
+                               codes + ((size_t)b * cap + e) * dn,
+                               scales + ((size_t)b * cap + e) * ng,
+                               rope + ((size_t)b * cap + e) * d_rope);
+        }
+    }
+    free(y); free(y64); free(mag);
+    return worst;
+}
+
+/* ------------------------------------------------------------------ */
+/* (2) Lightning indexer scores  [N7] eq. I_{t,s}, [N9] "FP4"          */
+/* ------------------------------------------------------------------ */
+
+/* Exact FP4 dot of one indexer query head with one indexer key.
+ *   qc, kc : c/2 bytes, element 2i in the low nibble of byte i
+ *   qs, ks : c/32 ue8m0 bytes, one per block of 32 elements
+ * Block b's dot D_b = sum_{i in b} v(q_i) v(k_i) is exact (an integer
+ * multiple of 1/4, |D_b| <= 32*36).  The dot is the fp32 sum, in block
+ * order b = 0, 1, ..., of the terms t_b = D_b * 2^(eq_b + ek_b), each of
+ * which is an exact fp32 value.  With all scale bytes in [123, 127]
+ * (2^-4 .. 2^0) every partial sum is exact as well, so the result is the
+ * exact dot product, whatever the order; *inexact (if given) is set when a
+ * term or the sum is not exact. */
+float oracle_fp4_dot(const uint8_t* qc, const uint8_t* qs,
+                     const uint8_t* kc, const uint8_t* ks, int c, int* inexact)
+{
+    float acc = 0.0f;
+    double exact = 0.0;
+    for (int b = 0; b < c / 32; ++b) {
+        int64_t isum = 0;                             /* sum of (2q)(2k) */
+        for (int i = b * 32; i < b * 32 + 32; ++i) {
+            int qn = (qc[i >> 1] >> ((i & 1) * 4)) & 0xF;
+            int kn = (kc[i >> 1] >> ((i & 1) * 4)) & 0xF;
+            double qv = oracle_e2m1_value(qn), kv = oracle_e2m1_value(kn);
+            isum += (int64_t)llround(2.0 * qv) * (int64_t)llround(2.0 * kv);
+        }
+        double term = ldexp((double)isum, (int)qs[b] - 127 + (int)ks[b] - 127 - 2);
+        float t32 = (float)term;
+        if (inexact && (double)t32 != term) *inexact = 1;
+        acc = acc + t32;
+        exact += term;
+    }
+    if (inexact && (double)acc != exact) *inexact = 1;
+    return acc;
+}
+
+/* Index scores for B*Tq queries against Nc_cap indexer keys per sequence.
+ *   q_codes [B][Tq][Hi][c/2], q_sf [B][Tq][Hi][c/32], w [B][Tq][Hi] fp32
+ *   k_codes [B][Nc_cap][c/2], k_sf [B][Nc_cap][c/32]
+ *   q_pos   [B][Tq] absolute position t of each query
+ *   scores  [B][Tq][Nc_cap] fp32
+ * Eligibility (causal block rule): entry s exists for query t only if its
+ * block ends at or before t, i.e. (s+1)*m - 1 <= t.  Ineligible -> -inf.
+ * Score: acc = +0; for h = 0..Hi-1 in order: acc = acc + w_h * ReLU(dot_h)
+ * (fp32 multiply then fp32 add; ReLU(x) = x > 0 ? x : +0).
+ * One key per entry serves every indexer head (K^IComp_s carries no head
+ * index in [N7]).  Returns the number of inexact dots seen. */
+int64_t oracle_index_scores(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
+                            const uint8_t* k_codes, const uint8_t* k_sf,
+                            const int32_t* q_pos, int B, int Tq, int64_t Nc_cap,
+                            int Hi, int c, int m, float* scores)
+{
+    int64_t n_inexact = 0;
+    const int cb = c / 2, cs = c / 32;
+    for (int b = 0; b < B; ++b) {
+        for (int t = 0; t < Tq; ++t) {
+            int64_t pos = q_pos[(size_t)b * Tq + t];
+            int64_t elig = (pos + 1) / m;
+            if (elig > Nc_cap) elig = Nc_cap;
+            if (elig < 0) elig = 0;
+            float* row = scores + ((size_t)b * Tq + t) * Nc_cap;
+            const size_t qi = (size_t)b * Tq + t;
+            for (int64_t s = 0; s < Nc_cap; ++s) {
+                if (s >= elig) { row[s] = -INFINITY; continue; }
+                const uint8_t* kc = k_codes + ((size_t)b * Nc_cap + s) * cb;
+                const uint8_t* ks = k_sf + ((size_t)b * Nc_cap + s) * cs;
+                float acc = 0.0f;
+                for (int h = 0; h < Hi; ++h) {
+                    int inexact = 0;
+                    float dot = oracle_fp4_dot(q_codes + (qi * Hi + h) * cb, q_sf + (qi * Hi + h) * cs,
+                                               kc, ks, c, &inexact);
+                    n_inexact += inexact;
+                    float relu = dot > 0.0f ? dot : 0.0f;
+                    float term = w[qi * Hi + h] * relu;
+                    acc = acc + term;
+                }
+                row[s] = acc;
+            }
+        }
+    }
+    return n_inexact;
+}
+
+/* ------------------------------------------------------------------ */
+/* (3) Top-k selection  [N7] C^SprsComp_t = {C_s | I_{t,s} in Top-k(I_t,:)} */
+/* ------------------------------------------------------------------ */
+
+typedef struct { double v; int64_t i; } scored_t;
+
+static int cmp_score_desc_index_asc(const void* a, const void* b)
+{
+    const scored_t* x = (const scored_t*)a;
+    const scored_t* y = (const scored_t*)b;
+    if (x->v > y->v) return -1;
+    if (x->v < y->v) return 1;
+    return (x->i < y->i) ? -1 : (x->i > y->i);
+}
+static int cmp_i32(const void* a, const void* b)
+{
+    int32_t x = *(const int32_t*)a, y = *(const int32_t*)b;
+    return (x > y) - (x < y);
+}
+
+/* For each of R rows: the eligible entries are s < min(Nc_cap, (pos+1)/m).
+ * Take the min(k, #eligible) largest scores; scores compare as values
+ * (+0 == -0), equal scores go to the lower index.  idx[r][:] receives the
+ * chosen indices in ascending order, padded with -1; count[r] how many. */
+void oracle_topk(const float* scores, const int32_t* q_pos, int R, int64_t Nc_cap,
+                 int m, int k, int32_t* idx, int32_t* count)
+{
+    scored_t* buf = (scored_t*)malloc(sizeof(scored_t) * (Nc_cap > 0 ? Nc_cap : 1));
+    for (int r = 0; r < R; ++r) {
+        int64_t elig = ((int64_t)q_pos[r] + 1) / m;
+        if (elig > Nc_cap) elig = Nc_cap;
+        if (elig < 0) elig = 0;
+        const float* row = scores + (size_t)r * Nc_cap;
+        for (int64_t s = 0; s < elig; ++s) { buf[s].v = (double)row[s] + 0.0; buf[s].i = s; }
+        qsort(buf, (size_t)elig, sizeof(scored_t), cmp_score_desc_index_asc);
+        int64_t kk = elig < k ? elig : k;
+        int32_t* out = idx + (size_t)r * k;
+        for (int64_t j = 0; j < kk; ++j) out[j] = (int32_t)buf[j].i;
+        qsort(out, (size_t)kk, sizeof(int32_t), cmp_i32);
+        for (int64_t j = kk; j < k; ++j) out[j] = -1;
+        count[r] = (int32_t)kk;
+    }
+    free(buf);
+}
+
+/* ------------------------------------------------------------------ */
+/* (4) Core attention  [N7] shared key-value MQA + sliding window,      */
+/*     [N8] dense over all compressed entries, [HF] figures 3 and 4    */
+/* ------------------------------------------------------------------ */
+
+/* One query token, H heads, one joint softmax over a key list made of
+ *   - n_ent compressed entries ent[0..n_ent) of one sequence's cache
+ *     (codes [.][d-d_rope] e4m3fn, scales [.][(d-d_rope)/g], rope [.][d_rope]);
+ *     the entry is both key and value (shared key-value MQA), dequantised
+ *     exactly: code value * scale for the FP8 dims, the bf16 value for the
+ *     RoPE dims;
+ *   - n_win raw bf16 tokens win[0..n_win) ([n_win][d]), key = value = token.
+ * logit_j = softmax_scale * (q_h . k_j); p = softmax(logit); o_h = sum p_j k_j.
+ * All in fp64.  out [H][d] fp64, lse [H] fp64 (natural-log log-sum-exp of
+ * the scaled logits), either may be NULL.  With no keys at all, o = 0 and
+ * lse = -inf. */
+void oracle_attend(const uint16_t* q, int H, int d, int d_rope, int g,
+                   const uint8_t* codes, const float* scales, const uint16_t* rope,
+                   const int64_t* ent, int64_t n_ent,
+                   const uint16_t* win, int64_t n_win,
+                   float softmax_scale, double* out, double* lse)
+{
+    const int dn = d - d_rope, ng = dn / g;
+    const int64_t n = n_ent + n_win;
+    double* K = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * d);
+    for (int64_t j = 0; j < n_ent; ++j) {
+        const int64_t e = ent[j];
+        double* kr = K + (size_t)j * d;
+        for (int c = 0; c < dn; ++c)
+            kr[c] = oracle_e4m3_value(codes[(size_t)e * dn + c]) * (double)scales[(size_t)e * ng + c / g];
+        for (int c = dn; c < d; ++c)
+            kr[c] = (double)oracle_bf16_to_f32(rope[(size_t)e * d_rope + (c - dn)]);
+    }
+    for (int64_t j = 0; j < n_win; ++j) {
+        double* kr = K + (size_t)(n_ent + j) * d;
+        for (int c = 0; c < d; ++c) kr[c] = (double)oracle_bf16_to_f32(win[(size_t)j * d + c]);
+    }
+    double* logit = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    for (int h = 0; h < H; ++h) {
+        const uint16_t* qh = q + (size_t)h * d;
+        double mx = -INFINITY;
+        for (int64_t j = 0; j < n; ++j) {
+            double s = 0.0;
+            for (int c = 0; c < d; ++c) s += (double)oracle_bf16_to_f32(qh[c]) * K[(size_t)j * d + c];
+            logit[j] = (double)softmax_scale * s;
+            if (logit[j] > mx) mx = logit[j];
+        }
+        double den = 0.0;
+        for (int64_t j = 0; j < n; ++j) { logit[j] = exp(logit[j] - mx); den += logit[j]; }
+        if (out) {
+            for (int c = 0; c < d; ++c) {
+                double o = 0.0;
+                for (int64_t j = 0; j < n; ++j) o += logit[j] * K[(size_t)j * d + c];
+                out[(size_t)h * d + c] = n > 0 ? o / den : 0.0;
+            }
+        }
+        if (lse) lse[h] = n > 0 ? mx + log(den) : -INFINITY;
+    }
+    free(K); free(logit);
+}
