@@ -1,0 +1,433 @@
+#!/usr/bin/env python3
+"""Benchmark of the CSA + HCA decode hot path at 1M context on B200.
+
+Workload (default ``decode_b4_1m``): batch 4, one query token per sequence at
+position 1,048,575; one CSA layer (FP4 indexer over 262,144 compressed
+entries, exact top-1024, attention over 1,024 entries + 128 window tokens)
+and one HCA layer (dense attention over 8,192 entries + 128 window tokens),
+H = 64, d = 512.  A step is one pass of the whole hot path: index scores,
+top-k, CSA attention (split-K + log-sum-exp combine), HCA attention.
+
+Metric: query tokens per second (whole job: all ranks' query tokens / max
+over ranks of the device time).  Inputs are synthetic (hca_inputs recipes)
+and resident in HBM before the timed region; the decode step is one CUDA
+graph per replica, and four independently built replicas rotate so that the
+bytes one pass touches are out of L2 (126 MB) when the replica comes back.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode_b4_1m|decode_b16_64k|prefill_4096_131k|stack61_b32_256k]
+
+Multi-GPU: one process per GPU under torchrun; each rank runs its own
+replicas (the decode batch shards over sequences with no data exchange), so
+scaling is weak.  ``--impl reference`` times the CPU oracle on the host cores
+(rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import hca_inputs as inp  # noqa: E402
+
+MEASURED = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+NOMINAL_HBM_GBS = 8000.0
+
+
+def peaks():
+    try:
+        with open(MEASURED) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+
+    REASONS = {
+        "hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+        "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+        "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+        "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+        "hw_power_brake_slowdown": "nvmlClocksEventReasonHwPowerBrakeSlowdown",
+    }
+
+    def __init__(self, index: int):
+        self.samples, self.ok, self._stop = [], False, threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not inside:      # timed region shorter than one poll: nearest samples around it
+            inside = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:3]
+        mhz = sorted(s[1] for s in inside)
+        reasons = set()
+        for s in inside:
+            for name, attr in self.REASONS.items():
+                if s[2] & getattr(self.nv, attr, 0):
+                    reasons.add(name)
+        return {"sm_mhz": mhz[len(mhz) // 2] if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(inside)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+        pg = dist
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local, pg
+
+
+def max_over_ranks(value: float, pg) -> float:
+    if pg is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+# ------------------------------------------------------------------ algorithmic bytes (decode)
+def decode_bytes(wl):
+    """Algorithmic HBM bytes of one decode step of a CSA + HCA layer pair:
+    FP4 indexer keys of every eligible CSA entry (64 B codes + 4 B scales),
+    the k selected CSA entries and every HCA entry (448 B FP8 + 28 B scales
+    + 128 B bf16 RoPE = 604 B), the 128-token bf16 windows, queries in and
+    outputs out.  Scores and split partials stay on chip / in L2."""
+    dn = wl.d - wl.d_rope
+    entry = dn + 4 * (dn // wl.g) + 2 * wl.d_rope
+    ikey = wl.c // 2 + wl.c // 32
+    T = wl.t + 1
+    nc, nh = T // 4, T // 128
+    qo = wl.H * wl.d * 2 * 2
+    per_seq = {
+        "indexer": nc * ikey + wl.Hi * (wl.c // 2 + wl.c // 32 + 4),
+        "csa_attn": min(wl.k, nc) * entry + wl.W * wl.d * 2 + qo + min(wl.k, nc) * 4,
+        "hca_attn": nh * entry + wl.W * wl.d * 2 + qo,
+    }
+    return {k: v * wl.B for k, v in per_seq.items()}
+
+
+# ------------------------------------------------------------------ CPU oracle timings
+def oracle_decode_sample(wl, seq_fraction=1.0, seed_offset=0):
+    """Build the inputs of one decode sequence on the CPU (seeded CPU draws;
+    HCA entries pooled by the oracle itself, untimed) and return a closure
+    that runs the oracle's decode of that sequence: index scores over the
+    first `seq_fraction` of the CSA entries, top-k, CSA attention, HCA
+    attention over the same fraction of HCA entries."""
+    import numpy as np
+    import oracle
+    T = wl.t + 1
+    nc = int((T // 4) * seq_fraction)
+    nh = max(1, int((T // 128) * seq_fraction))
+    d, dr, g = wl.d, wl.d_rope, wl.g
+    gen = lambda name, shape, std=1.0: inp.normal_bf16(shape, std, wl.seed + 1000 + seed_offset, name)
+    qb = inp.bf16_bits(gen("q", (wl.H, d)))
+    win = inp.bf16_bits(gen("win", (wl.W, d)))
+    # HCA entries: pool nh blocks of 128 raw tokens with the oracle (setup)
+    xr = inp.bf16_bits(gen("x", (1, nh * 128, d)))
+    gr = inp.bf16_bits(gen("gate", (1, nh * 128, d)))
+    b128 = inp.normal_f32((128, d), 0.5, wl.seed + 1000, "b128").numpy()
+    hc, hs, hr, _ = oracle.compress(xr, gr, b128, 128, nh, dr, g)
+    # CSA entries: only the selected ones are ever read; pool them on demand
+    x4 = inp.bf16_bits(gen("x4", (1, 4 * 2048, d)))
+    g4 = inp.bf16_bits(gen("g4", (1, 4 * 2048, d)))
+    b4 = inp.normal_f32((4, d), 0.5, wl.seed + 1000, "b4").numpy()
+    cc, cs, cr, _ = oracle.compress(x4, g4, b4, 4, 2048, dr, g)
+    qc = inp.uniform_bytes((1, 1, wl.Hi, wl.c // 2), wl.seed + 1000, "iq").numpy()
+    qs = inp.ue8m0_scales((1, 1, wl.Hi, wl.c // 32), wl.seed + 1000, "iqs").numpy()
+    w = inp.uniform_f32((1, 1, wl.Hi), wl.seed + 1000, "iw").numpy()
+    kc = inp.uniform_bytes((1, nc, wl.c // 2), wl.seed + 1000, "ik").numpy()
+    ks = inp.ue8m0_scales((1, nc, wl.c // 32), wl.seed + 1000, "iks").numpy()
+    pos = np.array([[4 * nc - 1]], np.int32)
+
+    def run():
+        s, _ = oracle.index_scores(qc, qs, w, kc, ks, pos, 4)
+        idx, cnt = oracle.topk(s[0], pos[0], 4, wl.k)
+        ent = idx[0, :cnt[0]] % 2048          # selected entries mapped onto the pooled sample
+        oracle.attend(qb, cc[0], cs[0], cr[0], ent, win, wl.softmax_scale, g)
+        oracle.attend(qb, hc[0], hs[0], hr[0], np.arange(nh), win, wl.softmax_scale, g)
+    return run
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args, wl):
+    """--impl reference: the CPU oracle, as it stands, on the host cores."""
+    import oracle
+    oracle.build()
+    frac = 1.0
+    run = oracle_decode_sample(wl, frac)
+    t0 = time.perf_counter(); run(); t_one = time.perf_counter() - t0
+    budget = 150.0
+    if t_one * (args.steps + args.warmup) > budget:
+        frac = max(1e-3, budget / ((args.steps + args.warmup) * t_one))
+        run = oracle_decode_sample(wl, frac)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = frac / dt
+    sample = (f"one query token (sequence) of {wl.name}: FP4 index scores over {frac:.3g} of its "
+              f"{(wl.t + 1) // 4} CSA entries, exact top-{wl.k}, CSA attention over {wl.k}+{wl.W} keys, "
+              f"HCA attention over {frac:.3g} of its {(wl.t + 1) // 128} entries + {wl.W} window tokens; "
+              "single-threaded C oracle (fp64 attention)")
+    line = {"metric": "1M-ctx CSA+HCA decode query-tok/s", "impl": "reference", "value": value,
+            "unit": "query-tok/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "global_batch": wl.B, "seq_len": wl.t + 1, "parallelism": "none"},
+            "cpu_baseline": {"value": value, "unit": "query-tok/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "query-tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm: decode
+def bench_decode(args, wl, world, rank, pg):
+    import long_context_attention_hca_b200 as hca
+    from hca_workloads import build_decode
+    from long_context_attention_hca_b200.pipeline import DecodeRunner
+
+    dev = torch.device("cuda")
+    n_rep = args.replicas
+    reps = []
+    for r in range(n_rep):
+        dw = build_decode(wl)
+        runner = DecodeRunner(dw.layers, wl.B, wl.H, wl.k, wl.t, wl.softmax_scale)
+        reps.append((dw, runner))
+    main = torch.cuda.current_stream()
+
+    # one graph per replica, with external timing events around each kernel class
+    graphs, evs = [], []
+    for dw, runner in reps:
+        s = torch.cuda.Stream()
+        s.wait_stream(main)
+        with torch.cuda.stream(s):
+            for _ in range(2):
+                runner.step(dw.q, dw.iq)
+        main.wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        ev = {}
+        runner.timing_events = ev
+        with torch.cuda.graph(g):
+            runner.step(dw.q, dw.iq, events=ev)
+        graphs.append(g)
+        evs.append(ev)
+    torch.cuda.synchronize()
+
+    for i in range(args.warmup):
+        graphs[i % n_rep].replay()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(torch.cuda.current_device()).start()
+    time.sleep(0.02)
+    barrier(pg)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.perf_counter()
+    e0.record()
+    for i in range(args.steps):
+        graphs[i % n_rep].replay()
+    e1.record()
+    torch.cuda.synchronize()
+    t_wall1 = time.perf_counter()
+    barrier(pg)
+    time.sleep(0.01)
+    clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    ms_max = max_over_ranks(ms, pg)
+
+    # per-kernel durations from the last replay of each replica graph
+    kern = {}
+    for ev in evs:
+        for name, (a, b) in ev.items():
+            kern.setdefault(name, []).append(a.elapsed_time(b))
+    kern_ms = {k: sum(v) / len(v) for k, v in kern.items()}
+
+    # ---------------- end to end through the public API: host q / indexer q in, outputs out
+    dw, runner = reps[0]
+    h_q = [t.to("cpu").pin_memory() for t in dw.q]
+    h_iq = [None if t is None else tuple(x.to("cpu").pin_memory() for x in t) for t in dw.iq]
+    h_out = [torch.empty_like(o, device="cpu").pin_memory() for o in runner.out]
+    d_q = [t.clone() for t in dw.q]
+    d_iq = [None if t is None else tuple(x.clone() for x in t) for t in dw.iq]
+    h2d = sum(t.numel() * t.element_size() for t in h_q) + sum(
+        sum(x.numel() * x.element_size() for x in t) for t in h_iq if t is not None)
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+
+    def e2e_step():
+        for a, b in zip(d_q, h_q):
+            a.copy_(b, non_blocking=True)
+        for a, b in zip(d_iq, h_iq):
+            if a is not None:
+                for x, y in zip(a, b):
+                    x.copy_(y, non_blocking=True)
+        runner.step(d_q, d_iq)
+        for a, b in zip(h_out, runner.out):
+            a.copy_(b, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    n_e2e = max(10, min(args.steps, 200))
+    barrier(pg)
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(n_e2e):
+        e2e_step()
+    f1.record()
+    torch.cuda.synchronize()
+    barrier(pg)
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / n_e2e, pg)
+
+    # ---------------- roofline of the dominant kernel
+    hbm, bf16, bf16s, src = peaks()
+    algo = decode_bytes(wl)
+    dominant = max(kern_ms, key=kern_ms.get) if kern_ms else None
+    roof = None
+    if dominant is not None:
+        ach = algo[dominant] / (kern_ms[dominant] * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": dominant, "achieved": ach, "peak": hbm, "unit": "GB/s",
+                "frac": ach / hbm, "peak_source": f"{src} (burst copy)", "traffic": None,
+                "algorithmic_bytes": algo[dominant], "avg_launch_us": kern_ms[dominant] * 1e3}
+    step_bytes = sum(algo.values())
+
+    value = world * wl.B / (ms_max * 1e-3)
+    line = {
+        "metric": "1M-ctx CSA+HCA decode query-tok/s", "value": value, "unit": "query-tok/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16/fp32 (FP8/FP4 storage)",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "global_batch": wl.B * world, "seq_len": wl.t + 1,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"inputs larger than L2: {n_rep} rotating replicas, {n_rep * step_bytes / 1e6:.0f} MB touched per cycle"},
+        "step_hbm": {"algorithmic_bytes": step_bytes, "achieved_gbs": step_bytes / (ms_max * 1e-3) / 1e9,
+                     "frac_of_measured": step_bytes / (ms_max * 1e-3) / 1e9 / hbm,
+                     "frac_of_8tbs": step_bytes / (ms_max * 1e-3) / 1e9 / NOMINAL_HBM_GBS},
+        "kernels_us": {k: v * 1e3 for k, v in kern_ms.items()},
+        "roofline": roof,
+        "clocks": clocks.summary(t_wall0, t_wall1),
+        "e2e": {"value": world * wl.B / (e2e_ms * 1e-3), "unit": "query-tok/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": reps[0][1].kernels_per_step * args.steps,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for g in graphs:
+        del g
+
+
+def cpu_baseline(wl):
+    import oracle
+    oracle.build()
+    run = oracle_decode_sample(wl, 1.0)
+    run()
+    t0 = time.perf_counter()
+    n = 0
+    while n < 3 and time.perf_counter() - t0 < 25.0:
+        run()
+        n += 1
+    dt = (time.perf_counter() - t0) / n
+    return {"value": 1.0 / dt, "unit": "query-tok/s", "cores": 1, "kind": "oracle",
+            "sample": f"one query token (sequence) of {wl.name} through the oracle: index scores over all "
+                      f"{(wl.t + 1) // 4} CSA entries, exact top-{wl.k}, CSA and HCA attention in fp64; "
+                      f"{n} repetitions, single thread"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode_b4_1m", choices=["decode_b4_1m", "decode_b16_64k"])
+    ap.add_argument("--replicas", type=int, default=4)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = inp.WORKLOADS[args.workload]
+    world, rank, local, pg = dist_setup(args.gpus)
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, wl)
+        if pg is not None:
+            pg.destroy_process_group()
+        return
+    bench_decode(args, wl, world, rank, pg)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,210 @@
+/*
+ * hca.h -- C ABI of the B200 (sm_100a) hot path of DeepSeek-V4's hybrid
+ * compressed attention: CSA (4x compression, FP4 lightning indexer, top-k)
+ * and HCA (128x compression, dense), both with the 128-token sliding window.
+ *
+ * Sources (page titles and sections):
+ *   "DeepSeek V4: Towards Highly Efficient Million Token Context
+ *    Intelligence" (papers.chlience.com reading note):
+ *      section 7 "CSA"  -- compressor (m = 4), lightning indexer
+ *                          I_{t,s} = sum_h w_{t,h} ReLU(q_{t,h} . K_s),
+ *                          Top-k selection, shared key-value MQA core
+ *                          attention, sliding-window branch;
+ *      section 8 "HCA"  -- compressor (m' = 128) equations
+ *                          S = Softmax_row(Z + B), C^Comp_i = sum_j S_j (.) C_j,
+ *                          dense attention over all compressed entries;
+ *      section 9        -- KV storage (RoPE dims BF16, the rest FP8),
+ *                          FP4 indexer, 128-token window.
+ *   "DeepSeek-V4: a million-token context that agents can actually use"
+ *    (Hugging Face blog), "Hybrid attention: CSA and HCA" and figures 3, 4.
+ *
+ * Conventions for every call
+ *   - Returns an hca_status.  Arguments are validated on the host before
+ *     anything is launched; a rejected call launches nothing.
+ *   - Every pointer is a DEVICE pointer unless stated otherwise, owned by
+ *     the caller, and must stay valid until the work queued on `stream`
+ *     has finished.  The library allocates no device memory: scratch comes
+ *     from the caller's `ws` buffer, sized by the matching *_workspace_size.
+ *   - Every pointer must be 16-byte aligned (HCA_ERR_INVALID_ARG otherwise).
+ *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream.  Calls are asynchronous and never synchronise the device.
+ *   - bf16 values travel as uint16_t bit patterns.
+ *   - Integer/byte results (FP8 codes, scales, top-k sets) are bit-exact
+ *     reproductions of the definitions below; attention outputs are fp32-
+ *     accumulated and rounded to bf16.
+ *
+ * KV cache layout (one cache per layer and compression ratio; structure of
+ * arrays, entry e of sequence b at row b*capacity + e):
+ *   codes  uint8  [B][capacity][d - d_rope]          FP8 e4m3fn
+ *   scales float  [B][capacity][(d - d_rope)/group]  fp32, amax/448
+ *   rope   bf16   [B][capacity][d_rope]
+ * Supported layouts: (d, d_rope, group) = (512, 64, 64) and (128, 32, 32).
+ */
+#ifndef HCA_B200_H
+#define HCA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HCA_OK = 0,
+    HCA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or index  */
+    HCA_ERR_UNSUPPORTED = 2,   /* valid but not implemented shape/layout       */
+    HCA_ERR_CUDA = 3,          /* a CUDA launch or query failed                */
+    HCA_ERR_WORKSPACE = 4      /* ws is NULL or smaller than required          */
+} hca_status;
+
+typedef struct {
+    int32_t d;             /* channels per entry (= attention head dim)       */
+    int32_t d_rope;        /* trailing channels stored as bf16                 */
+    int32_t scale_group;   /* FP8 channels sharing one fp32 scale              */
+} hca_kv_layout;
+
+typedef struct {
+    uint8_t*  codes;
+    float*    scales;
+    uint16_t* rope;
+    int64_t   capacity;    /* entries per sequence                             */
+} hca_kv_cache;
+
+/* Human-readable name of a status code (static string). */
+const char* hca_status_string(int status);
+/* The last cudaError_t seen by a call that returned HCA_ERR_CUDA (per thread). */
+int hca_last_cuda_error(void);
+
+/* ------------------------------------------------------------------ */
+/* Compression: softmax-gated pooling + FP8/BF16 storage.               */
+/* ------------------------------------------------------------------ */
+/* Pools n_blocks consecutive blocks of m tokens for each of B sequences
+ * (note, section 8 equations; section 7 for m = 4) and stores each pooled
+ * entry in the cache layout above (section 9).
+ *
+ *   x, gate   bf16 [B][x_seq_stride][d]: raw KV C and gate logits Z; row 0
+ *             of each sequence is the first token of block `entry_begin`
+ *             (the caller offsets the pointers), so block entry_begin+j is
+ *             rows j*m .. j*m+m-1.  Requires n_blocks*m <= x_seq_stride.
+ *   pos_bias  fp32 [m][d]: learned positional bias B, row i added to the
+ *             gate logit of the i-th token of every block.
+ *   out       entries entry_begin .. entry_begin+n_blocks-1 are written;
+ *             requires entry_begin + n_blocks <= out.capacity.
+ *
+ * Arithmetic (fixed so results are bit-exact; the pages give no precision):
+ * per channel c, z_i = fp32(gate) + bias (fp32), zmax = max z_i,
+ * e_i = E(z_i - zmax) with E the Cody-Waite / degree-7-Taylor exp in fp32,
+ * S and N = sum e_i and sum e_i*x_i accumulated from +0 in ascending i with
+ * every product and sum rounded (no FMA), y = N / S (IEEE division).  FP8
+ * channels: per group, scale = amax/448 (IEEE division; 0 when amax = 0,
+ * with codes 0), code = e4m3fn(y / scale) round-to-nearest-even,
+ * saturating at +-448.  RoPE channels: bf16(y), nearest-even.
+ * csa_compress uses m = 4, hca_compress m = 128. */
+int csa_compress(const uint16_t* x, const uint16_t* gate, int64_t x_seq_stride,
+                 const float* pos_bias, int32_t B, int64_t n_blocks,
+                 hca_kv_layout layout, hca_kv_cache out, int64_t entry_begin,
+                 void* stream);
+int hca_compress(const uint16_t* x, const uint16_t* gate, int64_t x_seq_stride,
+                 const float* pos_bias, int32_t B, int64_t n_blocks,
+                 hca_kv_layout layout, hca_kv_cache out, int64_t entry_begin,
+                 void* stream);
+
+/* ------------------------------------------------------------------ */
+/* Lightning indexer (section 7, eq. I_{t,s}; section 9: FP4).          */
+/* ------------------------------------------------------------------ */
+/*   q_codes  uint8 [B][Tq][Hi][c/2]  FP4 e2m1, element 2i in the low nibble
+ *   q_sf     uint8 [B][Tq][Hi][c/32] ue8m0 (2^(u-127)) per 32 elements
+ *   w        fp32  [B][Tq][Hi]       head weights w_{t,h}
+ *   k_codes  uint8 [B][Nc_cap][c/2]  one indexer key per compressed entry,
+ *   k_sf     uint8 [B][Nc_cap][c/32] shared by all Hi heads
+ *   q_pos    int32 [B][Tq]           absolute position t of each query
+ *   scores   fp32  [B][Tq][Nc_cap]   output
+ * Entry s is eligible for query t iff its block ends at or before t:
+ * (s+1)*m - 1 <= t; ineligible scores are -inf.
+ * dot_h = fp32 sum over blocks b = 0..c/32-1, in order, of
+ *         (exact block dot) * 2^(eq_b + ek_b - 254); with all scale bytes in
+ *         [123, 127] every term and partial sum is exact, so dot_h is the
+ *         exact FP4 dot product.
+ * score = fp32, from +0, for h = 0..Hi-1 in order: score += w_h * ReLU(dot_h)
+ *         (product rounded, then sum rounded).
+ * Supported: c in {64, 128}, 1 <= Hi <= 8, m >= 1. */
+int lightning_index(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
+                    const uint8_t* k_codes, const uint8_t* k_sf, const int32_t* q_pos,
+                    int32_t B, int32_t Tq, int64_t Nc_cap, int32_t Hi, int32_t c, int32_t m,
+                    float* scores, void* stream);
+
+/* ------------------------------------------------------------------ */
+/* Top-k selection (section 7: C^SprsComp_t = {C_s | I_{t,s} in Top-k}) */
+/* ------------------------------------------------------------------ */
+/*   scores  fp32 [R][Nc_cap]; row r belongs to the query at q_pos[r]
+ *   q_pos   int32 [R]
+ *   idx     int32 [R][k]  output: the chosen entry indices, ascending,
+ *                         padded with -1
+ *   count   int32 [R]     output: min(k, #eligible)
+ * Eligible entries are s < min(Nc_cap, (q_pos+1)/m).  The chosen set is the
+ * min(k, #eligible) largest scores under the total order (score descending,
+ * index ascending): scores compare as values (+0 == -0) and equal scores go
+ * to the lower index.  NaN scores are not supported.
+ * Supported: 1 <= k <= 4096, Nc_cap <= 2^24 (top-k splits a row over up to
+ * 16 cooperating blocks of at most 32768 scores each). */
+size_t topk_select_workspace_size(int32_t R, int64_t Nc_cap, int32_t k);
+int topk_select(const float* scores, const int32_t* q_pos, int32_t R, int64_t Nc_cap,
+                int32_t m, int32_t k, int32_t* idx, int32_t* count,
+                void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ */
+/* Core attention (section 7: shared key-value MQA + sliding window;    */
+/* section 8: dense over all compressed entries).                       */
+/* ------------------------------------------------------------------ */
+/* Decode: one query token per sequence, H heads sharing one KV head.
+ *   q        bf16 [B][H][d]
+ *   kv       the sequences' compressed cache (layout above)
+ *   idx      int32 [B][idx_stride]: CSA mode, the selected entries of each
+ *            sequence (e.g. topk_select output); only the first n_comp[b]
+ *            are read.  NULL: HCA (dense) mode, entries 0..n_comp[b]-1.
+ *   n_comp   int32 [B] (device): compressed keys of each sequence
+ *   max_comp host upper bound of n_comp[] (sizes the split-K plan)
+ *   window   bf16 [B][W][d]: the last W raw tokens, oldest first; key =
+ *            value = token (all W rows are used)
+ *   out      bf16 [B][H][d];  lse fp32 [B][H] (natural log) or NULL
+ * Per head: o = sum_j softmax_j(scale * q.k_j) k_j over the compressed keys
+ * (dequantised: code * scale, bf16 RoPE dims) and the window tokens, one
+ * joint softmax.  Split-K over the keys with a log-sum-exp combine; the
+ * contractions run on tensor cores with fp16 operands and fp32 accumulation.
+ * Supported: H in {8, 64} for d = 128 and H = 64 for d = 512; W <= 4096. */
+size_t compressed_attn_decode_workspace_size(int32_t B, int32_t H, hca_kv_layout layout,
+                                             int32_t max_comp, int32_t W);
+int compressed_attn_decode(const uint16_t* q, int32_t B, int32_t H,
+                           hca_kv_layout layout, hca_kv_cache kv,
+                           const int32_t* idx, int32_t idx_stride,
+                           const int32_t* n_comp, int32_t max_comp,
+                           const uint16_t* window, int32_t W,
+                           float softmax_scale, uint16_t* out, float* lse,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* Chunked prefill of one sequence: Tq query tokens at positions p0..p0+Tq-1,
+ * each with causal eligibility.
+ *   q       bf16 [Tq][H][d]
+ *   kv      the sequence's cache (B = 1), already holding every entry a
+ *           query can see (including the chunk's own complete blocks)
+ *   idx     int32 [Tq][idx_stride] + count int32 [Tq]: CSA mode, query i
+ *           attends to idx[i][0..count[i]);  idx = NULL: HCA (dense causal)
+ *           mode, query at position p attends to entries
+ *           s < min(kv.capacity, (p+1)/m)  (m is only used in this mode)
+ *   raw     bf16 [W-1+Tq][d]: raw tokens from position p0-(W-1) on; the
+ *           window of position p is tokens max(0, p-W+1) .. p
+ *   out     bf16 [Tq][H][d]
+ * Same attention rule as decode. */
+size_t compressed_attn_prefill_workspace_size(int32_t Tq, int32_t H, hca_kv_layout layout);
+int compressed_attn_prefill(const uint16_t* q, int32_t Tq, int32_t H, int32_t p0, int32_t m,
+                            hca_kv_layout layout, hca_kv_cache kv,
+                            const int32_t* idx, int32_t idx_stride, const int32_t* count,
+                            const uint16_t* raw, int32_t W,
+                            float softmax_scale, uint16_t* out,
+                            void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HCA_B200_H */

@@ -1,0 +1,183 @@
+// api.cu -- extern "C" entry points: argument validation, then the launch.
+// Every check happens on the host before any work is queued, so a rejected
+// call leaves the stream untouched.  See include/hca.h for the contract.
+#include <mutex>
+
+#include "common.cuh"
+
+namespace hca {
+
+int compress_launch(int m, const uint16_t* x, const uint16_t* gate, int64_t seq_stride,
+                    const float* bias, int B, int64_t n_blocks, const hca_kv_layout& L,
+                    const hca_kv_cache& out, int64_t entry_begin, cudaStream_t st);
+int index_launch(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
+                 const uint8_t* k_codes, const uint8_t* k_sf, const int32_t* q_pos,
+                 int B, int Tq, int64_t Nc_cap, int Hi, int c, int m, float* scores, cudaStream_t st);
+int topk_launch(const float* scores, const int32_t* q_pos, int R, int64_t Nc_cap, int m, int k,
+                int32_t* idx, int32_t* count, cudaStream_t st);
+size_t decode_ws_bytes(int B, int H, int D, int max_comp, int W);
+int attn_decode_launch(const uint16_t* q, int B, int H, const hca_kv_layout& L, const hca_kv_cache& kv,
+                       const int32_t* idx, int idx_stride, const int32_t* n_comp, int max_comp,
+                       const uint16_t* window, int W, float softmax_scale, uint16_t* out, float* lse,
+                       void* ws, size_t ws_bytes, cudaStream_t st);
+int attn_prefill_launch(const uint16_t* q, int Tq, int H, int p0, int m, const hca_kv_layout& L,
+                        const hca_kv_cache& kv, const int32_t* idx, int idx_stride, const int32_t* count,
+                        const uint16_t* raw, int W, float softmax_scale, uint16_t* out, cudaStream_t st);
+
+static thread_local int g_last_cuda_error = 0;
+void set_last_cuda_error(int e) { g_last_cuda_error = e; }
+
+int sm_count() {
+    static std::mutex mu;
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::lock_guard<std::mutex> lk(mu);
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+namespace {
+
+bool layout_ok(const hca_kv_layout& L) {
+    return (L.d == 512 && L.d_rope == 64 && L.scale_group == 64) ||
+           (L.d == 128 && L.d_rope == 32 && L.scale_group == 32);
+}
+
+bool cache_ptrs_ok(const hca_kv_cache& c) {
+    return c.codes && c.scales && c.rope && aligned16(c.codes) && aligned16(c.scales) && aligned16(c.rope) &&
+           c.capacity >= 0;
+}
+
+#define REQUIRE(cond) do { if (!(cond)) return HCA_ERR_INVALID_ARG; } while (0)
+#define REQ_PTR(p) REQUIRE((p) != nullptr && aligned16(p))
+
+int compress_common(int m, const uint16_t* x, const uint16_t* gate, int64_t x_seq_stride,
+                    const float* pos_bias, int32_t B, int64_t n_blocks, hca_kv_layout L,
+                    hca_kv_cache out, int64_t entry_begin, void* stream) {
+    REQUIRE(B >= 0 && n_blocks >= 0 && entry_begin >= 0);
+    if (!layout_ok(L)) return HCA_ERR_UNSUPPORTED;
+    if (B == 0 || n_blocks == 0) return HCA_OK;
+    REQ_PTR(x); REQ_PTR(gate); REQ_PTR(pos_bias);
+    REQUIRE(cache_ptrs_ok(out));
+    REQUIRE(n_blocks * m <= x_seq_stride);
+    REQUIRE(entry_begin + n_blocks <= out.capacity);
+    return compress_launch(m, x, gate, x_seq_stride, pos_bias, B, n_blocks, L, out, entry_begin,
+                           as_stream(stream));
+}
+
+}  // namespace
+}  // namespace hca
+
+using namespace hca;
+
+extern "C" {
+
+const char* hca_status_string(int status) {
+    switch (status) {
+        case HCA_OK: return "ok";
+        case HCA_ERR_INVALID_ARG: return "invalid argument";
+        case HCA_ERR_UNSUPPORTED: return "unsupported shape or layout";
+        case HCA_ERR_CUDA: return "CUDA error";
+        case HCA_ERR_WORKSPACE: return "workspace missing or too small";
+        default: return "unknown status";
+    }
+}
+
+int hca_last_cuda_error(void) { return g_last_cuda_error; }
+
+int csa_compress(const uint16_t* x, const uint16_t* gate, int64_t x_seq_stride, const float* pos_bias,
+                 int32_t B, int64_t n_blocks, hca_kv_layout layout, hca_kv_cache out,
+                 int64_t entry_begin, void* stream) {
+    return compress_common(4, x, gate, x_seq_stride, pos_bias, B, n_blocks, layout, out, entry_begin, stream);
+}
+
+int hca_compress(const uint16_t* x, const uint16_t* gate, int64_t x_seq_stride, const float* pos_bias,
+                 int32_t B, int64_t n_blocks, hca_kv_layout layout, hca_kv_cache out,
+                 int64_t entry_begin, void* stream) {
+    return compress_common(128, x, gate, x_seq_stride, pos_bias, B, n_blocks, layout, out, entry_begin, stream);
+}
+
+int lightning_index(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
+                    const uint8_t* k_codes, const uint8_t* k_sf, const int32_t* q_pos,
+                    int32_t B, int32_t Tq, int64_t Nc_cap, int32_t Hi, int32_t c, int32_t m,
+                    float* scores, void* stream) {
+    REQUIRE(B >= 0 && Tq >= 0 && Nc_cap >= 0 && m >= 1);
+    if (c != 64 && c != 128) return HCA_ERR_UNSUPPORTED;
+    if (Hi < 1 || Hi > 8) return HCA_ERR_UNSUPPORTED;
+    if (B == 0 || Tq == 0 || Nc_cap == 0) return HCA_OK;
+    REQ_PTR(q_codes); REQ_PTR(q_sf); REQ_PTR(w); REQ_PTR(k_codes); REQ_PTR(k_sf); REQ_PTR(q_pos); REQ_PTR(scores);
+    return index_launch(q_codes, q_sf, w, k_codes, k_sf, q_pos, B, Tq, Nc_cap, Hi, c, m, scores, as_stream(stream));
+}
+
+size_t topk_select_workspace_size(int32_t R, int64_t Nc_cap, int32_t k) {
+    (void)R; (void)Nc_cap; (void)k;
+    return 0;
+}
+
+int topk_select(const float* scores, const int32_t* q_pos, int32_t R, int64_t Nc_cap, int32_t m, int32_t k,
+                int32_t* idx, int32_t* count, void* ws, size_t ws_bytes, void* stream) {
+    (void)ws; (void)ws_bytes;
+    REQUIRE(R >= 0 && Nc_cap >= 0 && m >= 1);
+    if (k < 1 || k > 4096) return HCA_ERR_UNSUPPORTED;
+    if (Nc_cap > 16 * 32768LL) return HCA_ERR_UNSUPPORTED;
+    if (R == 0) return HCA_OK;
+    REQ_PTR(q_pos); REQ_PTR(idx); REQ_PTR(count);
+    if (Nc_cap > 0) REQ_PTR(scores);
+    return topk_launch(scores, q_pos, R, Nc_cap, m, k, idx, count, as_stream(stream));
+}
+
+size_t compressed_attn_decode_workspace_size(int32_t B, int32_t H, hca_kv_layout layout, int32_t max_comp, int32_t W) {
+    if (B <= 0 || max_comp < 0 || W < 0 || !layout_ok(layout)) return 0;
+    return decode_ws_bytes(B, H, layout.d, max_comp, W);
+}
+
+int compressed_attn_decode(const uint16_t* q, int32_t B, int32_t H, hca_kv_layout layout, hca_kv_cache kv,
+                           const int32_t* idx, int32_t idx_stride, const int32_t* n_comp, int32_t max_comp,
+                           const uint16_t* window, int32_t W, float softmax_scale, uint16_t* out, float* lse,
+                           void* ws, size_t ws_bytes, void* stream) {
+    REQUIRE(B >= 0 && max_comp >= 0 && W >= 0);
+    if (!layout_ok(layout)) return HCA_ERR_UNSUPPORTED;
+    if (!((layout.d == 512 && H == 64) || (layout.d == 128 && (H == 64 || (H >= 1 && H <= 16)))))
+        return HCA_ERR_UNSUPPORTED;
+    if (W > 4096) return HCA_ERR_UNSUPPORTED;
+    if (B == 0) return HCA_OK;
+    REQ_PTR(q); REQ_PTR(n_comp); REQ_PTR(out);
+    REQUIRE(cache_ptrs_ok(kv));
+    if (W > 0) REQ_PTR(window);
+    if (idx) { REQUIRE(aligned16(idx) && idx_stride >= max_comp); }
+    if (lse) REQUIRE(aligned16(lse));
+    if (ws) REQUIRE(aligned16(ws));
+    return attn_decode_launch(q, B, H, layout, kv, idx, idx_stride, n_comp, max_comp, window, W, softmax_scale,
+                              out, lse, ws, ws_bytes, as_stream(stream));
+}
+
+size_t compressed_attn_prefill_workspace_size(int32_t Tq, int32_t H, hca_kv_layout layout) {
+    (void)Tq; (void)H; (void)layout;
+    return 0;
+}
+
+int compressed_attn_prefill(const uint16_t* q, int32_t Tq, int32_t H, int32_t p0, int32_t m,
+                            hca_kv_layout layout, hca_kv_cache kv, const int32_t* idx, int32_t idx_stride,
+                            const int32_t* count, const uint16_t* raw, int32_t W, float softmax_scale,
+                            uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+    (void)ws; (void)ws_bytes;
+    REQUIRE(Tq >= 0 && p0 >= 0 && W >= 1);
+    if (!layout_ok(layout)) return HCA_ERR_UNSUPPORTED;
+    if (!((layout.d == 512 && H == 64) || (layout.d == 128 && (H == 64 || (H >= 1 && H <= 16)))))
+        return HCA_ERR_UNSUPPORTED;
+    if (W > 4096) return HCA_ERR_UNSUPPORTED;
+    if (Tq == 0) return HCA_OK;
+    REQ_PTR(q); REQ_PTR(out); REQ_PTR(raw);
+    REQUIRE(cache_ptrs_ok(kv));
+    if (idx) { REQUIRE(aligned16(idx) && count != nullptr && aligned16(count) && idx_stride >= 0); }
+    else { REQUIRE(m >= 1); }
+    return attn_prefill_launch(q, Tq, H, p0, m, layout, kv, idx, idx_stride, count, raw, W, softmax_scale, out,
+                               as_stream(stream));
+}
+
+}  // extern "C"

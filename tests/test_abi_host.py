@@ -1,0 +1,93 @@
+"""CPU tests of the C-ABI library: it loads, exports every symbol the header
+declares, and rejects bad arguments on the host before touching the GPU
+(these calls return before any CUDA call, so they run without a device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hca.h")
+
+
+def _build_lib():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("_hca_build",
+                                                  os.path.join(ROOT, "long_context_attention_hca_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return ctypes.CDLL(_build_lib())
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+([a-z_][a-z0-9_]*)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_six_calls():
+    names = declared_functions()
+    for n in ("csa_compress", "hca_compress", "lightning_index", "topk_select", "compressed_attn_decode",
+              "compressed_attn_prefill"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    lib.hca_status_string.restype = ctypes.c_char_p
+    assert lib.hca_status_string(0) == b"ok"
+    assert lib.hca_status_string(1) == b"invalid argument"
+    assert lib.hca_status_string(4) == b"workspace missing or too small"
+
+
+class Layout(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("d_rope", ctypes.c_int32), ("scale_group", ctypes.c_int32)]
+
+
+class Cache(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("rope", ctypes.c_void_p),
+                ("capacity", ctypes.c_int64)]
+
+
+def test_host_validation_without_gpu(lib):
+    V, I32, I64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    lib.csa_compress.argtypes = [V, V, I64, V, I32, I64, Layout, Cache, I64, V]
+    good = Layout(512, 64, 64)
+    cache = Cache(None, None, None, 10)
+    # unsupported layout is reported before pointers are looked at
+    assert lib.csa_compress(None, None, 8, None, 1, 1, Layout(256, 64, 64), cache, 0, None) == 2
+    # null pointers
+    assert lib.csa_compress(None, None, 8, None, 1, 1, good, cache, 0, None) == 1
+    # misaligned pointer
+    assert lib.csa_compress(V(0x1008), V(0x1000), 8, V(0x1000), 1, 1, good,
+                            Cache(0x1000, 0x1000, 0x1000, 10), 0, None) == 1
+    # empty work is a no-op
+    assert lib.csa_compress(None, None, 0, None, 0, 0, good, cache, 0, None) == 0
+    lib.lightning_index.argtypes = [V, V, V, V, V, V, I32, I32, I64, I32, I32, I32, V, V]
+    assert lib.lightning_index(None, None, None, None, None, None, 1, 1, 10, 4, 96, 4, None, None) == 2  # c
+    assert lib.lightning_index(None, None, None, None, None, None, 1, 1, 10, 9, 128, 4, None, None) == 2  # Hi
+    assert lib.lightning_index(None, None, None, None, None, None, 1, 1, 10, 4, 128, 0, None, None) == 1  # m
+    lib.topk_select.argtypes = [V, V, I32, I64, I32, I32, V, V, V, ctypes.c_size_t, V]
+    assert lib.topk_select(None, None, 1, 100, 4, 0, None, None, None, 0, None) == 2       # k = 0
+    assert lib.topk_select(None, None, 1, 1 << 20, 4, 8, None, None, None, 0, None) == 2   # Nc too large
+    assert lib.topk_select(None, None, 1, 100, 4, 8, None, None, None, 0, None) == 1       # null pointers
+    lib.compressed_attn_decode.argtypes = [V, I32, I32, Layout, Cache, V, I32, V, I32, V, I32, ctypes.c_float,
+                                           V, V, V, ctypes.c_size_t, V]
+    assert lib.compressed_attn_decode(None, 1, 32, good, cache, None, 0, None, 10, None, 128, 0.1,
+                                      None, None, None, 0, None) == 2                      # H = 32 at d = 512
+    assert lib.compressed_attn_decode(None, 1, 64, good, cache, None, 0, None, 10, None, 128, 0.1,
+                                      None, None, None, 0, None) == 1
+    lib.compressed_attn_decode_workspace_size.argtypes = [I32, I32, Layout, I32, I32]
+    lib.compressed_attn_decode_workspace_size.restype = ctypes.c_size_t
+    assert lib.compressed_attn_decode_workspace_size(0, 64, good, 10, 128) == 0

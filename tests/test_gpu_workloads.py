@@ -1,0 +1,170 @@
+"""GPU parity on the five synthetic workloads, run through the same runners
+(and launch configuration) that bench.py times.
+
+tiny_decode_1k      everything compared in full.
+decode_b16_64k,     compressed entries: sampled blocks (raw rows copied to the
+decode_b4_1m        host while they exist); index scores, top-k sets and both
+                    attention outputs: every sequence in full.
+prefill_4096_131k   the chunk's compressed entries in full, prefix entries
+                    sampled; index scores / top-k / attention on sampled
+                    query positions (first, last, block and tile edges).
+stack61_b32_256k    layers 0, 1, 2, 59, 60 and sequences 0 and 31 sampled.
+"""
+import numpy as np
+import pytest
+import torch
+
+import hca_inputs as inp
+import oracle
+from gpu_util import assert_attn_close, cache_host, host
+
+pytestmark = pytest.mark.gpu
+
+hca = pytest.importorskip("long_context_attention_hca_b200")
+from hca_workloads import build_decode, build_prefill  # noqa: E402
+from long_context_attention_hca_b200.pipeline import DecodeRunner, PrefillRunner  # noqa: E402
+
+
+class RawSampler:
+    """on_raw hook: copies the raw rows of chosen blocks to the host."""
+
+    def __init__(self, picks):
+        self.picks = picks            # {layer: [(b, j), ...]}  (block index j of that layer's ratio)
+        self.got = {}
+
+    def __call__(self, li, r, x, gate, bias):
+        for (b, j) in self.picks.get(li, []):
+            self.got[(li, b, j)] = (host(x[b:b + 1, j * r:(j + 1) * r]), host(gate[b:b + 1, j * r:(j + 1) * r]),
+                                    host(bias))
+
+
+def check_sampled_entries(wl, layers, sampler):
+    for (li, b, j), (xr, gr, br) in sampler.got.items():
+        L = layers[li]
+        c, s, r, _ = oracle.compress(xr, gr, br, L.ratio, 1, wl.d_rope, wl.g)
+        gc, gs, grp = host(L.cache.codes[b, j]), host(L.cache.scales[b, j]), host(L.cache.rope[b, j])
+        assert np.array_equal(gc, c[0, 0]), (li, b, j)
+        assert np.array_equal(gs.view(np.uint32), s[0, 0].view(np.uint32)), (li, b, j)
+        assert np.array_equal(grp, r[0, 0]), (li, b, j)
+
+
+def check_decode_layer(wl, dw, runner, li, seqs):
+    L = dw.layers[li]
+    qh = host(dw.q[li])
+    out = host(runner.out[li])
+    win = host(L.window)
+    codes, scales, rope = cache_host(L.cache)
+    if L.ratio == 4:
+        qc, qs, w = (host(t) for t in dw.iq[li])
+        kc, ks = host(L.k_codes), host(L.k_sf)
+        gpu_scores = host(runner.scores[li])
+        gpu_idx, gpu_cnt = host(runner.idx[li]), host(runner.count[li])
+    for b in seqs:
+        if L.ratio == 4:
+            pos = np.array([[wl.t]], np.int32)
+            s, n_inexact = oracle.index_scores(qc[b:b + 1], qs[b:b + 1], w[b:b + 1], kc[b:b + 1], ks[b:b + 1], pos, 4)
+            assert n_inexact == 0
+            assert np.array_equal(gpu_scores[b, 0].view(np.uint32), s[0, 0].view(np.uint32)), f"scores layer {li} b {b}"
+            idx, cnt = oracle.topk(s[0], pos[0], 4, wl.k)
+            assert gpu_cnt[b] == cnt[0] and np.array_equal(gpu_idx[b], idx[0]), f"top-k layer {li} b {b}"
+            ent = idx[0, :cnt[0]]
+        else:
+            ent = np.arange(L.n_entries)
+        ref, _ = oracle.attend(qh[b], codes[b], scales[b], rope[b], ent, win[b], wl.softmax_scale, wl.g)
+        assert_attn_close(out[b], ref, f"layer {li} (ratio {L.ratio}) seq {b}")
+
+
+def _decode_case(name, n_samples, seqs=None, layers=None):
+    wl = inp.WORKLOADS[name]
+    rng = np.random.default_rng(wl.seed)
+    ratios = [4, 128] if wl.layers == 1 else [128 if (i < 2 or i % 2) else 4 for i in range(wl.layers)]
+    check_layers = list(range(len(ratios))) if layers is None else layers
+    picks = {}
+    T = wl.t + 1
+    for li in check_layers:
+        nb = T // ratios[li]
+        js = [0, nb - 1] + list(rng.integers(0, nb, n_samples))
+        picks[li] = [(int(rng.integers(0, wl.B)), int(j)) for j in js]
+    sampler = RawSampler(picks)
+    dw = build_decode(wl, on_raw=sampler)
+    runner = DecodeRunner(dw.layers, wl.B, wl.H, wl.k, wl.t, wl.softmax_scale)
+    runner.step(dw.q, dw.iq)
+    torch.cuda.synchronize()
+    check_sampled_entries(wl, dw.layers, sampler)
+    for li in check_layers:
+        check_decode_layer(wl, dw, runner, li, range(wl.B) if seqs is None else seqs)
+    del dw, runner
+    torch.cuda.empty_cache()
+
+
+def test_tiny_decode_1k_full():
+    wl = inp.WORKLOADS["tiny_decode_1k"]
+    raw = {}
+    dw = build_decode(wl, on_raw=lambda li, r, x, g, b: raw.setdefault(li, (host(x), host(g), host(b))))
+    runner = DecodeRunner(dw.layers, wl.B, wl.H, wl.k, wl.t, wl.softmax_scale)
+    runner.step(dw.q, dw.iq)
+    torch.cuda.synchronize()
+    for li, L in enumerate(dw.layers):
+        x, g, b = raw[li]
+        c, s, r, _ = oracle.compress(x, g, b, L.ratio, L.n_entries, wl.d_rope, wl.g)
+        gc, gs, gr = cache_host(L.cache)
+        assert np.array_equal(gc, c) and np.array_equal(gs.view(np.uint32), s.view(np.uint32)) and np.array_equal(gr, r)
+        check_decode_layer(wl, dw, runner, li, range(wl.B))
+
+
+def test_decode_b16_64k():
+    _decode_case("decode_b16_64k", n_samples=40)
+
+
+def test_decode_b4_1m():
+    _decode_case("decode_b4_1m", n_samples=40)
+
+
+def test_stack61_b32_256k_sampled():
+    _decode_case("stack61_b32_256k", n_samples=6, seqs=[0, 31], layers=[0, 1, 2, 59, 60])
+
+
+def test_prefill_4096_131k_sampled():
+    wl = inp.WORKLOADS["prefill_4096_131k"]
+    pw = build_prefill(wl, keep_raw=True)
+    st = pw.state
+    runner = PrefillRunner(st, wl.t, wl.Tq, wl.H, wl.k, wl.W, wl.softmax_scale)
+    runner.step(pw.raw_chunk, pw.gate_chunk, pw.raw_window, pw.q, pw.iq)
+    torch.cuda.synchronize()
+    p0, Tq = wl.t, wl.Tq
+    # chunk entries in full, a sample of the cached prefix
+    xc, gc = host(pw.raw_chunk), host(pw.gate_chunk)
+    for cache, m, bias in ((st.csa, 4, st.bias4), (st.hca, 128, st.bias128)):
+        c, s, r, _ = oracle.compress(xc, gc, host(bias), m, Tq // m, wl.d_rope, wl.g)
+        e0 = p0 // m
+        assert np.array_equal(host(cache.codes[0, e0:]), c[0])
+        assert np.array_equal(host(cache.scales[0, e0:]).view(np.uint32), s[0].view(np.uint32))
+        assert np.array_equal(host(cache.rope[0, e0:]), r[0])
+        for j in (0, 1, e0 // 2, e0 - 1):
+            xr, gr = host(pw.x_all[:, j * m:(j + 1) * m]), host(pw.gate_all[:, j * m:(j + 1) * m])
+            c1, s1, r1, _ = oracle.compress(xr, gr, host(bias), m, 1, wl.d_rope, wl.g)
+            assert np.array_equal(host(cache.codes[0, j]), c1[0, 0])
+            assert np.array_equal(host(cache.scales[0, j]).view(np.uint32), s1[0, 0].view(np.uint32))
+    # sampled query positions
+    rows = [0, 1, 2, 3, 4, 127, 128, 511, 2047, 2048, 4094, 4095]
+    qc, qs, w = (host(t) for t in pw.iq)
+    kc, ks = host(st.k_codes), host(st.k_sf)
+    codes4, scales4, rope4 = (a[0] for a in cache_host(st.csa))
+    codes128, scales128, rope128 = (a[0] for a in cache_host(st.hca))
+    gs, gi, gcnt = host(runner.scores), host(runner.idx), host(runner.count)
+    qh, rawh = host(pw.q), host(pw.raw_window)
+    oc, oh = host(runner.out_csa), host(runner.out_hca)
+    for i in rows:
+        p = p0 + i
+        pos = np.array([[p]], np.int32)
+        s, n_inexact = oracle.index_scores(qc[:, i:i + 1], qs[:, i:i + 1], w[:, i:i + 1], kc, ks, pos, 4)
+        assert n_inexact == 0
+        assert np.array_equal(gs[0, i].view(np.uint32), s[0, 0].view(np.uint32)), f"scores row {i}"
+        idx, cnt = oracle.topk(s[0], pos[0], 4, wl.k)
+        assert gcnt[i] == cnt[0] and np.array_equal(gi[i], idx[0]), f"top-k row {i}"
+        win = rawh[i:i + wl.W]                     # positions p-127 .. p
+        ref, _ = oracle.attend(qh[i], codes4, scales4, rope4, idx[0, :cnt[0]], win, wl.softmax_scale, wl.g)
+        assert_attn_close(oc[i], ref, f"CSA pos {p}")
+        ref, _ = oracle.attend(qh[i], codes128, scales128, rope128, np.arange((p + 1) // 128), win,
+                               wl.softmax_scale, wl.g)
+        assert_attn_close(oh[i], ref, f"HCA pos {p}")

@@ -1,0 +1,88 @@
+"""CPU tests of host-side logic: the layer schedule and the KV-footprint
+figure against the pages (tests/golden), the workload parameters, and the
+multi-process timing plumbing of bench.py (gloo, world size 2)."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+GOLD = os.path.join(ROOT, "tests", "golden")
+
+
+def _golden(name):
+    rows = []
+    for line in open(os.path.join(GOLD, name)):
+        line = line.split("#", 1)[0].strip()
+        if line:
+            rows.append(line.split())
+    return rows
+
+
+@pytest.fixture(scope="module")
+def pipeline():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("_hca_build",
+                                                  os.path.join(ROOT, "long_context_attention_hca_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    from long_context_attention_hca_b200 import pipeline as p
+    return p
+
+
+def test_pro_schedule_matches_pages(pipeline):
+    gold = {int(a): int(b) for a, b in _golden("pro_layer_schedule.txt")}
+    assert len(gold) == 61
+    ratios = pipeline.pro_layer_ratios(61)
+    assert ratios == [gold[i] for i in range(61)]
+    assert ratios.count(4) == 30 and ratios.count(128) == 31
+
+
+def test_workload_parameters_match_pages():
+    import hca_inputs as inp
+    gold = {k: float(v) for k, v in _golden("page_parameters.txt")}
+    for wl in inp.WORKLOADS.values():
+        assert wl.m_csa == gold["csa_ratio"] and wl.m_hca == gold["hca_ratio"] and wl.W == gold["window"]
+        if wl.d == 512:
+            assert wl.c == gold["indexer_head_dim"]
+    assert inp.WORKLOADS["decode_b4_1m"].k == gold["topk_pro"]
+    assert inp.WORKLOADS["decode_b16_64k"].k == gold["topk_flash"]
+
+
+def test_kv_footprint_is_about_two_percent_of_gqa8(pipeline):
+    """The pages: the KV cache is about 2% of a bf16 GQA-8 (head dim 128)
+    cache.  The stack workload's resident state against that baseline."""
+    gold = {k: float(v) for k, v in _golden("page_parameters.txt")}
+    B, T = 32, 262144
+    ours = pipeline.kv_resident_bytes(B, T, pipeline.pro_layer_ratios(61))
+    gqa = pipeline.gqa_bf16_bytes(B, T, 61)
+    ratio = ours / gqa
+    assert abs(ratio - gold["kv_ratio_vs_gqa8_bf16_hd128"]) < 0.005, ratio
+    assert 43.0e9 < ours < 44.5e9
+
+
+_CHILD = r"""
+import os, sys, torch
+sys.path.insert(0, os.environ["HCA_ROOT"])
+import bench
+world, rank, local, pg = bench.dist_setup(2)
+v = bench.max_over_ranks(float(rank + 1) * 1.5, pg)
+bench.barrier(pg)
+assert v == 3.0, v
+open(os.path.join(os.environ["HCA_OUT"], "rank%d" % rank), "w").write("ok %s" % v)
+pg.destroy_process_group()
+"""
+
+
+def test_bench_max_over_ranks_gloo_world2(tmp_path):
+    env = dict(os.environ, HCA_ROOT=ROOT, HCA_OUT=str(tmp_path), MASTER_ADDR="127.0.0.1", CUDA_VISIBLE_DEVICES="")
+    script = tmp_path / "child.py"
+    script.write_text(_CHILD)
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr", "127.0.0.1", "--master-port", "29533", str(script)]
+    r = subprocess.run(cmd, env=env, capture_output=True, text=True, timeout=240)
+    assert r.returncode == 0, r.stdout + r.stderr
+    for rank in (0, 1):
+        assert (tmp_path / f"rank{rank}").read_text() == "ok 3.0"
