@@ -55,7 +55,9 @@ typedef enum {
     HCA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or index  */
     HCA_ERR_UNSUPPORTED = 2,   /* valid but not implemented shape/layout       */
     HCA_ERR_CUDA = 3,          /* a CUDA launch or query failed                */
-    HCA_ERR_WORKSPACE = 4      /* ws is NULL or smaller than required          */
+    HCA_ERR_WORKSPACE = 4,     /* ws is NULL or smaller than required          */
+    HCA_ERR_SCRATCH_LIMIT = 5  /* request needs more than the library's built-in
+                                  scratch (compressed_attn_decode_noalloc)     */
 } hca_status;
 
 typedef struct {
@@ -182,6 +184,41 @@ int compressed_attn_decode(const uint16_t* q, int32_t B, int32_t H,
                            const uint16_t* window, int32_t W,
                            float softmax_scale, uint16_t* out, float* lse,
                            void* ws, size_t ws_bytes, void* stream);
+
+/* Decode attention for callers that cannot allocate device memory.
+ * No passage of the pages corresponds to this call: it is the same
+ * computation as compressed_attn_decode (same arguments minus ws/ws_bytes,
+ * same split-K plan and kernels, so the same outputs), but the split-K
+ * partials go to a scratch array built into the library instead of a
+ * caller-provided workspace.  It is meant for code that has no way to get
+ * device memory at the point of the call: for example a plug-in running
+ * inside a host engine that owns every byte of device memory and forbids
+ * allocation after start-up, or a latency-critical path where the implicit
+ * device synchronisation of cudaMalloc/cudaFree is not acceptable.  The call
+ * itself allocates nothing (no cudaMalloc, no cudaFree, no library
+ * allocator).
+ *   - Limit: the scratch is 16 MiB
+ *     (HCA_NOALLOC_SCRATCH_BYTES); a request whose split-K workspace
+ *     (compressed_attn_decode_workspace_size) exceeds it is rejected with
+ *     HCA_ERR_SCRATCH_LIMIT and nothing is launched.
+ *   - The scratch is a per-device global of the library: every GPU on which
+ *     the library is used keeps those 16 MiB until the process exits.
+ *   - The first call on a device looks up the scratch's device address with
+ *     that device current (a one-time set-up per device); make that first
+ *     call before any stream capture.
+ *   - Every call on a device shares the one scratch array, which keeps the
+ *     previous call's contents; the kernels overwrite every partial they
+ *     read, so nothing needs clearing.  Calls whose work overlaps on the GPU
+ *     (different streams, or different host threads, without ordering
+ *     between them) race on the scratch and give wrong results: order them. */
+#define HCA_NOALLOC_SCRATCH_BYTES (16u << 20)
+int compressed_attn_decode_noalloc(const uint16_t* q, int32_t B, int32_t H,
+                                   hca_kv_layout layout, hca_kv_cache kv,
+                                   const int32_t* idx, int32_t idx_stride,
+                                   const int32_t* n_comp, int32_t max_comp,
+                                   const uint16_t* window, int32_t W,
+                                   float softmax_scale, uint16_t* out, float* lse,
+                                   void* stream);
 
 /* Chunked prefill of one sequence: Tq query tokens at positions p0..p0+Tq-1,
  * each with causal eligibility.

@@ -27,7 +27,7 @@ if not os.path.exists(LIB_PATH):
 
 _lib = ctypes.CDLL(LIB_PATH)
 
-HCA_OK, HCA_ERR_INVALID_ARG, HCA_ERR_UNSUPPORTED, HCA_ERR_CUDA, HCA_ERR_WORKSPACE = range(5)
+HCA_OK, HCA_ERR_INVALID_ARG, HCA_ERR_UNSUPPORTED, HCA_ERR_CUDA, HCA_ERR_WORKSPACE, HCA_ERR_SCRATCH_LIMIT = range(6)
 
 EXPORTED = (
     "hca_status_string", "hca_last_cuda_error", "csa_compress", "hca_compress", "lightning_index",

@@ -84,6 +84,7 @@ const char* hca_status_string(int status) {
         case HCA_ERR_UNSUPPORTED: return "unsupported shape or layout";
         case HCA_ERR_CUDA: return "CUDA error";
         case HCA_ERR_WORKSPACE: return "workspace missing or too small";
+        case HCA_ERR_SCRATCH_LIMIT: return "request exceeds the library's built-in scratch (16 MiB)";
         default: return "unknown status";
     }
 }

@@ -18,6 +18,8 @@
 // output accumulator in registers:  warp (hg, half) owns heads
 // 16*hg .. 16*hg+15 and output dims half*D/2 .. ; the two halves exchange
 // their partial q.k sums through shared memory so both see the same logits.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace hca {
@@ -491,4 +493,85 @@ int attn_prefill_launch(const uint16_t* q, int Tq, int H, int p0, int m, const h
     return dispatch(p, L.d, Tq, st);
 }
 
+// ------------------------------------------------------------------
+// Decode attention without a caller workspace.
+//
+// For callers that cannot allocate device memory when they call us (a
+// plug-in inside an engine that owns all device memory and allows no
+// allocation after start-up; a latency-critical path that cannot afford
+// cudaMalloc's implicit synchronisation), the split-K partials live in this
+// file-scope array instead of a caller buffer.  The array is a global of the
+// loaded library, so every device it runs on keeps HCA_NOALLOC_SCRATCH_BYTES
+// until the process exits.  Host code must not pass `g_noalloc_scratch`
+// itself to a kernel: in host code that name is only a host-side stand-in.
+// The device address is looked up once per device, with that device
+// current, by cudaGetSymbolAddress (so the first call on a device should
+// come before any stream capture), and that address is what the kernels get.
+// All calls on a device share the array; the kernels write every partial
+// before reading it, so no clearing is needed, but calls that overlap on the
+// GPU race on it.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[HCA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+void* noalloc_scratch_address(int* status) {
+    static std::mutex mu;
+    static void* addr[64] = {nullptr};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64) {
+        set_last_cuda_error(static_cast<int>(e));
+        *status = HCA_ERR_CUDA;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lk(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || p == nullptr) {
+            set_last_cuda_error(static_cast<int>(e));
+            *status = HCA_ERR_CUDA;
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    *status = HCA_OK;
+    return addr[dev];
+}
+
+bool noalloc_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
 }  // namespace hca
+
+extern "C" int compressed_attn_decode_noalloc(const uint16_t* q, int32_t B, int32_t H, hca_kv_layout layout,
+                                              hca_kv_cache kv, const int32_t* idx, int32_t idx_stride,
+                                              const int32_t* n_comp, int32_t max_comp, const uint16_t* window,
+                                              int32_t W, float softmax_scale, uint16_t* out, float* lse,
+                                              void* stream) {
+    using namespace hca;
+    // the same argument rules as compressed_attn_decode
+    if (!(B >= 0 && max_comp >= 0 && W >= 0)) return HCA_ERR_INVALID_ARG;
+    const bool layout_ok = (layout.d == 512 && layout.d_rope == 64 && layout.scale_group == 64) ||
+                           (layout.d == 128 && layout.d_rope == 32 && layout.scale_group == 32);
+    if (!layout_ok) return HCA_ERR_UNSUPPORTED;
+    if (!((layout.d == 512 && H == 64) || (layout.d == 128 && (H == 64 || (H >= 1 && H <= 16)))))
+        return HCA_ERR_UNSUPPORTED;
+    if (W > 4096) return HCA_ERR_UNSUPPORTED;
+    if (B == 0) return HCA_OK;
+    if (!q || !noalloc_aligned16(q) || !n_comp || !noalloc_aligned16(n_comp) || !out || !noalloc_aligned16(out))
+        return HCA_ERR_INVALID_ARG;
+    if (!kv.codes || !kv.scales || !kv.rope || !noalloc_aligned16(kv.codes) || !noalloc_aligned16(kv.scales) ||
+        !noalloc_aligned16(kv.rope) || kv.capacity < 0)
+        return HCA_ERR_INVALID_ARG;
+    if (W > 0 && (!window || !noalloc_aligned16(window))) return HCA_ERR_INVALID_ARG;
+    if (idx && (!noalloc_aligned16(idx) || idx_stride < max_comp)) return HCA_ERR_INVALID_ARG;
+    if (lse && !noalloc_aligned16(lse)) return HCA_ERR_INVALID_ARG;
+    const size_t need = decode_ws_bytes(B, H, layout.d, max_comp, W);
+    if (need > HCA_NOALLOC_SCRATCH_BYTES) return HCA_ERR_SCRATCH_LIMIT;
+    int st = HCA_OK;
+    void* scratch = noalloc_scratch_address(&st);
+    if (st != HCA_OK) return st;
+    return attn_decode_launch(q, B, H, layout, kv, idx, idx_stride, n_comp, max_comp, window, W, softmax_scale,
+                              out, lse, scratch, HCA_NOALLOC_SCRATCH_BYTES, as_stream(stream));
+}
