@@ -165,6 +165,7 @@ def decode_bytes(wl):
         "indexer": nc * ikey + wl.Hi * (wl.c // 2 + wl.c // 32 + 4),
         "csa_attn": min(wl.k, nc) * entry + wl.W * wl.d * 2 + qo + min(wl.k, nc) * 4,
         "hca_attn": nh * entry + wl.W * wl.d * 2 + qo,
+        "topk": nc * 4 + wl.k * 4 + 8,          # scores read (L2-resident at this size), indices written
     }
     return {k: v * wl.B for k, v in per_seq.items()}
 
@@ -389,6 +390,112 @@ def bench_decode(args, wl, world, rank, pg):
         del g
 
 
+def prefill_flops(wl):
+    """Algorithmic work of one prefill chunk: attention 4*H*d flop per
+    (query, key) pair over each query's CSA keys (min(k, eligible) + window)
+    and HCA keys (eligible entries + window); indexer 2*Hi*c int ops per
+    (query, eligible CSA entry)."""
+    p0, Tq, W = wl.t, wl.Tq, wl.W
+    att = ind = 0
+    for p in range(p0, p0 + Tq):
+        e4, e128 = (p + 1) // 4, (p + 1) // 128
+        win = min(W, p + 1)
+        att += min(wl.k, e4) + win + e128 + win
+        ind += e4
+    return 4 * wl.H * wl.d * att, 2 * wl.Hi * wl.c * ind
+
+
+def bench_prefill(args, wl, world, rank, pg):
+    from hca_workloads import build_prefill
+    from long_context_attention_hca_b200.pipeline import PrefillRunner
+    pw = build_prefill(wl)
+    runner = PrefillRunner(pw.state, wl.t, wl.Tq, wl.H, wl.k, wl.W, wl.softmax_scale)
+    args_step = (pw.raw_chunk, pw.gate_chunk, pw.raw_window, pw.q, pw.iq)
+    for _ in range(max(1, args.warmup)):
+        runner.step(*args_step, events=None)
+    torch.cuda.synchronize()
+    ev = {}
+    runner.step(*args_step, events=ev)
+    torch.cuda.synchronize()
+    kern_ms = {k: a.elapsed_time(b) for k, (a, b) in ev.items()}
+    clocks = ClockSampler(torch.cuda.current_device()).start()
+    barrier(pg)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    e0.record()
+    for _ in range(args.steps):
+        runner.step(*args_step)
+    e1.record()
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    barrier(pg)
+    clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, pg)
+    fl_att, op_ind = prefill_flops(wl)
+    hbm, bf16, bf16s, src = peaks()
+    line = {"metric": "prefill tokens/s", "value": world * wl.Tq / (ms * 1e-3), "unit": "tok/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp16/fp32 (FP8/FP4 storage)", "data": "synthetic",
+            "config": {"workload": wl.name, "chunk": wl.Tq, "p0": wl.t, "parallelism": "single GPU"},
+            "tflops": {"attention": fl_att / (ms * 1e-3) / 1e12, "indexer_int": op_ind / (ms * 1e-3) / 1e12,
+                       "total": (fl_att + op_ind) / (ms * 1e-3) / 1e12,
+                       "frac_of_bf16_measured": (fl_att + op_ind) / (ms * 1e-3) / 1e12 / bf16},
+            "kernels_us": {k: v * 1e3 for k, v in kern_ms.items()},
+            "clocks": clocks.summary(t0, t1)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def bench_stack(args, wl, world, rank, pg):
+    from hca_workloads import build_decode
+    from long_context_attention_hca_b200.pipeline import (DecodeRunner, gqa_bf16_bytes, kv_resident_bytes,
+                                                           pro_layer_ratios)
+    dw = build_decode(wl)
+    runner = DecodeRunner(dw.layers, wl.B, wl.H, wl.k, wl.t, wl.softmax_scale)
+    main = torch.cuda.current_stream()
+    s = torch.cuda.Stream()
+    s.wait_stream(main)
+    with torch.cuda.stream(s):
+        runner.step(dw.q, dw.iq)
+    main.wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    ev = {}
+    with torch.cuda.graph(g):
+        runner.step(dw.q, dw.iq, events=ev)
+    for _ in range(max(1, args.warmup)):
+        g.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(torch.cuda.current_device()).start()
+    barrier(pg)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    e0.record()
+    for _ in range(args.steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    barrier(pg)
+    clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, pg)
+    per = {k: a.elapsed_time(b) * 1e3 for k, (a, b) in ev.items()}
+    ratios = pro_layer_ratios(wl.layers)
+    resident = kv_resident_bytes(wl.B, wl.t + 1, ratios)
+    gqa = gqa_bf16_bytes(wl.B, wl.t + 1, wl.layers)
+    line = {"metric": "61-layer decode step", "value": world * wl.B / (ms * 1e-3), "unit": "query-tok/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16/fp32 (FP8/FP4 storage)",
+            "data": "synthetic", "config": {"workload": wl.name, "global_batch": wl.B, "seq_len": wl.t + 1,
+                                            "layers": wl.layers, "parallelism": "single GPU"},
+            "kv_resident_bytes": resident, "gqa8_bf16_bytes": gqa, "kv_ratio": resident / gqa,
+            "kernels_us_last_replay": per, "clocks": clocks.summary(t0, t1)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def cpu_baseline(wl):
     import oracle
     oracle.build()
@@ -412,7 +519,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode_b4_1m", choices=["decode_b4_1m", "decode_b16_64k"])
+    ap.add_argument("--workload", default="decode_b4_1m",
+                    choices=["decode_b4_1m", "decode_b16_64k", "prefill_4096_131k", "stack61_b32_256k"])
     ap.add_argument("--replicas", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -424,7 +532,12 @@ def main():
         if pg is not None:
             pg.destroy_process_group()
         return
-    bench_decode(args, wl, world, rank, pg)
+    if wl.prefill:
+        bench_prefill(args, wl, world, rank, pg)
+    elif wl.layers > 1:
+        bench_stack(args, wl, world, rank, pg)
+    else:
+        bench_decode(args, wl, world, rank, pg)
     if pg is not None:
         pg.destroy_process_group()
 

@@ -77,6 +77,11 @@ typedef struct {
 const char* hca_status_string(int status);
 /* The last cudaError_t seen by a call that returned HCA_ERR_CUDA (per thread). */
 int hca_last_cuda_error(void);
+/* Device-side error word of the current device: non-zero when a kernel gave
+ * up a bounded wait on its own pipeline barriers (its outputs are then NaN).
+ * Reads and clears the word; synchronises with the device.  -1 if the word
+ * cannot be read. */
+int hca_take_device_error(void);
 
 /* ------------------------------------------------------------------ */
 /* Compression: softmax-gated pooling + FP8/BF16 storage.               */

@@ -50,6 +50,13 @@ _lib.hca_status_string.argtypes = [ctypes.c_int]
 _lib.hca_status_string.restype = ctypes.c_char_p
 _lib.hca_last_cuda_error.argtypes = []
 _lib.hca_last_cuda_error.restype = ctypes.c_int
+_lib.hca_take_device_error.argtypes = []
+_lib.hca_take_device_error.restype = ctypes.c_int
+
+
+def take_device_error() -> int:
+    """Read and clear the device error word (non-zero: a kernel gave up a bounded wait)."""
+    return int(_lib.hca_take_device_error())
 for _name in ("csa_compress", "hca_compress"):
     getattr(_lib, _name).argtypes = [_V, _V, _I64, _V, _I32, _I64, Layout, CacheStruct, _I64, _V]
     getattr(_lib, _name).restype = ctypes.c_int

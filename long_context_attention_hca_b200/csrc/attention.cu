@@ -431,6 +431,18 @@ int heads_padded(int D, int H) { return (D == 128 && H <= 16) ? 16 : 64; }
 
 }  // namespace
 
+// tensor-core (tcgen05) path for d = 512, H = 64: attention_tc.cu
+void tc_decode_plan(int B, int max_comp, int W, bool sparse, int& n_splits, int& tiles_per_split);
+size_t tc_decode_ws_bytes(int B, int max_comp, int W, bool sparse);
+int tc_attn_decode_launch(const uint16_t* q, int B, int H, const hca_kv_cache& kv, const int32_t* idx,
+                          int idx_stride, const int32_t* n_comp, int max_comp, const uint16_t* window, int W,
+                          float softmax_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
+                          cudaStream_t st);
+int tc_attn_prefill_launch(const uint16_t* q, int Tq, int H, int p0, int m, const hca_kv_cache& kv,
+                           const int32_t* idx, int idx_stride, const int32_t* count, const uint16_t* raw, int W,
+                           float softmax_scale, uint16_t* out, cudaStream_t st);
+static bool use_tc(int D, int H) { return D == 512 && H == 64; }
+
 // split-K plan shared by the workspace query and the launch
 void decode_plan(int B, int max_comp, int W, int& n_splits, int& tiles_per_split) {
     const int n_tiles = static_cast<int>(ceil_div(static_cast<int64_t>(max_comp) + W, attn::TK));
@@ -442,6 +454,10 @@ void decode_plan(int B, int max_comp, int W, int& n_splits, int& tiles_per_split
 }
 
 size_t decode_ws_bytes(int B, int H, int D, int max_comp, int W) {
+    if (use_tc(D, H)) {
+        const size_t a = tc_decode_ws_bytes(B, max_comp, W, true), b = tc_decode_ws_bytes(B, max_comp, W, false);
+        return a > b ? a : b;
+    }
     int ns, tps;
     decode_plan(B, max_comp, W, ns, tps);
     if (ns <= 1) return 0;
@@ -454,6 +470,9 @@ int attn_decode_launch(const uint16_t* q, int B, int H, const hca_kv_layout& L, 
                        const uint16_t* window, int W, float softmax_scale, uint16_t* out, float* lse,
                        void* ws, size_t ws_bytes, cudaStream_t st) {
     if (B == 0) return HCA_OK;
+    if (use_tc(L.d, H))
+        return tc_attn_decode_launch(q, B, H, kv, idx, idx_stride, n_comp, max_comp, window, W, softmax_scale, out,
+                                     lse, ws, ws_bytes, st);
     attn::Params p = {};
     p.q = q; p.H = H;
     p.codes = kv.codes; p.scales = kv.scales; p.rope = kv.rope; p.cap = kv.capacity;
@@ -478,6 +497,8 @@ int attn_prefill_launch(const uint16_t* q, int Tq, int H, int p0, int m, const h
                         const hca_kv_cache& kv, const int32_t* idx, int idx_stride, const int32_t* count,
                         const uint16_t* raw, int W, float softmax_scale, uint16_t* out, cudaStream_t st) {
     if (Tq == 0) return HCA_OK;
+    if (use_tc(L.d, H))
+        return tc_attn_prefill_launch(q, Tq, H, p0, m, kv, idx, idx_stride, count, raw, W, softmax_scale, out, st);
     attn::Params p = {};
     p.q = q; p.H = H;
     p.codes = kv.codes; p.scales = kv.scales; p.rope = kv.rope; p.cap = kv.capacity;

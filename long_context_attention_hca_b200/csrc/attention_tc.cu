@@ -1,0 +1,647 @@
+// attention_tc.cu -- core attention of CSA and HCA on the sm_100a tensor
+// cores (tcgen05 + TMEM), for decode (split-K) and chunked prefill, d = 512,
+// H = 64 query heads sharing one KV head.
+//
+// "DeepSeek V4: Towards Highly Efficient Million Token Context Intelligence"
+// (papers.chlience.com reading note), section 7: shared key-value MQA (the
+// compressed entry is both key and value) plus the sliding-window branch;
+// section 8: HCA attends densely to every compressed entry; section 9: FP8
+// entries with BF16 RoPE dims.  One joint softmax over compressed and window
+// keys.
+//
+// One CTA = one (query token, split): 64 heads against a run of 64-key tiles.
+//   S    = Q . K^T      M = 64 heads (TMEM lanes 32w + r, r < 16), N = 64 keys,
+//                       K = 512; Q (fp16, K-major SW128) stays in shared memory.
+//   O^T += V^T . P^T    M = 128 output dims (4 M-tiles), N = 64 heads,
+//                       K = 64 keys; V^T is the key tile itself read MN-major,
+//                       P^T the softmax probabilities stored K-major.
+// TMEM: S in NBUF buffers of 32 columns + O^T (4 x 64 columns).
+// Warp roles (512 threads):
+//   warps 0-3   softmax: one thread per head row of S (lanes 0..15 of each
+//               warp); online softmax in base 2 with a lazy rescale (O^T and
+//               l are rescaled only when a head's running max grows by more
+//               than 8, so P <= 2^8 in fp16); all 128 threads (= the 128
+//               TMEM lanes of O^T) apply a rescale and run the epilogue.
+//   warps 4-15  three producer groups; group g dequantises tiles g, g+3,
+//               ... (FP8 code x fp32 scale -> fp16, bf16 -> fp16) into key
+//               buffer g; each thread holds one tile's raw loads (8 units of
+//               16 dims) and issues them before it waits for the buffer, and
+//               prefetches the gather indices of its next tile, so three
+//               tiles of HBM reads are in flight per SM.  Once the group has
+//               stored a tile, one of its threads issues that tile's QK
+//               MMAs, so the tensor pipe computes ahead of the softmax.
+//   The softmax issues PV(i) (thread 0) once all four warps stored P(i).
+//   tcgen05.commit tracks the issuing thread's own MMAs, so each issuer
+//   signals the barriers of the work it issued.
+// Every mbarrier wait is bounded; a timeout sets the device error word,
+// raises the CTA's abort flag, drains the issued MMAs and frees TMEM.
+#include <mutex>
+
+#include "common.cuh"
+
+namespace hca {
+
+__device__ int g_tc_device_error = 0;
+
+namespace tc {
+
+constexpr int D = 512;
+constexpr int HP = 64;
+constexpr int TK = 32;                       // keys per tile
+constexpr int NBUF = 3;                      // key tiles (and S tiles) in flight
+constexpr int NSOFT = 4, GROUP_WARPS = 4, NPROD = NBUF * GROUP_WARPS;
+constexpr int NWARPS = NSOFT + NPROD;
+constexpr int NTHREADS = NWARPS * 32;        // 512
+constexpr int QBLK = 8192;                   // Q column block: 64 head rows x 128 B (SW128)
+constexpr int KBLK = TK * 128;               // key column block: 32 key rows x 128 B
+constexpr int Q_OFF = 0;                     // 8 column blocks (64 KB)
+constexpr int K_OFF = 8 * QBLK;              // NBUF buffers x 8 column blocks (3 x 32 KB)
+constexpr int P_OFF = K_OFF + NBUF * 8 * KBLK;   // 64 head rows x 128 B (keys 0..31 used)
+constexpr int SMEM_BYTES = P_OFF + QBLK + 1024;  // + alignment slack
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t S_COL = 0;                // S buffer b at columns 32 b
+constexpr uint32_t O_COL = 128;              // O^T M-tile mt at 128 + 64 mt
+constexpr float RESCALE_THRESHOLD = 8.0f;    // log2 units
+constexpr long long WAIT_LIMIT = 1ll << 24;  // polls before a wait is declared stuck
+
+struct Params {
+    const uint16_t* q;          // [units][H][D] bf16
+    int H;
+    const uint8_t* codes;
+    const float* scales;
+    const uint16_t* rope;
+    int64_t cap;
+    int prefill;
+    const int32_t* idx;
+    int idx_stride;
+    const int32_t* n_comp;
+    int dense_m;
+    int p0;
+    const uint16_t* win;
+    int W;
+    float scale_log2;
+    int n_splits, tiles_per_split;
+    uint16_t* out;
+    float* lse;
+    float* part_o;              // [units][splits][HP][D]
+    float* part_ml;             // [units][splits][2][HP]
+};
+
+// ------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ uint32_t mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok;
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(dst), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void mma_f16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                 :: "r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(bar) : "memory");
+}
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(n) : "memory"); }
+
+#define TMEM_LD16(taddr, r, o)                                                                                     \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];" \
+                 : "=r"(r[o + 0]), "=r"(r[o + 1]), "=r"(r[o + 2]), "=r"(r[o + 3]), "=r"(r[o + 4]), "=r"(r[o + 5]),    \
+                   "=r"(r[o + 6]), "=r"(r[o + 7]), "=r"(r[o + 8]), "=r"(r[o + 9]), "=r"(r[o + 10]), "=r"(r[o + 11]),  \
+                   "=r"(r[o + 12]), "=r"(r[o + 13]), "=r"(r[o + 14]), "=r"(r[o + 15])                                \
+                 : "r"(taddr))
+#define TMEM_ST16(taddr, r, o)                                                                                     \
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" \
+                 :: "r"(taddr), "r"(r[o + 0]), "r"(r[o + 1]), "r"(r[o + 2]), "r"(r[o + 3]), "r"(r[o + 4]),            \
+                   "r"(r[o + 5]), "r"(r[o + 6]), "r"(r[o + 7]), "r"(r[o + 8]), "r"(r[o + 9]), "r"(r[o + 10]),         \
+                   "r"(r[o + 11]), "r"(r[o + 12]), "r"(r[o + 13]), "r"(r[o + 14]), "r"(r[o + 15]) : "memory")
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// shared-memory matrix descriptor, 128-byte swizzle (sm_100 format)
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+           (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// instruction descriptor, kind::f16: fp16 A and B, fp32 accumulator
+__device__ __forceinline__ constexpr uint32_t idesc_f16(int M, int N, int a_mn, int b_mn) {
+    return (1u << 4) | (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16) |
+           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+// byte offset of (row, 16-byte chunk c in 0..7) inside an SW128 column block
+__device__ __forceinline__ uint32_t sw128(int row, int c) {
+    return static_cast<uint32_t>((row >> 3) * 1024 + (row & 7) * 128 + ((c ^ (row & 7)) << 4));
+}
+
+struct UnitKeys {
+    int n_c, n_w;
+    const int32_t* ent;
+    int64_t kv_row0;
+    const uint16_t* wrow;
+};
+
+__device__ __forceinline__ UnitKeys unit_keys(const Params& p, int64_t u) {
+    UnitKeys k;
+    if (!p.prefill) {
+        const int nc = p.n_comp[u];
+        k.n_c = nc < 0 ? 0 : nc;
+        k.ent = p.idx ? p.idx + u * p.idx_stride : nullptr;
+        k.kv_row0 = u * p.cap;
+        k.wrow = p.win + static_cast<size_t>(u) * p.W * D;
+        k.n_w = p.W;
+    } else {
+        const int64_t pos = p.p0 + u;
+        if (p.idx) {
+            const int nc = p.n_comp[u];
+            k.n_c = nc < 0 ? 0 : nc;
+            k.ent = p.idx + u * p.idx_stride;
+        } else {
+            const int64_t e = (pos + 1) / p.dense_m;
+            k.n_c = static_cast<int>(e > p.cap ? p.cap : e);
+            k.ent = nullptr;
+        }
+        k.kv_row0 = 0;
+        const int64_t first = pos - (p.W - 1) > 0 ? pos - (p.W - 1) : 0;
+        k.wrow = p.win + static_cast<size_t>(first - (p.p0 - (p.W - 1))) * D;
+        k.n_w = static_cast<int>(pos - first + 1);
+    }
+    return k;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+    return pack_half2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+}
+
+// Bounded wait; returns false on timeout (and records it).
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    for (long long it = 0; it < WAIT_LIMIT; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 1023) == 1023 && *abort_flag) return false;
+    }
+    *abort_flag = 1;
+    atomicExch(&g_tc_device_error, 1);
+    return false;
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ __align__(8) uint64_t bar_kempty[NBUF], bar_sfull[NBUF], bar_pempty, bar_drain;
+    __shared__ uint32_t tmem_base_slot;
+    __shared__ float s_alpha[HP], s_l[HP];
+    __shared__ int s_resc_w[NSOFT];
+    __shared__ volatile int s_abort;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t u = blockIdx.x;
+    const int split = blockIdx.y;
+    const UnitKeys uk = unit_keys(p, u);
+    const int n_tot = uk.n_c + uk.n_w;
+    const int n_tiles_all = (n_tot + TK - 1) / TK;
+    const int t_begin = split * p.tiles_per_split;
+    const int t_end = min(n_tiles_all, t_begin + p.tiles_per_split);
+    const int n_tiles = t_end > t_begin ? t_end - t_begin : 0;
+    const uint32_t sbase = smem_u32(smem);
+
+    if (tid == 0) {
+        for (int i = 0; i < NBUF; ++i) {
+            mbar_init(smem_u32(&bar_kempty[i]), 1);
+            mbar_init(smem_u32(&bar_sfull[i]), 1);
+        }
+        mbar_init(smem_u32(&bar_pempty), 1);
+        mbar_init(smem_u32(&bar_drain), NBUF + 1);   // the MMA-issuing threads
+        s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) { tmem_alloc(smem_u32(&tmem_base_slot), TMEM_COLS); tmem_relinquish(); }
+    // Q -> fp16, K-major SW128: column block cb = dims 64cb.., row = head
+    for (int w = tid; w < HP * (D / 8); w += NTHREADS) {
+        const int r = w / (D / 8), c = w % (D / 8);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (r < p.H) {
+            const uint4 b = __ldg(reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(u) * p.H + r) * D + c * 8));
+            v = make_uint4(bf16x2_to_f16x2(b.x), bf16x2_to_f16x2(b.y), bf16x2_to_f16x2(b.z), bf16x2_to_f16x2(b.w));
+        }
+        *reinterpret_cast<uint4*>(smem + Q_OFF + (c >> 3) * QBLK + sw128(r, c & 7)) = v;
+    }
+    fence_async_smem();
+    fence_before();
+    __syncthreads();
+    fence_after();
+    const uint32_t tmem = tmem_base_slot;
+
+    constexpr uint32_t id_qk = idesc_f16(64, TK, 0, 0);   // S[64 heads x 32 keys]
+    constexpr uint32_t id_pv = idesc_f16(128, HP, 1, 0);
+    if (warp >= NSOFT) {
+        // ------------------------------------------------------------ producers
+        const int grp = (warp - NSOFT) / GROUP_WARPS;                  // key buffer
+        const int pt = ((warp - NSOFT) % GROUP_WARPS) * 32 + lane;     // 0..127 within the group
+        const int c16 = pt & 31;                 // this thread's 16-dim unit (same for all its keys)
+        const int d0 = c16 * 16;
+        const int dn = D - 64;
+        // unit j of a tile: key row r = pt / 32 + 4 j
+        int32_t ent_next[8];
+        auto fetch_ent = [&](int i, int32_t (&e)[8]) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int slot = (t_begin + i) * TK + (pt >> 5) + 4 * j;
+                e[j] = (i < n_tiles && slot < uk.n_c) ? (uk.ent ? uk.ent[slot] : slot) : -1;
+            }
+        };
+        fetch_ent(grp, ent_next);
+        for (int i = grp; i < n_tiles; i += NBUF) {
+            int32_t ent[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) ent[j] = ent_next[j];
+            const int slot0 = (t_begin + i) * TK;
+            // raw loads of this tile (registers only: no buffer needed yet)
+            uint32_t raw[8][8];
+            float sc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = (pt >> 5) + 4 * j;
+                const int slot = slot0 + r;
+                sc[j] = 0.0f;
+#pragma unroll
+                for (int z = 0; z < 8; ++z) raw[j][z] = 0;
+                if (slot < uk.n_c) {
+                    const int64_t e = ent[j];
+                    if (e >= 0 && e < p.cap) {
+                        const int64_t er = uk.kv_row0 + e;
+                        if (d0 < dn) {
+                            const uint4 cv = __ldg(reinterpret_cast<const uint4*>(p.codes + er * dn + d0));
+                            raw[j][0] = cv.x; raw[j][1] = cv.y; raw[j][2] = cv.z; raw[j][3] = cv.w;
+                            sc[j] = __ldg(p.scales + er * (dn / 64) + d0 / 64);
+                        } else {
+                            const uint4* rp = reinterpret_cast<const uint4*>(p.rope + er * 64 + (d0 - dn));
+                            const uint4 a = __ldg(rp), bq = __ldg(rp + 1);
+                            raw[j][0] = a.x; raw[j][1] = a.y; raw[j][2] = a.z; raw[j][3] = a.w;
+                            raw[j][4] = bq.x; raw[j][5] = bq.y; raw[j][6] = bq.z; raw[j][7] = bq.w;
+                        }
+                    }
+                } else if (slot < n_tot) {
+                    const uint4* rp = reinterpret_cast<const uint4*>(uk.wrow + static_cast<size_t>(slot - uk.n_c) * D + d0);
+                    const uint4 a = __ldg(rp), bq = __ldg(rp + 1);
+                    raw[j][0] = a.x; raw[j][1] = a.y; raw[j][2] = a.z; raw[j][3] = a.w;
+                    raw[j][4] = bq.x; raw[j][5] = bq.y; raw[j][6] = bq.z; raw[j][7] = bq.w;
+                }
+            }
+            fetch_ent(i + NBUF, ent_next);       // gather indices of this group's next tile
+            const int use = i / NBUF;
+            if (use >= 1 && !wait_bar(smem_u32(&bar_kempty[grp]), (use - 1) & 1, &s_abort)) break;
+            uint8_t* kb = smem + K_OFF + grp * 8 * KBLK;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = (pt >> 5) + 4 * j;
+                const bool fp8 = slot0 + r < uk.n_c && d0 < dn;
+                uint32_t h[8];
+                if (fp8) {
+                    const float s_ = sc[j];
+#pragma unroll
+                    for (int z = 0; z < 4; ++z) {
+                        const float2 a = unpack_half2(e4m3x2_to_f16x2(static_cast<uint16_t>(raw[j][z] & 0xFFFFu)));
+                        const float2 bb = unpack_half2(e4m3x2_to_f16x2(static_cast<uint16_t>(raw[j][z] >> 16)));
+                        h[2 * z] = pack_half2(a.x * s_, a.y * s_);
+                        h[2 * z + 1] = pack_half2(bb.x * s_, bb.y * s_);
+                    }
+                } else {
+#pragma unroll
+                    for (int z = 0; z < 8; ++z) h[z] = bf16x2_to_f16x2(raw[j][z]);
+                }
+                // dims 16 c16 .. +15 = chunks 2 c16, 2 c16 + 1 of column block c16 / 4
+                uint8_t* blk = kb + (c16 >> 2) * KBLK;
+                const int c8 = (2 * c16) & 7;
+                *reinterpret_cast<uint4*>(blk + sw128(r, c8)) = make_uint4(h[0], h[1], h[2], h[3]);
+                *reinterpret_cast<uint4*>(blk + sw128(r, c8 + 1)) = make_uint4(h[4], h[5], h[6], h[7]);
+            }
+            fence_async_smem();
+            named_bar(2 + grp, GROUP_WARPS * 32);
+            if (pt == 0) {
+                fence_after();
+                const uint32_t kbuf = sbase + K_OFF + grp * 8 * KBLK;
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    mma_f16(tmem + S_COL + grp * TK, sdesc(sbase + Q_OFF + (kk >> 2) * QBLK + (kk & 3) * 32, 16, 1024),
+                            sdesc(kbuf + (kk >> 2) * KBLK + (kk & 3) * 32, 16, 1024), id_qk, kk > 0);
+                }
+                mma_commit(smem_u32(&bar_sfull[grp]));
+            }
+        }
+        if (pt == 0) mma_commit(smem_u32(&bar_drain));
+    } else {
+        // ------------------------------------------------------------ softmax (warps 0-3)
+        const int h = warp * 16 + lane;              // head row of S (valid for lane < 16)
+        const bool hrow = lane < 16;
+        float m_used = -INFINITY, l_run = 0.0f;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        bool ok = true;
+        for (int i = 0; i < n_tiles; ++i) {
+            const int b = i % NBUF;
+            if (!wait_bar(smem_u32(&bar_sfull[b]), (i / NBUF) & 1, &s_abort)) { ok = false; break; }
+            fence_after();
+            uint32_t sr[TK];
+            TMEM_LD16(lane_base + S_COL + b * TK + 0, sr, 0);
+            TMEM_LD16(lane_base + S_COL + b * TK + 16, sr, 16);
+            tmem_wait_ld();
+            const int nvalid = min(TK, n_tot - (t_begin + i) * TK);
+            float tmax = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < TK; ++c) {
+                const float v = c < nvalid ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
+                sr[c] = __float_as_uint(v);
+                tmax = fmaxf(tmax, v);
+            }
+            // the P buffer is free and O^T is stable once PV(i-1) has completed
+            if (i >= 1) {
+                if (!wait_bar(smem_u32(&bar_pempty), (i - 1) & 1, &s_abort)) { ok = false; break; }
+                fence_after();
+            }
+            bool resc = false;
+            float alpha = 1.0f;
+            if (hrow) {
+                const float m_new = fmaxf(m_used, tmax);
+                if (i == 0) {
+                    m_used = m_new;
+                } else if (m_new > m_used + RESCALE_THRESHOLD) {
+                    resc = true;
+                    alpha = exp2f(m_used - m_new);
+                    m_used = m_new;
+                    l_run *= alpha;
+                }
+                s_alpha[h] = alpha;
+            }
+            const unsigned wr = __ballot_sync(0xffffffffu, resc);
+            if (lane == 0) s_resc_w[warp] = wr != 0u;
+            named_bar(1, NSOFT * 32);
+            if (s_resc_w[0] | s_resc_w[1] | s_resc_w[2] | s_resc_w[3]) {
+                // this thread owns TMEM lane 32 warp + lane = one output dim of each M-tile
+#pragma unroll 1
+                for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll
+                    for (int c0 = 0; c0 < HP; c0 += 16) {
+                        uint32_t o[16];
+                        TMEM_LD16(lane_base + O_COL + mt * HP + c0, o, 0);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * s_alpha[c0 + j]);
+                        TMEM_ST16(lane_base + O_COL + mt * HP + c0, o, 0);
+                    }
+                }
+                tmem_wait_st();
+            }
+            if (hrow) {
+                float rs = 0.0f;
+#pragma unroll
+                for (int c8 = 0; c8 < TK / 8; ++c8) {
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int z = 0; z < 4; ++z) {
+                        const float a = exp2f(__uint_as_float(sr[c8 * 8 + 2 * z]) - m_used);
+                        const float bq = exp2f(__uint_as_float(sr[c8 * 8 + 2 * z + 1]) - m_used);
+                        pk[z] = pack_half2(a, bq);
+                        const float2 f = unpack_half2(pk[z]);
+                        rs += f.x + f.y;
+                    }
+                    *reinterpret_cast<uint4*>(smem + P_OFF + sw128(h, c8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+                l_run += rs;
+            }
+            fence_async_smem();
+            fence_before();
+            named_bar(1, NSOFT * 32);
+            if (tid == 0) {
+                fence_after();
+                const uint32_t kb = sbase + K_OFF + b * 8 * KBLK;
+                // V^T read MN-major from the key tile: dims in atoms of 64 (column blocks,
+                // KBLK apart), keys in atoms of 8 rows (1024 B apart)
+                for (int mt = 0; mt < 4; ++mt)
+                    for (int kk = 0; kk < TK / 16; ++kk)
+                        mma_f16(tmem + O_COL + mt * HP, sdesc(kb + 2 * mt * KBLK + kk * 2048, KBLK, 1024),
+                                sdesc(sbase + P_OFF + kk * 32, 16, 1024), id_pv, (i > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(smem_u32(&bar_pempty));
+                mma_commit(smem_u32(&bar_kempty[b]));
+            }
+        }
+        if (tid == 0) mma_commit(smem_u32(&bar_drain));
+        // ---- epilogue: wait for the last PV, then O^T / l -> out (or the split partials)
+        if (ok && n_tiles > 0) {
+            ok = wait_bar(smem_u32(&bar_pempty), (n_tiles - 1) & 1, &s_abort);
+            fence_after();
+        }
+        if (hrow) s_l[h] = l_run;
+        named_bar(1, NSOFT * 32);
+        const int L = warp * 32 + lane;              // output dim within each M-tile
+        const size_t uo = static_cast<size_t>(u);
+        const float qnan = __int_as_float(0x7fc00000);
+        if (p.n_splits == 1) {
+#pragma unroll 1
+            for (int mt = 0; mt < 4; ++mt) {
+                const int dim = mt * 128 + L;
+#pragma unroll
+                for (int c0 = 0; c0 < HP; c0 += 16) {
+                    uint32_t o[16];
+                    if (n_tiles > 0) {
+                        TMEM_LD16(lane_base + O_COL + mt * HP + c0, o, 0);
+                        tmem_wait_ld();
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int hh = c0 + j;
+                        if (hh < p.H) {
+                            const float l = s_l[hh];
+                            float v = (n_tiles > 0 && l > 0.0f) ? __uint_as_float(o[j]) / l : 0.0f;
+                            if (!ok) v = qnan;
+                            p.out[(uo * p.H + hh) * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+                        }
+                    }
+                }
+            }
+            if (p.lse && hrow && h < p.H)
+                p.lse[uo * p.H + h] = (l_run > 0.0f && ok) ? (m_used + log2f(l_run)) * 0.69314718055994531f
+                                                          : (ok ? -INFINITY : qnan);
+        } else {
+            const size_t ps = uo * p.n_splits + split;
+            float* po = p.part_o + ps * HP * D;
+            if (n_tiles > 0) {
+#pragma unroll 1
+                for (int mt = 0; mt < 4; ++mt) {
+                    const int dim = mt * 128 + L;
+#pragma unroll
+                    for (int c0 = 0; c0 < HP; c0 += 16) {
+                        uint32_t o[16];
+                        TMEM_LD16(lane_base + O_COL + mt * HP + c0, o, 0);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) po[static_cast<size_t>(c0 + j) * D + dim] = ok ? __uint_as_float(o[j]) : qnan;
+                    }
+                }
+            }
+            if (hrow) {
+                float* ml = p.part_ml + ps * 2 * HP;
+                ml[h] = m_used;
+                ml[HP + h] = ok ? l_run : qnan;
+            }
+        }
+    }
+    fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        // every issued MMA has completed before TMEM is freed
+        if (lane == 0)
+            for (long long it = 0; it < WAIT_LIMIT; ++it)
+                if (mbar_try_wait(smem_u32(&bar_drain), 0)) break;
+        __syncwarp();
+        fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// Log-sum-exp combine of split partials (base-2 maxima): grid (unit, head),
+// 128 threads x 4 dims.
+__global__ void __launch_bounds__(128) combine_tc_kernel(Params p) {
+    const int64_t u = blockIdx.x;
+    const int h = blockIdx.y;
+    const int S = p.n_splits;
+    const float* ml0 = p.part_ml + static_cast<size_t>(u) * S * 2 * HP;
+    float M = -INFINITY;
+    for (int s = 0; s < S; ++s) {
+        const float ls = ml0[s * 2 * HP + HP + h];
+        if (ls > 0.0f) M = fmaxf(M, ml0[s * 2 * HP + h]);
+    }
+    float L = 0.0f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+    bool bad = false;
+    const int d0 = threadIdx.x * 4;
+    for (int s = 0; s < S; ++s) {
+        const float ms = ml0[s * 2 * HP + h], ls = ml0[s * 2 * HP + HP + h];
+        if (ls != ls) bad = true;
+        if (!(ls > 0.0f)) continue;
+        const float wgt = exp2f(ms - M);
+        L += wgt * ls;
+        const float4 v = *reinterpret_cast<const float4*>(p.part_o + ((static_cast<size_t>(u) * S + s) * HP + h) * D + d0);
+        acc[0] += wgt * v.x; acc[1] += wgt * v.y; acc[2] += wgt * v.z; acc[3] += wgt * v.w;
+    }
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+    const float qnan = __int_as_float(0x7fc00000);
+    __nv_bfloat162 a = __floats2bfloat162_rn(bad ? qnan : acc[0] * inv, bad ? qnan : acc[1] * inv);
+    __nv_bfloat162 b = __floats2bfloat162_rn(bad ? qnan : acc[2] * inv, bad ? qnan : acc[3] * inv);
+    uint2 w;
+    w.x = *reinterpret_cast<uint32_t*>(&a);
+    w.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p.out + (static_cast<size_t>(u) * p.H + h) * D + d0) = w;
+    if (p.lse && threadIdx.x == 0)
+        p.lse[u * p.H + h] = bad ? qnan : (L > 0.0f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY);
+}
+
+}  // namespace tc
+
+// ---------------------------------------------------------------- host side
+namespace {
+
+int launch_tc(tc::Params& p, int64_t units, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         tc::SMEM_BYTES);
+    if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
+    tc::attn_tc_kernel<<<dim3(static_cast<unsigned>(units), p.n_splits), tc::NTHREADS, tc::SMEM_BYTES, st>>>(p);
+    HCA_CHECK_LAUNCH();
+    if (p.n_splits > 1) {
+        tc::combine_tc_kernel<<<dim3(static_cast<unsigned>(units), p.H), tc::D / 4, 0, st>>>(p);
+        HCA_CHECK_LAUNCH();
+    }
+    return HCA_OK;
+}
+
+}  // namespace
+
+// Split plan of the tensor-core decode path: sparse (CSA) lists favour many
+// short splits (latency after top-k); dense (HCA) lists favour a few tiles
+// per CTA so the pipeline fills and the partials stay small.
+void tc_decode_plan(int B, int max_comp, int W, bool sparse, int& n_splits, int& tiles_per_split) {
+    const int n_tiles = static_cast<int>(ceil_div(static_cast<int64_t>(max_comp) + W, tc::TK));
+    const int min_tps = sparse ? 4 : 12;      // tiles of 32 keys
+    int splits = sm_count() / (B > 0 ? B : 1);
+    const int cap_by_len = static_cast<int>(ceil_div(n_tiles > 0 ? n_tiles : 1, min_tps));
+    if (splits > cap_by_len) splits = cap_by_len;
+    if (splits < 1) splits = 1;
+    tiles_per_split = static_cast<int>(ceil_div(n_tiles > 0 ? n_tiles : 1, splits));
+    n_splits = static_cast<int>(ceil_div(n_tiles > 0 ? n_tiles : 1, tiles_per_split));
+}
+
+size_t tc_decode_ws_bytes(int B, int max_comp, int W, bool sparse) {
+    int ns, tps;
+    tc_decode_plan(B, max_comp, W, sparse, ns, tps);
+    if (ns <= 1) return 0;
+    return static_cast<size_t>(B) * ns * tc::HP * (static_cast<size_t>(tc::D) + 2) * sizeof(float) + 256;
+}
+
+int tc_attn_decode_launch(const uint16_t* q, int B, int H, const hca_kv_cache& kv, const int32_t* idx,
+                          int idx_stride, const int32_t* n_comp, int max_comp, const uint16_t* window, int W,
+                          float softmax_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
+                          cudaStream_t st) {
+    if (B == 0) return HCA_OK;
+    tc::Params p = {};
+    p.q = q; p.H = H;
+    p.codes = kv.codes; p.scales = kv.scales; p.rope = kv.rope; p.cap = kv.capacity;
+    p.prefill = 0;
+    p.idx = idx; p.idx_stride = idx_stride; p.n_comp = n_comp;
+    p.win = window; p.W = W;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    tc_decode_plan(B, max_comp, W, idx != nullptr, p.n_splits, p.tiles_per_split);
+    p.out = out; p.lse = lse;
+    if (p.n_splits > 1) {
+        const size_t need = tc_decode_ws_bytes(B, max_comp, W, idx != nullptr);
+        if (ws == nullptr || ws_bytes < need) return HCA_ERR_WORKSPACE;
+        p.part_o = reinterpret_cast<float*>(ws);
+        p.part_ml = p.part_o + static_cast<size_t>(B) * p.n_splits * tc::HP * tc::D;
+    }
+    return launch_tc(p, B, st);
+}
+
+int tc_attn_prefill_launch(const uint16_t* q, int Tq, int H, int p0, int m, const hca_kv_cache& kv,
+                           const int32_t* idx, int idx_stride, const int32_t* count, const uint16_t* raw, int W,
+                           float softmax_scale, uint16_t* out, cudaStream_t st) {
+    if (Tq == 0) return HCA_OK;
+    tc::Params p = {};
+    p.q = q; p.H = H;
+    p.codes = kv.codes; p.scales = kv.scales; p.rope = kv.rope; p.cap = kv.capacity;
+    p.prefill = 1;
+    p.idx = idx; p.idx_stride = idx_stride; p.n_comp = count;
+    p.dense_m = m; p.p0 = p0;
+    p.win = raw; p.W = W;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.n_splits = 1;
+    p.tiles_per_split = 1 << 28;
+    p.out = out; p.lse = nullptr;
+    return launch_tc(p, Tq, st);
+}
+
+// Reads and clears the device error word of the tensor-core attention
+// (a bounded wait that gave up).  Synchronous.
+int tc_take_device_error() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_tc_device_error, sizeof(int)) != cudaSuccess) return -1;
+    if (v) {
+        const int z = 0;
+        cudaMemcpyToSymbol(g_tc_device_error, &z, sizeof(int));
+    }
+    return v;
+}
+
+}  // namespace hca

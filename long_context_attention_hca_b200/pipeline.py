@@ -176,22 +176,40 @@ class PrefillRunner:
         self.side = torch.cuda.Stream(device=dev)
         self.kernels_per_step = 6
 
-    def step(self, raw_chunk, gate_chunk, raw_window, q, iq):
+    def step(self, raw_chunk, gate_chunk, raw_window, q, iq, events: Optional[dict] = None):
         """raw_chunk, gate_chunk: [1][Tq][d] bf16 tokens p0..p0+Tq-1;
         raw_window: [(W-1)+Tq][d] bf16 tokens from p0-(W-1); q: [Tq][H][d];
-        iq = (codes [1][Tq][Hi][c/2], sf, w [1][Tq][Hi])."""
+        iq = (codes [1][Tq][Hi][c/2], sf, w [1][Tq][Hi]).  events: as in
+        DecodeRunner.step (names compress, indexer, topk, csa_attn, hca_attn)."""
         st, p0, Tq = self.st, self.p0, self.Tq
         main = torch.cuda.current_stream()
-        csa_compress(raw_chunk, gate_chunk, st.bias4, Tq // CSA_RATIO, st.csa, entry_begin=p0 // CSA_RATIO)
-        hca_compress(raw_chunk, gate_chunk, st.bias128, Tq // HCA_RATIO, st.hca, entry_begin=p0 // HCA_RATIO)
+
+        def timed(name, fn):
+            if events is None:
+                return fn()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            events[name] = (a, b)
+
+        def compress():
+            csa_compress(raw_chunk, gate_chunk, st.bias4, Tq // CSA_RATIO, st.csa, entry_begin=p0 // CSA_RATIO)
+            hca_compress(raw_chunk, gate_chunk, st.bias128, Tq // HCA_RATIO, st.hca, entry_begin=p0 // HCA_RATIO)
+
+        timed("compress", compress)
         self.side.wait_stream(main)
         with torch.cuda.stream(self.side):
             qc, qs, w = iq
-            lightning_index(qc, qs, w, st.k_codes, st.k_sf, self.q_pos, CSA_RATIO, scores=self.scores)
-            topk_select(self.scores.view(Tq, -1), self.q_pos.view(-1), CSA_RATIO, self.k, idx=self.idx,
-                        count=self.count)
-            compressed_attn_prefill(q, p0, CSA_RATIO, st.csa, raw_window, self.W, self.scale, idx=self.idx,
-                                    count=self.count, out=self.out_csa)
-        compressed_attn_prefill(q, p0, HCA_RATIO, st.hca, raw_window, self.W, self.scale, out=self.out_hca)
+            timed("indexer", lambda: lightning_index(qc, qs, w, st.k_codes, st.k_sf, self.q_pos, CSA_RATIO,
+                                                     scores=self.scores))
+            timed("topk", lambda: topk_select(self.scores.view(Tq, -1), self.q_pos.view(-1), CSA_RATIO, self.k,
+                                              idx=self.idx, count=self.count))
+            timed("csa_attn", lambda: compressed_attn_prefill(q, p0, CSA_RATIO, st.csa, raw_window, self.W,
+                                                              self.scale, idx=self.idx, count=self.count,
+                                                              out=self.out_csa))
+        timed("hca_attn", lambda: compressed_attn_prefill(q, p0, HCA_RATIO, st.hca, raw_window, self.W, self.scale,
+                                                          out=self.out_hca))
         main.wait_stream(self.side)
         return self.out_csa, self.out_hca
