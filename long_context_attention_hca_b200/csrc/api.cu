@@ -25,6 +25,7 @@ int attn_prefill_launch(const uint16_t* q, int Tq, int H, int p0, int m, const h
                         const uint16_t* raw, int W, float softmax_scale, uint16_t* out, cudaStream_t st);
 
 int tc_take_device_error();
+int index_take_device_error();
 
 static thread_local int g_last_cuda_error = 0;
 void set_last_cuda_error(int e) { g_last_cuda_error = e; }
@@ -93,7 +94,10 @@ const char* hca_status_string(int status) {
 
 int hca_last_cuda_error(void) { return g_last_cuda_error; }
 
-int hca_take_device_error(void) { return tc_take_device_error(); }
+int hca_take_device_error(void) {
+    const int a = tc_take_device_error(), b = index_take_device_error();
+    return (a < 0 || b < 0) ? -1 : (a | b);
+}
 
 int csa_compress(const uint16_t* x, const uint16_t* gate, int64_t x_seq_stride, const float* pos_bias,
                  int32_t B, int64_t n_blocks, hca_kv_layout layout, hca_kv_cache out,

@@ -56,8 +56,8 @@ constexpr int QBLK = 8192;                   // Q column block: 64 head rows x 1
 constexpr int KBLK = TK * 128;               // key column block: 32 key rows x 128 B
 constexpr int Q_OFF = 0;                     // 8 column blocks (64 KB)
 constexpr int K_OFF = 8 * QBLK;              // NBUF buffers x 8 column blocks (3 x 32 KB)
-constexpr int P_OFF = K_OFF + NBUF * 8 * KBLK;   // 64 head rows x 128 B (keys 0..31 used)
-constexpr int SMEM_BYTES = P_OFF + QBLK + 1024;  // + alignment slack
+constexpr int P_OFF = K_OFF + NBUF * 8 * KBLK;   // 2 x (64 head rows x 128 B, keys 0..31 used)
+constexpr int SMEM_BYTES = P_OFF + 2 * QBLK + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t S_COL = 0;                // S buffer b at columns 32 b
 constexpr uint32_t O_COL = 128;              // O^T M-tile mt at 128 + 64 mt
@@ -134,6 +134,21 @@ __device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.syn
                  :: "r"(taddr), "r"(r[o + 0]), "r"(r[o + 1]), "r"(r[o + 2]), "r"(r[o + 3]), "r"(r[o + 4]),            \
                    "r"(r[o + 5]), "r"(r[o + 6]), "r"(r[o + 7]), "r"(r[o + 8]), "r"(r[o + 9]), "r"(r[o + 10]),         \
                    "r"(r[o + 11]), "r"(r[o + 12]), "r"(r[o + 13]), "r"(r[o + 14]), "r"(r[o + 15]) : "memory")
+#define TMEM_LD32(taddr, r)                                                                                        \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"    \
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                           \
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),      \
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), \
+                   "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),          \
+                   "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),          \
+                   "=r"(r[30]), "=r"(r[31])                                                                         \
+                 : "r"(taddr))
+// 2^x with the special-function unit (approximate; x = -inf gives +0)
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -205,7 +220,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
 __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t bar_kempty[NBUF], bar_sfull[NBUF], bar_pempty, bar_drain;
+    __shared__ __align__(8) uint64_t bar_kempty[NBUF], bar_sfull[NBUF], bar_pempty[2], bar_drain;
     __shared__ uint32_t tmem_base_slot;
     __shared__ float s_alpha[HP], s_l[HP];
     __shared__ int s_resc_w[NSOFT];
@@ -227,7 +242,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
             mbar_init(smem_u32(&bar_kempty[i]), 1);
             mbar_init(smem_u32(&bar_sfull[i]), 1);
         }
-        mbar_init(smem_u32(&bar_pempty), 1);
+        mbar_init(smem_u32(&bar_pempty[0]), 1);
+        mbar_init(smem_u32(&bar_pempty[1]), 1);
         mbar_init(smem_u32(&bar_drain), NBUF + 1);   // the MMA-issuing threads
         s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -337,10 +353,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
             named_bar(2 + grp, GROUP_WARPS * 32);
             if (pt == 0) {
                 fence_after();
-                const uint32_t kbuf = sbase + K_OFF + grp * 8 * KBLK;
+                // descriptors differ per k-step only in the start address (bits 0..13, units of 16 B)
+                const uint64_t qd = sdesc(sbase + Q_OFF, 16, 1024);
+                const uint64_t kd = sdesc(sbase + K_OFF + grp * 8 * KBLK, 16, 1024);
+                const uint32_t dst = tmem + S_COL + grp * TK;
+#pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    mma_f16(tmem + S_COL + grp * TK, sdesc(sbase + Q_OFF + (kk >> 2) * QBLK + (kk & 3) * 32, 16, 1024),
-                            sdesc(kbuf + (kk >> 2) * KBLK + (kk & 3) * 32, 16, 1024), id_qk, kk > 0);
+                    const uint32_t qo = static_cast<uint32_t>(((kk >> 2) * QBLK + (kk & 3) * 32) >> 4);
+                    const uint32_t ko = static_cast<uint32_t>(((kk >> 2) * KBLK + (kk & 3) * 32) >> 4);
+                    mma_f16(dst, qd + qo, kd + ko, id_qk, kk > 0);
                 }
                 mma_commit(smem_u32(&bar_sfull[grp]));
             }
@@ -348,50 +369,65 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
         if (pt == 0) mma_commit(smem_u32(&bar_drain));
     } else {
         // ------------------------------------------------------------ softmax (warps 0-3)
-        const int h = warp * 16 + lane;              // head row of S (valid for lane < 16)
-        const bool hrow = lane < 16;
+        // head h = 16 warp + (lane & 15); lanes 0-15 hold keys 0..15 of the tile, lanes
+        // 16-31 keys 16..31 (S row h lives in TMEM lane 32 warp + (lane & 15)).
+        const int h = warp * 16 + (lane & 15);
+        const int kh = lane >> 4;
         float m_used = -INFINITY, l_run = 0.0f;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
         bool ok = true;
         for (int i = 0; i < n_tiles; ++i) {
-            const int b = i % NBUF;
+            const int b = i % NBUF, pb = i & 1;
             if (!wait_bar(smem_u32(&bar_sfull[b]), (i / NBUF) & 1, &s_abort)) { ok = false; break; }
             fence_after();
             uint32_t sr[TK];
-            TMEM_LD16(lane_base + S_COL + b * TK + 0, sr, 0);
-            TMEM_LD16(lane_base + S_COL + b * TK + 16, sr, 16);
+            TMEM_LD32(lane_base + S_COL + b * TK, sr);
             tmem_wait_ld();
             const int nvalid = min(TK, n_tot - (t_begin + i) * TK);
+            float v[16];
             float tmax = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < TK; ++c) {
-                const float v = c < nvalid ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
-                sr[c] = __float_as_uint(v);
-                tmax = fmaxf(tmax, v);
+            for (int j = 0; j < 16; ++j) {
+                const uint32_t up = __shfl_up_sync(0xffffffffu, sr[16 + j], 16);
+                const float x = __uint_as_float(kh ? up : sr[j]);
+                v[j] = (kh * 16 + j < nvalid) ? x * p.scale_log2 : -INFINITY;
+                tmax = fmaxf(tmax, v[j]);
             }
-            // the P buffer is free and O^T is stable once PV(i-1) has completed
-            if (i >= 1) {
-                if (!wait_bar(smem_u32(&bar_pempty), (i - 1) & 1, &s_abort)) { ok = false; break; }
-                fence_after();
-            }
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
             bool resc = false;
             float alpha = 1.0f;
-            if (hrow) {
-                const float m_new = fmaxf(m_used, tmax);
-                if (i == 0) {
-                    m_used = m_new;
-                } else if (m_new > m_used + RESCALE_THRESHOLD) {
-                    resc = true;
-                    alpha = exp2f(m_used - m_new);
-                    m_used = m_new;
-                    l_run *= alpha;
-                }
-                s_alpha[h] = alpha;
+            const float m_new = fmaxf(m_used, tmax);
+            if (i == 0) {
+                m_used = m_new;
+            } else if (m_new > m_used + RESCALE_THRESHOLD) {
+                resc = true;
+                alpha = ex2(m_used - m_new);
+                m_used = m_new;
+                l_run *= alpha;
             }
+            // probabilities in registers before any wait (fp16, the sum of the rounded values)
+            uint32_t pk[8];
+            float rs = 0.0f;
+#pragma unroll
+            for (int z = 0; z < 8; ++z) {
+                pk[z] = pack_half2(ex2(v[2 * z] - m_used), ex2(v[2 * z + 1] - m_used));
+                const float2 f = unpack_half2(pk[z]);
+                rs += f.x + f.y;
+            }
+            rs += __shfl_xor_sync(0xffffffffu, rs, 16);
+            l_run += rs;
+            if (lane < 16) s_alpha[h] = alpha;
             const unsigned wr = __ballot_sync(0xffffffffu, resc);
             if (lane == 0) s_resc_w[warp] = wr != 0u;
+            // P buffer pb is free once PV(i-2) has completed
+            if (i >= 2) {
+                if (!wait_bar(smem_u32(&bar_pempty[pb]), ((i - 2) >> 1) & 1, &s_abort)) { ok = false; break; }
+            }
             named_bar(1, NSOFT * 32);
             if (s_resc_w[0] | s_resc_w[1] | s_resc_w[2] | s_resc_w[3]) {
+                // O^T must be stable: PV(i-1) complete
+                if (i >= 1 && !wait_bar(smem_u32(&bar_pempty[(i - 1) & 1]), ((i - 1) >> 1) & 1, &s_abort)) { ok = false; break; }
+                fence_after();
                 // this thread owns TMEM lane 32 warp + lane = one output dim of each M-tile
 #pragma unroll 1
                 for (int mt = 0; mt < 4; ++mt) {
@@ -407,45 +443,35 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
                 }
                 tmem_wait_st();
             }
-            if (hrow) {
-                float rs = 0.0f;
-#pragma unroll
-                for (int c8 = 0; c8 < TK / 8; ++c8) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int z = 0; z < 4; ++z) {
-                        const float a = exp2f(__uint_as_float(sr[c8 * 8 + 2 * z]) - m_used);
-                        const float bq = exp2f(__uint_as_float(sr[c8 * 8 + 2 * z + 1]) - m_used);
-                        pk[z] = pack_half2(a, bq);
-                        const float2 f = unpack_half2(pk[z]);
-                        rs += f.x + f.y;
-                    }
-                    *reinterpret_cast<uint4*>(smem + P_OFF + sw128(h, c8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                }
-                l_run += rs;
-            }
+            uint8_t* pbuf = smem + P_OFF + pb * QBLK;
+            *reinterpret_cast<uint4*>(pbuf + sw128(h, 2 * kh)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(pbuf + sw128(h, 2 * kh + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             fence_async_smem();
             fence_before();
             named_bar(1, NSOFT * 32);
             if (tid == 0) {
                 fence_after();
-                const uint32_t kb = sbase + K_OFF + b * 8 * KBLK;
                 // V^T read MN-major from the key tile: dims in atoms of 64 (column blocks,
                 // KBLK apart), keys in atoms of 8 rows (1024 B apart)
+                const uint64_t vd = sdesc(sbase + K_OFF + b * 8 * KBLK, KBLK, 1024);
+                const uint64_t pd = sdesc(sbase + P_OFF + pb * QBLK, 16, 1024);
+#pragma unroll
                 for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
                     for (int kk = 0; kk < TK / 16; ++kk)
-                        mma_f16(tmem + O_COL + mt * HP, sdesc(kb + 2 * mt * KBLK + kk * 2048, KBLK, 1024),
-                                sdesc(sbase + P_OFF + kk * 32, 16, 1024), id_pv, (i > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(smem_u32(&bar_pempty));
+                        mma_f16(tmem + O_COL + mt * HP, vd + static_cast<uint32_t>((2 * mt * KBLK + kk * 2048) >> 4),
+                                pd + static_cast<uint32_t>((kk * 32) >> 4), id_pv, (i > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(smem_u32(&bar_pempty[pb]));
                 mma_commit(smem_u32(&bar_kempty[b]));
             }
         }
         if (tid == 0) mma_commit(smem_u32(&bar_drain));
         // ---- epilogue: wait for the last PV, then O^T / l -> out (or the split partials)
         if (ok && n_tiles > 0) {
-            ok = wait_bar(smem_u32(&bar_pempty), (n_tiles - 1) & 1, &s_abort);
+            ok = wait_bar(smem_u32(&bar_pempty[(n_tiles - 1) & 1]), ((n_tiles - 1) >> 1) & 1, &s_abort);
             fence_after();
         }
+        const bool hrow = lane < 16;
         if (hrow) s_l[h] = l_run;
         named_bar(1, NSOFT * 32);
         const int L = warp * 32 + lane;              // output dim within each M-tile

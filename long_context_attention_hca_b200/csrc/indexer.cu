@@ -12,6 +12,8 @@
 // of an entry (NB = c/32), so 8 (c = 128) or 16 (c = 64) entries per warp
 // step and a 16-byte load per lane; the query's int8 expansion for the
 // lane's block stays in registers for the whole stream.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace hca {
@@ -326,6 +328,257 @@ index_mma_kernel(const uint8_t* __restrict__ q_codes, const uint8_t* __restrict_
     }
 }
 
+// ------------------------------------------------------------------ tcgen05 path (c = 128, Hi = 4)
+// The tensor cores read FP4 e2m1 operands straight from shared memory
+// (tcgen05.mma kind::f8f6f4, fp32 accumulation), laid out as 16-element
+// groups in 16-byte slots (8 data bytes, then 8 bytes of zero padding) in the
+// K-major 128-byte-swizzled layout.  A = 128 keys (one per TMEM lane),
+// B = 16 columns per query: column (block b, head h) holds head h's values on
+// block b's 32 elements and zeros elsewhere, so every accumulator column is
+// one exact 32-element block dot.  The thread that owns a TMEM lane (one
+// key) applies the two ue8m0 exponents exactly and sums blocks and heads in
+// the order the C ABI defines.
+namespace itc {
+
+constexpr int kThreads = 128;
+constexpr int kStages = 4;               // key tiles resident in shared memory
+constexpr int kAhead = 4;                // key tiles of raw loads in flight per thread
+constexpr int TILE = 128;
+constexpr int TILE_BYTES = TILE * 128;   // 16 KB
+constexpr long long kWaitLimit = 1ll << 24;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ uint32_t mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok;
+}
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr) {   // K-major SW128, 8-row groups 1024 B apart
+    return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
+           (static_cast<uint64_t>(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+__device__ __forceinline__ uint32_t sw128(int row, int slot) {
+    return static_cast<uint32_t>((row >> 3) * 1024 + (row & 7) * 128 + ((slot ^ (row & 7)) << 4));
+}
+
+__device__ int g_index_device_error = 0;    // a bounded wait gave up (outputs are NaN)
+
+// QG queries per CTA (N = 16 QG accumulator columns, NBD accumulator buffers)
+template <int QG, int NBD>
+__global__ void __launch_bounds__(kThreads)
+index_tc_kernel(const uint8_t* __restrict__ q_codes, const uint8_t* __restrict__ q_sf,
+                const float* __restrict__ w, const uint8_t* __restrict__ k_codes,
+                const uint8_t* __restrict__ k_sf, const int32_t* __restrict__ q_pos,
+                int Tq, int64_t Nc_cap, int m, int64_t chunk, float* __restrict__ scores) {
+    constexpr int N = 16 * QG;
+    constexpr uint32_t NCOLS = (N * NBD) <= 32 ? 32 : (N * NBD <= 64 ? 64 : (N * NBD <= 128 ? 128 : (N * NBD <= 256 ? 256 : 512)));
+    constexpr uint32_t IDESC = (1u << 4) | (5u << 7) | (5u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+                               (static_cast<uint32_t>(TILE >> 4) << 24);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;                                  // kStages x 16 KB
+    uint8_t* sB = smem + kStages * TILE_BYTES;           // N rows x 128 B
+    __shared__ __align__(8) uint64_t bar_d[NBD];
+    __shared__ uint32_t tmem_slot;
+    __shared__ int s_eq[QG][16];                         // (uq - 127) - 127 per (query, block*4+head)
+    __shared__ float s_w[QG][4];
+    __shared__ int64_t s_elig[QG];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t qrow0 = static_cast<int64_t>(blockIdx.x) * QG;     // first query row (b * Tq + t)
+    const int64_t b = qrow0 / Tq;                                    // all QG rows share a sequence
+    const int64_t s_begin = static_cast<int64_t>(blockIdx.y) * chunk;
+    const int64_t s_end = min(s_begin + chunk, Nc_cap);
+
+    if (tid == 0) {
+        for (int i = 0; i < NBD; ++i) mbar_init(smem_u32(&bar_d[i]), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(smem_u32(&tmem_slot)), "r"(NCOLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    // query operand: row n = q*16 + blk*4 + h; slot j (elements 16j..16j+15) is block j/2
+    for (int x = tid; x < N * 8; x += kThreads) {
+        const int n = x >> 3, j = x & 7;
+        const int q = n >> 4, blk = (n >> 2) & 3, h = n & 3;
+        uint2 v = make_uint2(0, 0);
+        if ((j >> 1) == blk) v = __ldg(reinterpret_cast<const uint2*>(q_codes + ((qrow0 + q) * 4 + h) * 64 + j * 8));
+        *reinterpret_cast<uint4*>(sB + sw128(n, j)) = make_uint4(v.x, v.y, 0u, 0u);
+    }
+    for (int x = tid; x < QG * 16; x += kThreads) {
+        const int q = x >> 4, blk = (x >> 2) & 3, h = x & 3;
+        s_eq[q][x & 15] = static_cast<int>(__ldg(q_sf + ((qrow0 + q) * 4 + h) * 4 + blk)) - 254;
+    }
+    for (int x = tid; x < QG * 4; x += kThreads) s_w[x >> 2][x & 3] = __ldg(w + (qrow0 + (x >> 2)) * 4 + (x & 3));
+    if (tid < QG) {
+        int64_t e = (static_cast<int64_t>(q_pos[qrow0 + tid]) + 1) / m;
+        s_elig[tid] = e < 0 ? 0 : (e > Nc_cap ? Nc_cap : e);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = tmem_slot;
+    int64_t elig_max = 0;
+    for (int q = 0; q < QG; ++q) elig_max = max(elig_max, s_elig[q]);
+    const int64_t s_live = min(s_end, elig_max);
+    const int n_tiles = s_live > s_begin ? static_cast<int>((s_live - s_begin + TILE - 1) / TILE) : 0;
+
+    // ineligible part of the chunk: -inf (per query)
+    for (int q = 0; q < QG; ++q) {
+        float* orow = scores + static_cast<size_t>(qrow0 + q) * Nc_cap;
+        for (int64_t s = max(s_begin, s_elig[q]) + tid; s < s_end; s += kThreads) orow[s] = -INFINITY;
+    }
+
+    const uint8_t* kc = k_codes + static_cast<size_t>(b) * Nc_cap * 64;
+    const uint32_t* ks = reinterpret_cast<const uint32_t*>(k_sf + static_cast<size_t>(b) * Nc_cap * 4);
+    uint4 raw[kAhead][4];
+    uint32_t rsc[kAhead];
+    auto fetch = [&](int t, int slot) {
+        const int64_t e = s_begin + static_cast<int64_t>(t) * TILE + tid;
+        if (t < n_tiles && e < s_live) {
+            const uint4* src = reinterpret_cast<const uint4*>(kc + e * 64);
+#pragma unroll
+            for (int z = 0; z < 4; ++z) raw[slot][z] = __ldg(src + z);
+            rsc[slot] = __ldg(ks + e);
+        } else {
+#pragma unroll
+            for (int z = 0; z < 4; ++z) raw[slot][z] = make_uint4(0, 0, 0, 0);
+            rsc[slot] = 0x7F7F7F7Fu;
+        }
+    };
+#pragma unroll
+    for (int a = 0; a < kAhead; ++a) fetch(a, a);
+    uint32_t cur_sc[2] = {0u, 0u};                       // scale words of the tile whose MMA is in flight
+    bool ok = true;
+
+    auto epilogue = [&](int t, uint32_t sw) {
+        const int nb = t % NBD;
+        bool done = false;
+        for (long long it = 0; it < kWaitLimit && !done; ++it) done = mbar_try_wait(smem_u32(&bar_d[nb]), (t / NBD) & 1);
+        if (!done) { ok = false; atomicExch(&g_index_device_error, 1); }
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const int64_t e = s_begin + static_cast<int64_t>(t) * TILE + tid;
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(nb * N);
+        int ek[4];
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) ek[blk] = static_cast<int>((sw >> (8 * blk)) & 0xFFu);
+#pragma unroll 1
+        for (int q = 0; q < QG; ++q) {
+            uint32_t r[16];
+            asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                         : "r"(taddr + q * 16));
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            if (e < s_end && e < s_elig[q]) {
+                float sc = 0.0f;
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    float dot = 0.0f;
+#pragma unroll
+                    for (int blk = 0; blk < 4; ++blk) {
+                        const float t_ = __fmul_rn(__uint_as_float(r[blk * 4 + h]), pow2i(s_eq[q][blk * 4 + h] + ek[blk]));
+                        dot = blk == 0 ? t_ : __fadd_rn(dot, t_);
+                    }
+                    sc = __fadd_rn(sc, __fmul_rn(s_w[q][h], dot > 0.0f ? dot : 0.0f));
+                }
+                scores[static_cast<size_t>(qrow0 + q) * Nc_cap + e] = ok ? sc : __int_as_float(0x7fc00000);
+            }
+        }
+    };
+
+    for (int t = 0; t < n_tiles; ++t) {
+        const int st = t % kStages;
+        // stage st was last read by MMA(t - kStages), whose epilogue ran in an earlier iteration
+        uint8_t* a = sA + st * TILE_BYTES;
+#pragma unroll
+        for (int z = 0; z < 4; ++z) {
+            const uint4 v = raw[0][z];
+            *reinterpret_cast<uint4*>(a + sw128(tid, 2 * z)) = make_uint4(v.x, v.y, 0u, 0u);
+            *reinterpret_cast<uint4*>(a + sw128(tid, 2 * z + 1)) = make_uint4(v.z, v.w, 0u, 0u);
+        }
+        const uint32_t sw_t = rsc[0];
+#pragma unroll
+        for (int x = 0; x < kAhead - 1; ++x) {
+#pragma unroll
+            for (int z = 0; z < 4; ++z) raw[x][z] = raw[x + 1][z];
+            rsc[x] = rsc[x + 1];
+        }
+        fetch(t + kAhead, kAhead - 1);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        __syncthreads();
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        if (tid == 0) {
+            const uint32_t abase = smem_u32(a), bbase = smem_u32(sB);
+            const uint32_t d = tmem + static_cast<uint32_t>((t % NBD) * N);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                             "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+                             :: "r"(d), "l"(sdesc(abase + kk * 32)), "l"(sdesc(bbase + kk * 32)), "r"(IDESC), "r"(kk)
+                             : "memory");
+            }
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                         :: "r"(smem_u32(&bar_d[t % NBD])) : "memory");
+        }
+        if (t >= 1) epilogue(t - 1, cur_sc[(t - 1) & 1]);
+        cur_sc[t & 1] = sw_t;
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    }
+    if (n_tiles >= 1) epilogue(n_tiles - 1, cur_sc[(n_tiles - 1) & 1]);
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(NCOLS) : "memory");
+    }
+}
+
+template <int QG, int NBD>
+int launch_tc(const uint8_t* q_codes, const uint8_t* q_sf, const float* w, const uint8_t* k_codes,
+              const uint8_t* k_sf, const int32_t* q_pos, int64_t rows, int Tq, int64_t Nc_cap, int m,
+              float* scores, cudaStream_t st, int64_t want_ctas) {
+    const int64_t groups = rows / QG;
+    int64_t chunk = ceil_div(Nc_cap, std::max<int64_t>(1, want_ctas / std::max<int64_t>(groups, 1)));
+    chunk = ceil_div(chunk, TILE) * TILE;
+    if (chunk < TILE) chunk = TILE;
+    if (ceil_div(Nc_cap, chunk) > 65535) chunk = ceil_div(ceil_div(Nc_cap, 65535), TILE) * TILE;
+    size_t smem = static_cast<size_t>(kStages) * TILE_BYTES + 16 * QG * 128 + 1024;
+    // a CTA that takes all 512 TMEM columns must be alone on its SM: ask for
+    // more than half of the SM's shared memory
+    if (16 * QG * NBD >= 512 && smem < 120 * 1024) smem = 120 * 1024;
+    cudaError_t e = cudaFuncSetAttribute(index_tc_kernel<QG, NBD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
+    const dim3 grid(static_cast<unsigned>(groups), static_cast<unsigned>(ceil_div(Nc_cap, chunk)));
+    index_tc_kernel<QG, NBD><<<grid, kThreads, smem, st>>>(q_codes, q_sf, w, k_codes, k_sf, q_pos, Tq, Nc_cap, m,
+                                                           chunk, scores);
+    HCA_CHECK_LAUNCH();
+    return HCA_OK;
+}
+
+}  // namespace itc
+
+}  // namespace
+
+int index_take_device_error() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, itc::g_index_device_error, sizeof(int)) != cudaSuccess) return -1;
+    if (v) {
+        const int z = 0;
+        cudaMemcpyToSymbol(itc::g_index_device_error, &z, sizeof(int));
+    }
+    return v;
+}
+
+namespace {
 }  // namespace
 
 int index_launch(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
@@ -347,6 +600,15 @@ int index_launch(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
     const dim3 grid(static_cast<unsigned>(rows), static_cast<unsigned>(ceil_div(Nc_cap, chunk)));
     if (rows > 0x7FFFFFFFLL) return HCA_ERR_UNSUPPORTED;
     const bool small = Hi <= 4;
+    if (c == 128 && Hi == 4) {
+        // tensor cores on FP4 straight from shared memory: 16 queries per CTA when
+        // a sequence has many query rows (prefill), else one
+        if (Tq % 16 == 0 && Tq >= 64)
+            return itc::launch_tc<16, 2>(q_codes, q_sf, w, k_codes, k_sf, q_pos, rows, Tq, Nc_cap, m, scores, st,
+                                         4LL * sm_count());
+        return itc::launch_tc<1, 4>(q_codes, q_sf, w, k_codes, k_sf, q_pos, rows, Tq, Nc_cap, m, scores, st,
+                                    3LL * sm_count());
+    }
     if (c == 128 && Hi == 4) {
         int64_t ch = 8192;
         if (rows * ceil_div(Nc_cap, ch) < want_blocks) {
