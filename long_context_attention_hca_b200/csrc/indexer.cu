@@ -14,6 +14,8 @@
 // lane's block stays in registers for the whole stream.
 #include <algorithm>
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace hca {
@@ -43,10 +45,13 @@ __device__ __forceinline__ void fp4x8_to_i8x8(uint32_t w, uint32_t& lo, uint32_t
     }
 }
 
-// 2^(e) for an integer exponent, exact; e outside the normal range goes through ldexpf.
-__device__ __forceinline__ float pow2i(int e) {
-    if (e >= -126 && e <= 127) return __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
-    return ldexpf(1.0f, e);
+// v * 2^e rounded once (round to nearest even), for any integer e: a plain
+// product by the exact power of two when 2^e is a normal float, else ldexpf
+// (which scales with a single rounding into the subnormal range and to +-inf
+// on overflow, and keeps 0 * 2^e = 0 where 2^e itself would overflow).
+__device__ __forceinline__ float scale_pow2(float v, int e) {
+    if (e >= -126 && e <= 127) return __fmul_rn(v, __uint_as_float(static_cast<uint32_t>(e + 127) << 23));
+    return ldexpf(v, e);
 }
 
 constexpr int kWarps = 8;
@@ -131,7 +136,7 @@ index_kernel(const uint8_t* __restrict__ q_codes, const uint8_t* __restrict__ q_
 #pragma unroll
                 for (int i = 0; i < 8; ++i) acc = __dp4a(static_cast<int>(kv[i]), static_cast<int>(qv[h][i]), acc);
                 // block dot = acc / 4 exactly; times 2^(eq + ek - 254)
-                const float t = __fmul_rn(static_cast<float>(acc), pow2i(qe[h] + ke[j] - 2));
+                const float t = scale_pow2(static_cast<float>(acc), qe[h] + ke[j] - 2);
                 // ordered block sum on the entry's first lane: ((t0 + t1) + t2) + t3
                 float a = t;
 #pragma unroll
@@ -287,8 +292,8 @@ index_mma_kernel(const uint8_t* __restrict__ q_codes, const uint8_t* __restrict_
             const int ekB = static_cast<int>((sw >> (8 * (2 + (q >> 1)))) & 0xFFu);
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                tA[j][r] = __fmul_rn(D0[j + 2 * r], pow2i(eqv[0][j] + ekA));
-                tB[j][r] = __fmul_rn(D1[j + 2 * r], pow2i(eqv[1][j] + ekB));
+                tA[j][r] = scale_pow2(D0[j + 2 * r], eqv[0][j] + ekA);
+                tB[j][r] = scale_pow2(D1[j + 2 * r], eqv[1][j] + ekB);
             }
         }
         // lanes q = 0, 1 hold blocks 0 and 2; lanes q = 2, 3 blocks 1 and 3 (same heads as q - 2)
@@ -331,20 +336,30 @@ index_mma_kernel(const uint8_t* __restrict__ q_codes, const uint8_t* __restrict_
 // ------------------------------------------------------------------ tcgen05 path (c = 128, Hi = 4)
 // The tensor cores read FP4 e2m1 operands straight from shared memory
 // (tcgen05.mma kind::f8f6f4, fp32 accumulation), laid out as 16-element
-// groups in 16-byte slots (8 data bytes, then 8 bytes of zero padding) in the
-// K-major 128-byte-swizzled layout.  A = 128 keys (one per TMEM lane),
-// B = 16 columns per query: column (block b, head h) holds head h's values on
-// block b's 32 elements and zeros elsewhere, so every accumulator column is
-// one exact 32-element block dot.  The thread that owns a TMEM lane (one
-// key) applies the two ue8m0 exponents exactly and sums blocks and heads in
-// the order the C ABI defines.
+// groups in 16-byte slots (8 data bytes, then 8 bytes of padding) in the
+// K-major 128-byte-swizzled layout.  The key tiles arrive in exactly that
+// layout from the tensor memory accelerator: a tensor map of type
+// 16U4_ALIGN16B spreads 64 packed bytes per key over a 128-byte row.  It
+// writes only the data bytes (the padding is zeroed once per CTA) and its
+// transaction count is the packed size, 64 bytes per key.
+// A = 128 keys (one per TMEM lane), B = 16 columns per query: column
+// (block b, head h) holds head h's values on block b's 32 elements and zeros
+// elsewhere, so every accumulator column is one exact 32-element block dot.
+// The thread that owns a TMEM lane (one key) applies the two ue8m0 exponents
+// exactly and sums blocks and heads in the order the C ABI defines.
+//
+// Warp roles: warp 0 issues the tensor-map loads of key codes and key scales
+// into a ring of KS stages, warp 1 issues the MMAs into NBD accumulator
+// buffers, warps 2.. run the epilogue (EG warps per TMEM lane quarter, each
+// taking every EG-th query).  Every wait is bounded; a wait that gives up
+// raises the device error word and the scores of that CTA become NaN.
 namespace itc {
 
-constexpr int kThreads = 128;
-constexpr int kStages = 4;               // key tiles resident in shared memory
-constexpr int kAhead = 4;                // key tiles of raw loads in flight per thread
-constexpr int TILE = 128;
-constexpr int TILE_BYTES = TILE * 128;   // 16 KB
+constexpr int TILE = 128;                    // keys per tile (MMA M)
+constexpr int CODE_BYTES = TILE * 128;       // 16 KB of unpacked FP4 per tile
+constexpr int CODE_TX_BYTES = TILE * 64;     // the load's transaction count: packed bytes read
+constexpr int SCALE_BYTES = TILE * 4;        // ue8m0 x 4 per key
+constexpr int STAGE_BYTES = CODE_BYTES + 1024;
 constexpr long long kWaitLimit = 1ll << 24;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
@@ -357,6 +372,20 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint32_t bar, uint32_t parity)
                  : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
     return ok;
 }
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+                 :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void tma_load_1d(uint32_t dst, const CUtensorMap* map, int x, uint32_t bar) {
+    asm volatile("cp.async.bulk.tensor.1d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2}], [%3];"
+                 :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(bar) : "memory");
+}
 __device__ __forceinline__ uint64_t sdesc(uint32_t addr) {   // K-major SW128, 8-row groups 1024 B apart
     return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
            (static_cast<uint64_t>(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
@@ -367,26 +396,39 @@ __device__ __forceinline__ uint32_t sw128(int row, int slot) {
 
 __device__ int g_index_device_error = 0;    // a bounded wait gave up (outputs are NaN)
 
-// QG queries per CTA (N = 16 QG accumulator columns, NBD accumulator buffers)
-template <int QG, int NBD>
-__global__ void __launch_bounds__(kThreads)
-index_tc_kernel(const uint8_t* __restrict__ q_codes, const uint8_t* __restrict__ q_sf,
-                const float* __restrict__ w, const uint8_t* __restrict__ k_codes,
-                const uint8_t* __restrict__ k_sf, const int32_t* __restrict__ q_pos,
+// bounded wait; on give-up raise the CTA's abort flag and the device error word
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    for (long long it = 0; it < kWaitLimit; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 1023) == 1023 && *abort_flag) return false;
+    }
+    *abort_flag = 1;
+    atomicExch(&g_index_device_error, 1);
+    return false;
+}
+
+// QG queries per CTA (N = 16 QG accumulator columns), NBD accumulator buffers,
+// KS key stages, EG epilogue warps per TMEM lane quarter.
+template <int QG, int NBD, int KS, int EG>
+__global__ void __launch_bounds__(64 + 128 * EG)
+index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
+                const uint8_t* __restrict__ q_codes, const uint8_t* __restrict__ q_sf,
+                const float* __restrict__ w, const int32_t* __restrict__ q_pos,
                 int Tq, int64_t Nc_cap, int m, int64_t chunk, float* __restrict__ scores) {
     constexpr int N = 16 * QG;
     constexpr uint32_t NCOLS = (N * NBD) <= 32 ? 32 : (N * NBD <= 64 ? 64 : (N * NBD <= 128 ? 128 : (N * NBD <= 256 ? 256 : 512)));
     constexpr uint32_t IDESC = (1u << 4) | (5u << 7) | (5u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
                                (static_cast<uint32_t>(TILE >> 4) << 24);
+    constexpr int EPI = 4 * EG;                         // epilogue warps
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sA = smem;                                  // kStages x 16 KB
-    uint8_t* sB = smem + kStages * TILE_BYTES;           // N rows x 128 B
-    __shared__ __align__(8) uint64_t bar_d[NBD];
+    uint8_t* sB = smem + KS * STAGE_BYTES;              // N rows x 128 B (query operand)
+    __shared__ __align__(8) uint64_t bar_full[KS], bar_empty[KS], bar_accf[NBD], bar_acce[NBD], bar_drain;
     __shared__ uint32_t tmem_slot;
-    __shared__ int s_eq[QG][16];                         // (uq - 127) - 127 per (query, block*4+head)
+    __shared__ int s_eq[QG][16];                        // (uq - 127) - 127 per (query, block*4+head)
     __shared__ float s_w[QG][4];
     __shared__ int64_t s_elig[QG];
+    __shared__ int s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t qrow0 = static_cast<int64_t>(blockIdx.x) * QG;     // first query row (b * Tq + t)
@@ -395,26 +437,34 @@ index_tc_kernel(const uint8_t* __restrict__ q_codes, const uint8_t* __restrict__
     const int64_t s_end = min(s_begin + chunk, Nc_cap);
 
     if (tid == 0) {
-        for (int i = 0; i < NBD; ++i) mbar_init(smem_u32(&bar_d[i]), 1);
+        for (int i = 0; i < KS; ++i) { mbar_init(smem_u32(&bar_full[i]), 1); mbar_init(smem_u32(&bar_empty[i]), EPI); }
+        for (int i = 0; i < NBD; ++i) { mbar_init(smem_u32(&bar_accf[i]), 1); mbar_init(smem_u32(&bar_acce[i]), EPI); }
+        mbar_init(smem_u32(&bar_drain), 1);
+        s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0) {
+    if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(smem_u32(&tmem_slot)), "r"(NCOLS) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
+    // the loads write only the 8 data bytes of each 16-byte slot: zero the padding once
+    for (int x = tid; x < KS * (CODE_BYTES / 16); x += blockDim.x) {
+        const int st = x / (CODE_BYTES / 16), o = x % (CODE_BYTES / 16);
+        *reinterpret_cast<uint4*>(smem + st * STAGE_BYTES + o * 16) = make_uint4(0u, 0u, 0u, 0u);
+    }
     // query operand: row n = q*16 + blk*4 + h; slot j (elements 16j..16j+15) is block j/2
-    for (int x = tid; x < N * 8; x += kThreads) {
+    for (int x = tid; x < N * 8; x += blockDim.x) {
         const int n = x >> 3, j = x & 7;
         const int q = n >> 4, blk = (n >> 2) & 3, h = n & 3;
         uint2 v = make_uint2(0, 0);
         if ((j >> 1) == blk) v = __ldg(reinterpret_cast<const uint2*>(q_codes + ((qrow0 + q) * 4 + h) * 64 + j * 8));
         *reinterpret_cast<uint4*>(sB + sw128(n, j)) = make_uint4(v.x, v.y, 0u, 0u);
     }
-    for (int x = tid; x < QG * 16; x += kThreads) {
+    for (int x = tid; x < QG * 16; x += blockDim.x) {
         const int q = x >> 4, blk = (x >> 2) & 3, h = x & 3;
         s_eq[q][x & 15] = static_cast<int>(__ldg(q_sf + ((qrow0 + q) * 4 + h) * 4 + blk)) - 254;
     }
-    for (int x = tid; x < QG * 4; x += kThreads) s_w[x >> 2][x & 3] = __ldg(w + (qrow0 + (x >> 2)) * 4 + (x & 3));
+    for (int x = tid; x < QG * 4; x += blockDim.x) s_w[x >> 2][x & 3] = __ldg(w + (qrow0 + (x >> 2)) * 4 + (x & 3));
     if (tid < QG) {
         int64_t e = (static_cast<int64_t>(q_pos[qrow0 + tid]) + 1) / m;
         s_elig[tid] = e < 0 ? 0 : (e > Nc_cap ? Nc_cap : e);
@@ -432,134 +482,221 @@ index_tc_kernel(const uint8_t* __restrict__ q_codes, const uint8_t* __restrict__
     // ineligible part of the chunk: -inf (per query)
     for (int q = 0; q < QG; ++q) {
         float* orow = scores + static_cast<size_t>(qrow0 + q) * Nc_cap;
-        for (int64_t s = max(s_begin, s_elig[q]) + tid; s < s_end; s += kThreads) orow[s] = -INFINITY;
+        for (int64_t s = max(s_begin, s_elig[q]) + tid; s < s_end; s += blockDim.x) orow[s] = -INFINITY;
     }
+    const int row0 = static_cast<int>(b * Nc_cap + s_begin);        // tensor-map row of the chunk's first key
 
-    const uint8_t* kc = k_codes + static_cast<size_t>(b) * Nc_cap * 64;
-    const uint32_t* ks = reinterpret_cast<const uint32_t*>(k_sf + static_cast<size_t>(b) * Nc_cap * 4);
-    uint4 raw[kAhead][4];
-    uint32_t rsc[kAhead];
-    auto fetch = [&](int t, int slot) {
-        const int64_t e = s_begin + static_cast<int64_t>(t) * TILE + tid;
-        if (t < n_tiles && e < s_live) {
-            const uint4* src = reinterpret_cast<const uint4*>(kc + e * 64);
-#pragma unroll
-            for (int z = 0; z < 4; ++z) raw[slot][z] = __ldg(src + z);
-            rsc[slot] = __ldg(ks + e);
-        } else {
-#pragma unroll
-            for (int z = 0; z < 4; ++z) raw[slot][z] = make_uint4(0, 0, 0, 0);
-            rsc[slot] = 0x7F7F7F7Fu;
-        }
-    };
-#pragma unroll
-    for (int a = 0; a < kAhead; ++a) fetch(a, a);
-    uint32_t cur_sc[2] = {0u, 0u};                       // scale words of the tile whose MMA is in flight
-    bool ok = true;
-
-    auto epilogue = [&](int t, uint32_t sw) {
-        const int nb = t % NBD;
-        bool done = false;
-        for (long long it = 0; it < kWaitLimit && !done; ++it) done = mbar_try_wait(smem_u32(&bar_d[nb]), (t / NBD) & 1);
-        if (!done) { ok = false; atomicExch(&g_index_device_error, 1); }
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const int64_t e = s_begin + static_cast<int64_t>(t) * TILE + tid;
-        const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(nb * N);
-        int ek[4];
-#pragma unroll
-        for (int blk = 0; blk < 4; ++blk) ek[blk] = static_cast<int>((sw >> (8 * blk)) & 0xFFu);
-#pragma unroll 1
-        for (int q = 0; q < QG; ++q) {
-            uint32_t r[16];
-            asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-                         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-                           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-                         : "r"(taddr + q * 16));
-            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-            if (e < s_end && e < s_elig[q]) {
-                float sc = 0.0f;
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    float dot = 0.0f;
-#pragma unroll
-                    for (int blk = 0; blk < 4; ++blk) {
-                        const float t_ = __fmul_rn(__uint_as_float(r[blk * 4 + h]), pow2i(s_eq[q][blk * 4 + h] + ek[blk]));
-                        dot = blk == 0 ? t_ : __fadd_rn(dot, t_);
-                    }
-                    sc = __fadd_rn(sc, __fmul_rn(s_w[q][h], dot > 0.0f ? dot : 0.0f));
-                }
-                scores[static_cast<size_t>(qrow0 + q) * Nc_cap + e] = ok ? sc : __int_as_float(0x7fc00000);
-            }
-        }
-    };
-
-    for (int t = 0; t < n_tiles; ++t) {
-        const int st = t % kStages;
-        // stage st was last read by MMA(t - kStages), whose epilogue ran in an earlier iteration
-        uint8_t* a = sA + st * TILE_BYTES;
-#pragma unroll
-        for (int z = 0; z < 4; ++z) {
-            const uint4 v = raw[0][z];
-            *reinterpret_cast<uint4*>(a + sw128(tid, 2 * z)) = make_uint4(v.x, v.y, 0u, 0u);
-            *reinterpret_cast<uint4*>(a + sw128(tid, 2 * z + 1)) = make_uint4(v.z, v.w, 0u, 0u);
-        }
-        const uint32_t sw_t = rsc[0];
-#pragma unroll
-        for (int x = 0; x < kAhead - 1; ++x) {
-#pragma unroll
-            for (int z = 0; z < 4; ++z) raw[x][z] = raw[x + 1][z];
-            rsc[x] = rsc[x + 1];
-        }
-        fetch(t + kAhead, kAhead - 1);
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        __syncthreads();
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        if (tid == 0) {
-            const uint32_t abase = smem_u32(a), bbase = smem_u32(sB);
-            const uint32_t d = tmem + static_cast<uint32_t>((t % NBD) * N);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                             "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
-                             :: "r"(d), "l"(sdesc(abase + kk * 32)), "l"(sdesc(bbase + kk * 32)), "r"(IDESC), "r"(kk)
-                             : "memory");
-            }
-            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                         :: "r"(smem_u32(&bar_d[t % NBD])) : "memory");
-        }
-        if (t >= 1) epilogue(t - 1, cur_sc[(t - 1) & 1]);
-        cur_sc[t & 1] = sw_t;
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    }
-    if (n_tiles >= 1) epilogue(n_tiles - 1, cur_sc[(n_tiles - 1) & 1]);
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    __syncthreads();
     if (warp == 0) {
+        // ---------------------------------------------------------------- loads
+        if (lane == 0) {
+            for (int t = 0; t < n_tiles; ++t) {
+                const int st = t % KS;
+                if (t >= KS && !wait_bar(smem_u32(&bar_empty[st]), ((t / KS) - 1) & 1, &s_abort)) break;
+                const uint32_t full = smem_u32(&bar_full[st]);
+                uint8_t* stage = smem + st * STAGE_BYTES;
+                mbar_expect_tx(full, CODE_TX_BYTES + SCALE_BYTES);
+                tma_load_2d(smem_u32(stage), &tm_codes, 0, row0 + t * TILE, full);
+                tma_load_1d(smem_u32(stage + CODE_BYTES), &tm_scales, row0 + t * TILE, full);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issue
+        if (lane == 0) {
+            const uint32_t bbase = smem_u32(sB);
+            for (int t = 0; t < n_tiles; ++t) {
+                const int st = t % KS, nb = t % NBD;
+                if (!wait_bar(smem_u32(&bar_full[st]), (t / KS) & 1, &s_abort)) break;
+                if (t >= NBD && !wait_bar(smem_u32(&bar_acce[nb]), ((t / NBD) - 1) & 1, &s_abort)) break;
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const uint32_t abase = smem_u32(smem + st * STAGE_BYTES);
+                const uint32_t d = tmem + static_cast<uint32_t>(nb * N);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                                 "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+                                 :: "r"(d), "l"(sdesc(abase + kk * 32)), "l"(sdesc(bbase + kk * 32)), "r"(IDESC), "r"(kk)
+                                 : "memory");
+                }
+                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                             :: "r"(smem_u32(&bar_accf[nb])) : "memory");
+            }
+            // completes once every MMA issued above has finished
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                         :: "r"(smem_u32(&bar_drain)) : "memory");
+        }
+    } else {
+        // ---------------------------------------------------------------- epilogue
+        // items i = (tile t, j-th query of this warp), in order; the TMEM load of item
+        // i + 1 is in flight while item i is scored
+        constexpr int QPW = QG / EG;                   // queries per epilogue warp
+        const int quarter = warp & 3;                  // TMEM lanes 32 quarter .. +31
+        const int eg = (warp - 2) >> 2;                // this warp's share of the queries
+        const int row = quarter * 32 + lane;           // key row of the tile
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        const int n_items = n_tiles * QPW;
+        int eq1[16];                                   // exponents of the only query (QG == 1)
+#pragma unroll
+        for (int j = 0; j < 16; ++j) eq1[j] = s_eq[0][j];
+        uint32_t rn[16];
+        auto tmem_ld = [&](int i) {
+            const int t = i / QPW, q = eg + EG * (i % QPW);
+            asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                         : "=r"(rn[0]), "=r"(rn[1]), "=r"(rn[2]), "=r"(rn[3]), "=r"(rn[4]), "=r"(rn[5]), "=r"(rn[6]), "=r"(rn[7]),
+                           "=r"(rn[8]), "=r"(rn[9]), "=r"(rn[10]), "=r"(rn[11]), "=r"(rn[12]), "=r"(rn[13]), "=r"(rn[14]), "=r"(rn[15])
+                         : "r"(lane_base + static_cast<uint32_t>((t % NBD) * N + q * 16)));
+        };
+        // a tile's accumulators are complete (and its stage's loads visible) after these waits
+        auto tile_ready = [&](int t) {
+            if (!wait_bar(smem_u32(&bar_accf[t % NBD]), (t / NBD) & 1, &s_abort)) return false;
+            if (!wait_bar(smem_u32(&bar_full[t % KS]), (t / KS) & 1, &s_abort)) return false;
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            return true;
+        };
+        bool ok = true;
+        if (n_items > 0) {
+            if (tile_ready(0)) tmem_ld(0); else ok = false;
+        }
+        uint32_t sw = 0;
+        for (int i = 0; i < n_items && ok; ++i) {
+            const int t = i / QPW, j = i % QPW, q = eg + EG * j;
+            const int st = t % KS, nb = t % NBD;
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            uint32_t r[16];
+#pragma unroll
+            for (int z = 0; z < 16; ++z) r[z] = rn[z];
+            if (j == 0) sw = *reinterpret_cast<const uint32_t*>(smem + st * STAGE_BYTES + CODE_BYTES + row * 4);
+            if (j == QPW - 1) {
+                // every load of tile t has completed and its scale word is read: release
+                // the accumulator buffer and the key stage
+                asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) { mbar_arrive(smem_u32(&bar_acce[nb])); mbar_arrive(smem_u32(&bar_empty[st])); }
+            }
+            if (i + 1 < n_items) {
+                if ((i + 1) % QPW == 0 && !tile_ready(t + 1)) { ok = false; }
+                else tmem_ld(i + 1);
+            }
+            int eq[16];
+#pragma unroll
+            for (int z = 0; z < 16; ++z) eq[z] = QG == 1 ? eq1[z] : s_eq[q][z];
+            // fast path: every exponent eq + ek in [-126, 127], so 2^(eq+ek) is a
+            // normal float whose bits are (eq + ek + 127) << 23
+            bool normal = true;
+#pragma unroll
+            for (int z = 0; z < 16; ++z) {
+                const int x = eq[z] + static_cast<int>((sw >> (8 * (z >> 2))) & 0xFFu);
+                normal &= (x >= -126) & (x <= 127);
+            }
+            float tv[16];
+            if (__all_sync(0xffffffffu, normal)) {
+#pragma unroll
+                for (int z = 0; z < 16; ++z) {
+                    const uint32_t bits = static_cast<uint32_t>(eq[z] + 127 + static_cast<int>((sw >> (8 * (z >> 2))) & 0xFFu)) << 23;
+                    tv[z] = __fmul_rn(__uint_as_float(r[z]), __uint_as_float(bits));
+                }
+            } else {
+#pragma unroll
+                for (int z = 0; z < 16; ++z)
+                    tv[z] = scale_pow2(__uint_as_float(r[z]), eq[z] + static_cast<int>((sw >> (8 * (z >> 2))) & 0xFFu));
+            }
+            float sc = 0.0f;
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                // column blk*4 + h: ordered block sum ((t0 + t1) + t2) + t3
+                const float dot = __fadd_rn(__fadd_rn(__fadd_rn(tv[h], tv[4 + h]), tv[8 + h]), tv[12 + h]);
+                sc = __fadd_rn(sc, __fmul_rn(s_w[q][h], dot > 0.0f ? dot : 0.0f));
+            }
+            const int64_t e = s_begin + static_cast<int64_t>(t) * TILE + row;
+            if (e < s_end && e < s_elig[q])
+                scores[static_cast<size_t>(qrow0 + q) * Nc_cap + e] = ok ? sc : __int_as_float(0x7fc00000);
+        }
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        if (!ok) {
+            // scores of the tiles this warp did not reach: NaN
+            for (int q = eg; q < QG; q += EG)
+                for (int64_t e = s_begin + row; e < s_live; e += TILE)
+                    if (e < s_elig[q]) scores[static_cast<size_t>(qrow0 + q) * Nc_cap + e] = __int_as_float(0x7fc00000);
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        // no MMA may still write TMEM when it is released
+        if (lane == 0) wait_bar(smem_u32(&bar_drain), 0, &s_abort);
+        __syncwarp();
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(NCOLS) : "memory");
     }
 }
 
-template <int QG, int NBD>
+// tensor maps of the keys: codes as [rows][128] 4-bit values (64 B a row,
+// unpacked to 128 B a row in shared memory), scales as [rows] 32-bit words
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// false when the key buffers do not meet the tensor-map rules (the caller
+// then takes the CUDA-core path)
+bool make_maps(const uint8_t* k_codes, const uint8_t* k_sf, int64_t rows, int64_t nc_cap, CUtensorMap* codes,
+               CUtensorMap* scales) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    if ((reinterpret_cast<uintptr_t>(k_codes) & 31u) || (reinterpret_cast<uintptr_t>(k_sf) & 15u)) return false;
+    if (rows <= 0 || rows > 0x7FFFFFFFLL) return false;
+    // a tile's scale words start at x = row (32-bit elements): x * 4 must be a
+    // multiple of 16 bytes, so every sequence must start on a multiple of 4 rows
+    if (nc_cap % 4 != 0) return false;
+    const cuuint64_t cdim[2] = {128, static_cast<cuuint64_t>(rows)};
+    const cuuint64_t cstride[1] = {64};
+    const cuuint32_t cbox[2] = {128, TILE};
+    const cuuint32_t ones[2] = {1, 1};
+    if (fn(codes, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<uint8_t*>(k_codes), cdim, cstride, cbox, ones,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    const cuuint64_t sdim[1] = {static_cast<cuuint64_t>(rows)};
+    const cuuint64_t sstride[1] = {4};   // unused at rank 1
+    const cuuint32_t sbox[1] = {TILE};
+    if (fn(scales, CU_TENSOR_MAP_DATA_TYPE_UINT32, 1, const_cast<uint8_t*>(k_sf), sdim, sstride, sbox, ones,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    return true;
+}
+
+// returns HCA_ERR_UNSUPPORTED (nothing launched) when the tensor maps cannot be made
+template <int QG, int NBD, int KS, int EG>
 int launch_tc(const uint8_t* q_codes, const uint8_t* q_sf, const float* w, const uint8_t* k_codes,
-              const uint8_t* k_sf, const int32_t* q_pos, int64_t rows, int Tq, int64_t Nc_cap, int m,
+              const uint8_t* k_sf, const int32_t* q_pos, int64_t rows, int B, int Tq, int64_t Nc_cap, int m,
               float* scores, cudaStream_t st, int64_t want_ctas) {
+    CUtensorMap tm_codes, tm_scales;
+    if (!make_maps(k_codes, k_sf, static_cast<int64_t>(B) * Nc_cap, Nc_cap, &tm_codes, &tm_scales)) return HCA_ERR_UNSUPPORTED;
     const int64_t groups = rows / QG;
     int64_t chunk = ceil_div(Nc_cap, std::max<int64_t>(1, want_ctas / std::max<int64_t>(groups, 1)));
     chunk = ceil_div(chunk, TILE) * TILE;
     if (chunk < TILE) chunk = TILE;
     if (ceil_div(Nc_cap, chunk) > 65535) chunk = ceil_div(ceil_div(Nc_cap, 65535), TILE) * TILE;
-    size_t smem = static_cast<size_t>(kStages) * TILE_BYTES + 16 * QG * 128 + 1024;
+    size_t smem = static_cast<size_t>(KS) * STAGE_BYTES + 16 * QG * 128 + 1024;
     // a CTA that takes all 512 TMEM columns must be alone on its SM: ask for
     // more than half of the SM's shared memory
     if (16 * QG * NBD >= 512 && smem < 120 * 1024) smem = 120 * 1024;
-    cudaError_t e = cudaFuncSetAttribute(index_tc_kernel<QG, NBD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    auto kern = index_tc_kernel<QG, NBD, KS, EG>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
     const dim3 grid(static_cast<unsigned>(groups), static_cast<unsigned>(ceil_div(Nc_cap, chunk)));
-    index_tc_kernel<QG, NBD><<<grid, kThreads, smem, st>>>(q_codes, q_sf, w, k_codes, k_sf, q_pos, Tq, Nc_cap, m,
-                                                           chunk, scores);
+    kern<<<grid, 64 + 128 * EG, smem, st>>>(tm_codes, tm_scales, q_codes, q_sf, w, q_pos, Tq, Nc_cap, m, chunk, scores);
     HCA_CHECK_LAUNCH();
     return HCA_OK;
 }
@@ -601,13 +738,17 @@ int index_launch(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
     if (rows > 0x7FFFFFFFLL) return HCA_ERR_UNSUPPORTED;
     const bool small = Hi <= 4;
     if (c == 128 && Hi == 4) {
-        // tensor cores on FP4 straight from shared memory: 16 queries per CTA when
-        // a sequence has many query rows (prefill), else one
+        // tensor cores on FP4 fed by the tensor memory accelerator: 16 queries per
+        // CTA when a sequence has many query rows (prefill), else one
+        int rc;
         if (Tq % 16 == 0 && Tq >= 64)
-            return itc::launch_tc<16, 2>(q_codes, q_sf, w, k_codes, k_sf, q_pos, rows, Tq, Nc_cap, m, scores, st,
-                                         4LL * sm_count());
-        return itc::launch_tc<1, 4>(q_codes, q_sf, w, k_codes, k_sf, q_pos, rows, Tq, Nc_cap, m, scores, st,
-                                    3LL * sm_count());
+            rc = itc::launch_tc<16, 2, 4, 2>(q_codes, q_sf, w, k_codes, k_sf, q_pos, rows, B, Tq, Nc_cap, m, scores, st,
+                                             2LL * sm_count());
+        else
+            rc = itc::launch_tc<1, 4, 4, 1>(q_codes, q_sf, w, k_codes, k_sf, q_pos, rows, B, Tq, Nc_cap, m, scores, st,
+                                            3LL * sm_count());
+        if (rc != HCA_ERR_UNSUPPORTED) return rc;
+        // unaligned key buffers: CUDA-core tensor path below
     }
     if (c == 128 && Hi == 4) {
         int64_t ch = 8192;

@@ -116,6 +116,54 @@ def test_indexer_full_scale_range_ordered_sum():
     assert np.array_equal(host(s).view(np.uint32), want.view(np.uint32))
 
 
+def _same_scores(got, want):
+    """Bit-identical, except that any NaN matches any NaN (payloads differ between CPU and GPU)."""
+    g, w_ = got.view(np.uint32), want.view(np.uint32)
+    nan_g, nan_w = np.isnan(got), np.isnan(want)
+    return np.array_equal(nan_g, nan_w) and np.array_equal(g[~nan_g], w_[~nan_w])
+
+
+@pytest.mark.parametrize("Tq,Nc", [(3, 512), (3, 511), (64, 512), (64, 509)])
+def test_indexer_extreme_exponents(Tq, Nc):
+    """ue8m0 bytes at both ends of their range: 2^(uq+uk-254) overflows fp32 (a zero
+    block must still give 0, a nonzero one inf) or lies far in the subnormal range
+    (the product is rounded once).  Covers the tensor-map path (Nc a multiple of 4),
+    the fallback path (Nc not), one query per CTA (Tq = 3) and 16 per CTA (Tq = 64)."""
+    B, Hi, c, m = 2, 4, 128, 1
+    qc, qs, w, kc, ks = _fp4_inputs(B, Tq, Hi, c, Nc, 7 * Tq + Nc)
+    g = _gen(Tq + Nc)
+    ends = torch.tensor([0, 1, 2, 3, 60, 127, 200, 250, 253, 254, 255], dtype=torch.uint8, device=DEV)
+    qs = ends[torch.randint(0, len(ends), qs.shape, generator=g, device=DEV)]
+    ks = ends[torch.randint(0, len(ends), ks.shape, generator=g, device=DEV)]
+    # zero whole 32-element blocks of some keys (0 * 2^e must stay 0 when 2^e overflows)
+    zero = torch.rand((B, Nc, c // 32), generator=g, device=DEV) < 0.3
+    kc = kc.view(B, Nc, c // 32, 16).masked_fill(zero[..., None], 0).view(B, Nc, c // 2).contiguous()
+    w[..., 0] = 0.0                                     # 0 * inf = NaN in head 0 where its dot overflows
+    pos = torch.full((B, Tq), 10 ** 6, dtype=torch.int32, device=DEV)
+    pos[1, 0] = Nc // 2
+    s = hca.lightning_index(qc, qs, w, kc, ks, pos, m)
+    torch.cuda.synchronize()
+    want, _ = oracle.index_scores(host(qc), host(qs), host(w), host(kc), host(ks), host(pos), m)
+    got = host(s)
+    assert np.isinf(want).any() and np.isnan(want).any()          # the planted cases occur
+    assert _same_scores(got, want)
+
+
+@pytest.mark.parametrize("Tq,Nc", [(64, 1000), (64, 4099), (80, 2048)])
+def test_indexer_sixteen_queries_per_cta(Tq, Nc):
+    """Prefill-shaped calls (Tq a multiple of 16, >= 64): 16 queries share each key
+    tile; causal positions cut the eligible range inside tiles."""
+    B, Hi, c, m = 2, 4, 128, 4
+    qc, qs, w, kc, ks = _fp4_inputs(B, Tq, Hi, c, Nc, Tq * 31 + Nc)
+    base = torch.arange(Tq, dtype=torch.int32, device=DEV) * 37
+    pos = torch.stack([base + 4 * Nc - 37 * Tq, base + 5]).to(torch.int32)
+    s = hca.lightning_index(qc, qs, w, kc, ks, pos, m)
+    torch.cuda.synchronize()
+    want, n_inexact = oracle.index_scores(host(qc), host(qs), host(w), host(kc), host(ks), host(pos), m)
+    assert n_inexact == 0
+    assert np.array_equal(host(s).view(np.uint32), want.view(np.uint32))
+
+
 # ------------------------------------------------------------------ top-k
 @pytest.mark.parametrize("Nc,k", [(1, 1), (100, 7), (5000, 32), (33000, 1024), (70000, 512), (140000, 4096)])
 def test_topk_bit_exact(Nc, k):
