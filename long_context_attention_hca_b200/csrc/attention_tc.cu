@@ -15,24 +15,36 @@
 //   O^T += V^T . P^T    M = 128 output dims (4 M-tiles), N = 64 heads,
 //                       K = 64 keys; V^T is the key tile itself read MN-major,
 //                       P^T the softmax probabilities stored K-major.
-// TMEM: S in NBUF buffers of 32 columns + O^T (4 x 64 columns).
-// Warp roles (512 threads):
-//   warps 0-3   softmax: one thread per head row of S (lanes 0..15 of each
-//               warp); online softmax in base 2 with a lazy rescale (O^T and
-//               l are rescaled only when a head's running max grows by more
-//               than 8, so P <= 2^8 in fp16); all 128 threads (= the 128
-//               TMEM lanes of O^T) apply a rescale and run the epilogue.
-//   warps 4-15  three producer groups; group g dequantises tiles g, g+3,
-//               ... (FP8 code x fp32 scale -> fp16, bf16 -> fp16) into key
-//               buffer g; each thread holds one tile's raw loads (8 units of
-//               16 dims) and issues them before it waits for the buffer, and
-//               prefetches the gather indices of its next tile, so three
-//               tiles of HBM reads are in flight per SM.  Once the group has
-//               stored a tile, one of its threads issues that tile's QK
-//               MMAs, so the tensor pipe computes ahead of the softmax.
-//   The softmax issues PV(i) (thread 0) once all four warps stored P(i).
-//   tcgen05.commit tracks the issuing thread's own MMAs, so each issuer
-//   signals the barriers of the work it issued.
+// TMEM: S in NBUF buffers of 64 columns + O^T (4 x 64 columns).
+// Warp roles (704 threads):
+//   warps 0-3   softmax: head h = 16 w + (lane & 15); lanes 0-15 take keys
+//               0..31 of the tile, lanes 16-31 keys 32..63; online softmax
+//               in base 2 with a lazy rescale (O^T and l are rescaled only
+//               when a head's running max grows by more than 8, so P <= 2^8
+//               in fp16); all 128 threads (= the 128 TMEM lanes of O^T)
+//               apply a rescale and run the epilogue.
+//   warps 4-19  producers: tile i goes to key buffer i % 2 (FP8 code x
+//               scale -> fp16, bf16 -> fp16).  Warp w converts column block
+//               w % 8 (64 dims) of key rows 32 (w / 8) .. + 31: lane l takes
+//               16-dim unit l / 8 of that block and rows l % 8 + 8 j, so the
+//               eight lanes that write one 16-byte chunk position hit eight
+//               different swizzled bank groups.  Each thread issues the raw
+//               loads of tile i + 1 as soon as tile i is stored (before it
+//               waits for the buffer), and prefetches the gather indices one
+//               tile ahead.
+//   warps 20-21 QK issue, one warp per key buffer: once the producers have
+//               stored tile i, lane 0 of warp 20 + i % 2 issues its 32 MMAs,
+//               so the QK of consecutive tiles overlaps.
+//   All threads load Q (bf16 -> fp16) at the start, every load in flight at once.
+// Per 64-key tile the MMAs read 128 KB of shared memory (Q and K for QK) and
+// 96 KB (V^T and P, four M-tiles, for PV) and the stores write 72 KB: at
+// 128 B per clock that is ~2300 clocks, the bound of this data flow.
+//   The softmax issues PV(i) from four threads (lane 0 of each warp, one
+//   M-tile each) once all four warps stored P(i): a thread issues
+//   tcgen05.mma one at a time, so four issuers cut the issue latency by
+//   four.  tcgen05.commit tracks the issuing thread's own MMAs, so each
+//   issuer signals the barriers of the work it issued (the PV barriers
+//   count four arrivals).
 // Every mbarrier wait is bounded; a timeout sets the device error word,
 // raises the CTA's abort flag, drains the issued MMAs and frees TMEM.
 #include <mutex>
@@ -47,20 +59,22 @@ namespace tc {
 
 constexpr int D = 512;
 constexpr int HP = 64;
-constexpr int TK = 32;                       // keys per tile
-constexpr int NBUF = 3;                      // key tiles (and S tiles) in flight
-constexpr int NSOFT = 4, GROUP_WARPS = 4, NPROD = NBUF * GROUP_WARPS;
-constexpr int NWARPS = NSOFT + NPROD;
-constexpr int NTHREADS = NWARPS * 32;        // 512
+constexpr int TK = 64;                       // keys per tile
+constexpr int NBUF = 2;                      // key tiles (and S tiles) in flight
+constexpr int NSOFT = 4, NPROD = 16, NISSUE = NBUF;
+constexpr int NWARPS = NSOFT + NPROD + NISSUE;
+constexpr int NTHREADS = NWARPS * 32;        // 704
+constexpr int ROWS_PER_THREAD = TK / NPROD;  // key rows a producer thread converts (4)
 constexpr int QBLK = 8192;                   // Q column block: 64 head rows x 128 B (SW128)
-constexpr int KBLK = TK * 128;               // key column block: 32 key rows x 128 B
+constexpr int KBLK = TK * 128;               // key column block: 64 key rows x 128 B
+constexpr int PBLK = 64 * 128;               // P^T: 64 head rows x 64 keys fp16 (one SW128 block)
 constexpr int Q_OFF = 0;                     // 8 column blocks (64 KB)
-constexpr int K_OFF = 8 * QBLK;              // NBUF buffers x 8 column blocks (3 x 32 KB)
-constexpr int P_OFF = K_OFF + NBUF * 8 * KBLK;   // 2 x (64 head rows x 128 B, keys 0..31 used)
-constexpr int SMEM_BYTES = P_OFF + 2 * QBLK + 1024;  // + alignment slack
+constexpr int K_OFF = 8 * QBLK;              // NBUF buffers x 8 column blocks (2 x 64 KB)
+constexpr int P_OFF = K_OFF + NBUF * 8 * KBLK;   // 2 P^T buffers
+constexpr int SMEM_BYTES = P_OFF + 2 * PBLK + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t S_COL = 0;                // S buffer b at columns 32 b
-constexpr uint32_t O_COL = 128;              // O^T M-tile mt at 128 + 64 mt
+constexpr uint32_t S_COL = 0;                // S buffer b at columns 64 b
+constexpr uint32_t O_COL = NBUF * TK;        // O^T M-tile mt at 128 + 64 mt
 constexpr float RESCALE_THRESHOLD = 8.0f;    // log2 units
 constexpr long long WAIT_LIMIT = 1ll << 24;  // polls before a wait is declared stuck
 
@@ -143,6 +157,18 @@ __device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.syn
                    "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),          \
                    "=r"(r[30]), "=r"(r[31])                                                                         \
                  : "r"(taddr))
+// 16 TMEM lanes x 32 columns, twice: threads 0-15 read lanes base + t at columns
+// c .. c + 31, threads 16-31 the same lanes at columns c + 32 .. c + 63 (the M = 64
+// accumulator layout keeps a warp's 16 rows in the first 16 lanes of its quarter)
+#define TMEM_LD_16X32BX2_32(taddr, r)                                                                              \
+    asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15," \
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], 32;"                       \
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),      \
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), \
+                   "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),          \
+                   "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),          \
+                   "=r"(r[30]), "=r"(r[31])                                                                         \
+                 : "r"(taddr))
 // 2^x with the special-function unit (approximate; x = -inf gives +0)
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -202,6 +228,12 @@ __device__ __forceinline__ UnitKeys unit_keys(const Params& p, int64_t u) {
     return k;
 }
 
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
     return pack_half2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
 }
@@ -220,7 +252,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
 __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t bar_kempty[NBUF], bar_sfull[NBUF], bar_pempty[2], bar_drain;
+    __shared__ __align__(8) uint64_t bar_kempty[NBUF], bar_kfull[NBUF], bar_sfull[NBUF], bar_pempty[2], bar_drain;
     __shared__ uint32_t tmem_base_slot;
     __shared__ float s_alpha[HP], s_l[HP];
     __shared__ int s_resc_w[NSOFT];
@@ -239,25 +271,38 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
 
     if (tid == 0) {
         for (int i = 0; i < NBUF; ++i) {
-            mbar_init(smem_u32(&bar_kempty[i]), 1);
+            mbar_init(smem_u32(&bar_kempty[i]), 4);  // freed by the four PV issuers
+            mbar_init(smem_u32(&bar_kfull[i]), NPROD);  // one arrival per producer warp
             mbar_init(smem_u32(&bar_sfull[i]), 1);
         }
-        mbar_init(smem_u32(&bar_pempty[0]), 1);
-        mbar_init(smem_u32(&bar_pempty[1]), 1);
-        mbar_init(smem_u32(&bar_drain), NBUF + 1);   // the MMA-issuing threads
+        mbar_init(smem_u32(&bar_pempty[0]), 4);      // the four PV issuers
+        mbar_init(smem_u32(&bar_pempty[1]), 4);
+        mbar_init(smem_u32(&bar_drain), NISSUE + 4);   // the MMA-issuing threads
         s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) { tmem_alloc(smem_u32(&tmem_base_slot), TMEM_COLS); tmem_relinquish(); }
-    // Q -> fp16, K-major SW128: column block cb = dims 64cb.., row = head
-    for (int w = tid; w < HP * (D / 8); w += NTHREADS) {
-        const int r = w / (D / 8), c = w % (D / 8);
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (r < p.H) {
-            const uint4 b = __ldg(reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(u) * p.H + r) * D + c * 8));
-            v = make_uint4(bf16x2_to_f16x2(b.x), bf16x2_to_f16x2(b.y), bf16x2_to_f16x2(b.z), bf16x2_to_f16x2(b.w));
+    {
+        // Q -> fp16, K-major SW128: column block cb = dims 64cb.., row = head; all of
+        // a thread's loads are issued before the first conversion
+        constexpr int QV = HP * (D / 8);                      // 16-byte vectors of Q
+        constexpr int QPT = (QV + NTHREADS - 1) / NTHREADS;   // per thread
+        uint4 qv[QPT];
+#pragma unroll
+        for (int k = 0; k < QPT; ++k) {
+            const int w = tid + k * NTHREADS, r = w / (D / 8), c = w % (D / 8);
+            qv[k] = (w < QV && r < p.H)
+                        ? __ldg(reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(u) * p.H + r) * D + c * 8))
+                        : make_uint4(0, 0, 0, 0);
         }
-        *reinterpret_cast<uint4*>(smem + Q_OFF + (c >> 3) * QBLK + sw128(r, c & 7)) = v;
+#pragma unroll
+        for (int k = 0; k < QPT; ++k) {
+            const int w = tid + k * NTHREADS, r = w / (D / 8), c = w % (D / 8);
+            if (w < QV)
+                *reinterpret_cast<uint4*>(smem + Q_OFF + (c >> 3) * QBLK + sw128(r, c & 7)) =
+                    make_uint4(bf16x2_to_f16x2(qv[k].x), bf16x2_to_f16x2(qv[k].y), bf16x2_to_f16x2(qv[k].z),
+                               bf16x2_to_f16x2(qv[k].w));
+        }
     }
     fence_async_smem();
     fence_before();
@@ -265,40 +310,58 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
     fence_after();
     const uint32_t tmem = tmem_base_slot;
 
-    constexpr uint32_t id_qk = idesc_f16(64, TK, 0, 0);   // S[64 heads x 32 keys]
+    constexpr uint32_t id_qk = idesc_f16(64, TK, 0, 0);   // S[64 heads x 64 keys]
     constexpr uint32_t id_pv = idesc_f16(128, HP, 1, 0);
-    if (warp >= NSOFT) {
+    if (warp >= NSOFT + NPROD) {
+        // ------------------------------------------------------------ QK issue
+        const int b = warp - (NSOFT + NPROD);             // this warp's key buffer
+        if (lane == 0) {
+            const uint64_t qd = sdesc(sbase + Q_OFF, 16, 1024);
+            const uint64_t kd = sdesc(sbase + K_OFF + b * 8 * KBLK, 16, 1024);
+            const uint32_t dst = tmem + S_COL + b * TK;
+            for (int i = b; i < n_tiles; i += NBUF) {
+                if (!wait_bar(smem_u32(&bar_kfull[b]), (i / NBUF) & 1, &s_abort)) break;
+                fence_after();
+                // descriptors differ per k-step only in the start address (bits 0..13, units of 16 B)
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t qo = static_cast<uint32_t>(((kk >> 2) * QBLK + (kk & 3) * 32) >> 4);
+                    const uint32_t ko = static_cast<uint32_t>(((kk >> 2) * KBLK + (kk & 3) * 32) >> 4);
+                    mma_f16(dst, qd + qo, kd + ko, id_qk, kk > 0);
+                }
+                mma_commit(smem_u32(&bar_sfull[b]));
+            }
+            mma_commit(smem_u32(&bar_drain));
+        }
+    } else if (warp >= NSOFT) {
         // ------------------------------------------------------------ producers
-        const int grp = (warp - NSOFT) / GROUP_WARPS;                  // key buffer
-        const int pt = ((warp - NSOFT) % GROUP_WARPS) * 32 + lane;     // 0..127 within the group
-        const int c16 = pt & 31;                 // this thread's 16-dim unit (same for all its keys)
+        const int pw = warp - NSOFT;                   // 0..15
+        const int pt = pw * 32 + lane;                 // 0..511
+        const int c16 = (pw & 7) * 4 + (lane >> 3);    // this thread's 16-dim unit (same for all its keys)
+        const int row0 = (pw >> 3) * 32 + (lane & 7);  // its rows: row0 + 8 j
         const int d0 = c16 * 16;
         const int dn = D - 64;
-        // unit j of a tile: key row r = pt / 32 + 4 j
-        int32_t ent_next[8];
-        auto fetch_ent = [&](int i, int32_t (&e)[8]) {
+        int32_t ent_next[ROWS_PER_THREAD];
+        auto fetch_ent = [&](int i, int32_t (&e)[ROWS_PER_THREAD]) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int slot = (t_begin + i) * TK + (pt >> 5) + 4 * j;
+            for (int j = 0; j < ROWS_PER_THREAD; ++j) {
+                const int slot = (t_begin + i) * TK + row0 + 8 * j;
                 e[j] = (i < n_tiles && slot < uk.n_c) ? (uk.ent ? uk.ent[slot] : slot) : -1;
             }
         };
-        fetch_ent(grp, ent_next);
-        for (int i = grp; i < n_tiles; i += NBUF) {
-            int32_t ent[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) ent[j] = ent_next[j];
+        uint32_t raw[ROWS_PER_THREAD][8];
+        float sc[ROWS_PER_THREAD];
+        // raw loads of tile i (registers only: no buffer needed yet)
+        auto load_tile = [&](int i, const int32_t (&ent)[ROWS_PER_THREAD]) {
             const int slot0 = (t_begin + i) * TK;
-            // raw loads of this tile (registers only: no buffer needed yet)
-            uint32_t raw[8][8];
-            float sc[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int r = (pt >> 5) + 4 * j;
+            for (int j = 0; j < ROWS_PER_THREAD; ++j) {
+                const int r = row0 + 8 * j;
                 const int slot = slot0 + r;
                 sc[j] = 0.0f;
 #pragma unroll
                 for (int z = 0; z < 8; ++z) raw[j][z] = 0;
+                if (i >= n_tiles) continue;
                 if (slot < uk.n_c) {
                     const int64_t e = ent[j];
                     if (e >= 0 && e < p.cap) {
@@ -321,23 +384,44 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
                     raw[j][4] = bq.x; raw[j][5] = bq.y; raw[j][6] = bq.z; raw[j][7] = bq.w;
                 }
             }
-            fetch_ent(i + NBUF, ent_next);       // gather indices of this group's next tile
-            const int use = i / NBUF;
-            if (use >= 1 && !wait_bar(smem_u32(&bar_kempty[grp]), (use - 1) & 1, &s_abort)) break;
-            uint8_t* kb = smem + K_OFF + grp * 8 * KBLK;
+        };
+        {
+            int32_t ent0[ROWS_PER_THREAD];
+            fetch_ent(0, ent0);
+            load_tile(0, ent0);
+            fetch_ent(1, ent_next);
+        }
+        for (int i = 0; i < n_tiles; ++i) {
+            const int b = i % NBUF, use = i / NBUF;
+            const int slot0 = (t_begin + i) * TK;
+            // key buffer b is free once PV(i - 2) has completed
+            if (use >= 1 && !wait_bar(smem_u32(&bar_kempty[b]), (use - 1) & 1, &s_abort)) break;
+            uint8_t* kb = smem + K_OFF + b * 8 * KBLK;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int r = (pt >> 5) + 4 * j;
+            for (int j = 0; j < ROWS_PER_THREAD; ++j) {
+                const int r = row0 + 8 * j;
                 const bool fp8 = slot0 + r < uk.n_c && d0 < dn;
                 uint32_t h[8];
                 if (fp8) {
                     const float s_ = sc[j];
+                    if (s_ >= 6.103515625e-05f && s_ <= 65504.0f) {
+                        // scale is a normal fp16: code (exact in fp16) x fp16(scale), one
+                        // fp16 rounding per product, two elements per instruction
+                        const uint32_t s2 = pack_half2(s_, s_);
 #pragma unroll
-                    for (int z = 0; z < 4; ++z) {
-                        const float2 a = unpack_half2(e4m3x2_to_f16x2(static_cast<uint16_t>(raw[j][z] & 0xFFFFu)));
-                        const float2 bb = unpack_half2(e4m3x2_to_f16x2(static_cast<uint16_t>(raw[j][z] >> 16)));
-                        h[2 * z] = pack_half2(a.x * s_, a.y * s_);
-                        h[2 * z + 1] = pack_half2(bb.x * s_, bb.y * s_);
+                        for (int z = 0; z < 4; ++z) {
+                            h[2 * z] = hmul2_u32(e4m3x2_to_f16x2(static_cast<uint16_t>(raw[j][z] & 0xFFFFu)), s2);
+                            h[2 * z + 1] = hmul2_u32(e4m3x2_to_f16x2(static_cast<uint16_t>(raw[j][z] >> 16)), s2);
+                        }
+                    } else {
+                        // tiny, zero or huge scale: fp32 product, rounded once to fp16
+#pragma unroll
+                        for (int z = 0; z < 4; ++z) {
+                            const float2 a = unpack_half2(e4m3x2_to_f16x2(static_cast<uint16_t>(raw[j][z] & 0xFFFFu)));
+                            const float2 bb = unpack_half2(e4m3x2_to_f16x2(static_cast<uint16_t>(raw[j][z] >> 16)));
+                            h[2 * z] = pack_half2(a.x * s_, a.y * s_);
+                            h[2 * z + 1] = pack_half2(bb.x * s_, bb.y * s_);
+                        }
                     }
                 } else {
 #pragma unroll
@@ -350,27 +434,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
                 *reinterpret_cast<uint4*>(blk + sw128(r, c8 + 1)) = make_uint4(h[4], h[5], h[6], h[7]);
             }
             fence_async_smem();
-            named_bar(2 + grp, GROUP_WARPS * 32);
-            if (pt == 0) {
-                fence_after();
-                // descriptors differ per k-step only in the start address (bits 0..13, units of 16 B)
-                const uint64_t qd = sdesc(sbase + Q_OFF, 16, 1024);
-                const uint64_t kd = sdesc(sbase + K_OFF + grp * 8 * KBLK, 16, 1024);
-                const uint32_t dst = tmem + S_COL + grp * TK;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bar_kfull[b]));
+            // next tile's raw loads fly while this thread waits for its buffer
+            int32_t ent[ROWS_PER_THREAD];
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t qo = static_cast<uint32_t>(((kk >> 2) * QBLK + (kk & 3) * 32) >> 4);
-                    const uint32_t ko = static_cast<uint32_t>(((kk >> 2) * KBLK + (kk & 3) * 32) >> 4);
-                    mma_f16(dst, qd + qo, kd + ko, id_qk, kk > 0);
-                }
-                mma_commit(smem_u32(&bar_sfull[grp]));
-            }
+            for (int j = 0; j < ROWS_PER_THREAD; ++j) ent[j] = ent_next[j];
+            load_tile(i + 1, ent);
+            fetch_ent(i + 2, ent_next);
         }
-        if (pt == 0) mma_commit(smem_u32(&bar_drain));
     } else {
         // ------------------------------------------------------------ softmax (warps 0-3)
-        // head h = 16 warp + (lane & 15); lanes 0-15 hold keys 0..15 of the tile, lanes
-        // 16-31 keys 16..31 (S row h lives in TMEM lane 32 warp + (lane & 15)).
+        // head h = 16 warp + (lane & 15); lanes 0-15 hold keys 0..31 of the tile, lanes
+        // 16-31 keys 32..63 (S row h lives in TMEM lane 32 warp + (lane & 15)).
         const int h = warp * 16 + (lane & 15);
         const int kh = lane >> 4;
         float m_used = -INFINITY, l_run = 0.0f;
@@ -380,18 +456,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
             const int b = i % NBUF, pb = i & 1;
             if (!wait_bar(smem_u32(&bar_sfull[b]), (i / NBUF) & 1, &s_abort)) { ok = false; break; }
             fence_after();
-            uint32_t sr[TK];
-            TMEM_LD32(lane_base + S_COL + b * TK, sr);
-            tmem_wait_ld();
             const int nvalid = min(TK, n_tot - (t_begin + i) * TK);
-            float v[16];
+            float v[32];
             float tmax = -INFINITY;
+            {
+                // row h, keys 32 kh .. 32 kh + 31
+                uint32_t sr[32];
+                TMEM_LD_16X32BX2_32(lane_base + S_COL + b * TK, sr);
+                tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const uint32_t up = __shfl_up_sync(0xffffffffu, sr[16 + j], 16);
-                const float x = __uint_as_float(kh ? up : sr[j]);
-                v[j] = (kh * 16 + j < nvalid) ? x * p.scale_log2 : -INFINITY;
-                tmax = fmaxf(tmax, v[j]);
+                for (int j = 0; j < 32; ++j) {
+                    v[j] = (kh * 32 + j < nvalid) ? __uint_as_float(sr[j]) * p.scale_log2 : -INFINITY;
+                    tmax = fmaxf(tmax, v[j]);
+                }
             }
             tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
             bool resc = false;
@@ -406,10 +483,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
                 l_run *= alpha;
             }
             // probabilities in registers before any wait (fp16, the sum of the rounded values)
-            uint32_t pk[8];
+            uint32_t pk[16];
             float rs = 0.0f;
 #pragma unroll
-            for (int z = 0; z < 8; ++z) {
+            for (int z = 0; z < 16; ++z) {
                 pk[z] = pack_half2(ex2(v[2 * z] - m_used), ex2(v[2 * z + 1] - m_used));
                 const float2 f = unpack_half2(pk[z]);
                 rs += f.x + f.y;
@@ -428,44 +505,51 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
                 // O^T must be stable: PV(i-1) complete
                 if (i >= 1 && !wait_bar(smem_u32(&bar_pempty[(i - 1) & 1]), ((i - 1) >> 1) & 1, &s_abort)) { ok = false; break; }
                 fence_after();
-                // this thread owns TMEM lane 32 warp + lane = one output dim of each M-tile
+                // this thread owns TMEM lane 32 warp + lane = one output dim of each M-tile;
+                // 16 head columns at a time (their factors stay in registers for the 4 M-tiles)
 #pragma unroll 1
-                for (int mt = 0; mt < 4; ++mt) {
+                for (int c0 = 0; c0 < HP; c0 += 16) {
+                    float al[16];
 #pragma unroll
-                    for (int c0 = 0; c0 < HP; c0 += 16) {
+                    for (int j = 0; j < 16; ++j) al[j] = s_alpha[c0 + j];
+#pragma unroll 1
+                    for (int mt = 0; mt < 4; ++mt) {
                         uint32_t o[16];
                         TMEM_LD16(lane_base + O_COL + mt * HP + c0, o, 0);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * s_alpha[c0 + j]);
+                        for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * al[j]);
                         TMEM_ST16(lane_base + O_COL + mt * HP + c0, o, 0);
                     }
                 }
                 tmem_wait_st();
             }
-            uint8_t* pbuf = smem + P_OFF + pb * QBLK;
-            *reinterpret_cast<uint4*>(pbuf + sw128(h, 2 * kh)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            *reinterpret_cast<uint4*>(pbuf + sw128(h, 2 * kh + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            // P^T row h: keys 32 kh .. 32 kh + 31 are 16-byte chunks 4 kh .. 4 kh + 3
+            uint8_t* pbuf = smem + P_OFF + pb * PBLK;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                *reinterpret_cast<uint4*>(pbuf + sw128(h, 4 * kh + c)) =
+                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
             fence_async_smem();
             fence_before();
             named_bar(1, NSOFT * 32);
-            if (tid == 0) {
+            if (lane == 0) {
                 fence_after();
                 // V^T read MN-major from the key tile: dims in atoms of 64 (column blocks,
-                // KBLK apart), keys in atoms of 8 rows (1024 B apart)
+                // KBLK apart), keys in atoms of 8 rows (1024 B apart).  Lane 0 of warp w
+                // issues M-tile w (output dims 128 w .. 128 w + 127).
                 const uint64_t vd = sdesc(sbase + K_OFF + b * 8 * KBLK, KBLK, 1024);
-                const uint64_t pd = sdesc(sbase + P_OFF + pb * QBLK, 16, 1024);
+                const uint64_t pd = sdesc(sbase + P_OFF + pb * PBLK, 16, 1024);
+                const int mt = warp;
 #pragma unroll
-                for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-                    for (int kk = 0; kk < TK / 16; ++kk)
-                        mma_f16(tmem + O_COL + mt * HP, vd + static_cast<uint32_t>((2 * mt * KBLK + kk * 2048) >> 4),
-                                pd + static_cast<uint32_t>((kk * 32) >> 4), id_pv, (i > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < TK / 16; ++kk)
+                    mma_f16(tmem + O_COL + mt * HP, vd + static_cast<uint32_t>((2 * mt * KBLK + kk * 2048) >> 4),
+                            pd + static_cast<uint32_t>((kk * 32) >> 4), id_pv, (i > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(smem_u32(&bar_pempty[pb]));
                 mma_commit(smem_u32(&bar_kempty[b]));
             }
         }
-        if (tid == 0) mma_commit(smem_u32(&bar_drain));
+        if (lane == 0) mma_commit(smem_u32(&bar_drain));
         // ---- epilogue: wait for the last PV, then O^T / l -> out (or the split partials)
         if (ok && n_tiles > 0) {
             ok = wait_bar(smem_u32(&bar_pempty[(n_tiles - 1) & 1]), ((n_tiles - 1) >> 1) & 1, &s_abort);
@@ -601,7 +685,7 @@ int launch_tc(tc::Params& p, int64_t units, cudaStream_t st) {
 // per CTA so the pipeline fills and the partials stay small.
 void tc_decode_plan(int B, int max_comp, int W, bool sparse, int& n_splits, int& tiles_per_split) {
     const int n_tiles = static_cast<int>(ceil_div(static_cast<int64_t>(max_comp) + W, tc::TK));
-    const int min_tps = sparse ? 4 : 12;      // tiles of 32 keys
+    const int min_tps = sparse ? 2 : 6;       // tiles of 64 keys
     int splits = sm_count() / (B > 0 ? B : 1);
     const int cap_by_len = static_cast<int>(ceil_div(n_tiles > 0 ? n_tiles : 1, min_tps));
     if (splits > cap_by_len) splits = cap_by_len;

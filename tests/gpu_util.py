@@ -8,6 +8,8 @@ Codes, scales, index scores and top-k sets are compared bit for bit.
 """
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
@@ -37,6 +39,10 @@ def attn_errors(gpu_bits: np.ndarray, ref64: np.ndarray):
 
 def assert_attn_close(gpu_bits, ref64, what=""):
     mx, mr = attn_errors(gpu_bits, ref64)
+    log = os.environ.get("HCA_ATTN_ERROR_LOG")
+    if log:                                   # margin report: one line per comparison
+        with open(log, "a") as f:
+            f.write(f"{os.environ.get('PYTEST_CURRENT_TEST', '?').split(' ')[0]} {what} max_abs={mx:.3e} mean_rel={mr:.3e}\n")
     assert mx <= MAX_ABS and mr <= MEAN_REL, f"{what}: max-abs {mx:.3e} (<= {MAX_ABS}), mean-rel {mr:.3e} (<= {MEAN_REL})"
     return mx, mr
 
