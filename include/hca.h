@@ -153,8 +153,16 @@ int lightning_index(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
  * min(k, #eligible) largest scores under the total order (score descending,
  * index ascending): scores compare as values (+0 == -0) and equal scores go
  * to the lower index.  NaN scores are not supported.
- * Supported: 1 <= k <= 4096, Nc_cap <= 2^24 (top-k splits a row over up to
- * 16 cooperating blocks of at most 32768 scores each). */
+ * Supported: 1 <= k <= 4096.
+ * Workspace: topk_select_workspace_size(R, Nc_cap, k) bytes (0 when the call
+ * needs none), 256-byte aligned, owned by the caller, contents need not be
+ * initialised and are clobbered.  Few long rows (R * ceil(Nc_cap / 16384)
+ * <= the device's SM count, Nc_cap >= 8192) and rows longer than 2^19 scores
+ * go through histogram passes
+ * spread over the whole device and use it; otherwise a row is split over a
+ * thread-block cluster of up to 16 blocks of at most 32768 scores each
+ * (Nc_cap <= 2^19) and the workspace is ignored.  A row longer than 2^19
+ * scores without an adequate workspace returns HCA_ERR_WORKSPACE. */
 size_t topk_select_workspace_size(int32_t R, int64_t Nc_cap, int32_t k);
 int topk_select(const float* scores, const int32_t* q_pos, int32_t R, int64_t Nc_cap,
                 int32_t m, int32_t k, int32_t* idx, int32_t* count,

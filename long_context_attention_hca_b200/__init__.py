@@ -181,8 +181,13 @@ def lightning_index(q_codes, q_sf, w, k_codes, k_sf, q_pos, m, scores=None, stre
     return scores
 
 
-def topk_select(scores, q_pos, m, k, idx=None, count=None, stream=None):
-    """scores [R][Nc] (any leading shape flattened), q_pos [R] -> (idx [R][k] ascending, -1 padded; count [R])."""
+def topk_workspace_size(R, Nc, k) -> int:
+    return int(_lib.topk_select_workspace_size(R, Nc, k))
+
+
+def topk_select(scores, q_pos, m, k, idx=None, count=None, ws=None, stream=None):
+    """scores [R][Nc] (any leading shape flattened), q_pos [R] -> (idx [R][k] ascending, -1 padded; count [R]).
+    ws: optional uint8 workspace of topk_workspace_size(R, Nc, k) bytes (allocated here when None)."""
     _need(scores, torch.float32, "scores"); _need(q_pos, torch.int32, "q_pos")
     Nc = scores.shape[-1]
     R = scores.numel() // Nc if Nc else q_pos.numel()
@@ -190,8 +195,11 @@ def topk_select(scores, q_pos, m, k, idx=None, count=None, stream=None):
         idx = torch.empty((R, k), dtype=torch.int32, device=scores.device)
     if count is None:
         count = torch.empty((R,), dtype=torch.int32, device=scores.device)
-    ws_bytes = _lib.topk_select_workspace_size(R, Nc, k)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=scores.device) if ws_bytes else None
+    ws_bytes = topk_workspace_size(R, Nc, k)
+    if ws_bytes and (ws is None or ws.numel() < ws_bytes):
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=scores.device)
+    elif not ws_bytes:
+        ws = None
     _check(_lib.topk_select(_p(scores), _p(q_pos), R, Nc, m, k, _p(idx), _p(count), _p(ws), ws_bytes,
                             _stream(stream)), "topk_select")
     return idx, count

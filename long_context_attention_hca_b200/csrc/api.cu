@@ -14,7 +14,9 @@ int index_launch(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
                  const uint8_t* k_codes, const uint8_t* k_sf, const int32_t* q_pos,
                  int B, int Tq, int64_t Nc_cap, int Hi, int c, int m, float* scores, cudaStream_t st);
 int topk_launch(const float* scores, const int32_t* q_pos, int R, int64_t Nc_cap, int m, int k,
-                int32_t* idx, int32_t* count, cudaStream_t st);
+                int32_t* idx, int32_t* count, void* ws, size_t ws_bytes, cudaStream_t st);
+bool topk_wide_preferred(int R, int64_t Nc_cap);
+size_t topk_wide_ws_bytes(int R, int64_t Nc_cap);
 size_t decode_ws_bytes(int B, int H, int D, int max_comp, int W);
 int attn_decode_launch(const uint16_t* q, int B, int H, const hca_kv_layout& L, const hca_kv_cache& kv,
                        const int32_t* idx, int idx_stride, const int32_t* n_comp, int max_comp,
@@ -124,20 +126,20 @@ int lightning_index(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
 }
 
 size_t topk_select_workspace_size(int32_t R, int64_t Nc_cap, int32_t k) {
-    (void)R; (void)Nc_cap; (void)k;
-    return 0;
+    (void)k;
+    if (R <= 0 || Nc_cap <= 0 || !topk_wide_preferred(R, Nc_cap)) return 0;
+    return topk_wide_ws_bytes(R, Nc_cap);
 }
 
 int topk_select(const float* scores, const int32_t* q_pos, int32_t R, int64_t Nc_cap, int32_t m, int32_t k,
                 int32_t* idx, int32_t* count, void* ws, size_t ws_bytes, void* stream) {
-    (void)ws; (void)ws_bytes;
     REQUIRE(R >= 0 && Nc_cap >= 0 && m >= 1);
     if (k < 1 || k > 4096) return HCA_ERR_UNSUPPORTED;
-    if (Nc_cap > 16 * 32768LL) return HCA_ERR_UNSUPPORTED;
     if (R == 0) return HCA_OK;
     REQ_PTR(q_pos); REQ_PTR(idx); REQ_PTR(count);
     if (Nc_cap > 0) REQ_PTR(scores);
-    return topk_launch(scores, q_pos, R, Nc_cap, m, k, idx, count, as_stream(stream));
+    if (Nc_cap > 16 * 32768LL && ws_bytes < topk_select_workspace_size(R, Nc_cap, k)) return HCA_ERR_WORKSPACE;
+    return topk_launch(scores, q_pos, R, Nc_cap, m, k, idx, count, ws, ws_bytes, as_stream(stream));
 }
 
 size_t compressed_attn_decode_workspace_size(int32_t B, int32_t H, hca_kv_layout layout, int32_t max_comp, int32_t W) {

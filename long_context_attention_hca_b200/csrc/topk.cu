@@ -21,6 +21,8 @@
 // compaction writes the indices ascending, with per-warp and per-CTA offsets
 // from block and cluster prefix sums.  Hardware cluster barriers order
 // everything: no flag spinning.
+#include <algorithm>
+
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -317,11 +319,395 @@ cudaError_t launch_cl(int R, int64_t slice, const float* scores, const int32_t* 
     return cudaLaunchKernelEx(&cfg, topk_kernel<CL>, scores, q_pos, Nc_cap, m, k, slice, idx, count);
 }
 
+// ------------------------------------------------------------------ few long rows
+// Used when there are few rows (decode: one per sequence) of many scores.
+// No clusters: three short kernels, each spread over the whole device.
+//   hist     per row, a 2048-bin histogram of the top 11 bits of the
+//            order-preserving key (shared-memory histogram per CTA, then
+//            global atomics of the non-zero bins).
+//   mark     every CTA of a row finds the same threshold bin T1 (the bin of
+//            the k-th largest key) from the histogram; keys in higher bins
+//            are selected (one bitmap word per warp ballot, no atomics);
+//            keys in bin T1 are appended to the row's candidate list.
+//   resolve  one CTA per row: two histogram passes over the candidates' low
+//            21 bits give the exact key T of the k-th largest score and how
+//            many keys equal to T are still needed; keys above T are marked
+//            selected, keys equal to T are marked in a tie bitmap.  An
+//            ordered scan of both bitmaps then takes the ties lowest index
+//            first and writes the indices ascending.
+// Workspace per row (256-byte aligned): hist u32[2048], header u32[8]
+// (candidate count, T1, keys needed from bin T1), selected and tie bitmaps
+// u32[ceil(Nc_cap / 32)] each, candidates u64[Nc_cap] (key << 32 | index).
+// The histogram, header and bitmaps are cleared by a memset on the stream.
+namespace wide {
+
+constexpr int kBins = 2048;
+constexpr int kThreads = 256;
+constexpr int kResolveThreads = 1024;
+constexpr int kMaxIt = 64;                 // mark: at most 64 x 256 keys per CTA
+
+struct Layout {
+    int64_t words;          // bitmap words per row
+    size_t row_bytes;       // per-row stride
+    size_t clear_bytes;     // bytes cleared per row (hist, header, bitmaps)
+};
+
+__host__ __device__ inline Layout layout(int64_t Nc_cap) {
+    Layout L;
+    L.words = (Nc_cap + 31) / 32;
+    L.clear_bytes = static_cast<size_t>(kBins) * 4 + 32 + static_cast<size_t>(2 * L.words) * 4;
+    L.clear_bytes = (L.clear_bytes + 255) & ~static_cast<size_t>(255);
+    L.row_bytes = L.clear_bytes + ((static_cast<size_t>(Nc_cap) * 8 + 255) & ~static_cast<size_t>(255));
+    return L;
+}
+
+struct RowWs {
+    uint32_t* hist;
+    uint32_t* hdr;          // [0] candidate count, [1] T1, [2] needed from bin T1
+    uint32_t* sel;
+    uint32_t* tie;
+    unsigned long long* cand;
+};
+
+__device__ __forceinline__ RowWs row_ws(uint8_t* ws, int64_t Nc_cap, int64_t r) {
+    const Layout L = layout(Nc_cap);
+    uint8_t* base = ws + static_cast<size_t>(r) * L.row_bytes;
+    RowWs w;
+    w.hist = reinterpret_cast<uint32_t*>(base);
+    w.hdr = w.hist + kBins;
+    w.sel = w.hdr + 8;
+    w.tie = w.sel + L.words;
+    w.cand = reinterpret_cast<unsigned long long*>(base + L.clear_bytes);
+    return w;
+}
+
+__device__ __forceinline__ int64_t n_eligible(const int32_t* q_pos, int64_t r, int m, int64_t Nc_cap) {
+    const int64_t e = (static_cast<int64_t>(q_pos[r]) + 1) / m;
+    return e < 0 ? 0 : (e > Nc_cap ? Nc_cap : e);
+}
+
+__global__ void __launch_bounds__(kThreads)
+hist_kernel(const float* __restrict__ scores, const int32_t* __restrict__ q_pos, int64_t Nc_cap, int m,
+            int64_t chunk, uint8_t* __restrict__ ws) {
+    __shared__ uint32_t sh[kBins];
+    const int64_t r = blockIdx.y;
+    const int64_t n = n_eligible(q_pos, r, m, Nc_cap);
+    const int64_t e0 = static_cast<int64_t>(blockIdx.x) * chunk;
+    const int64_t e1 = min(e0 + chunk, n);
+    if (e0 >= e1) return;
+    for (int i = threadIdx.x; i < kBins; i += kThreads) sh[i] = 0;
+    __syncthreads();
+    const float* row = scores + static_cast<size_t>(r) * Nc_cap;
+    // eight loads in flight per thread before the shared-memory atomics
+    for (int64_t e = e0 + threadIdx.x; e < e1; e += kThreads * 8) {
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = e + j * kThreads < e1 ? row[e + j * kThreads] : 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (e + j * kThreads < e1) atomicAdd(&sh[order_key(v[j]) >> 21], 1u);
+    }
+    __syncthreads();
+    RowWs w = row_ws(ws, Nc_cap, r);
+    for (int i = threadIdx.x; i < kBins; i += kThreads)
+        if (sh[i]) atomicAdd(&w.hist[i], sh[i]);
+}
+
+// Threshold bin of a row from its histogram (the same result in every CTA):
+// T1 = the highest bin whose suffix count reaches kk; returns the number of
+// keys needed from bin T1 (kk - keys in higher bins).  Block-wide.
+__device__ uint32_t find_t1(const uint32_t* __restrict__ hist, uint32_t kk, uint32_t* sh_cnt, int* t1_out) {
+    // thread t sums bins [2048 - 8 (t + 1), 2048 - 8 t) (thread 0 holds the top bins)
+    const int t = threadIdx.x;
+    uint32_t c[8], tot = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) { c[j] = hist[kBins - 8 * t - 1 - j]; tot += c[j]; }
+    sh_cnt[t] = tot;
+    __syncthreads();
+    // inclusive prefix over threads (from the top bins down), Hillis-Steele in shared memory
+    for (int off = 1; off < kThreads; off <<= 1) {
+        const uint32_t v = t >= off ? sh_cnt[t - off] : 0u;
+        __syncthreads();
+        sh_cnt[t] += v;
+        __syncthreads();
+    }
+    const uint32_t before = t > 0 ? sh_cnt[t - 1] : 0u;   // keys in bins above this thread's range
+    if (before < kk && before + tot >= kk) {
+        uint32_t acc = before;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (acc + c[j] >= kk) { *t1_out = kBins - 8 * t - 1 - j; sh_cnt[kThreads] = kk - acc; break; }
+            acc += c[j];
+        }
+    }
+    __syncthreads();
+    return sh_cnt[kThreads];
+}
+
+__global__ void __launch_bounds__(kThreads)
+mark_kernel(const float* __restrict__ scores, const int32_t* __restrict__ q_pos, int64_t Nc_cap, int m, int k,
+            int64_t chunk, uint8_t* __restrict__ ws) {
+    __shared__ uint32_t sh_cnt[kThreads + 1];
+    __shared__ int s_t1;
+    const int64_t r = blockIdx.y;
+    const int64_t n = n_eligible(q_pos, r, m, Nc_cap);
+    const uint32_t kk = static_cast<uint32_t>(min(static_cast<int64_t>(k), n));
+    const int64_t e0 = static_cast<int64_t>(blockIdx.x) * chunk;
+    const int64_t e1 = min(e0 + chunk, n);
+    if (kk == 0 || e0 >= e1) return;
+    RowWs w = row_ws(ws, Nc_cap, r);
+    if (threadIdx.x == 0) s_t1 = -1;
+    const uint32_t need1 = find_t1(w.hist, kk, sh_cnt, &s_t1);
+    const uint32_t t1 = static_cast<uint32_t>(s_t1);
+    if (blockIdx.x == 0 && threadIdx.x == 0) { w.hdr[1] = t1; w.hdr[2] = need1; }
+    const float* row = scores + static_cast<size_t>(r) * Nc_cap;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // chunk is a multiple of 256 and at most kMaxIt * 256: each warp owns whole bitmap
+    // words.  Pass A marks the keys above bin T1 and keeps the ballot of bin-T1 keys per
+    // (warp, step); one atomic per CTA reserves the candidate slots; pass B writes them.
+    __shared__ uint32_t s_mask[kThreads / 32][kMaxIt];
+    __shared__ uint32_t s_wcnt[kThreads / 32];
+    __shared__ uint32_t s_base;
+    const int n_it = static_cast<int>((e1 - e0 + kThreads - 1) / kThreads);
+    uint32_t cnt = 0;
+    for (int it0 = 0; it0 < n_it; it0 += 4) {
+        float v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t e = e0 + static_cast<int64_t>(it0 + j) * kThreads + warp * 32 + lane;
+            v[j] = e < e1 ? row[e] : 0.0f;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int it = it0 + j;
+            if (it >= n_it) break;
+            const int64_t base = e0 + static_cast<int64_t>(it) * kThreads + warp * 32;
+            const bool live = base + lane < e1;
+            const uint32_t bin = order_key(v[j]) >> 21;
+            const unsigned above = __ballot_sync(0xffffffffu, live && bin > t1);
+            const unsigned in_t1 = __ballot_sync(0xffffffffu, live && bin == t1);
+            if (lane == 0) {
+                if (above) w.sel[base >> 5] = above;
+                s_mask[warp][it] = in_t1;
+            }
+            cnt += __popc(in_t1);
+        }
+    }
+    if (lane == 0) s_wcnt[warp] = cnt;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t tot = 0;
+        for (int q = 0; q < kThreads / 32; ++q) { const uint32_t c = s_wcnt[q]; s_wcnt[q] = tot; tot += c; }
+        s_base = tot ? atomicAdd(&w.hdr[0], tot) : 0u;
+    }
+    __syncthreads();
+    uint32_t pos = s_base + s_wcnt[warp];
+    for (int it = 0; it < n_it; ++it) {
+        const uint32_t mask = s_mask[warp][it];
+        if (!mask) continue;
+        const int64_t e = e0 + static_cast<int64_t>(it) * kThreads + warp * 32 + lane;
+        if ((mask >> lane) & 1u)
+            w.cand[pos + __popc(mask & ((1u << lane) - 1u))] =
+                (static_cast<unsigned long long>(order_key(row[e])) << 32) | static_cast<uint32_t>(e);
+        pos += __popc(mask);
+    }
+}
+
+// block-wide exclusive prefix sum of one value per thread (kResolveThreads)
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* sh_warp, uint32_t* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) sh_warp[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t s = sh_warp[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += y;
+        }
+        sh_warp[lane] = s;                       // inclusive per warp
+    }
+    __syncthreads();
+    const uint32_t warp_off = warp > 0 ? sh_warp[warp - 1] : 0u;
+    *total = sh_warp[31];
+    const uint32_t r = warp_off + x - v;
+    __syncthreads();
+    return r;
+}
+
+__global__ void __launch_bounds__(kResolveThreads, 1)
+resolve_kernel(const int32_t* __restrict__ q_pos, int64_t Nc_cap, int m, int k, uint8_t* __restrict__ ws,
+               int32_t* __restrict__ idx, int32_t* __restrict__ count) {
+    __shared__ uint32_t hist2[kBins];
+    __shared__ uint32_t sh_warp[32];
+    __shared__ uint32_t s_digit, s_need;
+    const int64_t r = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int64_t n = n_eligible(q_pos, r, m, Nc_cap);
+    const uint32_t kk = static_cast<uint32_t>(min(static_cast<int64_t>(k), n));
+    int32_t* orow = idx + static_cast<size_t>(r) * k;
+    if (tid == 0) count[r] = static_cast<int32_t>(kk);
+    if (kk == 0) {
+        for (int j = tid; j < k; j += kResolveThreads) orow[j] = -1;
+        return;
+    }
+    RowWs w = row_ws(ws, Nc_cap, r);
+    const uint32_t n_cand = w.hdr[0], t1 = w.hdr[1], need1 = w.hdr[2];
+    // exact threshold key T among the candidates (all share the top 11 bits t1)
+    uint32_t prefix = t1 << 21, need = need1;
+    if (need1 < n_cand) {
+        // pass 1: bits 20..10 (2048 bins); pass 2: bits 9..0 (1024 bins) of keys matching the prefix
+#pragma unroll 1
+        for (int pass = 0; pass < 2; ++pass) {
+            const int shift = pass == 0 ? 10 : 0;
+            const uint32_t nb = pass == 0 ? 2048u : 1024u;
+            const uint32_t mask_hi = pass == 0 ? 0xFFE00000u : 0xFFFFFC00u;   // bits already fixed
+            for (uint32_t i = tid; i < nb; i += kResolveThreads) hist2[i] = 0;
+            __syncthreads();
+            for (uint32_t c = tid; c < n_cand; c += kResolveThreads) {
+                const uint32_t key = static_cast<uint32_t>(w.cand[c] >> 32);
+                if ((key & mask_hi) == prefix) atomicAdd(&hist2[(key >> shift) & (nb - 1)], 1u);
+            }
+            __syncthreads();
+            {
+                // from the top digit down: the digit where the running count reaches need.
+                // Thread t holds digits nb-1-bpt*t .. nb-bpt*(t+1) (top first); a block
+                // scan gives the count above its digits.
+                const uint32_t bpt = nb / kResolveThreads;     // 2 or 1
+                uint32_t cnt[2] = {0u, 0u}, tot = 0;
+                for (uint32_t j = 0; j < bpt; ++j) { cnt[j] = hist2[nb - 1 - bpt * tid - j]; tot += cnt[j]; }
+                uint32_t all;
+                const uint32_t above = block_excl_scan(tot, sh_warp, &all);
+                if (above < need && above + tot >= need) {
+                    uint32_t acc = above;
+                    for (uint32_t j = 0; j < bpt; ++j) {
+                        if (acc + cnt[j] >= need) { s_digit = nb - 1 - bpt * tid - j; s_need = need - acc; break; }
+                        acc += cnt[j];
+                    }
+                }
+            }
+            __syncthreads();
+            prefix |= s_digit << shift;
+            need = s_need;
+            __syncthreads();
+        }
+        // keys above T: selected; keys equal to T: ties (need of them, lowest index first)
+        for (uint32_t c = tid; c < n_cand; c += kResolveThreads) {
+            const unsigned long long v = w.cand[c];
+            const uint32_t key = static_cast<uint32_t>(v >> 32), e = static_cast<uint32_t>(v);
+            if (key > prefix) atomicOr(&w.sel[e >> 5], 1u << (e & 31));
+            else if (key == prefix) atomicOr(&w.tie[e >> 5], 1u << (e & 31));
+        }
+    } else {
+        for (uint32_t c = tid; c < n_cand; c += kResolveThreads) {
+            const uint32_t e = static_cast<uint32_t>(w.cand[c]);
+            atomicOr(&w.sel[e >> 5], 1u << (e & 31));
+        }
+        need = 0;
+    }
+    __syncthreads();
+    // ordered output over the eligible words: thread t owns a contiguous run of words
+    const int64_t words = (n + 31) / 32;
+    const int64_t per = (words + kResolveThreads - 1) / kResolveThreads;
+    const int64_t w0 = min(words, per * tid), w1 = min(words, w0 + per);
+    uint32_t n_tie = 0;
+    for (int64_t q0 = w0; q0 < w1; q0 += 8) {
+        uint32_t t[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) t[j] = q0 + j < w1 ? w.tie[q0 + j] : 0u;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) n_tie += __popc(t[j]);
+    }
+    uint32_t tie_total;
+    uint32_t tie_before = block_excl_scan(n_tie, sh_warp, &tie_total);
+    uint32_t n_sel = 0;
+    {
+        uint32_t tb = tie_before;
+        for (int64_t q0 = w0; q0 < w1; q0 += 8) {
+            uint32_t t[8], sl[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                t[j] = q0 + j < w1 ? w.tie[q0 + j] : 0u;
+                sl[j] = q0 + j < w1 ? w.sel[q0 + j] : 0u;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t nt = __popc(t[j]);
+                const uint32_t take = tb >= need ? 0u : min(nt, need - tb);
+                n_sel += __popc(sl[j]) + take;
+                tb += nt;
+            }
+        }
+    }
+    uint32_t sel_total;
+    uint32_t out = block_excl_scan(n_sel, sh_warp, &sel_total);
+    {
+        uint32_t tb = tie_before;
+        for (int64_t q = w0; q < w1; ++q) {
+            uint32_t bits = w.sel[q];
+            uint32_t t = w.tie[q];
+            // the lowest ties of this word while the row still needs ties
+            while (t && tb < need) { const uint32_t lo = t & (~t + 1u); bits |= lo; t ^= lo; ++tb; }
+            tb += __popc(t);
+            while (bits) {
+                const int b = __ffs(bits) - 1;
+                bits &= bits - 1u;
+                if (out < static_cast<uint32_t>(k)) orow[out] = static_cast<int32_t>(q * 32 + b);
+                ++out;
+            }
+        }
+    }
+    for (int j = static_cast<int>(kk) + tid; j < k; j += kResolveThreads) orow[j] = -1;
+}
+
+}  // namespace wide
+
 }  // namespace
 
+// few long rows, or rows too long for a 16-block cluster
+bool topk_wide_preferred(int R, int64_t Nc_cap) {
+    if (R <= 0 || Nc_cap < 8192) return false;
+    return Nc_cap > 16 * kSliceMax || static_cast<int64_t>(R) * ceil_div(Nc_cap, kSlicePref) <= sm_count();
+}
+
+size_t topk_wide_ws_bytes(int R, int64_t Nc_cap) {
+    return static_cast<size_t>(R) * wide::layout(Nc_cap).row_bytes;
+}
+
+int topk_wide_launch(const float* scores, const int32_t* q_pos, int R, int64_t Nc_cap, int m, int k,
+                     int32_t* idx, int32_t* count, void* ws, cudaStream_t st) {
+    const wide::Layout L = wide::layout(Nc_cap);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    // clear each row's histogram, header and bitmaps
+    cudaError_t e = cudaMemset2DAsync(w, L.row_bytes, 0, L.clear_bytes, static_cast<size_t>(R), st);
+    if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
+    const int64_t ctas_per_row = std::max<int64_t>(1, ceil_div(2LL * sm_count(), R));
+    int64_t chunk = ceil_div(Nc_cap, ctas_per_row);
+    chunk = std::max<int64_t>(256, ceil_div(chunk, 256) * 256);       // whole bitmap words per warp
+    chunk = std::min<int64_t>(chunk, static_cast<int64_t>(wide::kMaxIt) * wide::kThreads);
+    const dim3 grid(static_cast<unsigned>(ceil_div(Nc_cap, chunk)), static_cast<unsigned>(R));
+    wide::hist_kernel<<<grid, wide::kThreads, 0, st>>>(scores, q_pos, Nc_cap, m, chunk, w);
+    HCA_CHECK_LAUNCH();
+    wide::mark_kernel<<<grid, wide::kThreads, 0, st>>>(scores, q_pos, Nc_cap, m, k, chunk, w);
+    HCA_CHECK_LAUNCH();
+    wide::resolve_kernel<<<R, wide::kResolveThreads, 0, st>>>(q_pos, Nc_cap, m, k, w, idx, count);
+    HCA_CHECK_LAUNCH();
+    return HCA_OK;
+}
+
 int topk_launch(const float* scores, const int32_t* q_pos, int R, int64_t Nc_cap, int m, int k,
-                int32_t* idx, int32_t* count, cudaStream_t st) {
+                int32_t* idx, int32_t* count, void* ws, size_t ws_bytes, cudaStream_t st) {
     if (R == 0) return HCA_OK;
+    if (topk_wide_preferred(R, Nc_cap) && ws != nullptr && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0 &&
+        ws_bytes >= topk_wide_ws_bytes(R, Nc_cap) && R <= 65535 && Nc_cap <= 0x7FFFFFFFLL)
+        return topk_wide_launch(scores, q_pos, R, Nc_cap, m, k, idx, count, ws, st);
+    if (Nc_cap > 16 * kSliceMax) return HCA_ERR_WORKSPACE;   // only the workspace path takes such rows
     if (g_max_cluster == 0) {
         // probe once whether 16-CTA clusters of this kernel fit the device
         cudaError_t e = cudaFuncSetAttribute(topk_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -19,7 +19,7 @@ from typing import List, Optional
 import torch
 
 from . import (KVCache, compressed_attn_decode, compressed_attn_prefill, csa_compress, decode_workspace_size,
-               hca_compress, lightning_index, topk_select)
+               hca_compress, lightning_index, topk_select, topk_workspace_size)
 
 CSA_RATIO = 4
 HCA_RATIO = 128
@@ -66,8 +66,12 @@ class DecodeLayer:
 class DecodeRunner:
     """Queues one decode step over a list of layers.  Per layer: CSA ->
     lightning_index, topk_select, compressed_attn_decode(sparse); HCA ->
-    compressed_attn_decode(dense).  CSA chains run on `side`, HCA on the
-    current stream; the step ends with both joined."""
+    compressed_attn_decode(dense).  CSA chains run on `side`, a stream of
+    higher priority, and HCA on the current stream; the step ends with both
+    joined.  An HCA launch waits for the indexer queued before it: the
+    indexer fills every SM anyway, and the top-k that follows it needs whole
+    clusters of free SMs, which the HCA CTAs (one per SM) would otherwise
+    hold when the indexer drains."""
 
     def __init__(self, layers: List[DecodeLayer], B: int, H: int, k: int, pos: int, softmax_scale: float,
                  device="cuda"):
@@ -79,20 +83,23 @@ class DecodeRunner:
         self.q_pos = torch.full((B, 1), pos, dtype=torch.int32, device=dev)
         self.out = [torch.empty((B, H, d), dtype=torch.bfloat16, device=dev) for _ in layers]
         self.n_dense = {}
-        self.scores, self.idx, self.count, self.ws = {}, {}, {}, {}
+        self.scores, self.idx, self.count, self.ws, self.topk_ws = {}, {}, {}, {}, {}
         W = layers[0].window.shape[1]
         for li, L in enumerate(layers):
             if L.ratio == CSA_RATIO:
                 self.scores[li] = torch.empty((B, 1, L.n_entries), dtype=torch.float32, device=dev)
                 self.idx[li] = torch.empty((B, k), dtype=torch.int32, device=dev)
                 self.count[li] = torch.empty((B,), dtype=torch.int32, device=dev)
+                self.topk_ws[li] = torch.empty(max(topk_workspace_size(B, L.n_entries, k), 16), dtype=torch.uint8,
+                                               device=dev)
                 mc = min(k, L.n_entries)
             else:
                 self.n_dense[li] = torch.full((B,), L.n_entries, dtype=torch.int32, device=dev)
                 mc = L.n_entries
             nbytes = decode_workspace_size(B, H, L.cache.layout, mc, W)
             self.ws[li] = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
-        self.side = torch.cuda.Stream(device=dev)
+        lo, hi = torch.cuda.Stream.priority_range()
+        self.side = torch.cuda.Stream(device=dev, priority=hi)
         self.kernels_per_step = self._count_kernels()
 
     def _count_kernels(self) -> int:
@@ -124,18 +131,24 @@ class DecodeRunner:
             b.record()
             events[key] = (a, b)
 
+        after_index = None
         for li, L in enumerate(self.layers):
             if L.ratio == CSA_RATIO:
                 with torch.cuda.stream(self.side):
                     qc, qs, w = iq[li]
                     timed("indexer", li, lambda: lightning_index(qc, qs, w, L.k_codes, L.k_sf, self.q_pos, CSA_RATIO,
                                                                  scores=self.scores[li]))
+                    after_index = torch.cuda.Event()
+                    after_index.record(self.side)
                     timed("topk", li, lambda: topk_select(self.scores[li].view(self.B, -1), self.q_pos.view(-1),
-                                                          CSA_RATIO, self.k, idx=self.idx[li], count=self.count[li]))
+                                                          CSA_RATIO, self.k, idx=self.idx[li], count=self.count[li],
+                                                          ws=self.topk_ws[li]))
                     timed("csa_attn", li, lambda: compressed_attn_decode(
                         q[li], L.cache, self.count[li], min(self.k, L.n_entries), L.window, self.scale,
                         idx=self.idx[li], out=self.out[li], ws=self.ws[li]))
             else:
+                if after_index is not None:
+                    main.wait_event(after_index)
                 timed("hca_attn", li, lambda: compressed_attn_decode(
                     q[li], L.cache, self.n_dense[li], L.n_entries, L.window, self.scale, out=self.out[li],
                     ws=self.ws[li]))
@@ -173,7 +186,8 @@ class PrefillRunner:
         d = st.csa.layout[0]
         self.out_csa = torch.empty((Tq, H, d), dtype=torch.bfloat16, device=dev)
         self.out_hca = torch.empty((Tq, H, d), dtype=torch.bfloat16, device=dev)
-        self.side = torch.cuda.Stream(device=dev)
+        lo, hi = torch.cuda.Stream.priority_range()
+        self.side = torch.cuda.Stream(device=dev, priority=hi)
         self.kernels_per_step = 6
 
     def step(self, raw_chunk, gate_chunk, raw_window, q, iq, events: Optional[dict] = None):

@@ -80,7 +80,12 @@ def test_host_validation_without_gpu(lib):
     assert lib.lightning_index(None, None, None, None, None, None, 1, 1, 10, 4, 128, 0, None, None) == 1  # m
     lib.topk_select.argtypes = [V, V, I32, I64, I32, I32, V, V, V, ctypes.c_size_t, V]
     assert lib.topk_select(None, None, 1, 100, 4, 0, None, None, None, 0, None) == 2       # k = 0
-    assert lib.topk_select(None, None, 1, 1 << 20, 4, 8, None, None, None, 0, None) == 2   # Nc too large
+    # a row longer than 2^19 scores needs the workspace path
+    assert lib.topk_select(V(0x1000), V(0x1000), 1, 1 << 20, 4, 8, V(0x1000), V(0x1000), None, 0, None) == 4
+    lib.topk_select_workspace_size.argtypes = [I32, I64, I32]
+    lib.topk_select_workspace_size.restype = ctypes.c_size_t
+    assert lib.topk_select_workspace_size(4, 262144, 1024) >= 4 * 262144 * 8   # few long rows: histogram path
+    assert lib.topk_select_workspace_size(4096, 33000, 512) == 0               # many rows: clusters, no workspace
     assert lib.topk_select(None, None, 1, 100, 4, 8, None, None, None, 0, None) == 1       # null pointers
     lib.compressed_attn_decode.argtypes = [V, I32, I32, Layout, Cache, V, I32, V, I32, V, I32, ctypes.c_float,
                                            V, V, V, ctypes.c_size_t, V]

@@ -165,7 +165,8 @@ def test_indexer_sixteen_queries_per_cta(Tq, Nc):
 
 
 # ------------------------------------------------------------------ top-k
-@pytest.mark.parametrize("Nc,k", [(1, 1), (100, 7), (5000, 32), (33000, 1024), (70000, 512), (140000, 4096)])
+@pytest.mark.parametrize("Nc,k", [(1, 1), (100, 7), (5000, 32), (33000, 1024), (70000, 512), (140000, 4096),
+                                  (600000, 4096)])
 def test_topk_bit_exact(Nc, k):
     R, m = 5, 4
     g = _gen(Nc + k)
@@ -178,6 +179,22 @@ def test_topk_bit_exact(Nc, k):
     idx, cnt = hca.topk_select(scores, pos, m, k)
     torch.cuda.synchronize()
     wi, wc = oracle.topk(host(scores), host(pos), m, k)
+    assert np.array_equal(host(cnt), wc)
+    assert np.array_equal(host(idx), wi)
+
+
+@pytest.mark.parametrize("R,Nc,k", [(4, 262144, 1024), (2, 70001, 777)])
+def test_topk_crowded_threshold_bin(R, Nc, k):
+    """Scores packed into a narrow range (one top-11-bit histogram bin holds most of
+    them), duplicated so that the k-th score is tied: the exact key and the
+    lowest-index ties must be found among the candidates."""
+    g = _gen(R * Nc + k)
+    base = 1.0 + torch.randint(0, 3000, (R, Nc), generator=g, device=DEV).float() * 2.0 ** -13
+    pos = torch.full((R,), 4 * Nc - 1, dtype=torch.int32, device=DEV)
+    pos[-1] = 4 * (Nc // 2) + 1
+    idx, cnt = hca.topk_select(base, pos, 4, k)
+    torch.cuda.synchronize()
+    wi, wc = oracle.topk(host(base), host(pos), 4, k)
     assert np.array_equal(host(cnt), wc)
     assert np.array_equal(host(idx), wi)
 
