@@ -103,11 +103,16 @@ class DecodeRunner:
         self.kernels_per_step = self._count_kernels()
 
     def _count_kernels(self) -> int:
+        """Kernels of this library launched per step: attention (+ split combine) per
+        layer; per CSA layer the indexer and the top-k (three kernels on the
+        histogram path, one on the cluster path)."""
         n = 0
         for li, L in enumerate(self.layers):
             mc = min(self.k, L.n_entries) if L.ratio == CSA_RATIO else L.n_entries
             split = decode_workspace_size(self.B, self.H, L.cache.layout, mc, L.window.shape[1]) > 0
-            n += (1 + int(split)) + (2 if L.ratio == CSA_RATIO else 0)
+            n += 1 + int(split)
+            if L.ratio == CSA_RATIO:
+                n += 1 + (3 if topk_workspace_size(self.B, L.n_entries, self.k) > 0 else 1)
         return n
 
     def step(self, q: List[torch.Tensor], iq: List[Optional[tuple]], events: Optional[dict] = None):
