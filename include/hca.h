@@ -83,6 +83,21 @@ int hca_last_cuda_error(void);
  * cannot be read. */
 int hca_take_device_error(void);
 
+/* Launch budget: a scheduling knob with no counterpart on the pages.  It
+ * caps the CTAs (splits x sequences) of one decode attention launch on the
+ * tensor-core path (d = 512, H = 64) so that
+ * the launch occupies only part of the device and another stream's kernels
+ * (the CSA chain: indexer, top-k, sparse attention) run beside it.
+ *   op        HCA_BUDGET_DENSE_DECODE or HCA_BUDGET_SPARSE_DECODE
+ *   max_ctas  > 0: at most max(max_ctas, B) CTAs; 0: the default (one CTA
+ *             per SM at most)
+ * Process-wide; applies to workspace sizing and launches made after the
+ * call, so size workspaces after setting it.  Returns the previous value,
+ * or -1 for an unknown op or a negative max_ctas. */
+#define HCA_BUDGET_DENSE_DECODE 0
+#define HCA_BUDGET_SPARSE_DECODE 1
+int hca_set_launch_budget(int op, int max_ctas);
+
 /* ------------------------------------------------------------------ */
 /* Compression: softmax-gated pooling + FP8/BF16 storage.               */
 /* ------------------------------------------------------------------ */

@@ -54,6 +54,20 @@ _lib.hca_take_device_error.argtypes = []
 _lib.hca_take_device_error.restype = ctypes.c_int
 
 
+BUDGET_DENSE_DECODE, BUDGET_SPARSE_DECODE = 0, 1
+_lib.hca_set_launch_budget.argtypes = [ctypes.c_int, ctypes.c_int]
+_lib.hca_set_launch_budget.restype = ctypes.c_int
+
+
+def set_launch_budget(op: int, max_ctas: int) -> int:
+    """Cap the CTAs of decode attention launches (op: BUDGET_DENSE_DECODE or
+    BUDGET_SPARSE_DECODE; 0 = default).  Process-wide; returns the previous value."""
+    prev = int(_lib.hca_set_launch_budget(op, max_ctas))
+    if prev < 0:
+        raise ValueError("set_launch_budget: unknown op or negative budget")
+    return prev
+
+
 def take_device_error() -> int:
     """Read and clear the device error word (non-zero: a kernel gave up a bounded wait)."""
     return int(_lib.hca_take_device_error())

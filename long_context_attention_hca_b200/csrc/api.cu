@@ -3,6 +3,8 @@
 // call leaves the stream untouched.  See include/hca.h for the contract.
 #include <mutex>
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace hca {
@@ -76,6 +78,10 @@ int compress_common(int m, const uint16_t* x, const uint16_t* gate, int64_t x_se
 }
 
 }  // namespace
+
+static std::atomic<int> g_launch_budget[2] = {{0}, {0}};
+int launch_budget(int op) { return (op == 0 || op == 1) ? g_launch_budget[op].load() : 0; }
+
 }  // namespace hca
 
 using namespace hca;
@@ -95,6 +101,12 @@ const char* hca_status_string(int status) {
 }
 
 int hca_last_cuda_error(void) { return g_last_cuda_error; }
+
+
+int hca_set_launch_budget(int op, int max_ctas) {
+    if ((op != HCA_BUDGET_DENSE_DECODE && op != HCA_BUDGET_SPARSE_DECODE) || max_ctas < 0) return -1;
+    return hca::g_launch_budget[op].exchange(max_ctas);
+}
 
 int hca_take_device_error(void) {
     const int a = tc_take_device_error(), b = index_take_device_error();

@@ -625,29 +625,68 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
 }
 
 // Log-sum-exp combine of split partials (base-2 maxima): grid (unit, head),
-// 128 threads x 4 dims.
+// 128 threads x 4 dims.  All (m, l) pairs are read first, then the partial
+// outputs 8 splits at a time, so the L2 reads are in flight together.
 __global__ void __launch_bounds__(128) combine_tc_kernel(Params p) {
+    constexpr int MAXS = 256;
+    __shared__ float s_w[MAXS];
+    __shared__ float s_L;
+    __shared__ int s_bad;
     const int64_t u = blockIdx.x;
     const int h = blockIdx.y;
     const int S = p.n_splits;
     const float* ml0 = p.part_ml + static_cast<size_t>(u) * S * 2 * HP;
-    float M = -INFINITY;
-    for (int s = 0; s < S; ++s) {
-        const float ls = ml0[s * 2 * HP + HP + h];
-        if (ls > 0.0f) M = fmaxf(M, ml0[s * 2 * HP + h]);
+    if (threadIdx.x < 32) {
+        // split weights 2^(m_s - M) (0 for empty splits), their l-weighted sum, NaN flag
+        float M = -INFINITY;
+        for (int s = threadIdx.x; s < S; s += 32) {
+            const float ls = ml0[s * 2 * HP + HP + h];
+            if (ls > 0.0f) M = fmaxf(M, ml0[s * 2 * HP + h]);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float L = 0.0f;
+        int bad = 0;
+        for (int s = threadIdx.x; s < S; s += 32) {
+            const float ms = ml0[s * 2 * HP + h], ls = ml0[s * 2 * HP + HP + h];
+            if (ls != ls) bad = 1;
+            const float wgt = ls > 0.0f ? exp2f(ms - M) : 0.0f;
+            if (s < MAXS) s_w[s] = wgt;
+            L += wgt * (ls > 0.0f ? ls : 0.0f);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            L += __shfl_xor_sync(0xffffffffu, L, o);
+            bad |= __shfl_xor_sync(0xffffffffu, bad, o);
+        }
+        if (threadIdx.x == 0) {
+            s_L = L;
+            s_bad = bad;
+            if (p.lse)
+                p.lse[u * p.H + h] = bad ? __int_as_float(0x7fc00000)
+                                         : (L > 0.0f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY);
+        }
     }
-    float L = 0.0f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-    bool bad = false;
+    __syncthreads();
     const int d0 = threadIdx.x * 4;
-    for (int s = 0; s < S; ++s) {
-        const float ms = ml0[s * 2 * HP + h], ls = ml0[s * 2 * HP + HP + h];
-        if (ls != ls) bad = true;
-        if (!(ls > 0.0f)) continue;
-        const float wgt = exp2f(ms - M);
-        L += wgt * ls;
-        const float4 v = *reinterpret_cast<const float4*>(p.part_o + ((static_cast<size_t>(u) * S + s) * HP + h) * D + d0);
-        acc[0] += wgt * v.x; acc[1] += wgt * v.y; acc[2] += wgt * v.z; acc[3] += wgt * v.w;
+    const float* po = p.part_o + (static_cast<size_t>(u) * S * HP + h) * D + d0;
+    const size_t split_stride = static_cast<size_t>(HP) * D;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int s0 = 0; s0 < S; s0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            v[j] = (s0 + j < S && s_w[s0 + j] != 0.0f)
+                       ? *reinterpret_cast<const float4*>(po + static_cast<size_t>(s0 + j) * split_stride)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float wgt = s0 + j < S ? s_w[s0 + j] : 0.0f;
+            acc[0] += wgt * v[j].x; acc[1] += wgt * v[j].y; acc[2] += wgt * v[j].z; acc[3] += wgt * v[j].w;
+        }
     }
+    const bool bad = s_bad != 0;
+    const float L = s_L;
     const float inv = L > 0.0f ? 1.0f / L : 0.0f;
     const float qnan = __int_as_float(0x7fc00000);
     __nv_bfloat162 a = __floats2bfloat162_rn(bad ? qnan : acc[0] * inv, bad ? qnan : acc[1] * inv);
@@ -656,8 +695,6 @@ __global__ void __launch_bounds__(128) combine_tc_kernel(Params p) {
     w.x = *reinterpret_cast<uint32_t*>(&a);
     w.y = *reinterpret_cast<uint32_t*>(&b);
     *reinterpret_cast<uint2*>(p.out + (static_cast<size_t>(u) * p.H + h) * D + d0) = w;
-    if (p.lse && threadIdx.x == 0)
-        p.lse[u * p.H + h] = bad ? qnan : (L > 0.0f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY);
 }
 
 }  // namespace tc
@@ -685,10 +722,12 @@ int launch_tc(tc::Params& p, int64_t units, cudaStream_t st) {
 // per CTA so the pipeline fills and the partials stay small.
 void tc_decode_plan(int B, int max_comp, int W, bool sparse, int& n_splits, int& tiles_per_split) {
     const int n_tiles = static_cast<int>(ceil_div(static_cast<int64_t>(max_comp) + W, tc::TK));
-    const int min_tps = sparse ? 2 : 6;       // tiles of 64 keys
-    int splits = sm_count() / (B > 0 ? B : 1);
+    const int min_tps = sparse ? 1 : 6;       // tiles of 64 keys
+    const int budget = launch_budget(sparse ? HCA_BUDGET_SPARSE_DECODE : HCA_BUDGET_DENSE_DECODE);
+    int splits = (budget > 0 ? budget : sm_count()) / (B > 0 ? B : 1);
     const int cap_by_len = static_cast<int>(ceil_div(n_tiles > 0 ? n_tiles : 1, min_tps));
     if (splits > cap_by_len) splits = cap_by_len;
+    if (splits > 256) splits = 256;           // the combine keeps one weight per split in shared memory
     if (splits < 1) splits = 1;
     tiles_per_split = static_cast<int>(ceil_div(n_tiles > 0 ? n_tiles : 1, splits));
     n_splits = static_cast<int>(ceil_div(n_tiles > 0 ? n_tiles : 1, tiles_per_split));

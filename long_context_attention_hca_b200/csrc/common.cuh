@@ -30,6 +30,8 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Number of SMs of the current device (queried once per process and device).
 int sm_count();
+// process-wide CTA cap of a decode attention launch (0: none); see hca_set_launch_budget
+int launch_budget(int op);
 
 // ---------------------------------------------------------------- device
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) {

@@ -470,15 +470,15 @@ mark_kernel(const float* __restrict__ scores, const int32_t* __restrict__ q_pos,
     __shared__ uint32_t s_base;
     const int n_it = static_cast<int>((e1 - e0 + kThreads - 1) / kThreads);
     uint32_t cnt = 0;
-    for (int it0 = 0; it0 < n_it; it0 += 4) {
-        float v[4];
+    for (int it0 = 0; it0 < n_it; it0 += 8) {
+        float v[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 8; ++j) {
             const int64_t e = e0 + static_cast<int64_t>(it0 + j) * kThreads + warp * 32 + lane;
             v[j] = e < e1 ? row[e] : 0.0f;
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 8; ++j) {
             const int it = it0 + j;
             if (it >= n_it) break;
             const int64_t base = e0 + static_cast<int64_t>(it) * kThreads + warp * 32;
@@ -544,7 +544,10 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* sh_war
 __global__ void __launch_bounds__(kResolveThreads, 1)
 resolve_kernel(const int32_t* __restrict__ q_pos, int64_t Nc_cap, int m, int k, uint8_t* __restrict__ ws,
                int32_t* __restrict__ idx, int32_t* __restrict__ count) {
+    constexpr int kCandCache = 4096;          // candidates kept in shared memory (else read from L2)
+    constexpr int kRegWords = 8;              // bitmap words a thread keeps in registers
     __shared__ uint32_t hist2[kBins];
+    __shared__ unsigned long long s_cand[kCandCache];
     __shared__ uint32_t sh_warp[32];
     __shared__ uint32_t s_digit, s_need;
     const int64_t r = blockIdx.x;
@@ -559,6 +562,20 @@ resolve_kernel(const int32_t* __restrict__ q_pos, int64_t Nc_cap, int m, int k, 
     }
     RowWs w = row_ws(ws, Nc_cap, r);
     const uint32_t n_cand = w.hdr[0], t1 = w.hdr[1], need1 = w.hdr[2];
+    const bool cached = n_cand <= static_cast<uint32_t>(kCandCache);
+    if (cached) {
+        // one round of loads for all candidates
+        unsigned long long v[kCandCache / kResolveThreads];
+#pragma unroll
+        for (int j = 0; j < kCandCache / kResolveThreads; ++j) {
+            const uint32_t c = tid + j * kResolveThreads;
+            v[j] = c < n_cand ? w.cand[c] : 0ull;
+        }
+#pragma unroll
+        for (int j = 0; j < kCandCache / kResolveThreads; ++j) s_cand[tid + j * kResolveThreads] = v[j];
+        __syncthreads();
+    }
+    auto cand = [&](uint32_t c) { return cached ? s_cand[c] : w.cand[c]; };
     // exact threshold key T among the candidates (all share the top 11 bits t1)
     uint32_t prefix = t1 << 21, need = need1;
     if (need1 < n_cand) {
@@ -571,7 +588,7 @@ resolve_kernel(const int32_t* __restrict__ q_pos, int64_t Nc_cap, int m, int k, 
             for (uint32_t i = tid; i < nb; i += kResolveThreads) hist2[i] = 0;
             __syncthreads();
             for (uint32_t c = tid; c < n_cand; c += kResolveThreads) {
-                const uint32_t key = static_cast<uint32_t>(w.cand[c] >> 32);
+                const uint32_t key = static_cast<uint32_t>(cand(c) >> 32);
                 if ((key & mask_hi) == prefix) atomicAdd(&hist2[(key >> shift) & (nb - 1)], 1u);
             }
             __syncthreads();
@@ -599,60 +616,78 @@ resolve_kernel(const int32_t* __restrict__ q_pos, int64_t Nc_cap, int m, int k, 
         }
         // keys above T: selected; keys equal to T: ties (need of them, lowest index first)
         for (uint32_t c = tid; c < n_cand; c += kResolveThreads) {
-            const unsigned long long v = w.cand[c];
+            const unsigned long long v = cand(c);
             const uint32_t key = static_cast<uint32_t>(v >> 32), e = static_cast<uint32_t>(v);
             if (key > prefix) atomicOr(&w.sel[e >> 5], 1u << (e & 31));
             else if (key == prefix) atomicOr(&w.tie[e >> 5], 1u << (e & 31));
         }
     } else {
         for (uint32_t c = tid; c < n_cand; c += kResolveThreads) {
-            const uint32_t e = static_cast<uint32_t>(w.cand[c]);
+            const uint32_t e = static_cast<uint32_t>(cand(c));
             atomicOr(&w.sel[e >> 5], 1u << (e & 31));
         }
         need = 0;
     }
-    __syncthreads();
+    __syncthreads();       // the bitmap updates above are visible to the whole block
     // ordered output over the eligible words: thread t owns a contiguous run of words
     const int64_t words = (n + 31) / 32;
     const int64_t per = (words + kResolveThreads - 1) / kResolveThreads;
     const int64_t w0 = min(words, per * tid), w1 = min(words, w0 + per);
-    uint32_t n_tie = 0;
-    for (int64_t q0 = w0; q0 < w1; q0 += 8) {
-        uint32_t t[8];
+    if (per <= kRegWords) {
+        // the thread's words in registers: one round of loads for both scans and the write
+        uint32_t sl[kRegWords], tw[kRegWords];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) t[j] = q0 + j < w1 ? w.tie[q0 + j] : 0u;
+        for (int j = 0; j < kRegWords; ++j) {
+            sl[j] = w0 + j < w1 ? w.sel[w0 + j] : 0u;
+            tw[j] = w0 + j < w1 ? w.tie[w0 + j] : 0u;
+        }
+        uint32_t n_tie = 0;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) n_tie += __popc(t[j]);
-    }
-    uint32_t tie_total;
-    uint32_t tie_before = block_excl_scan(n_tie, sh_warp, &tie_total);
-    uint32_t n_sel = 0;
-    {
-        uint32_t tb = tie_before;
-        for (int64_t q0 = w0; q0 < w1; q0 += 8) {
-            uint32_t t[8], sl[8];
+        for (int j = 0; j < kRegWords; ++j) n_tie += __popc(tw[j]);
+        uint32_t tie_total;
+        const uint32_t tie_before = block_excl_scan(n_tie, sh_warp, &tie_total);
+        // take the lowest ties while the row still needs them
+        uint32_t tb = tie_before, n_sel = 0;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                t[j] = q0 + j < w1 ? w.tie[q0 + j] : 0u;
-                sl[j] = q0 + j < w1 ? w.sel[q0 + j] : 0u;
+        for (int j = 0; j < kRegWords; ++j) {
+            uint32_t t = tw[j];
+            while (t && tb < need) { const uint32_t lo = t & (~t + 1u); sl[j] |= lo; t ^= lo; ++tb; }
+            tb += __popc(t);
+            n_sel += __popc(sl[j]);
+        }
+        uint32_t sel_total;
+        uint32_t out = block_excl_scan(n_sel, sh_warp, &sel_total);
+#pragma unroll
+        for (int j = 0; j < kRegWords; ++j) {
+            uint32_t bits = sl[j];
+            while (bits) {
+                const int b = __ffs(bits) - 1;
+                bits &= bits - 1u;
+                if (out < static_cast<uint32_t>(k)) orow[out] = static_cast<int32_t>((w0 + j) * 32 + b);
+                ++out;
             }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t nt = __popc(t[j]);
+        }
+    } else {
+        uint32_t n_tie = 0;
+        for (int64_t q = w0; q < w1; ++q) n_tie += __popc(w.tie[q]);
+        uint32_t tie_total;
+        const uint32_t tie_before = block_excl_scan(n_tie, sh_warp, &tie_total);
+        uint32_t n_sel = 0;
+        {
+            uint32_t tb = tie_before;
+            for (int64_t q = w0; q < w1; ++q) {
+                const uint32_t nt = __popc(w.tie[q]);
                 const uint32_t take = tb >= need ? 0u : min(nt, need - tb);
-                n_sel += __popc(sl[j]) + take;
+                n_sel += __popc(w.sel[q]) + take;
                 tb += nt;
             }
         }
-    }
-    uint32_t sel_total;
-    uint32_t out = block_excl_scan(n_sel, sh_warp, &sel_total);
-    {
+        uint32_t sel_total;
+        uint32_t out = block_excl_scan(n_sel, sh_warp, &sel_total);
         uint32_t tb = tie_before;
         for (int64_t q = w0; q < w1; ++q) {
             uint32_t bits = w.sel[q];
             uint32_t t = w.tie[q];
-            // the lowest ties of this word while the row still needs ties
             while (t && tb < need) { const uint32_t lo = t & (~t + 1u); bits |= lo; t ^= lo; ++tb; }
             tb += __popc(t);
             while (bits) {

@@ -19,7 +19,8 @@ from typing import List, Optional
 import torch
 
 from . import (KVCache, compressed_attn_decode, compressed_attn_prefill, csa_compress, decode_workspace_size,
-               hca_compress, lightning_index, topk_select, topk_workspace_size)
+               hca_compress, lightning_index, topk_select, topk_workspace_size, set_launch_budget,
+               BUDGET_DENSE_DECODE)
 
 CSA_RATIO = 4
 HCA_RATIO = 128
@@ -74,7 +75,16 @@ class DecodeRunner:
     hold when the indexer drains."""
 
     def __init__(self, layers: List[DecodeLayer], B: int, H: int, k: int, pos: int, softmax_scale: float,
-                 device="cuda"):
+                 device="cuda", schedule: str = "after_index", dense_budget: int = 0):
+        """schedule: "after_index" -- an HCA launch waits for the indexer queued
+        before it; "hca_first" -- all HCA launches are queued first and start at
+        once, with dense_budget (if > 0) capping their CTAs so that the CSA
+        chain runs beside them on the remaining SMs."""
+        if schedule not in ("after_index", "hca_first"):
+            raise ValueError(schedule)
+        self.schedule = schedule
+        if dense_budget:
+            set_launch_budget(BUDGET_DENSE_DECODE, dense_budget)
         self.layers, self.B, self.H, self.k, self.pos = layers, B, H, k, pos
         self.scale = softmax_scale
         d = layers[0].cache.layout[0]
@@ -137,7 +147,12 @@ class DecodeRunner:
             events[key] = (a, b)
 
         after_index = None
-        for li, L in enumerate(self.layers):
+        order = list(range(len(self.layers)))
+        if self.schedule == "hca_first":
+            order = [li for li in order if self.layers[li].ratio != CSA_RATIO] + \
+                    [li for li in order if self.layers[li].ratio == CSA_RATIO]
+        for li in order:
+            L = self.layers[li]
             if L.ratio == CSA_RATIO:
                 with torch.cuda.stream(self.side):
                     qc, qs, w = iq[li]
@@ -152,7 +167,7 @@ class DecodeRunner:
                         q[li], L.cache, self.count[li], min(self.k, L.n_entries), L.window, self.scale,
                         idx=self.idx[li], out=self.out[li], ws=self.ws[li]))
             else:
-                if after_index is not None:
+                if after_index is not None and self.schedule == "after_index":
                     main.wait_event(after_index)
                 timed("hca_attn", li, lambda: compressed_attn_decode(
                     q[li], L.cache, self.n_dense[li], L.n_entries, L.window, self.scale, out=self.out[li],

@@ -291,6 +291,29 @@ def test_decode_many_splits_match_single_split():
         assert_attn_close(host(out)[b], ref, f"b={b}")
 
 
+@pytest.mark.parametrize("budget", [2, 7, 40])
+def test_decode_launch_budget(budget):
+    """A CTA budget changes the split plan of the dense decode attention, not its
+    result (the workspace is sized for the larger of the sparse and dense plans)."""
+    layout = (512, 64, 64)
+    B, cap, W = 2, 9000, 128
+    cache = _random_cache(B, cap, layout, 41)
+    q = _bf16((B, 64, 512), 42)
+    win = _bf16((B, W, 512), 43)
+    n_comp = torch.tensor([cap, 4321], dtype=torch.int32, device=DEV)
+    prev = hca.set_launch_budget(hca.BUDGET_DENSE_DECODE, budget)
+    try:
+        out = hca.compressed_attn_decode(q, cache, n_comp, cap, win, 512 ** -0.5)
+        torch.cuda.synchronize()
+    finally:
+        hca.set_launch_budget(hca.BUDGET_DENSE_DECODE, prev)
+    codes, scales, rope = cache_host(cache)
+    for b in range(B):
+        ref, _ = oracle.attend(host(q)[b], codes[b], scales[b], rope[b], np.arange(host(n_comp)[b]), host(win)[b],
+                               512 ** -0.5, 64)
+        assert_attn_close(host(out)[b], ref, f"budget={budget} b={b}")
+
+
 @pytest.mark.parametrize("layout,H,p0", [((512, 64, 64), 64, 1000), ((128, 32, 32), 8, 10)])
 def test_prefill_dense_and_sparse(layout, H, p0):
     d, dr, g = layout
