@@ -192,6 +192,7 @@ def decode_bytes(wl):
         "hca_attn": nh * entry + wl.W * wl.d * 2 + qo,
         "topk": nc * 4 + wl.k * 4 + 8,          # scores read (L2-resident at this size), indices written
     }
+    per_seq["index_topk"] = per_seq["indexer"] + per_seq["topk"]
     return {k: v * wl.B for k, v in per_seq.items()}
 
 

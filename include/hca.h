@@ -184,6 +184,26 @@ int topk_select(const float* scores, const int32_t* q_pos, int32_t R, int64_t Nc
                 void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------ */
+/* Fused decode selection: lightning_index (Tq = 1) then topk_select.   */
+/* ------------------------------------------------------------------ */
+/* The same results as lightning_index(..., Tq = 1, ...) followed by
+ * topk_select(scores, q_pos, B, Nc_cap, m, k, ...): scores [B][Nc_cap]
+ * are written, idx [B][k] and count [B] as topk_select.  With a workspace of
+ * lightning_index_topk_workspace_size(B, Nc_cap, k) bytes (256-byte
+ * aligned), c = 128 and Hi = 4, the indexer kernel also builds each row's
+ * key histogram, which saves the top-k one pass over the scores; otherwise
+ * the two calls run one after the other.  index_done (a cudaEvent_t, may
+ * be NULL) is recorded on the stream once the scores are written, before the
+ * top-k work: a scheduler can start other streams' work there.  Error
+ * behaviour as the two calls. */
+size_t lightning_index_topk_workspace_size(int32_t B, int64_t Nc_cap, int32_t k);
+int lightning_index_topk(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
+                         const uint8_t* k_codes, const uint8_t* k_sf, const int32_t* q_pos,
+                         int32_t B, int64_t Nc_cap, int32_t Hi, int32_t c, int32_t m, int32_t k,
+                         float* scores, int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
+                         void* index_done, void* stream);
+
+/* ------------------------------------------------------------------ */
 /* Core attention (section 7: shared key-value MQA + sliding window;    */
 /* section 8: dense over all compressed entries).                       */
 /* ------------------------------------------------------------------ */

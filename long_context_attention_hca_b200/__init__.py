@@ -31,7 +31,8 @@ HCA_OK, HCA_ERR_INVALID_ARG, HCA_ERR_UNSUPPORTED, HCA_ERR_CUDA, HCA_ERR_WORKSPAC
 
 EXPORTED = (
     "hca_status_string", "hca_last_cuda_error", "csa_compress", "hca_compress", "lightning_index",
-    "topk_select_workspace_size", "topk_select", "compressed_attn_decode_workspace_size",
+    "topk_select_workspace_size", "topk_select", "lightning_index_topk_workspace_size", "lightning_index_topk",
+    "compressed_attn_decode_workspace_size",
     "compressed_attn_decode", "compressed_attn_prefill_workspace_size", "compressed_attn_prefill",
 )
 
@@ -217,6 +218,50 @@ def topk_select(scores, q_pos, m, k, idx=None, count=None, ws=None, stream=None)
     _check(_lib.topk_select(_p(scores), _p(q_pos), R, Nc, m, k, _p(idx), _p(count), _p(ws), ws_bytes,
                             _stream(stream)), "topk_select")
     return idx, count
+
+
+_lib.lightning_index_topk_workspace_size.argtypes = [_I32, _I64, _I32]
+_lib.lightning_index_topk_workspace_size.restype = _SZ
+_lib.lightning_index_topk.argtypes = [_V, _V, _V, _V, _V, _V, _I32, _I64, _I32, _I32, _I32, _I32, _V, _V, _V, _V, _SZ,
+                                      _V, _V]
+_lib.lightning_index_topk.restype = ctypes.c_int
+
+
+def lightning_index_topk(q_codes, q_sf, w, k_codes, k_sf, q_pos, m, k, scores=None, idx=None, count=None, ws=None,
+                         index_done=None, stream=None):
+    """Decode (one query per sequence): index scores and top-k in one call.
+    q_codes [B][1][Hi][c/2], q_sf [B][1][Hi][c/32], w [B][1][Hi]; k_codes [B][Nc][c/2], k_sf [B][Nc][c/32];
+    q_pos [B] or [B][1].  index_done: optional torch.cuda.Event recorded once the scores
+    are written (it must have been recorded once before, so that it exists).
+    Returns (scores [B][1][Nc], idx [B][k], count [B])."""
+    ev = None
+    if index_done is not None:
+        ev = ctypes.c_void_p(index_done.cuda_event)
+        if not ev.value:
+            raise ValueError("lightning_index_topk: index_done has no CUDA event yet (record it once first)")
+    for t, dt, n in ((q_codes, torch.uint8, "q_codes"), (q_sf, torch.uint8, "q_sf"), (w, torch.float32, "w"),
+                     (k_codes, torch.uint8, "k_codes"), (k_sf, torch.uint8, "k_sf"), (q_pos, torch.int32, "q_pos")):
+        _need(t, dt, n)
+    B, Tq, Hi, half_c = q_codes.shape
+    if Tq != 1:
+        raise ValueError("lightning_index_topk: one query per sequence")
+    Nc = k_codes.shape[1]
+    dev = q_codes.device
+    if scores is None:
+        scores = torch.empty((B, 1, Nc), dtype=torch.float32, device=dev)
+    if idx is None:
+        idx = torch.empty((B, k), dtype=torch.int32, device=dev)
+    if count is None:
+        count = torch.empty((B,), dtype=torch.int32, device=dev)
+    need = int(_lib.lightning_index_topk_workspace_size(B, Nc, k))
+    if need and (ws is None or ws.numel() < need):
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    elif not need:
+        ws = None
+    _check(_lib.lightning_index_topk(_p(q_codes), _p(q_sf), _p(w), _p(k_codes), _p(k_sf), _p(q_pos), B, Nc, Hi,
+                                     2 * half_c, m, k, _p(scores), _p(idx), _p(count), _p(ws), need, ev,
+                                     _stream(stream)), "lightning_index_topk")
+    return scores, idx, count
 
 
 def decode_workspace_size(B, H, layout, max_comp, W) -> int:

@@ -19,6 +19,14 @@ int topk_launch(const float* scores, const int32_t* q_pos, int R, int64_t Nc_cap
                 int32_t* idx, int32_t* count, void* ws, size_t ws_bytes, cudaStream_t st);
 bool topk_wide_preferred(int R, int64_t Nc_cap);
 size_t topk_wide_ws_bytes(int R, int64_t Nc_cap);
+int topk_wide_clear(void* ws, int R, int64_t Nc_cap, cudaStream_t st);
+uint32_t* topk_wide_hist(void* ws, int64_t Nc_cap, int64_t* stride_u32);
+int topk_wide_select(const float* scores, const int32_t* q_pos, int R, int64_t Nc_cap, int m, int k,
+                     int32_t* idx, int32_t* count, void* ws, cudaStream_t st);
+int index_launch_hist(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
+                      const uint8_t* k_codes, const uint8_t* k_sf, const int32_t* q_pos,
+                      int B, int64_t Nc_cap, int Hi, int c, int m, float* scores, uint32_t* hist,
+                      int64_t hist_stride, cudaStream_t st);
 size_t decode_ws_bytes(int B, int H, int D, int max_comp, int W);
 int attn_decode_launch(const uint16_t* q, int B, int H, const hca_kv_layout& L, const hca_kv_cache& kv,
                        const int32_t* idx, int idx_stride, const int32_t* n_comp, int max_comp,
@@ -152,6 +160,56 @@ int topk_select(const float* scores, const int32_t* q_pos, int32_t R, int64_t Nc
     if (Nc_cap > 0) REQ_PTR(scores);
     if (Nc_cap > 16 * 32768LL && ws_bytes < topk_select_workspace_size(R, Nc_cap, k)) return HCA_ERR_WORKSPACE;
     return topk_launch(scores, q_pos, R, Nc_cap, m, k, idx, count, ws, ws_bytes, as_stream(stream));
+}
+
+static int record_event(void* ev, cudaStream_t st) {
+    if (ev == nullptr) return HCA_OK;
+    const cudaError_t e = cudaEventRecord(static_cast<cudaEvent_t>(ev), st);
+    if (e != cudaSuccess) { hca::set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
+    return HCA_OK;
+}
+
+size_t lightning_index_topk_workspace_size(int32_t B, int64_t Nc_cap, int32_t k) {
+    return topk_select_workspace_size(B, Nc_cap, k);
+}
+
+int lightning_index_topk(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
+                         const uint8_t* k_codes, const uint8_t* k_sf, const int32_t* q_pos,
+                         int32_t B, int64_t Nc_cap, int32_t Hi, int32_t c, int32_t m, int32_t k,
+                         float* scores, int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
+                         void* index_done, void* stream) {
+    REQUIRE(B >= 0 && Nc_cap >= 0 && m >= 1);
+    if (c != 64 && c != 128) return HCA_ERR_UNSUPPORTED;
+    if (Hi < 1 || Hi > 8) return HCA_ERR_UNSUPPORTED;
+    if (k < 1 || k > 4096) return HCA_ERR_UNSUPPORTED;
+    if (B == 0) return HCA_OK;
+    REQ_PTR(q_pos); REQ_PTR(idx); REQ_PTR(count);
+    if (Nc_cap > 0) { REQ_PTR(q_codes); REQ_PTR(q_sf); REQ_PTR(w); REQ_PTR(k_codes); REQ_PTR(k_sf); REQ_PTR(scores); }
+    const size_t need = topk_select_workspace_size(B, Nc_cap, k);
+    if (Nc_cap > 16 * 32768LL && ws_bytes < need) return HCA_ERR_WORKSPACE;
+    cudaStream_t st = as_stream(stream);
+    if (need > 0 && ws != nullptr && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0) {
+        // fused: the indexer also builds each row's key histogram
+        int rc = topk_wide_clear(ws, B, Nc_cap, st);
+        if (rc != HCA_OK) return rc;
+        int64_t stride = 0;
+        uint32_t* hist = topk_wide_hist(ws, Nc_cap, &stride);
+        rc = index_launch_hist(q_codes, q_sf, w, k_codes, k_sf, q_pos, B, Nc_cap, Hi, c, m, scores, hist, stride, st);
+        if (rc == HCA_OK) {
+            rc = record_event(index_done, st);
+            if (rc != HCA_OK) return rc;
+            return topk_wide_select(scores, q_pos, B, Nc_cap, m, k, idx, count, ws, st);
+        }
+        if (rc != HCA_ERR_UNSUPPORTED) return rc;
+    }
+    // separate calls
+    if (Nc_cap > 0) {
+        const int rc = index_launch(q_codes, q_sf, w, k_codes, k_sf, q_pos, B, 1, Nc_cap, Hi, c, m, scores, st);
+        if (rc != HCA_OK) return rc;
+    }
+    const int rc = record_event(index_done, st);
+    if (rc != HCA_OK) return rc;
+    return topk_launch(scores, q_pos, B, Nc_cap, m, k, idx, count, ws, ws_bytes, st);
 }
 
 size_t compressed_attn_decode_workspace_size(int32_t B, int32_t H, hca_kv_layout layout, int32_t max_comp, int32_t W) {

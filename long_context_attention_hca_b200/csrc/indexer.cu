@@ -409,12 +409,23 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
 
 // QG queries per CTA (N = 16 QG accumulator columns), NBD accumulator buffers,
 // KS key stages, EG epilogue warps per TMEM lane quarter.
+// Larger key = larger score; +0 and -0 map to the same key (the top-k's order).
+__device__ __forceinline__ uint32_t score_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    if ((u << 1) == 0u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// hist (optional, one query per CTA): the query row's 2048-bin histogram of the
+// top 11 bits of each eligible score's key, hist + row * hist_stride (u32),
+// accumulated in shared memory and added with global atomics at the end.
 template <int QG, int NBD, int KS, int EG>
 __global__ void __launch_bounds__(64 + 128 * EG)
 index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
                 const uint8_t* __restrict__ q_codes, const uint8_t* __restrict__ q_sf,
                 const float* __restrict__ w, const int32_t* __restrict__ q_pos,
-                int Tq, int64_t Nc_cap, int m, int64_t chunk, float* __restrict__ scores) {
+                int Tq, int64_t Nc_cap, int m, int64_t chunk, float* __restrict__ scores,
+                uint32_t* __restrict__ hist, int64_t hist_stride) {
     constexpr int N = 16 * QG;
     constexpr uint32_t NCOLS = (N * NBD) <= 32 ? 32 : (N * NBD <= 64 ? 64 : (N * NBD <= 128 ? 128 : (N * NBD <= 256 ? 256 : 512)));
     constexpr uint32_t IDESC = (1u << 4) | (5u << 7) | (5u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
@@ -423,9 +434,11 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sB = smem + KS * STAGE_BYTES;              // N rows x 128 B (query operand)
+    uint32_t* sh_hist = reinterpret_cast<uint32_t*>(sB + N * 128);   // 2048 bins when hist != nullptr
     __shared__ __align__(8) uint64_t bar_full[KS], bar_empty[KS], bar_accf[NBD], bar_acce[NBD], bar_drain;
     __shared__ uint32_t tmem_slot;
     __shared__ int s_eq[QG][16];                        // (uq - 127) - 127 per (query, block*4+head)
+    __shared__ int s_klo[QG][4], s_khi[QG][4];          // key exponent range of the fast path per block
     __shared__ float s_w[QG][4];
     __shared__ int64_t s_elig[QG];
     __shared__ int s_abort;
@@ -437,8 +450,10 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
     const int64_t s_end = min(s_begin + chunk, Nc_cap);
 
     if (tid == 0) {
-        for (int i = 0; i < KS; ++i) { mbar_init(smem_u32(&bar_full[i]), 1); mbar_init(smem_u32(&bar_empty[i]), EPI); }
-        for (int i = 0; i < NBD; ++i) { mbar_init(smem_u32(&bar_accf[i]), 1); mbar_init(smem_u32(&bar_acce[i]), EPI); }
+        // warps that release a tile: all epilogue warps, or (one query per CTA) the 4 of the tile's group
+        constexpr int REL = QG == 1 ? 4 : EPI;
+        for (int i = 0; i < KS; ++i) { mbar_init(smem_u32(&bar_full[i]), 1); mbar_init(smem_u32(&bar_empty[i]), REL); }
+        for (int i = 0; i < NBD; ++i) { mbar_init(smem_u32(&bar_accf[i]), 1); mbar_init(smem_u32(&bar_acce[i]), REL); }
         mbar_init(smem_u32(&bar_drain), 1);
         s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -447,6 +462,8 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(smem_u32(&tmem_slot)), "r"(NCOLS) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
+    if (QG == 1 && hist)
+        for (int x = tid; x < 2048; x += blockDim.x) sh_hist[x] = 0u;
     // the loads write only the 8 data bytes of each 16-byte slot: zero the padding once
     for (int x = tid; x < KS * (CODE_BYTES / 16); x += blockDim.x) {
         const int st = x / (CODE_BYTES / 16), o = x % (CODE_BYTES / 16);
@@ -465,6 +482,19 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
         s_eq[q][x & 15] = static_cast<int>(__ldg(q_sf + ((qrow0 + q) * 4 + h) * 4 + blk)) - 254;
     }
     for (int x = tid; x < QG * 4; x += blockDim.x) s_w[x >> 2][x & 3] = __ldg(w + (qrow0 + (x >> 2)) * 4 + (x & 3));
+    for (int x = tid; x < QG * 4; x += blockDim.x) {
+        // fast path of a (query, block): every head's 2^(eq + ek) is a normal float and
+        // |block dot| * 2^(eq + ek) < 2^127, i.e. eq + ek in [-126, 116] for all heads
+        const int q = x >> 2, blk = x & 3;
+        int mn = 1 << 20, mx = -(1 << 20);
+        for (int h = 0; h < 4; ++h) {
+            const int e = static_cast<int>(__ldg(q_sf + ((qrow0 + q) * 4 + h) * 4 + blk)) - 254;
+            mn = min(mn, e);
+            mx = max(mx, e);
+        }
+        s_klo[q][blk] = -126 - mn;
+        s_khi[q][blk] = 116 - mx;
+    }
     if (tid < QG) {
         int64_t e = (static_cast<int64_t>(q_pos[qrow0 + tid]) + 1) / m;
         s_elig[tid] = e < 0 ? 0 : (e > Nc_cap ? Nc_cap : e);
@@ -528,18 +558,26 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
         // ---------------------------------------------------------------- epilogue
         // items i = (tile t, j-th query of this warp), in order; the TMEM load of item
         // i + 1 is in flight while item i is scored
-        constexpr int QPW = QG / EG;                   // queries per epilogue warp
+        // one query per CTA: the EG warps of a lane quarter take alternate tiles; else
+        // they split the queries of every tile
+        constexpr int QPW = QG == 1 ? 1 : QG / EG;     // queries per epilogue warp and tile
+        constexpr int TS = QG == 1 ? EG : 1;           // tile stride
+        constexpr int QE = QG == 1 ? 1 : EG;           // query stride
         const int quarter = warp & 3;                  // TMEM lanes 32 quarter .. +31
-        const int eg = (warp - 2) >> 2;                // this warp's share of the queries
+        const int eg = (warp - 2) >> 2;                // this warp's share of the tiles or queries
+        const int t0 = QG == 1 ? eg : 0, q0 = QG == 1 ? 0 : eg;
         const int row = quarter * 32 + lane;           // key row of the tile
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-        const int n_items = n_tiles * QPW;
-        int eq1[16];                                   // exponents of the only query (QG == 1)
+        const int n_mine = n_tiles > t0 ? (n_tiles - t0 + TS - 1) / TS : 0;
+        const int n_items = n_mine * QPW;
+        int eq1[16], klo1[4], khi1[4];                 // the only query's exponents (QG == 1)
 #pragma unroll
         for (int j = 0; j < 16; ++j) eq1[j] = s_eq[0][j];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) { klo1[j] = s_klo[0][j]; khi1[j] = s_khi[0][j]; }
         uint32_t rn[16];
         auto tmem_ld = [&](int i) {
-            const int t = i / QPW, q = eg + EG * (i % QPW);
+            const int t = t0 + TS * (i / QPW), q = q0 + QE * (i % QPW);
             asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
                          : "=r"(rn[0]), "=r"(rn[1]), "=r"(rn[2]), "=r"(rn[3]), "=r"(rn[4]), "=r"(rn[5]), "=r"(rn[6]), "=r"(rn[7]),
                            "=r"(rn[8]), "=r"(rn[9]), "=r"(rn[10]), "=r"(rn[11]), "=r"(rn[12]), "=r"(rn[13]), "=r"(rn[14]), "=r"(rn[15])
@@ -554,11 +592,11 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
         };
         bool ok = true;
         if (n_items > 0) {
-            if (tile_ready(0)) tmem_ld(0); else ok = false;
+            if (tile_ready(t0)) tmem_ld(0); else ok = false;
         }
         uint32_t sw = 0;
         for (int i = 0; i < n_items && ok; ++i) {
-            const int t = i / QPW, j = i % QPW, q = eg + EG * j;
+            const int t = t0 + TS * (i / QPW), j = i % QPW, q = q0 + QE * j;
             const int st = t % KS, nb = t % NBD;
             asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
             uint32_t r[16];
@@ -573,52 +611,70 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
                 if (lane == 0) { mbar_arrive(smem_u32(&bar_acce[nb])); mbar_arrive(smem_u32(&bar_empty[st])); }
             }
             if (i + 1 < n_items) {
-                if ((i + 1) % QPW == 0 && !tile_ready(t + 1)) { ok = false; }
+                if ((i + 1) % QPW == 0 && !tile_ready(t + TS)) { ok = false; }
                 else tmem_ld(i + 1);
             }
             int eq[16];
 #pragma unroll
             for (int z = 0; z < 16; ++z) eq[z] = QG == 1 ? eq1[z] : s_eq[q][z];
-            // fast path: every exponent eq + ek in [-126, 127], so 2^(eq+ek) is a
-            // normal float whose bits are (eq + ek + 127) << 23
-            bool normal = true;
+            int ek[4];
+            bool fast = true;
 #pragma unroll
-            for (int z = 0; z < 16; ++z) {
-                const int x = eq[z] + static_cast<int>((sw >> (8 * (z >> 2))) & 0xFFu);
-                normal &= (x >= -126) & (x <= 127);
+            for (int blk = 0; blk < 4; ++blk) {
+                ek[blk] = static_cast<int>((sw >> (8 * blk)) & 0xFFu);
+                const int lo = QG == 1 ? klo1[blk] : s_klo[q][blk], hi = QG == 1 ? khi1[blk] : s_khi[q][blk];
+                fast &= (ek[blk] >= lo) & (ek[blk] <= hi);
             }
-            float tv[16];
-            if (__all_sync(0xffffffffu, normal)) {
+            float dot[4];
+            if (__all_sync(0xffffffffu, fast)) {
+                // every term is an exact product (a normal power of two, no overflow), so
+                // fma(D, 2^e, acc) rounds exactly as the ordered sum acc + D * 2^e does
 #pragma unroll
-                for (int z = 0; z < 16; ++z) {
-                    const uint32_t bits = static_cast<uint32_t>(eq[z] + 127 + static_cast<int>((sw >> (8 * (z >> 2))) & 0xFFu)) << 23;
-                    tv[z] = __fmul_rn(__uint_as_float(r[z]), __uint_as_float(bits));
+                for (int h = 0; h < 4; ++h) {
+#pragma unroll
+                    for (int blk = 0; blk < 4; ++blk) {
+                        const int z = blk * 4 + h;
+                        const float s2 = __uint_as_float(static_cast<uint32_t>(eq[z] + 127 + ek[blk]) << 23);
+                        dot[h] = blk == 0 ? __fmul_rn(__uint_as_float(r[z]), s2)
+                                          : __fmaf_rn(__uint_as_float(r[z]), s2, dot[h]);
+                    }
                 }
             } else {
 #pragma unroll
-                for (int z = 0; z < 16; ++z)
-                    tv[z] = scale_pow2(__uint_as_float(r[z]), eq[z] + static_cast<int>((sw >> (8 * (z >> 2))) & 0xFFu));
+                for (int h = 0; h < 4; ++h) {
+                    // column blk*4 + h: ordered block sum ((t0 + t1) + t2) + t3, each term rounded once
+                    float a = scale_pow2(__uint_as_float(r[h]), eq[h] + ek[0]);
+#pragma unroll
+                    for (int blk = 1; blk < 4; ++blk)
+                        a = __fadd_rn(a, scale_pow2(__uint_as_float(r[blk * 4 + h]), eq[blk * 4 + h] + ek[blk]));
+                    dot[h] = a;
+                }
             }
             float sc = 0.0f;
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                // column blk*4 + h: ordered block sum ((t0 + t1) + t2) + t3
-                const float dot = __fadd_rn(__fadd_rn(__fadd_rn(tv[h], tv[4 + h]), tv[8 + h]), tv[12 + h]);
-                sc = __fadd_rn(sc, __fmul_rn(s_w[q][h], dot > 0.0f ? dot : 0.0f));
-            }
+            for (int h = 0; h < 4; ++h) sc = __fadd_rn(sc, __fmul_rn(s_w[q][h], dot[h] > 0.0f ? dot[h] : 0.0f));
             const int64_t e = s_begin + static_cast<int64_t>(t) * TILE + row;
-            if (e < s_end && e < s_elig[q])
+            if (e < s_end && e < s_elig[q]) {
                 scores[static_cast<size_t>(qrow0 + q) * Nc_cap + e] = ok ? sc : __int_as_float(0x7fc00000);
+                if (QG == 1 && hist) atomicAdd(&sh_hist[score_key(sc) >> 21], 1u);
+            }
         }
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
         if (!ok) {
             // scores of the tiles this warp did not reach: NaN
-            for (int q = eg; q < QG; q += EG)
+            for (int q = q0; q < QG; q += QE)
                 for (int64_t e = s_begin + row; e < s_live; e += TILE)
                     if (e < s_elig[q]) scores[static_cast<size_t>(qrow0 + q) * Nc_cap + e] = __int_as_float(0x7fc00000);
         }
     }
     __syncthreads();
+    if (QG == 1 && hist) {
+        uint32_t* gh = hist + qrow0 * hist_stride;
+        for (int x = tid; x < 2048; x += blockDim.x) {
+            const uint32_t v = sh_hist[x];
+            if (v) atomicAdd(&gh[x], v);
+        }
+    }
     if (warp == 1) {
         // no MMA may still write TMEM when it is released
         if (lane == 0) wait_bar(smem_u32(&bar_drain), 0, &s_abort);
@@ -680,7 +736,7 @@ bool make_maps(const uint8_t* k_codes, const uint8_t* k_sf, int64_t rows, int64_
 template <int QG, int NBD, int KS, int EG>
 int launch_tc(const uint8_t* q_codes, const uint8_t* q_sf, const float* w, const uint8_t* k_codes,
               const uint8_t* k_sf, const int32_t* q_pos, int64_t rows, int B, int Tq, int64_t Nc_cap, int m,
-              float* scores, cudaStream_t st, int64_t want_ctas) {
+              float* scores, cudaStream_t st, int64_t want_ctas, uint32_t* hist = nullptr, int64_t hist_stride = 0) {
     CUtensorMap tm_codes, tm_scales;
     if (!make_maps(k_codes, k_sf, static_cast<int64_t>(B) * Nc_cap, Nc_cap, &tm_codes, &tm_scales)) return HCA_ERR_UNSUPPORTED;
     const int64_t groups = rows / QG;
@@ -688,7 +744,7 @@ int launch_tc(const uint8_t* q_codes, const uint8_t* q_sf, const float* w, const
     chunk = ceil_div(chunk, TILE) * TILE;
     if (chunk < TILE) chunk = TILE;
     if (ceil_div(Nc_cap, chunk) > 65535) chunk = ceil_div(ceil_div(Nc_cap, 65535), TILE) * TILE;
-    size_t smem = static_cast<size_t>(KS) * STAGE_BYTES + 16 * QG * 128 + 1024;
+    size_t smem = static_cast<size_t>(KS) * STAGE_BYTES + 16 * QG * 128 + 1024 + (hist ? 2048 * 4 : 0);
     // a CTA that takes all 512 TMEM columns must be alone on its SM: ask for
     // more than half of the SM's shared memory
     if (16 * QG * NBD >= 512 && smem < 120 * 1024) smem = 120 * 1024;
@@ -696,7 +752,8 @@ int launch_tc(const uint8_t* q_codes, const uint8_t* q_sf, const float* w, const
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
     const dim3 grid(static_cast<unsigned>(groups), static_cast<unsigned>(ceil_div(Nc_cap, chunk)));
-    kern<<<grid, 64 + 128 * EG, smem, st>>>(tm_codes, tm_scales, q_codes, q_sf, w, q_pos, Tq, Nc_cap, m, chunk, scores);
+    kern<<<grid, 64 + 128 * EG, smem, st>>>(tm_codes, tm_scales, q_codes, q_sf, w, q_pos, Tq, Nc_cap, m, chunk, scores,
+                                            hist, hist_stride);
     HCA_CHECK_LAUNCH();
     return HCA_OK;
 }
@@ -717,6 +774,18 @@ int index_take_device_error() {
 
 namespace {
 }  // namespace
+
+// Decode index scores plus each row's key histogram (see index_tc_kernel); only
+// the tensor-map path (c = 128, Hi = 4, Tq = 1) supports it.  HCA_ERR_UNSUPPORTED:
+// nothing was launched.
+int index_launch_hist(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
+                      const uint8_t* k_codes, const uint8_t* k_sf, const int32_t* q_pos,
+                      int B, int64_t Nc_cap, int Hi, int c, int m, float* scores, uint32_t* hist,
+                      int64_t hist_stride, cudaStream_t st) {
+    if (c != 128 || Hi != 4 || B <= 0 || Nc_cap <= 0) return HCA_ERR_UNSUPPORTED;
+    return itc::launch_tc<1, 4, 5, 2>(q_codes, q_sf, w, k_codes, k_sf, q_pos, B, B, 1, Nc_cap, m, scores, st,
+                                      2LL * sm_count(), hist, hist_stride);
+}
 
 int index_launch(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
                  const uint8_t* k_codes, const uint8_t* k_sf, const int32_t* q_pos,
@@ -745,8 +814,8 @@ int index_launch(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
             rc = itc::launch_tc<16, 2, 4, 2>(q_codes, q_sf, w, k_codes, k_sf, q_pos, rows, B, Tq, Nc_cap, m, scores, st,
                                              2LL * sm_count());
         else
-            rc = itc::launch_tc<1, 4, 4, 1>(q_codes, q_sf, w, k_codes, k_sf, q_pos, rows, B, Tq, Nc_cap, m, scores, st,
-                                            3LL * sm_count());
+            rc = itc::launch_tc<1, 4, 5, 2>(q_codes, q_sf, w, k_codes, k_sf, q_pos, rows, B, Tq, Nc_cap, m, scores, st,
+                                            2LL * sm_count());
         if (rc != HCA_ERR_UNSUPPORTED) return rc;
         // unaligned key buffers: CUDA-core tensor path below
     }

@@ -715,25 +715,49 @@ size_t topk_wide_ws_bytes(int R, int64_t Nc_cap) {
     return static_cast<size_t>(R) * wide::layout(Nc_cap).row_bytes;
 }
 
-int topk_wide_launch(const float* scores, const int32_t* q_pos, int R, int64_t Nc_cap, int m, int k,
-                     int32_t* idx, int32_t* count, void* ws, cudaStream_t st) {
+// clear each row's histogram, header and bitmaps
+int topk_wide_clear(void* ws, int R, int64_t Nc_cap, cudaStream_t st) {
     const wide::Layout L = wide::layout(Nc_cap);
-    uint8_t* w = static_cast<uint8_t*>(ws);
-    // clear each row's histogram, header and bitmaps
-    cudaError_t e = cudaMemset2DAsync(w, L.row_bytes, 0, L.clear_bytes, static_cast<size_t>(R), st);
+    cudaError_t e = cudaMemset2DAsync(ws, L.row_bytes, 0, L.clear_bytes, static_cast<size_t>(R), st);
     if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
+    return HCA_OK;
+}
+
+// row r's key histogram (u32[2048]) starts at ws + r * stride u32 words
+uint32_t* topk_wide_hist(void* ws, int64_t Nc_cap, int64_t* stride_u32) {
+    *stride_u32 = static_cast<int64_t>(wide::layout(Nc_cap).row_bytes / 4);
+    return static_cast<uint32_t*>(ws);
+}
+
+static int64_t wide_chunk(int R, int64_t Nc_cap) {
     const int64_t ctas_per_row = std::max<int64_t>(1, ceil_div(2LL * sm_count(), R));
     int64_t chunk = ceil_div(Nc_cap, ctas_per_row);
     chunk = std::max<int64_t>(256, ceil_div(chunk, 256) * 256);       // whole bitmap words per warp
-    chunk = std::min<int64_t>(chunk, static_cast<int64_t>(wide::kMaxIt) * wide::kThreads);
+    return std::min<int64_t>(chunk, static_cast<int64_t>(wide::kMaxIt) * wide::kThreads);
+}
+
+// mark + resolve, given the rows' histograms (by hist_kernel or by the indexer)
+int topk_wide_select(const float* scores, const int32_t* q_pos, int R, int64_t Nc_cap, int m, int k,
+                     int32_t* idx, int32_t* count, void* ws, cudaStream_t st) {
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    const int64_t chunk = wide_chunk(R, Nc_cap);
     const dim3 grid(static_cast<unsigned>(ceil_div(Nc_cap, chunk)), static_cast<unsigned>(R));
-    wide::hist_kernel<<<grid, wide::kThreads, 0, st>>>(scores, q_pos, Nc_cap, m, chunk, w);
-    HCA_CHECK_LAUNCH();
     wide::mark_kernel<<<grid, wide::kThreads, 0, st>>>(scores, q_pos, Nc_cap, m, k, chunk, w);
     HCA_CHECK_LAUNCH();
     wide::resolve_kernel<<<R, wide::kResolveThreads, 0, st>>>(q_pos, Nc_cap, m, k, w, idx, count);
     HCA_CHECK_LAUNCH();
     return HCA_OK;
+}
+
+int topk_wide_launch(const float* scores, const int32_t* q_pos, int R, int64_t Nc_cap, int m, int k,
+                     int32_t* idx, int32_t* count, void* ws, cudaStream_t st) {
+    const int rc = topk_wide_clear(ws, R, Nc_cap, st);
+    if (rc != HCA_OK) return rc;
+    const int64_t chunk = wide_chunk(R, Nc_cap);
+    const dim3 grid(static_cast<unsigned>(ceil_div(Nc_cap, chunk)), static_cast<unsigned>(R));
+    wide::hist_kernel<<<grid, wide::kThreads, 0, st>>>(scores, q_pos, Nc_cap, m, chunk, static_cast<uint8_t*>(ws));
+    HCA_CHECK_LAUNCH();
+    return topk_wide_select(scores, q_pos, R, Nc_cap, m, k, idx, count, ws, st);
 }
 
 int topk_launch(const float* scores, const int32_t* q_pos, int R, int64_t Nc_cap, int m, int k,

@@ -19,8 +19,8 @@ from typing import List, Optional
 import torch
 
 from . import (KVCache, compressed_attn_decode, compressed_attn_prefill, csa_compress, decode_workspace_size,
-               hca_compress, lightning_index, topk_select, topk_workspace_size, set_launch_budget,
-               BUDGET_DENSE_DECODE)
+               hca_compress, lightning_index, lightning_index_topk, topk_select, topk_workspace_size,
+               set_launch_budget, BUDGET_DENSE_DECODE)
 
 CSA_RATIO = 4
 HCA_RATIO = 128
@@ -75,7 +75,7 @@ class DecodeRunner:
     hold when the indexer drains."""
 
     def __init__(self, layers: List[DecodeLayer], B: int, H: int, k: int, pos: int, softmax_scale: float,
-                 device="cuda", schedule: str = "after_index", dense_budget: int = 0):
+                 device="cuda", schedule: str = "after_index", dense_budget: int = 0, fused_select: bool = True):
         """schedule: "after_index" -- an HCA launch waits for the indexer queued
         before it; "hca_first" -- all HCA launches are queued first and start at
         once, with dense_budget (if > 0) capping their CTAs so that the CSA
@@ -93,7 +93,8 @@ class DecodeRunner:
         self.q_pos = torch.full((B, 1), pos, dtype=torch.int32, device=dev)
         self.out = [torch.empty((B, H, d), dtype=torch.bfloat16, device=dev) for _ in layers]
         self.n_dense = {}
-        self.scores, self.idx, self.count, self.ws, self.topk_ws = {}, {}, {}, {}, {}
+        self.scores, self.idx, self.count, self.ws, self.topk_ws, self.fused_select = {}, {}, {}, {}, {}, {}
+        self.index_done = {}
         W = layers[0].window.shape[1]
         for li, L in enumerate(layers):
             if L.ratio == CSA_RATIO:
@@ -102,6 +103,11 @@ class DecodeRunner:
                 self.count[li] = torch.empty((B,), dtype=torch.int32, device=dev)
                 self.topk_ws[li] = torch.empty(max(topk_workspace_size(B, L.n_entries, k), 16), dtype=torch.uint8,
                                                device=dev)
+                # the fused index + top-k call pays off when top-k takes the histogram path
+                self.fused_select[li] = fused_select and topk_workspace_size(B, L.n_entries, k) > 0
+                # recorded inside the fused call once the scores exist (created here, outside any capture)
+                self.index_done[li] = torch.cuda.Event()
+                self.index_done[li].record(torch.cuda.current_stream(dev))
                 mc = min(k, L.n_entries)
             else:
                 self.n_dense[li] = torch.full((B,), L.n_entries, dtype=torch.int32, device=dev)
@@ -122,7 +128,9 @@ class DecodeRunner:
             split = decode_workspace_size(self.B, self.H, L.cache.layout, mc, L.window.shape[1]) > 0
             n += 1 + int(split)
             if L.ratio == CSA_RATIO:
-                n += 1 + (3 if topk_workspace_size(self.B, L.n_entries, self.k) > 0 else 1)
+                wide = topk_workspace_size(self.B, L.n_entries, self.k) > 0
+                # indexer + (histogram,) mark, resolve on the histogram path; else the cluster kernel
+                n += 1 + ((2 if self.fused_select[li] else 3) if wide else 1)
         return n
 
     def step(self, q: List[torch.Tensor], iq: List[Optional[tuple]], events: Optional[dict] = None):
@@ -156,13 +164,21 @@ class DecodeRunner:
             if L.ratio == CSA_RATIO:
                 with torch.cuda.stream(self.side):
                     qc, qs, w = iq[li]
-                    timed("indexer", li, lambda: lightning_index(qc, qs, w, L.k_codes, L.k_sf, self.q_pos, CSA_RATIO,
-                                                                 scores=self.scores[li]))
-                    after_index = torch.cuda.Event()
-                    after_index.record(self.side)
-                    timed("topk", li, lambda: topk_select(self.scores[li].view(self.B, -1), self.q_pos.view(-1),
-                                                          CSA_RATIO, self.k, idx=self.idx[li], count=self.count[li],
-                                                          ws=self.topk_ws[li]))
+                    if self.fused_select[li]:
+                        # indexer (with the top-k's key histogram) + top-k passes in one call
+                        timed("index_topk", li, lambda: lightning_index_topk(
+                            qc, qs, w, L.k_codes, L.k_sf, self.q_pos.view(-1), CSA_RATIO, self.k,
+                            scores=self.scores[li], idx=self.idx[li], count=self.count[li], ws=self.topk_ws[li],
+                            index_done=self.index_done[li], stream=self.side))
+                        after_index = self.index_done[li]
+                    else:
+                        timed("indexer", li, lambda: lightning_index(qc, qs, w, L.k_codes, L.k_sf, self.q_pos,
+                                                                     CSA_RATIO, scores=self.scores[li]))
+                        after_index = torch.cuda.Event()
+                        after_index.record(self.side)
+                        timed("topk", li, lambda: topk_select(self.scores[li].view(self.B, -1), self.q_pos.view(-1),
+                                                              CSA_RATIO, self.k, idx=self.idx[li],
+                                                              count=self.count[li], ws=self.topk_ws[li]))
                     timed("csa_attn", li, lambda: compressed_attn_decode(
                         q[li], L.cache, self.count[li], min(self.k, L.n_entries), L.window, self.scale,
                         idx=self.idx[li], out=self.out[li], ws=self.ws[li]))

@@ -199,6 +199,28 @@ def test_topk_crowded_threshold_bin(R, Nc, k):
     assert np.array_equal(host(idx), wi)
 
 
+@pytest.mark.parametrize("Nc,k,zero_w", [(20000, 512, False), (5000, 64, False), (70001, 1024, False),
+                                         (20000, 777, True)])
+def test_lightning_index_topk_fused(Nc, k, zero_w):
+    """The fused decode call (indexer building the top-k histogram) equals the
+    oracle's scores and selection; Nc = 5000 takes the cluster top-k, Nc = 70001
+    (not a multiple of 4) the separate kernels; zero weights make every score
+    0, so the selection is all ties (lowest indices)."""
+    B, Hi, c, m = 3, 4, 128, 4
+    qc, qs, w, kc, ks = _fp4_inputs(B, 1, Hi, c, Nc, Nc + k)
+    if zero_w:
+        w.zero_()
+    pos = torch.tensor([4 * Nc - 1, 4 * 1234 + 1, 4 * 600], dtype=torch.int32, device=DEV)
+    s, idx, cnt = hca.lightning_index_topk(qc, qs, w, kc, ks, pos, m, k)
+    torch.cuda.synchronize()
+    want, n_inexact = oracle.index_scores(host(qc), host(qs), host(w), host(kc), host(ks), host(pos).reshape(B, 1), m)
+    assert n_inexact == 0
+    assert np.array_equal(host(s).view(np.uint32), want.view(np.uint32))
+    wi, wc = oracle.topk(want.reshape(B, Nc), host(pos), m, k)
+    assert np.array_equal(host(cnt), wc)
+    assert np.array_equal(host(idx), wi)
+
+
 def test_topk_from_index_scores_pipeline():
     """Index scores straight into top-k: the sets must match the oracle's."""
     B, Hi, c, Nc, m, k = 3, 4, 128, 20000, 4, 512
