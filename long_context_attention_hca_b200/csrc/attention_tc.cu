@@ -282,6 +282,64 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) { tmem_alloc(smem_u32(&tmem_base_slot), TMEM_COLS); tmem_relinquish(); }
+    // ---- producer state (warps 4-19), declared here so that the first tile's
+    // gathers are in flight while every thread loads Q
+    const bool producer = warp >= NSOFT && warp < NSOFT + NPROD;
+    const int pw = warp - NSOFT;                   // 0..15
+    const int c16 = (pw & 7) * 4 + (lane >> 3);    // this thread's 16-dim unit (same for all its keys)
+    const int row0 = (pw >> 3) * 32 + (lane & 7);  // its rows: row0 + 8 j
+    const int d0 = c16 * 16;
+    const int dn = D - 64;
+    int32_t ent_next[ROWS_PER_THREAD];
+    auto fetch_ent = [&](int i, int32_t (&e)[ROWS_PER_THREAD]) {
+#pragma unroll
+        for (int j = 0; j < ROWS_PER_THREAD; ++j) {
+            const int slot = (t_begin + i) * TK + row0 + 8 * j;
+            e[j] = (i < n_tiles && slot < uk.n_c) ? (uk.ent ? uk.ent[slot] : slot) : -1;
+        }
+    };
+    uint32_t raw[ROWS_PER_THREAD][8];
+    float sc[ROWS_PER_THREAD];
+    // raw loads of tile i (registers only: no buffer needed yet)
+    auto load_tile = [&](int i, const int32_t (&ent)[ROWS_PER_THREAD]) {
+        const int slot0 = (t_begin + i) * TK;
+#pragma unroll
+        for (int j = 0; j < ROWS_PER_THREAD; ++j) {
+            const int r = row0 + 8 * j;
+            const int slot = slot0 + r;
+            sc[j] = 0.0f;
+#pragma unroll
+            for (int z = 0; z < 8; ++z) raw[j][z] = 0;
+            if (i >= n_tiles) continue;
+            if (slot < uk.n_c) {
+                const int64_t e = ent[j];
+                if (e >= 0 && e < p.cap) {
+                    const int64_t er = uk.kv_row0 + e;
+                    if (d0 < dn) {
+                        const uint4 cv = __ldg(reinterpret_cast<const uint4*>(p.codes + er * dn + d0));
+                        raw[j][0] = cv.x; raw[j][1] = cv.y; raw[j][2] = cv.z; raw[j][3] = cv.w;
+                        sc[j] = __ldg(p.scales + er * (dn / 64) + d0 / 64);
+                    } else {
+                        const uint4* rp = reinterpret_cast<const uint4*>(p.rope + er * 64 + (d0 - dn));
+                        const uint4 a = __ldg(rp), bq = __ldg(rp + 1);
+                        raw[j][0] = a.x; raw[j][1] = a.y; raw[j][2] = a.z; raw[j][3] = a.w;
+                        raw[j][4] = bq.x; raw[j][5] = bq.y; raw[j][6] = bq.z; raw[j][7] = bq.w;
+                    }
+                }
+            } else if (slot < n_tot) {
+                const uint4* rp = reinterpret_cast<const uint4*>(uk.wrow + static_cast<size_t>(slot - uk.n_c) * D + d0);
+                const uint4 a = __ldg(rp), bq = __ldg(rp + 1);
+                raw[j][0] = a.x; raw[j][1] = a.y; raw[j][2] = a.z; raw[j][3] = a.w;
+                raw[j][4] = bq.x; raw[j][5] = bq.y; raw[j][6] = bq.z; raw[j][7] = bq.w;
+            }
+        }
+    };
+    if (producer) {
+        int32_t ent0[ROWS_PER_THREAD];
+        fetch_ent(0, ent0);
+        load_tile(0, ent0);
+        fetch_ent(1, ent_next);
+    }
     {
         // Q -> fp16, K-major SW128: column block cb = dims 64cb.., row = head; all of
         // a thread's loads are issued before the first conversion
@@ -335,62 +393,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
         }
     } else if (warp >= NSOFT) {
         // ------------------------------------------------------------ producers
-        const int pw = warp - NSOFT;                   // 0..15
-        const int pt = pw * 32 + lane;                 // 0..511
-        const int c16 = (pw & 7) * 4 + (lane >> 3);    // this thread's 16-dim unit (same for all its keys)
-        const int row0 = (pw >> 3) * 32 + (lane & 7);  // its rows: row0 + 8 j
-        const int d0 = c16 * 16;
-        const int dn = D - 64;
-        int32_t ent_next[ROWS_PER_THREAD];
-        auto fetch_ent = [&](int i, int32_t (&e)[ROWS_PER_THREAD]) {
-#pragma unroll
-            for (int j = 0; j < ROWS_PER_THREAD; ++j) {
-                const int slot = (t_begin + i) * TK + row0 + 8 * j;
-                e[j] = (i < n_tiles && slot < uk.n_c) ? (uk.ent ? uk.ent[slot] : slot) : -1;
-            }
-        };
-        uint32_t raw[ROWS_PER_THREAD][8];
-        float sc[ROWS_PER_THREAD];
-        // raw loads of tile i (registers only: no buffer needed yet)
-        auto load_tile = [&](int i, const int32_t (&ent)[ROWS_PER_THREAD]) {
-            const int slot0 = (t_begin + i) * TK;
-#pragma unroll
-            for (int j = 0; j < ROWS_PER_THREAD; ++j) {
-                const int r = row0 + 8 * j;
-                const int slot = slot0 + r;
-                sc[j] = 0.0f;
-#pragma unroll
-                for (int z = 0; z < 8; ++z) raw[j][z] = 0;
-                if (i >= n_tiles) continue;
-                if (slot < uk.n_c) {
-                    const int64_t e = ent[j];
-                    if (e >= 0 && e < p.cap) {
-                        const int64_t er = uk.kv_row0 + e;
-                        if (d0 < dn) {
-                            const uint4 cv = __ldg(reinterpret_cast<const uint4*>(p.codes + er * dn + d0));
-                            raw[j][0] = cv.x; raw[j][1] = cv.y; raw[j][2] = cv.z; raw[j][3] = cv.w;
-                            sc[j] = __ldg(p.scales + er * (dn / 64) + d0 / 64);
-                        } else {
-                            const uint4* rp = reinterpret_cast<const uint4*>(p.rope + er * 64 + (d0 - dn));
-                            const uint4 a = __ldg(rp), bq = __ldg(rp + 1);
-                            raw[j][0] = a.x; raw[j][1] = a.y; raw[j][2] = a.z; raw[j][3] = a.w;
-                            raw[j][4] = bq.x; raw[j][5] = bq.y; raw[j][6] = bq.z; raw[j][7] = bq.w;
-                        }
-                    }
-                } else if (slot < n_tot) {
-                    const uint4* rp = reinterpret_cast<const uint4*>(uk.wrow + static_cast<size_t>(slot - uk.n_c) * D + d0);
-                    const uint4 a = __ldg(rp), bq = __ldg(rp + 1);
-                    raw[j][0] = a.x; raw[j][1] = a.y; raw[j][2] = a.z; raw[j][3] = a.w;
-                    raw[j][4] = bq.x; raw[j][5] = bq.y; raw[j][6] = bq.z; raw[j][7] = bq.w;
-                }
-            }
-        };
-        {
-            int32_t ent0[ROWS_PER_THREAD];
-            fetch_ent(0, ent0);
-            load_tile(0, ent0);
-            fetch_ent(1, ent_next);
-        }
         for (int i = 0; i < n_tiles; ++i) {
             const int b = i % NBUF, use = i / NBUF;
             const int slot0 = (t_begin + i) * TK;
