@@ -116,6 +116,8 @@ class DecodeRunner:
             self.ws[li] = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
         lo, hi = torch.cuda.Stream.priority_range()
         self.side = torch.cuda.Stream(device=dev, priority=hi)
+        self.copy_in = torch.cuda.Stream(device=dev)     # step_host: attention queries in
+        self.copy_out = torch.cuda.Stream(device=dev)    # step_host: outputs out
         self.kernels_per_step = self._count_kernels()
 
     def _count_kernels(self) -> int:
@@ -133,12 +135,48 @@ class DecodeRunner:
                 n += 1 + ((2 if self.fused_select[li] else 3) if wide else 1)
         return n
 
-    def step(self, q: List[torch.Tensor], iq: List[Optional[tuple]], events: Optional[dict] = None):
+    def step_host(self, h_q: List[torch.Tensor], h_iq: List[Optional[tuple]], h_out: List[torch.Tensor],
+                  d_q: List[torch.Tensor], d_iq: List[Optional[tuple]]):
+        """One decode step from pinned host memory to pinned host memory.  The
+        indexer queries (a few hundred bytes) are copied first, on the current
+        stream; the attention queries stream in on a copy stream while the
+        indexer runs, and each layer's output streams out as soon as its
+        attention is done.  d_q / d_iq are the device buffers of the inputs."""
+        main = torch.cuda.current_stream()
+        for a, b in zip(d_iq, h_iq):
+            if a is not None:
+                for x, y in zip(a, b):
+                    x.copy_(y, non_blocking=True)
+        self.copy_in.wait_stream(main)
+        q_ready = {}
+        with torch.cuda.stream(self.copy_in):
+            for li, (a, b) in enumerate(zip(d_q, h_q)):
+                a.copy_(b, non_blocking=True)
+                q_ready[li] = torch.cuda.Event()
+                q_ready[li].record(self.copy_in)
+        self.copy_out.wait_stream(main)
+
+        def on_out(li, stream):
+            done = torch.cuda.Event()
+            done.record(stream)
+            self.copy_out.wait_event(done)
+            with torch.cuda.stream(self.copy_out):
+                h_out[li].copy_(self.out[li], non_blocking=True)
+
+        self.step(d_q, d_iq, q_ready=q_ready, on_out=on_out)
+        main.wait_stream(self.copy_in)
+        main.wait_stream(self.copy_out)
+        return h_out
+
+    def step(self, q: List[torch.Tensor], iq: List[Optional[tuple]], events: Optional[dict] = None,
+             q_ready: Optional[dict] = None, on_out=None):
         """q[li]: [B][H][d] bf16; iq[li]: (codes [B][1][Hi][c/2], sf, w [B][1][Hi]) for CSA layers.
         events: if a dict is given, timing events (recorded as graph nodes
         when captured) bracket each launch: events[name] = (start, end) with
         name in indexer/topk/csa_attn/hca_attn (suffixed by the layer index
-        when there are several layers)."""
+        when there are several layers).  q_ready: optional {layer: event} that
+        an attention launch waits for (its query copy); on_out(layer, stream):
+        called after each attention launch (to stream the output out)."""
         main = torch.cuda.current_stream()
         self.side.wait_stream(main)
         multi = len(self.layers) > 2
@@ -179,15 +217,23 @@ class DecodeRunner:
                         timed("topk", li, lambda: topk_select(self.scores[li].view(self.B, -1), self.q_pos.view(-1),
                                                               CSA_RATIO, self.k, idx=self.idx[li],
                                                               count=self.count[li], ws=self.topk_ws[li]))
+                    if q_ready is not None:
+                        self.side.wait_event(q_ready[li])
                     timed("csa_attn", li, lambda: compressed_attn_decode(
                         q[li], L.cache, self.count[li], min(self.k, L.n_entries), L.window, self.scale,
                         idx=self.idx[li], out=self.out[li], ws=self.ws[li]))
+                    if on_out is not None:
+                        on_out(li, self.side)
             else:
                 if after_index is not None and self.schedule == "after_index":
                     main.wait_event(after_index)
+                if q_ready is not None:
+                    main.wait_event(q_ready[li])
                 timed("hca_attn", li, lambda: compressed_attn_decode(
                     q[li], L.cache, self.n_dense[li], L.n_entries, L.window, self.scale, out=self.out[li],
                     ws=self.ws[li]))
+                if on_out is not None:
+                    on_out(li, main)
         main.wait_stream(self.side)
         return self.out
 
@@ -224,6 +270,8 @@ class PrefillRunner:
         self.out_hca = torch.empty((Tq, H, d), dtype=torch.bfloat16, device=dev)
         lo, hi = torch.cuda.Stream.priority_range()
         self.side = torch.cuda.Stream(device=dev, priority=hi)
+        self.copy_in = torch.cuda.Stream(device=dev)     # step_host: attention queries in
+        self.copy_out = torch.cuda.Stream(device=dev)    # step_host: outputs out
         self.kernels_per_step = 6
 
     def step(self, raw_chunk, gate_chunk, raw_window, q, iq, events: Optional[dict] = None):

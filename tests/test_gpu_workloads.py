@@ -112,6 +112,41 @@ def test_tiny_decode_1k_full():
         check_decode_layer(wl, dw, runner, li, range(wl.B))
 
 
+def test_step_host_matches_device_step():
+    """DecodeRunner.step_host (pinned host in and out, copies overlapped with the
+    kernels, captured in a CUDA graph) returns exactly what step() computes."""
+    wl = inp.WORKLOADS["decode_b16_64k"]
+    dw = build_decode(wl)
+    runner = DecodeRunner(dw.layers, wl.B, wl.H, wl.k, wl.t, wl.softmax_scale)
+    ref = [o.clone() for o in runner.step(dw.q, dw.iq)]
+    torch.cuda.synchronize()
+    h_q = [t.to("cpu").pin_memory() for t in dw.q]
+    h_iq = [None if t is None else tuple(x.to("cpu").pin_memory() for x in t) for t in dw.iq]
+    h_out = [torch.zeros_like(o, device="cpu").pin_memory() for o in runner.out]
+    d_q = [torch.zeros_like(t) for t in dw.q]
+    d_iq = [None if t is None else tuple(torch.zeros_like(x) for x in t) for t in dw.iq]
+    for o in runner.out:
+        o.zero_()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        runner.step_host(h_q, h_iq, h_out, d_q, d_iq)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    for a, b in zip(h_out, ref):
+        assert torch.equal(a.view(torch.int16), b.cpu().view(torch.int16))
+    # the same step captured in a graph and replayed
+    for h in h_out:
+        h.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        runner.step_host(h_q, h_iq, h_out, d_q, d_iq)
+    g.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(h_out, ref):
+        assert torch.equal(a.view(torch.int16), b.cpu().view(torch.int16))
+
+
 def test_decode_b16_64k():
     _decode_case("decode_b16_64k", n_samples=40)
 
