@@ -467,10 +467,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
                 TMEM_LD_16X32BX2_32(lane_base + S_COL + b * TK, sr);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
+                for (int j = 0; j < 32; ++j)
                     v[j] = (kh * 32 + j < nvalid) ? __uint_as_float(sr[j]) * p.scale_log2 : -INFINITY;
-                    tmax = fmaxf(tmax, v[j]);
-                }
+                // maximum as a tree (depth 5 instead of a 32-long chain)
+                float mx[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) mx[j] = fmaxf(v[j], v[j + 16]);
+#pragma unroll
+                for (int w2 = 8; w2 >= 1; w2 >>= 1)
+#pragma unroll
+                    for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
+                tmax = mx[0];
             }
             tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
             bool resc = false;
@@ -486,13 +493,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
             }
             // probabilities in registers before any wait (fp16, the sum of the rounded values)
             uint32_t pk[16];
-            float rs = 0.0f;
+            float ps[16];
 #pragma unroll
             for (int z = 0; z < 16; ++z) {
                 pk[z] = pack_half2(ex2(v[2 * z] - m_used), ex2(v[2 * z + 1] - m_used));
                 const float2 f = unpack_half2(pk[z]);
-                rs += f.x + f.y;
+                ps[z] = f.x + f.y;
             }
+            // row sum of the rounded probabilities as a tree
+#pragma unroll
+            for (int w2 = 8; w2 >= 1; w2 >>= 1)
+#pragma unroll
+                for (int j = 0; j < w2; ++j) ps[j] += ps[j + w2];
+            float rs = ps[0];
             rs += __shfl_xor_sync(0xffffffffu, rs, 16);
             l_run += rs;
             if (lane < 16) s_alpha[h] = alpha;
