@@ -153,8 +153,8 @@ def barrier(pg):
 # `python bench.py --steps 3 --warmup 3 --no-cpu-baseline` (summaries under profiles/),
 # valid only while the kernel's source is the one captured (first 16 hex of its sha256).
 MEASURED_TRAFFIC = {
-    "hca_attn": {"bytes": 20651008, "source": "long_context_attention_hca_b200/csrc/attention_tc.cu",
-                 "sha256_16": "df18d1cd972a338d", "profile": "profiles/attn_tc_HCA_decode_b4_1m.md"},
+    "hca_attn": {"bytes": 20651776, "source": "long_context_attention_hca_b200/csrc/attention_tc.cu",
+                 "sha256_16": "6cc15c7abc43b18b", "profile": "profiles/attn_tc_HCA_decode_b4_1m.md"},
     "indexer": {"bytes": 73379328, "source": "long_context_attention_hca_b200/csrc/indexer.cu",
                 "sha256_16": "34c10bfc9059ad78", "profile": "profiles/index_tc_decode_b4_1m.md"},
 }
