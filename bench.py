@@ -263,10 +263,10 @@ def run_reference(args, wl):
         run()
     dt = (time.perf_counter() - t0) / args.steps
     value = frac / dt
-    sample = (f"one query token (sequence) of {wl.name}: FP4 index scores over {frac:.3g} of its "
+    sample = (f"one query token (sequence) of {wl.name}: FP4 index scores over {100 * frac:.3g}% of its "
               f"{(wl.t + 1) // 4} CSA entries, exact top-{wl.k}, CSA attention over {wl.k}+{wl.W} keys, "
-              f"HCA attention over {frac:.3g} of its {(wl.t + 1) // 128} entries + {wl.W} window tokens; "
-              "single-threaded C oracle (fp64 attention)")
+              f"HCA attention over {100 * frac:.3g}% of its {(wl.t + 1) // 128} entries + {wl.W} window tokens; "
+              "single-threaded C oracle (fp64 attention); value = sampled fraction / time per step")
     line = {"metric": "1M-ctx CSA+HCA decode query-tok/s", "impl": "reference", "value": value,
             "unit": "query-tok/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
