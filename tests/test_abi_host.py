@@ -96,3 +96,41 @@ def test_host_validation_without_gpu(lib):
     lib.compressed_attn_decode_workspace_size.argtypes = [I32, I32, Layout, I32, I32]
     lib.compressed_attn_decode_workspace_size.restype = ctypes.c_size_t
     assert lib.compressed_attn_decode_workspace_size(0, 64, good, 10, 128) == 0
+
+
+def test_fused_selection_and_budget_host_paths(lib):
+    """The fused decode selection validates like its two parts; the launch budget is
+    a plain process-wide value (no device access on these paths)."""
+    V, I32, I64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    lib.lightning_index_topk.argtypes = [V, V, V, V, V, V, I32, I64, I32, I32, I32, I32, V, V, V, V,
+                                         ctypes.c_size_t, V, V]
+    P = V(0x1000)
+    # unsupported c, Hi, k
+    assert lib.lightning_index_topk(P, P, P, P, P, P, 2, 100, 4, 96, 4, 8, P, P, P, None, 0, None, None) == 2
+    assert lib.lightning_index_topk(P, P, P, P, P, P, 2, 100, 9, 128, 4, 8, P, P, P, None, 0, None, None) == 2
+    assert lib.lightning_index_topk(P, P, P, P, P, P, 2, 100, 4, 128, 4, 0, P, P, P, None, 0, None, None) == 2
+    # bad m, null and misaligned pointers
+    assert lib.lightning_index_topk(P, P, P, P, P, P, 2, 100, 4, 128, 0, 8, P, P, P, None, 0, None, None) == 1
+    assert lib.lightning_index_topk(P, P, P, P, P, None, 2, 100, 4, 128, 4, 8, P, P, P, None, 0, None, None) == 1
+    assert lib.lightning_index_topk(P, P, P, V(0x1004), P, P, 2, 100, 4, 128, 4, 8, P, P, P, None, 0, None,
+                                    None) == 1
+    # a row longer than 2^19 scores needs the workspace
+    assert lib.lightning_index_topk(P, P, P, P, P, P, 2, 1 << 20, 4, 128, 4, 8, P, P, P, None, 0, None,
+                                    None) == 4
+    # no sequences: nothing to do
+    assert lib.lightning_index_topk(None, None, None, None, None, None, 0, 100, 4, 128, 4, 8, None, None, None,
+                                    None, 0, None, None) == 0
+    lib.lightning_index_topk_workspace_size.argtypes = [I32, I64, I32]
+    lib.lightning_index_topk_workspace_size.restype = ctypes.c_size_t
+    lib.topk_select_workspace_size.argtypes = [I32, I64, I32]
+    lib.topk_select_workspace_size.restype = ctypes.c_size_t
+    assert lib.lightning_index_topk_workspace_size(4, 262144, 1024) == lib.topk_select_workspace_size(4, 262144, 1024)
+
+    lib.hca_set_launch_budget.argtypes = [ctypes.c_int, ctypes.c_int]
+    lib.hca_set_launch_budget.restype = ctypes.c_int
+    prev = lib.hca_set_launch_budget(0, 60)
+    assert prev >= 0
+    assert lib.hca_set_launch_budget(0, prev) == 60
+    assert lib.hca_set_launch_budget(1, 0) >= 0
+    assert lib.hca_set_launch_budget(2, 10) == -1       # unknown op
+    assert lib.hca_set_launch_budget(0, -1) == -1       # negative budget
