@@ -149,14 +149,15 @@ def barrier(pg):
 
 
 # ------------------------------------------------------------------ measured DRAM traffic
-# dram__bytes_read.sum + dram__bytes_write.sum of one launch, from an ncu capture of
-# `python bench.py --steps 3 --warmup 3 --no-cpu-baseline` (summaries under profiles/),
-# valid only while the kernel's source is the one captured (first 16 hex of its sha256).
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch of a kernel, taken
+# with ncu on the same workload, valid only while the kernel's source file is
+# the one that was captured (first 16 hex digits of its sha256); otherwise the
+# bench reports null.
 MEASURED_TRAFFIC = {
     "hca_attn": {"bytes": 20651776, "source": "long_context_attention_hca_b200/csrc/attention_tc.cu",
-                 "sha256_16": "6cc15c7abc43b18b", "profile": "profiles/attn_tc_HCA_decode_b4_1m.md"},
+                 "sha256_16": "6cc15c7abc43b18b"},
     "indexer": {"bytes": 73379328, "source": "long_context_attention_hca_b200/csrc/indexer.cu",
-                "sha256_16": "34c10bfc9059ad78", "profile": "profiles/index_tc_decode_b4_1m.md"},
+                "sha256_16": "34c10bfc9059ad78"},
 }
 
 
@@ -171,6 +172,61 @@ def measured_traffic(kernel: str):
     except OSError:
         return None
     return e["bytes"] if h == e["sha256_16"] else None
+
+
+# ------------------------------------------------------------------ tensor peaks measured in this run
+def gemm_peaks(n=8192, reps=20):
+    """Dense GEMM throughput of this GPU in TFLOP/s, measured here with torch
+    (cuBLAS / cuBLASLt): bf16 and fp16 n x n x n matmuls and an e4m3 x e4m3
+    scaled matmul (fp32 scales, bf16 out).  A short burst after warm-up, CUDA
+    events on the current stream; the denominators of the prefill fractions."""
+    out = {}
+    dev = torch.device("cuda")
+    a = torch.randn((n, n), device=dev)
+    b = torch.randn((n, n), device=dev)
+    flop = 2.0 * n * n * n
+
+    def timeit(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return flop * reps / (e0.elapsed_time(e1) * 1e-3) / 1e12
+
+    for name, dt in (("bf16", torch.bfloat16), ("fp16", torch.float16)):
+        x, y = a.to(dt), b.to(dt)
+        out[name] = timeit(lambda: torch.matmul(x, y))
+        del x, y
+    try:
+        x8 = a.to(torch.float8_e4m3fn)
+        y8 = b.to(torch.float8_e4m3fn).t().contiguous().t()       # column-major second operand
+        one = torch.ones((), device=dev)
+        out["fp8_e4m3"] = timeit(lambda: torch._scaled_mm(x8, y8, scale_a=one, scale_b=one,
+                                                          out_dtype=torch.bfloat16))
+        del x8, y8
+    except Exception as ex:                     # reported, not hidden
+        out["fp8_e4m3"] = None
+        out["fp8_error"] = str(ex)[:200]
+    del a, b
+    torch.cuda.empty_cache()
+    out["how"] = f"torch matmul / _scaled_mm, {n}x{n}x{n}, {reps} reps after 3 warm-up, CUDA events"
+    return out
+
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 # ------------------------------------------------------------------ algorithmic bytes (decode)
@@ -190,10 +246,16 @@ def decode_bytes(wl):
         "indexer": nc * ikey + wl.Hi * (wl.c // 2 + wl.c // 32 + 4),
         "csa_attn": min(wl.k, nc) * entry + wl.W * wl.d * 2 + qo + min(wl.k, nc) * 4,
         "hca_attn": nh * entry + wl.W * wl.d * 2 + qo,
-        "topk": nc * 4 + wl.k * 4 + 8,          # scores read (L2-resident at this size), indices written
+        "topk": nc * 4 + wl.k * 4 + 8,          # scores read (they stay in L2 at this size), indices written
     }
-    per_seq["index_topk"] = per_seq["indexer"] + per_seq["topk"]
     return {k: v * wl.B for k, v in per_seq.items()}
+
+
+def step_bytes_of(algo) -> int:
+    """HBM bytes one decode step must move: the indexer's key stream plus
+    both attention calls.  The scores the top-k reads and the split-K
+    partials stay in L2 and are not counted."""
+    return algo["indexer"] + algo["csa_attn"] + algo["hca_attn"]
 
 
 # ------------------------------------------------------------------ CPU oracle timings
@@ -249,6 +311,7 @@ def run_reference(args, wl):
     """--impl reference: the CPU oracle, as it stands, on the host cores."""
     import oracle
     oracle.build()
+    threads = oracle.set_threads(cpu_cores())
     frac = 1.0
     run = oracle_decode_sample(wl, frac)
     t0 = time.perf_counter(); run(); t_one = time.perf_counter() - t0
@@ -266,13 +329,14 @@ def run_reference(args, wl):
     sample = (f"one query token (sequence) of {wl.name}: FP4 index scores over {100 * frac:.3g}% of its "
               f"{(wl.t + 1) // 4} CSA entries, exact top-{wl.k}, CSA attention over {wl.k}+{wl.W} keys, "
               f"HCA attention over {100 * frac:.3g}% of its {(wl.t + 1) // 128} entries + {wl.W} window tokens; "
-              "single-threaded C oracle (fp64 attention); value = sampled fraction / time per step")
+              f"C oracle (fp64 attention) at {threads} threads; value = sampled fraction / time per step")
     line = {"metric": "1M-ctx CSA+HCA decode query-tok/s", "impl": "reference", "value": value,
             "unit": "query-tok/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic",
             "config": {"workload": wl.name, "global_batch": wl.B, "seq_len": wl.t + 1, "parallelism": "none"},
-            "cpu_baseline": {"value": value, "unit": "query-tok/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "query-tok/s", "cores": threads, "kind": "oracle",
+                             "cpu_model": cpu_model(), "sample": sample},
             "e2e": {"value": value, "unit": "query-tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -464,7 +528,7 @@ def bench_decode(args, wl, world, rank, pg):
                 "algorithmic_bytes": algo[dominant], "avg_launch_us": solo_ms[dominant] * 1e3,
                 "timing": "the kernel alone, CUDA events, inputs rotating over replicas (L2-cold)",
                 "solo_us": {k: v * 1e3 for k, v in solo_ms.items()}}
-    step_bytes = sum(algo.values())
+    step_bytes = step_bytes_of(algo)
 
     value = world * wl.B / (ms_max * 1e-3)
     line = {
@@ -510,44 +574,201 @@ def prefill_flops(wl):
     return 4 * wl.H * wl.d * att, 2 * wl.Hi * wl.c * ind
 
 
+def prefill_attn_flops(wl):
+    """Algorithmic flops of each prefill attention launch: 4*H*d per (query, key)."""
+    p0, Tq, W = wl.t, wl.Tq, wl.W
+    csa = hca_ = 0
+    for p in range(p0, p0 + Tq):
+        win = min(W, p + 1)
+        csa += min(wl.k, (p + 1) // 4) + win
+        hca_ += (p + 1) // 128 + win
+    f = 4 * wl.H * wl.d
+    return {"csa_attn": f * csa, "hca_attn": f * hca_}
+
+
+def oracle_prefill_sample(wl, rows):
+    """Host inputs for `rows` prefill queries of the workload, drawn on the CPU
+    (seeded), and a closure running the oracle's whole path for them: index
+    scores over every eligible CSA entry, top-k, CSA attention, HCA attention.
+    The compressed entries are pooled by the oracle itself (setup, untimed);
+    only a pool of 2048 CSA entries is built, and selected indices map onto it."""
+    import numpy as np
+    import oracle
+    d, dr, g = wl.d, wl.d_rope, wl.g
+    seed = wl.seed + 2000
+    gen = lambda name, shape, std=1.0: inp.bf16_bits(inp.normal_bf16(shape, std, seed, name))
+    nh = (wl.t + wl.Tq) // 128
+    x = gen("x", (1, nh * 128, d)); gt = gen("gate", (1, nh * 128, d))
+    b128 = inp.normal_f32((128, d), 0.5, seed, "b128").numpy()
+    hc, hs, hr, _ = oracle.compress(x, gt, b128, 128, nh, dr, g)
+    x4 = gen("x4", (1, 4 * 2048, d)); g4 = gen("g4", (1, 4 * 2048, d))
+    b4 = inp.normal_f32((4, d), 0.5, seed, "b4").numpy()
+    cc, cs, cr, _ = oracle.compress(x4, g4, b4, 4, 2048, dr, g)
+    nc = (wl.t + wl.Tq) // 4
+    kc = inp.uniform_bytes((1, nc, wl.c // 2), seed, "ik").numpy()
+    ks = inp.ue8m0_scales((1, nc, wl.c // 32), seed, "iks").numpy()
+    qb = gen("q", (len(rows), wl.H, d))
+    win = gen("win", (wl.W, d))
+    qc = inp.uniform_bytes((1, len(rows), wl.Hi, wl.c // 2), seed, "iq").numpy()
+    qs = inp.ue8m0_scales((1, len(rows), wl.Hi, wl.c // 32), seed, "iqs").numpy()
+    w = inp.uniform_f32((1, len(rows), wl.Hi), seed, "iw").numpy()
+
+    def run():
+        for j, i in enumerate(rows):
+            p = wl.t + i
+            pos = np.array([[p]], np.int32)
+            sc, _ = oracle.index_scores(qc[:, j:j + 1], qs[:, j:j + 1], w[:, j:j + 1], kc, ks, pos, 4)
+            idx, cnt = oracle.topk(sc[0], pos[0], 4, wl.k)
+            ent128, w0, w1 = oracle.causal_keys(p, 128, wl.W)
+            oracle.attend(qb[j], cc[0], cs[0], cr[0], idx[0, :cnt[0]] % 2048, win, wl.softmax_scale, g)
+            oracle.attend(qb[j], hc[0], hs[0], hr[0], ent128, win, wl.softmax_scale, g)
+    return run
+
+
 def bench_prefill(args, wl, world, rank, pg):
+    import long_context_attention_hca_b200 as hca
     from hca_workloads import build_prefill
     from long_context_attention_hca_b200.pipeline import PrefillRunner
     pw = build_prefill(wl)
     runner = PrefillRunner(pw.state, wl.t, wl.Tq, wl.H, wl.k, wl.W, wl.softmax_scale)
     args_step = (pw.raw_chunk, pw.gate_chunk, pw.raw_window, pw.q, pw.iq)
-    for _ in range(max(1, args.warmup)):
-        runner.step(*args_step, events=None)
+    main = torch.cuda.current_stream()
+    # warm-up eagerly, then one CUDA graph per chunk step (the inputs, 0.3 GB of
+    # queries alone, are larger than L2)
+    s = torch.cuda.Stream()
+    s.wait_stream(main)
+    with torch.cuda.stream(s):
+        runner.step(*args_step)
+    main.wait_stream(s)
     torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
     ev = {}
-    runner.step(*args_step, events=ev)
+    with torch.cuda.graph(g):
+        runner.step(*args_step, events=ev)
+    for _ in range(max(3, args.warmup)):
+        g.replay()
     torch.cuda.synchronize()
-    kern_ms = {k: a.elapsed_time(b) for k, (a, b) in ev.items()}
     clocks = ClockSampler(torch.cuda.current_device()).start()
+    time.sleep(0.02)
     barrier(pg)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0 = time.perf_counter()
     e0.record()
     for _ in range(args.steps):
-        runner.step(*args_step)
+        g.replay()
     e1.record()
     torch.cuda.synchronize()
     t1 = time.perf_counter()
     barrier(pg)
     clocks.stop()
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, pg)
+    kern_ms = {k: a.elapsed_time(b) for k, (a, b) in ev.items()}
+    del g
+
+    # each attention launch alone (CUDA events on the launching stream)
+    st = pw.state
+    solo = {}
+    calls = {
+        "hca_attn": lambda: hca.compressed_attn_prefill(pw.q, wl.t, 128, st.hca, pw.raw_window, wl.W,
+                                                        wl.softmax_scale, out=runner.out_hca, stream=s2),
+        "csa_attn": lambda: hca.compressed_attn_prefill(pw.q, wl.t, 4, st.csa, pw.raw_window, wl.W,
+                                                        wl.softmax_scale, idx=runner.idx, count=runner.count,
+                                                        out=runner.out_csa, stream=s2),
+    }
+    s2 = torch.cuda.Stream()
+    s2.wait_stream(main)
+    for name, fn in calls.items():
+        with torch.cuda.stream(s2):
+            fn()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            n_solo = 3
+            a.record(s2)
+            for _ in range(n_solo):
+                fn()
+            b.record(s2)
+            s2.synchronize()
+        solo[name] = a.elapsed_time(b) / n_solo
+    fl = prefill_attn_flops(wl)
     fl_att, op_ind = prefill_flops(wl)
+    gp = gemm_peaks()
     hbm, bf16, bf16s, src = peaks()
+    dominant = max(solo, key=solo.get)
+    ach = fl[dominant] / (solo[dominant] * 1e-3) / 1e12
+    fp16_peak = gp["fp16"]
+    roof = {"bound": "tensor", "kernel": dominant, "achieved": ach, "peak": fp16_peak, "unit": "TFLOP/s",
+            "frac": ach / fp16_peak, "peak_source": "fp16 dense GEMM measured in this run (cuBLAS, burst)",
+            "frac_of_fp8_measured": (ach / gp["fp8_e4m3"]) if gp.get("fp8_e4m3") else None,
+            "frac_of_bf16_measured": ach / gp["bf16"], "traffic": None,
+            "algorithmic_flops": fl[dominant], "avg_launch_us": solo[dominant] * 1e3,
+            "timing": "the kernel alone, CUDA events on its stream, 3 launches after one warm-up",
+            "solo_us": {k: v * 1e3 for k, v in solo.items()},
+            "solo_tflops": {k: fl[k] / (solo[k] * 1e-3) / 1e12 for k in solo}}
+
+    # end to end through the public API: the chunk's inputs from pinned host memory,
+    # both attention outputs back to pinned host memory, every step
+    h_in = [t.to("cpu").pin_memory() for t in (pw.raw_chunk, pw.gate_chunk, pw.raw_window, pw.q)]
+    h_iq = [t.to("cpu").pin_memory() for t in pw.iq]
+    d_in = [t.clone() for t in (pw.raw_chunk, pw.gate_chunk, pw.raw_window, pw.q)]
+    d_iq = [t.clone() for t in pw.iq]
+    h_out = [torch.empty_like(runner.out_csa, device="cpu").pin_memory(),
+             torch.empty_like(runner.out_hca, device="cpu").pin_memory()]
+    h2d = sum(t.numel() * t.element_size() for t in h_in + h_iq)
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+
+    def e2e_step():
+        for a_, b_ in zip(d_in + d_iq, h_in + h_iq):
+            a_.copy_(b_, non_blocking=True)
+        oc, oh = runner.step(d_in[0], d_in[1], d_in[2], d_in[3], tuple(d_iq))
+        h_out[0].copy_(oc, non_blocking=True)
+        h_out[1].copy_(oh, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    n_e2e = max(3, min(args.steps, 20))
+    barrier(pg)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(n_e2e):
+        e2e_step()
+    f1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / n_e2e, pg)
+
     line = {"metric": "prefill tokens/s", "value": world * wl.Tq / (ms * 1e-3), "unit": "tok/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "fp16/fp32 (FP8/FP4 storage)", "data": "synthetic",
-            "config": {"workload": wl.name, "chunk": wl.Tq, "p0": wl.t, "parallelism": "single GPU"},
+            "config": {"workload": wl.name, "chunk": wl.Tq, "p0": wl.t,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (queries alone 268 MB per chunk)"},
             "tflops": {"attention": fl_att / (ms * 1e-3) / 1e12, "indexer_int": op_ind / (ms * 1e-3) / 1e12,
                        "total": (fl_att + op_ind) / (ms * 1e-3) / 1e12,
-                       "frac_of_bf16_measured": (fl_att + op_ind) / (ms * 1e-3) / 1e12 / bf16},
+                       "frac_of_fp16_measured": (fl_att + op_ind) / (ms * 1e-3) / 1e12 / gp["fp16"],
+                       "frac_of_fp8_measured": ((fl_att + op_ind) / (ms * 1e-3) / 1e12 / gp["fp8_e4m3"])
+                       if gp.get("fp8_e4m3") else None},
+            "gemm_peaks_tflops": gp,
             "kernels_us": {k: v * 1e3 for k, v in kern_ms.items()},
-            "clocks": clocks.summary(t0, t1)}
+            "roofline": roof,
+            "clocks": clocks.summary(t0, t1),
+            "e2e": {"value": world * wl.Tq / (e2e_ms * 1e-3), "unit": "tok/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "how": "PrefillRunner.step from pinned host inputs (chunk raw KV "
+                    "and gates, window, queries, indexer queries) to pinned host outputs (CSA and HCA), eager"},
+            "gpu_launches": runner.kernels_per_step * args.steps}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        threads = oracle.set_threads(cpu_cores())
+        rows = [0, 1000, 2047, 4095]
+        run = oracle_prefill_sample(wl, rows)
+        run()
+        tt = time.perf_counter()
+        run()
+        dt = time.perf_counter() - tt
+        line["cpu_baseline"] = {"value": len(rows) / dt, "unit": "tok/s", "cores": threads, "kind": "oracle",
+                                "cpu_model": cpu_model(),
+                                "sample": f"{len(rows)} query positions of {wl.name} ({rows}) through the oracle: "
+                                          "index scores over every eligible CSA entry, exact top-k, CSA and HCA "
+                                          f"attention in fp64, at {threads} threads"}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -602,20 +823,29 @@ def bench_stack(args, wl, world, rank, pg):
 
 
 def cpu_baseline(wl):
+    """The oracle on the host cores: one query token of the workload (see
+    oracle_decode_sample), at all cores and at one thread."""
     import oracle
     oracle.build()
+    threads = oracle.set_threads(cpu_cores())
     run = oracle_decode_sample(wl, 1.0)
     run()
     t0 = time.perf_counter()
     n = 0
-    while n < 3 and time.perf_counter() - t0 < 25.0:
+    while n < 5 and time.perf_counter() - t0 < 15.0:
         run()
         n += 1
     dt = (time.perf_counter() - t0) / n
-    return {"value": 1.0 / dt, "unit": "query-tok/s", "cores": 1, "kind": "oracle",
+    oracle.set_threads(1)
+    t1 = time.perf_counter()
+    run()
+    dt1 = time.perf_counter() - t1
+    oracle.set_threads(threads)
+    return {"value": 1.0 / dt, "unit": "query-tok/s", "cores": threads, "kind": "oracle",
+            "cpu_model": cpu_model(), "single_thread_value": 1.0 / dt1,
             "sample": f"one query token (sequence) of {wl.name} through the oracle: index scores over all "
                       f"{(wl.t + 1) // 4} CSA entries, exact top-{wl.k}, CSA and HCA attention in fp64; "
-                      f"{n} repetitions, single thread"}
+                      f"{n} repetitions at {threads} threads (OpenMP over entries and heads), 1 at one thread"}
 
 
 def main():

@@ -25,6 +25,9 @@
  *     the caller, and must stay valid until the work queued on `stream`
  *     has finished.  The library allocates no device memory: scratch comes
  *     from the caller's `ws` buffer, sized by the matching *_workspace_size.
+ *     The one exception is compressed_attn_decode_noalloc, whose scratch is
+ *     a 16 MiB array built into the library: every device that loads the
+ *     library holds it until the process exits.
  *   - Every pointer must be 16-byte aligned (HCA_ERR_INVALID_ARG otherwise).
  *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
  *     stream.  Calls are asynchronous and never synchronise the device.
@@ -78,7 +81,9 @@ const char* hca_status_string(int status);
 /* The last cudaError_t seen by a call that returned HCA_ERR_CUDA (per thread). */
 int hca_last_cuda_error(void);
 /* Device-side error word of the current device: non-zero when a kernel gave
- * up a bounded wait on its own pipeline barriers (its outputs are then NaN).
+ * up a bounded wait on its own pipeline barriers (its outputs are then NaN;
+ * index scores of the CTA that gave up are NaN, and top-k sets and counts
+ * built from them are undefined).
  * Reads and clears the word; synchronises with the device.  -1 if the word
  * cannot be read. */
 int hca_take_device_error(void);
@@ -251,8 +256,9 @@ int compressed_attn_decode(const uint16_t* q, int32_t B, int32_t H,
  *     HCA_ERR_SCRATCH_LIMIT and nothing is launched.
  *   - The scratch is a per-device global of the library: every GPU on which
  *     the library is used keeps those 16 MiB until the process exits.
- *   - The first call on a device looks up the scratch's device address with
- *     that device current (a one-time set-up per device); make that first
+ *   - Every call looks up the scratch's device address for the current
+ *     device (cudaGetSymbolAddress; no allocation).  The first call on a
+ *     device also loads the library's device globals there: make that first
  *     call before any stream capture.
  *   - Every call on a device shares the one scratch array, which keeps the
  *     previous call's contents; the kernels overwrite every partial they

@@ -525,39 +525,27 @@ int attn_prefill_launch(const uint16_t* q, int Tq, int H, int p0, int m, const h
 // loaded library, so every device it runs on keeps HCA_NOALLOC_SCRATCH_BYTES
 // until the process exits.  Host code must not pass `g_noalloc_scratch`
 // itself to a kernel: in host code that name is only a host-side stand-in.
-// The device address is looked up once per device, with that device
-// current, by cudaGetSymbolAddress (so the first call on a device should
-// come before any stream capture), and that address is what the kernels get.
-// All calls on a device share the array; the kernels write every partial
-// before reading it, so no clearing is needed, but calls that overlap on the
-// GPU race on it.
+// Every call looks up the device address of the array for the current
+// device with cudaGetSymbolAddress (cheap; nothing is allocated), so an
+// address never outlives the context it came from.  The first call on a
+// device also loads the library's device globals there, so it should come
+// before any stream capture.  All calls on a device share the array; the
+// kernels write every partial before reading it, so no clearing is needed,
+// but calls that overlap on the GPU race on it.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[HCA_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 
 void* noalloc_scratch_address(int* status) {
-    static std::mutex mu;
-    static void* addr[64] = {nullptr};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess || dev < 0 || dev >= 64) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
         set_last_cuda_error(static_cast<int>(e));
         *status = HCA_ERR_CUDA;
         return nullptr;
     }
-    std::lock_guard<std::mutex> lk(mu);
-    if (addr[dev] == nullptr) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess || p == nullptr) {
-            set_last_cuda_error(static_cast<int>(e));
-            *status = HCA_ERR_CUDA;
-            return nullptr;
-        }
-        addr[dev] = p;
-    }
     *status = HCA_OK;
-    return addr[dev];
+    return p;
 }
 
 bool noalloc_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -656,7 +656,8 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
             const int64_t e = s_begin + static_cast<int64_t>(t) * TILE + row;
             if (e < s_end && e < s_elig[q]) {
                 scores[static_cast<size_t>(qrow0 + q) * Nc_cap + e] = ok ? sc : __int_as_float(0x7fc00000);
-                if (QG == 1 && hist) atomicAdd(&sh_hist[score_key(sc) >> 21], 1u);
+                // a NaN score is not counted: after a device error the top-k is undefined anyway
+                if (QG == 1 && hist && ok) atomicAdd(&sh_hist[score_key(sc) >> 21], 1u);
             }
         }
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");

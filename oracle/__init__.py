@@ -29,7 +29,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 _lock = threading.Lock()
 _lib = None
 
-GCC_FLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+GCC_FLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared"]
 
 
 def build(force: bool = False) -> str:
@@ -39,6 +39,14 @@ def build(force: bool = False) -> str:
         subprocess.check_call(["gcc", *GCC_FLAGS, "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
+
+
+def set_threads(n: int) -> int:
+    """Threads of the oracle's parallel loops (n <= 0: all cores).  Results
+    do not depend on it: each output is computed by one thread in the same
+    sequence.  Returns the thread count now in effect."""
+    lib().oracle_set_threads(int(n))
+    return int(lib().oracle_max_threads())
 
 
 def _P(t):
@@ -52,6 +60,10 @@ def lib():
             L = ctypes.CDLL(build())
             u8p, u16p, i32p, i64p = _P(ctypes.c_uint8), _P(ctypes.c_uint16), _P(ctypes.c_int32), _P(ctypes.c_int64)
             fp, dp = _P(ctypes.c_float), _P(ctypes.c_double)
+            L.oracle_set_threads.argtypes = [ctypes.c_int]
+            L.oracle_set_threads.restype = None
+            L.oracle_max_threads.argtypes = []
+            L.oracle_max_threads.restype = ctypes.c_int
             L.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
             L.oracle_bf16_to_f32.restype = ctypes.c_float
             L.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
@@ -66,6 +78,8 @@ def lib():
             L.oracle_ue8m0_value.restype = ctypes.c_double
             L.oracle_const.argtypes = [ctypes.c_int]
             L.oracle_const.restype = ctypes.c_float
+            L.oracle_f64_to_bf16_array.argtypes = [dp, u16p, ctypes.c_int64]
+            L.oracle_f64_to_bf16_array.restype = None
             L.oracle_f32_to_bf16_array.argtypes = [fp, u16p, ctypes.c_int64]
             L.oracle_f32_to_bf16_array.restype = None
             L.oracle_f32_to_e4m3_array.argtypes = [fp, u8p, ctypes.c_int64]
@@ -267,5 +281,28 @@ def attend(q_bits, codes, scales, rope, ent, win_bits, softmax_scale, g):
 
 
 def round_bf16(x64: np.ndarray) -> np.ndarray:
-    """fp64 -> bf16 bits via fp32 (both round to nearest even)."""
-    return f32_to_bf16(np.asarray(x64, dtype=np.float32))
+    """fp64 -> bf16 bits, rounded once to nearest (ties to even)."""
+    x = np.ascontiguousarray(np.asarray(x64, dtype=np.float64))
+    out = np.empty(x.shape, np.uint16)
+    lib().oracle_f64_to_bf16_array(_ptr(x, ctypes.c_double), _ptr(out, ctypes.c_uint16), x.size)
+    return out
+
+
+# ---------------------------------------------------------------- causal key sets
+def causal_keys(p: int, m: int, W: int, n_cap: int = None):
+    """Keys visible to a query at absolute position p ("DeepSeek V4 ..." note,
+    section 7: compressed entries plus the sliding window of the last n_win
+    uncompressed tokens; an entry exists once its block is complete).
+      entries: s = 0 .. min(n_cap, (p+1)//m) - 1, i.e. every block whose last
+               token (s+1)m - 1 is at or before p (m = 0: none, the branch is off)
+      window : raw positions max(0, p-W+1) .. p
+    Returns (entry indices, first window position, last window position + 1)."""
+    if m and m > 0:
+        e = (p + 1) // m
+        if n_cap is not None:
+            e = min(e, n_cap)
+    else:
+        e = 0
+    first = max(0, p - W + 1)
+    return np.arange(max(e, 0)), first, p + 1
+

@@ -26,11 +26,15 @@
  *   (2) index scores (which decide the top-k sets).
  * Everything else (attention) is computed in fp64.
  *
- * Build: gcc -O2 -std=c11 -ffp-contract=off -fPIC -shared -lm.
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fopenmp -fPIC -shared -lm.
  * -ffp-contract=off matters: every a*b+c below is two roundings unless it is
- * written as fmaf().
+ * written as fmaf().  OpenMP only spreads independent outputs (entries,
+ * scores, heads, rows) over threads; each output is computed by one thread
+ * in the same sequence whatever the thread count, so results do not depend
+ * on it.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -54,6 +58,37 @@ uint16_t oracle_f32_to_bf16(float f)
     uint32_t lsb = (u >> 16) & 1u;
     u += 0x7FFFu + lsb;
     return (uint16_t)(u >> 16);
+}
+
+/* Threads used by the parallel loops below (n <= 0: the OpenMP default). */
+void oracle_set_threads(int n) { omp_set_num_threads(n > 0 ? n : omp_get_num_procs()); }
+int oracle_max_threads(void) { return omp_get_max_threads(); }
+
+/* fp64 -> bf16 rounded once, to nearest with ties to even (no detour
+ * through fp32, whose own rounding could land on a bf16 midpoint).  With
+ * |x| = f 2^e, f in [0.5, 1), the bf16 spacing near x is 2^(e-8) for normal
+ * results and 2^-133 below 2^-126; x / spacing is exact in fp64 and
+ * nearbyint() rounds it to nearest-even.  Results of magnitude 2^128 or more
+ * are +-inf; NaN stays NaN. */
+uint16_t oracle_f64_to_bf16(double x)
+{
+    if (isnan(x)) return 0x7FC0u;
+    const uint16_t sign = signbit(x) ? 0x8000u : 0u;
+    const double a = fabs(x);
+    if (a == 0.0) return sign;
+    if (isinf(a)) return (uint16_t)(sign | 0x7F80u);
+    int e;
+    frexp(a, &e);
+    const int sp = e - 8 > -133 ? e - 8 : -133;       /* log2 of the bf16 spacing */
+    const double r = ldexp(nearbyint(ldexp(a, -sp)), sp);
+    if (r >= 0x1p128) return (uint16_t)(sign | 0x7F80u);
+    const float f = (float)r;                          /* exact: r is a bf16 value */
+    return (uint16_t)(sign | (bits_from_f32(f) >> 16));
+}
+
+void oracle_f64_to_bf16_array(const double* x, uint16_t* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_f64_to_bf16(x[i]);
 }
 
 void oracle_f32_to_bf16_array(const float* x, uint16_t* out, int64_t n)
@@ -251,12 +286,16 @@ double oracle_compress(const uint16_t* x, const uint16_t* gate, int64_t x_seq_st
                        int64_t cap, int64_t entry_begin)
 {
     int dn = d - d_rope, ng = dn / g;
-    float*  y   = (float*)malloc(sizeof(float) * d);
-    double* y64 = (double*)malloc(sizeof(double) * d);
-    double* mag = (double*)malloc(sizeof(double) * d);
     double worst = 0.0;
-    for (int b = 0; b < B; ++b) {
-        for (int64_t jj = 0; jj < n_blocks; ++jj) {
+    #pragma omp parallel reduction(max:worst)
+    {
+        float*  y   = (float*)malloc(sizeof(float) * d);
+        double* y64 = (double*)malloc(sizeof(double) * d);
+        double* mag = (double*)malloc(sizeof(double) * d);
+        #pragma omp for schedule(static)
+        for (int64_t be = 0; be < (int64_t)B * n_blocks; ++be) {
+            const int b = (int)(be / n_blocks);
+            const int64_t jj = be % n_blocks;
             const size_t row = (size_t)b * x_seq_stride + (size_t)jj * m;
             oracle_pool_block(x + row * d, gate + row * d, bias, m, d, y, y64, mag);
             for (int c = 0; c < d; ++c) {
@@ -270,8 +309,8 @@ double oracle_compress(const uint16_t* x, const uint16_t* gate, int64_t x_seq_st
                                scales + ((size_t)b * cap + e) * ng,
                                rope + ((size_t)b * cap + e) * d_rope);
         }
+        free(y); free(y64); free(mag);
     }
-    free(y); free(y64); free(mag);
     return worst;
 }
 
@@ -338,6 +377,7 @@ int64_t oracle_index_scores(const uint8_t* q_codes, const uint8_t* q_sf, const f
             if (elig < 0) elig = 0;
             float* row = scores + ((size_t)b * Tq + t) * Nc_cap;
             const size_t qi = (size_t)b * Tq + t;
+            #pragma omp parallel for schedule(static) reduction(+:n_inexact)
             for (int64_t s = 0; s < Nc_cap; ++s) {
                 if (s >= elig) { row[s] = -INFINITY; continue; }
                 const uint8_t* kc = k_codes + ((size_t)b * Nc_cap + s) * cb;
@@ -386,7 +426,10 @@ static int cmp_i32(const void* a, const void* b)
 void oracle_topk(const float* scores, const int32_t* q_pos, int R, int64_t Nc_cap,
                  int m, int k, int32_t* idx, int32_t* count)
 {
+    #pragma omp parallel
+    {
     scored_t* buf = (scored_t*)malloc(sizeof(scored_t) * (Nc_cap > 0 ? Nc_cap : 1));
+    #pragma omp for schedule(dynamic)
     for (int r = 0; r < R; ++r) {
         int64_t elig = ((int64_t)q_pos[r] + 1) / m;
         if (elig > Nc_cap) elig = Nc_cap;
@@ -402,6 +445,7 @@ void oracle_topk(const float* scores, const int32_t* q_pos, int R, int64_t Nc_ca
         count[r] = (int32_t)kk;
     }
     free(buf);
+    }
 }
 
 /* ------------------------------------------------------------------ */
@@ -441,7 +485,10 @@ void oracle_attend(const uint16_t* q, int H, int d, int d_rope, int g,
         double* kr = K + (size_t)(n_ent + j) * d;
         for (int c = 0; c < d; ++c) kr[c] = (double)oracle_bf16_to_f32(win[(size_t)j * d + c]);
     }
+    #pragma omp parallel
+    {
     double* logit = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    #pragma omp for schedule(static)
     for (int h = 0; h < H; ++h) {
         const uint16_t* qh = q + (size_t)h * d;
         double mx = -INFINITY;
@@ -462,5 +509,7 @@ void oracle_attend(const uint16_t* q, int H, int d, int d_rope, int g,
         }
         if (lse) lse[h] = n > 0 ? mx + log(den) : -INFINITY;
     }
-    free(K); free(logit);
+    free(logit);
+    }
+    free(K);
 }

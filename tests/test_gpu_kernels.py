@@ -364,10 +364,9 @@ def test_prefill_dense_and_sparse(layout, H, p0):
     qh, rh, idh, cth = host(q), host(raw), host(idx), host(cnt)
     for i in list(range(0, Tq, 7)) + [Tq - 1]:
         p = p0 + i
-        first = max(0, p - W + 1)
-        win = rh[first - (p0 - (W - 1)):p - (p0 - (W - 1)) + 1]
-        e = min(cap, (p + 1) // m)
-        ref, _ = oracle.attend(qh[i], codes, scales, rope, np.arange(e), win, scale, g)
+        ent, w0, w1 = oracle.causal_keys(p, m, W, n_cap=cap)
+        win = rh[w0 - (p0 - (W - 1)):w1 - (p0 - (W - 1))]
+        ref, _ = oracle.attend(qh[i], codes, scales, rope, ent, win, scale, g)
         assert_attn_close(host(out_d)[i], ref, f"dense pos {p}")
         refs, _ = oracle.attend(qh[i], codes, scales, rope, idh[i, :cth[i]], win, scale, g)
         assert_attn_close(host(out_s)[i], refs, f"sparse pos {p}")

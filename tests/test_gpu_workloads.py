@@ -197,9 +197,9 @@ def test_prefill_4096_131k_sampled():
         assert np.array_equal(gs[0, i].view(np.uint32), s[0, 0].view(np.uint32)), f"scores row {i}"
         idx, cnt = oracle.topk(s[0], pos[0], 4, wl.k)
         assert gcnt[i] == cnt[0] and np.array_equal(gi[i], idx[0]), f"top-k row {i}"
-        win = rawh[i:i + wl.W]                     # positions p-127 .. p
+        ent128, w0, w1 = oracle.causal_keys(p, 128, wl.W)
+        win = rawh[w0 - (p0 - (wl.W - 1)):w1 - (p0 - (wl.W - 1))]
         ref, _ = oracle.attend(qh[i], codes4, scales4, rope4, idx[0, :cnt[0]], win, wl.softmax_scale, wl.g)
         assert_attn_close(oc[i], ref, f"CSA pos {p}")
-        ref, _ = oracle.attend(qh[i], codes128, scales128, rope128, np.arange((p + 1) // 128), win,
-                               wl.softmax_scale, wl.g)
+        ref, _ = oracle.attend(qh[i], codes128, scales128, rope128, ent128, win, wl.softmax_scale, wl.g)
         assert_attn_close(oh[i], ref, f"HCA pos {p}")

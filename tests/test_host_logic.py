@@ -86,3 +86,42 @@ def test_bench_max_over_ranks_gloo_world2(tmp_path):
     assert r.returncode == 0, r.stdout + r.stderr
     for rank in (0, 1):
         assert (tmp_path / f"rank{rank}").read_text() == "ok 3.0"
+
+
+def test_decode_step_bytes_count_each_stream_once():
+    """The decode step's algorithmic HBM bytes are the indexer's key stream
+    plus the two attention calls (selected CSA entries, every HCA entry,
+    windows, queries, outputs), each counted once: 95.68 MB at decode_b4_1m.
+    The scores the top-k reads stay in L2 and are not part of the sum."""
+    import bench
+    import hca_inputs as inp
+    wl = inp.WORKLOADS["decode_b4_1m"]
+    algo = bench.decode_bytes(wl)
+    assert set(algo) == {"indexer", "csa_attn", "hca_attn", "topk"}
+    total = bench.step_bytes_of(algo)
+    assert total == algo["indexer"] + algo["csa_attn"] + algo["hca_attn"]
+    entry = 448 + 7 * 4 + 64 * 2
+    assert entry == 604
+    per_seq = (262144 * 68 + 4 * (64 + 4 + 4)) + (1024 * 604 + 128 * 1024 + 2 * 64 * 1024 + 1024 * 4) + \
+              (8192 * 604 + 128 * 1024 + 2 * 64 * 1024)
+    assert total == 4 * per_seq == 95683712
+
+
+def test_prefill_attention_flops_counts_causal_keys():
+    """Prefill attention work: 4*H*d flop per (query, key) over each query's
+    causal key set; for the CSA call min(k, eligible) + window keys."""
+    import bench
+    import hca_inputs as inp
+    import oracle
+    wl = inp.WORKLOADS["prefill_4096_131k"]
+    fl = bench.prefill_attn_flops(wl)
+    n_csa = n_hca = 0
+    for p in range(wl.t, wl.t + wl.Tq):
+        e4, w0, w1 = oracle.causal_keys(p, 4, wl.W)
+        e128, _, _ = oracle.causal_keys(p, 128, wl.W)
+        n_csa += min(wl.k, len(e4)) + (w1 - w0)
+        n_hca += len(e128) + (w1 - w0)
+    assert fl["csa_attn"] == 4 * 64 * 512 * n_csa
+    assert fl["hca_attn"] == 4 * 64 * 512 * n_hca
+    att, _ = bench.prefill_flops(wl)
+    assert att == fl["csa_attn"] + fl["hca_attn"]

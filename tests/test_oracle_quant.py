@@ -105,3 +105,48 @@ def test_quant_power_of_two_invariance():
         ck, sk, _ = oracle.quant_entry((y * np.float32(2.0 ** k)).astype(np.float32), 64, 64)
         assert np.array_equal(ck, c0)
         assert np.array_equal(sk, (s0 * np.float32(2.0 ** k)).astype(np.float32))
+
+
+def _bf16_exact(x: float) -> int:
+    """bf16 bits of x rounded once to nearest-even, by exact rational arithmetic."""
+    from fractions import Fraction
+    import math
+    if x == 0.0:
+        return 0x8000 if math.copysign(1.0, x) < 0 else 0
+    sign = 0x8000 if x < 0 else 0
+    a = Fraction(abs(x))
+    e = math.floor(math.log2(abs(x)))
+    if Fraction(2) ** e > a:
+        e -= 1
+    if Fraction(2) ** (e + 1) <= a:
+        e += 1
+    sp = max(e - 7, -133)                                  # spacing of bf16 values near x
+    q = a / Fraction(2) ** sp
+    n = math.floor(q)
+    rem = q - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    r = Fraction(n) * Fraction(2) ** sp
+    if r >= Fraction(2) ** 128:
+        return sign | 0x7F80
+    f = np.float32(float(r))                               # exact: a bf16 value
+    return sign | int(f.view(np.uint32)) >> 16
+
+
+def test_round_bf16_rounds_once_from_fp64():
+    """The attention tolerance compares against the fp64 result rounded to
+    bf16: one rounding.  1 + 2^-8 + 2^-30 lies above the bf16 midpoint
+    1 + 2^-8 but rounds to that midpoint in fp32, so a detour through fp32
+    would give 1.0 instead of 1 + 2^-7."""
+    x = 1.0 + 2.0 ** -8 + 2.0 ** -30
+    assert int(oracle.round_bf16(np.array([x]))[0]) == 0x3F81
+    assert int(oracle.round_bf16(np.array([-x]))[0]) == 0xBF81
+    assert int(oracle.round_bf16(np.array([1.0 + 2.0 ** -8]))[0]) == 0x3F80          # tie to even
+    assert int(oracle.round_bf16(np.array([1.0 + 3 * 2.0 ** -8]))[0]) == 0x3F82      # tie to even (up)
+    rng = np.random.default_rng(11)
+    xs = np.concatenate([rng.standard_normal(3000) * 10.0 ** rng.uniform(-40, 38, 3000),
+                         [0.0, -0.0, 3.3895313892515355e38, 3.4e38, 1e-40, -2.0 ** -133, 2.0 ** -134 * 1.5]])
+    got = oracle.round_bf16(xs)
+    want = np.array([_bf16_exact(float(v)) for v in xs], np.uint16)
+    assert np.array_equal(got, want)
+

@@ -180,3 +180,21 @@ def test_csa_with_k_covering_all_entries_equals_dense():
     o_sparse, _ = oracle.attend(q, codes, scales, rope, idx[0, :cnt[0]], win, 0.1, g)
     o_dense, _ = oracle.attend(q, codes, scales, rope, np.arange(Nc), win, 0.1, g)
     assert np.array_equal(o_sparse, o_dense)
+
+
+def test_causal_key_sets_by_enumeration():
+    """The causal rule of a prefill query at position p, enumerated token by
+    token: entry s is visible iff all m tokens of its block are at or before
+    p; the window holds the raw tokens in (p - W, p], none before 0."""
+    for m in (1, 4, 128):
+        for W in (1, 5, 128):
+            for p in list(range(0, 300)) + [1023, 131071, 135167]:
+                ent, w0, w1 = oracle.causal_keys(p, m, W)
+                want = [s for s in range(p // m + 2) if all(t <= p for t in range(s * m, s * m + m))]
+                assert list(ent) == want
+                assert list(range(w0, w1)) == [t for t in range(max(0, p - 2 * W), p + 1) if p - W < t]
+    ent, _, _ = oracle.causal_keys(1000, 4, 128, n_cap=100)
+    assert len(ent) == 100
+    ent, w0, w1 = oracle.causal_keys(50, 0, 128)
+    assert len(ent) == 0 and (w0, w1) == (0, 51)
+
