@@ -108,6 +108,21 @@ def lib():
                                         u8p, fp, u16p, i64p, ctypes.c_int64, u16p, ctypes.c_int64,
                                         ctypes.c_float, dp, dp]
             L.oracle_attend.restype = None
+            L.oracle_attend_ex.argtypes = [u16p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           u8p, fp, u16p, i64p, ctypes.c_int64, u16p, ctypes.c_int64,
+                                           ctypes.c_float, fp, ctypes.c_float, fp, fp, ctypes.c_int64, dp, dp]
+            L.oracle_attend_ex.restype = None
+            L.oracle_rmsnorm_f32.argtypes = [fp, ctypes.c_int, fp, ctypes.c_float, fp]
+            L.oracle_rmsnorm_f32.restype = None
+            L.oracle_rope_f64.argtypes = [dp, ctypes.c_int, ctypes.c_int64, fp, ctypes.c_int, dp]
+            L.oracle_rope_f64.restype = None
+            L.oracle_token_prep.argtypes = [u16p, i64p, ctypes.c_int64, ctypes.c_int, ctypes.c_int, fp,
+                                            ctypes.c_float, fp, u16p]
+            L.oracle_token_prep.restype = None
+            L.oracle_compress_ex.argtypes = [u16p, u16p, ctypes.c_int64, fp, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, u8p, fp, u16p,
+                                             ctypes.c_int64, ctypes.c_int64, fp, ctypes.c_float, fp]
+            L.oracle_compress_ex.restype = ctypes.c_double
             _lib = L
     return _lib
 
@@ -195,12 +210,24 @@ def quant_entry(y: np.ndarray, d_rope: int, g: int):
     return codes, scales, rope
 
 
-def compress(x_bits, gate_bits, bias, m, n_blocks, d_rope, g, cap=None, entry_begin=0):
+def _opt(a, dtype, ct):
+    if a is None:
+        return None, None
+    a = _c(a, dtype)
+    return a, _ptr(a, ct)
+
+
+def compress(x_bits, gate_bits, bias, m, n_blocks, d_rope, g, cap=None, entry_begin=0,
+             norm_w=None, eps=1e-6, inv_freq=None):
     """Pool + quantise n_blocks entries for each sequence.
     x_bits, gate_bits: [B][T][d] bf16 bits whose row 0 is the first token of
-    block ``entry_begin``.  Returns (codes [B][cap][dn], scales [B][cap][dn/g],
+    block ``entry_begin``.  norm_w [d] / inv_freq [d_rope/2] (optional): the
+    note's section 9 entry RMSNorm and partial RoPE (entry e at position e*m)
+    before storage.  Returns (codes [B][cap][dn], scales [B][cap][dn/g],
     rope [B][cap][d_rope], worst fp32-vs-fp64 relative deviation)."""
     x_bits, gate_bits, bias = _c(x_bits, np.uint16), _c(gate_bits, np.uint16), _c(bias, np.float32)
+    nw, nw_p = _opt(norm_w, np.float32, ctypes.c_float)
+    fq, fq_p = _opt(inv_freq, np.float32, ctypes.c_float)
     B, T, d = x_bits.shape
     assert n_blocks * m <= T
     cap = entry_begin + n_blocks if cap is None else cap
@@ -208,11 +235,44 @@ def compress(x_bits, gate_bits, bias, m, n_blocks, d_rope, g, cap=None, entry_be
     codes = np.zeros((B, cap, dn), np.uint8)
     scales = np.zeros((B, cap, dn // g), np.float32)
     rope = np.zeros((B, cap, d_rope), np.uint16)
-    worst = lib().oracle_compress(_ptr(x_bits, ctypes.c_uint16), _ptr(gate_bits, ctypes.c_uint16), T,
-                                  _ptr(bias, ctypes.c_float), m, B, n_blocks, d, d_rope, g,
-                                  _ptr(codes, ctypes.c_uint8), _ptr(scales, ctypes.c_float),
-                                  _ptr(rope, ctypes.c_uint16), cap, entry_begin)
+    worst = lib().oracle_compress_ex(_ptr(x_bits, ctypes.c_uint16), _ptr(gate_bits, ctypes.c_uint16), T,
+                                     _ptr(bias, ctypes.c_float), m, B, n_blocks, d, d_rope, g,
+                                     _ptr(codes, ctypes.c_uint8), _ptr(scales, ctypes.c_float),
+                                     _ptr(rope, ctypes.c_uint16), cap, entry_begin, nw_p, float(eps), fq_p)
     return codes, scales, rope, worst
+
+
+def rmsnorm_f32(y, w, eps=1e-6):
+    """RMSNorm of one vector in the defined fp32 sequence (pairwise-tree sum of
+    rounded squares, IEEE sqrt, (y / r) * w); note section 9."""
+    y, w = _c(y, np.float32), _c(w, np.float32)
+    out = np.empty_like(y)
+    lib().oracle_rmsnorm_f32(_ptr(y, ctypes.c_float), y.shape[0], _ptr(w, ctypes.c_float), float(eps),
+                             _ptr(out, ctypes.c_float))
+    return out
+
+
+def rope_f64(v, pos, inv_freq, sign=1):
+    """Partial RoPE of n_r values: pairs (2i, 2i+1) rotated by sign*pos*inv_freq[i], fp64."""
+    v, inv_freq = _c(v, np.float64), _c(inv_freq, np.float32)
+    out = np.empty_like(v)
+    lib().oracle_rope_f64(_ptr(v, ctypes.c_double), v.shape[0], int(pos), _ptr(inv_freq, ctypes.c_float),
+                          int(sign), _ptr(out, ctypes.c_double))
+    return out
+
+
+def token_prep(x_bits, pos, d_rope, norm_w=None, eps=1e-6, inv_freq=None):
+    """Window tokens for the state cache: RMSNorm and partial RoPE at each
+    token's position, stored bf16.  x_bits [n][d] bf16 bits, pos [n]."""
+    x_bits = _c(x_bits, np.uint16)
+    n, d = x_bits.shape
+    pos = _c(pos, np.int64).reshape(-1)
+    nw, nw_p = _opt(norm_w, np.float32, ctypes.c_float)
+    fq, fq_p = _opt(inv_freq, np.float32, ctypes.c_float)
+    out = np.empty_like(x_bits)
+    lib().oracle_token_prep(_ptr(x_bits, ctypes.c_uint16), _ptr(pos, ctypes.c_int64), n, d, d_rope, nw_p,
+                            float(eps), fq_p, _ptr(out, ctypes.c_uint16))
+    return out
 
 
 # ---------------------------------------------------------------- indexer
@@ -258,14 +318,21 @@ def topk(scores, q_pos, m, k):
 
 
 # ---------------------------------------------------------------- attention
-def attend(q_bits, codes, scales, rope, ent, win_bits, softmax_scale, g):
+def attend(q_bits, codes, scales, rope, ent, win_bits, softmax_scale, g, q_norm_w=None, eps=1e-6, sink=None,
+           inv_freq=None, q_pos=0):
     """Shared key-value MQA attention of one query token (H heads) over the
     listed compressed entries plus raw window tokens, one joint softmax, fp64
     ("DeepSeek V4 ..." note, sections 7-9; HF blog figures 3 and 4).
     q_bits [H][d] bf16 bits; codes/scales/rope: one sequence's cache;
     ent: entry indices; win_bits [n_win][d] bf16 bits.
+    Optional note section 9 extras: q_norm_w [d] (query-head RMSNorm), sink [H]
+    (per-head sink logit), inv_freq [d_rope/2] with q_pos (the query's RoPE
+    dims rotated to q_pos, the output's rotated back).
     Returns (out fp64 [H][d], lse fp64 [H])."""
     q_bits = _c(q_bits, np.uint16)
+    qn, qn_p = _opt(q_norm_w, np.float32, ctypes.c_float)
+    sk, sk_p = _opt(sink, np.float32, ctypes.c_float)
+    fq, fq_p = _opt(inv_freq, np.float32, ctypes.c_float)
     H, d = q_bits.shape
     codes, scales, rope = _c(codes, np.uint8), _c(scales, np.float32), _c(rope, np.uint16)
     d_rope = rope.shape[-1]
@@ -273,10 +340,11 @@ def attend(q_bits, codes, scales, rope, ent, win_bits, softmax_scale, g):
     win_bits = _c(win_bits, np.uint16).reshape(-1, d)
     out = np.empty((H, d), np.float64)
     lse = np.empty(H, np.float64)
-    lib().oracle_attend(_ptr(q_bits, ctypes.c_uint16), H, d, d_rope, g, _ptr(codes, ctypes.c_uint8),
-                        _ptr(scales, ctypes.c_float), _ptr(rope, ctypes.c_uint16), _ptr(ent, ctypes.c_int64),
-                        ent.shape[0], _ptr(win_bits, ctypes.c_uint16), win_bits.shape[0],
-                        float(softmax_scale), _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double))
+    lib().oracle_attend_ex(_ptr(q_bits, ctypes.c_uint16), H, d, d_rope, g, _ptr(codes, ctypes.c_uint8),
+                           _ptr(scales, ctypes.c_float), _ptr(rope, ctypes.c_uint16), _ptr(ent, ctypes.c_int64),
+                           ent.shape[0], _ptr(win_bits, ctypes.c_uint16), win_bits.shape[0],
+                           float(softmax_scale), qn_p, float(eps), sk_p, fq_p, int(q_pos),
+                           _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double))
     return out, lse
 
 

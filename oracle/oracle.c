@@ -272,6 +272,92 @@ void oracle_quant_entry(const float* y, int d, int d_rope, int g,
     for (int c = dn; c < d; ++c) rope[c - dn] = oracle_f32_to_bf16(y[c]);
 }
 
+/* ------------------------------------------------------------------ */
+/* Entry and query extras  [N9] "Query / KV entry RMSNorm", "Partial     */
+/* RoPE", "Attention Sink"                                              */
+/* ------------------------------------------------------------------ */
+
+/* RMSNorm of one d-vector (d a power of two) in a fixed fp32 sequence, so
+ * that the FP8 codes of a normalised entry can be bit-exact: every square is
+ * rounded; ss is the pairwise tree sum over consecutive pairs (level by
+ * level: t[i] = t[2i] + t[2i+1]); mean = ss / d; r = sqrt(mean + eps)
+ * (IEEE, correctly rounded); out_c = (y_c / r) * w_c.  The pages give no
+ * precision or epsilon; eps is an argument (1e-6 in the workloads).
+ * out may alias y. */
+void oracle_rmsnorm_f32(const float* y, int d, const float* w, float eps, float* out)
+{
+    float* t = (float*)malloc(sizeof(float) * (size_t)d);
+    for (int c = 0; c < d; ++c) t[c] = y[c] * y[c];
+    for (int n = d; n > 1; n >>= 1)
+        for (int i = 0; i < n / 2; ++i) t[i] = t[2 * i] + t[2 * i + 1];
+    const float mean = t[0] / (float)d;
+    const float r = sqrtf(mean + eps);
+    for (int c = 0; c < d; ++c) out[c] = (y[c] / r) * w[c];
+    free(t);
+}
+
+/* Partial RoPE on n_r values (the last n_r dims of a vector): pair i =
+ * (v[2i], v[2i+1]) is rotated by the angle sign * pos * f_i, where f_i =
+ * inv_freq[i] (fp32, the caller's frequency table) and pos an integer
+ * position, so the fp64 angle pos * f_i is exact.  fp64 throughout:
+ *   (a, b) -> (a cos - b sin, a sin + b cos).
+ * The pages fix neither the pairing nor the frequencies; the pairing taken is
+ * adjacent dims, the frequencies are an input. */
+void oracle_rope_f64(const double* v, int n_r, int64_t pos, const float* inv_freq, int sign, double* out)
+{
+    for (int i = 0; i < n_r / 2; ++i) {
+        const double ang = (double)pos * (double)inv_freq[i];
+        const double c = cos(ang), sn = (sign < 0 ? -1.0 : 1.0) * sin(ang);
+        const double a = v[2 * i], b = v[2 * i + 1];
+        const double x = a * c - b * sn;
+        const double y = a * sn + b * c;
+        out[2 * i] = x;
+        out[2 * i + 1] = y;
+    }
+}
+
+/* Storage of one entry with the [N9] extras: y (fp32, pooled) is RMS-
+ * normalised when norm_w is given; the FP8 dims are quantised as in
+ * oracle_quant_entry; the RoPE dims are rotated to the entry's position pos
+ * (fp64, then one rounding to bf16) when inv_freq is given. */
+static void quant_entry_ex(float* y, int d, int d_rope, int g, const float* norm_w, float eps,
+                           const float* inv_freq, int64_t pos, uint8_t* codes, float* scales, uint16_t* rope)
+{
+    if (norm_w) oracle_rmsnorm_f32(y, d, norm_w, eps, y);
+    oracle_quant_entry(y, d, d_rope, g, codes, scales, rope);
+    if (inv_freq) {
+        const int dn = d - d_rope;
+        double v[256], o[256];
+        for (int c = 0; c < d_rope; ++c) v[c] = (double)y[dn + c];
+        oracle_rope_f64(v, d_rope, pos, inv_freq, +1, o);
+        for (int c = 0; c < d_rope; ++c) rope[c] = oracle_f64_to_bf16(o[c]);
+    }
+}
+
+/* One raw token prepared for the sliding window of the state cache: RMSNorm
+ * (norm_w given) in the sequence of oracle_rmsnorm_f32, the non-RoPE dims
+ * rounded to bf16 from fp32, the RoPE dims rotated to the token's position in
+ * fp64 (inv_freq given) and rounded once to bf16.
+ *   x [n][d] bf16, pos [n], out [n][d] bf16. */
+void oracle_token_prep(const uint16_t* x, const int64_t* pos, int64_t n, int d, int d_rope,
+                       const float* norm_w, float eps, const float* inv_freq, uint16_t* out)
+{
+    float* y = (float*)malloc(sizeof(float) * (size_t)d);
+    const int dn = d - d_rope;
+    for (int64_t j = 0; j < n; ++j) {
+        for (int c = 0; c < d; ++c) y[c] = oracle_bf16_to_f32(x[(size_t)j * d + c]);
+        if (norm_w) oracle_rmsnorm_f32(y, d, norm_w, eps, y);
+        for (int c = 0; c < d; ++c) out[(size_t)j * d + c] = oracle_f32_to_bf16(y[c]);
+        if (inv_freq) {
+            double v[256], o[256];
+            for (int c = 0; c < d_rope; ++c) v[c] = (double)y[dn + c];
+            oracle_rope_f64(v, d_rope, pos[j], inv_freq, +1, o);
+            for (int c = 0; c < d_rope; ++c) out[(size_t)j * d + dn + c] = oracle_f64_to_bf16(o[c]);
+        }
+    }
+    free(y);
+}
+
 /* Pool and store n_blocks entries for each of B sequences.
  *   x, gate : [B][x_seq_stride][d] bf16; x points at the first token of
  *             block entry_begin, so block entry_begin+jj is rows jj*m..jj*m+m-1
@@ -279,11 +365,33 @@ void oracle_quant_entry(const float* y, int d, int d_rope, int g,
  *             rope [B][cap][d_rope]; entry entry_begin+jj is written.
  * Returns the largest |y32 - y64| / sum_i p_i |x_i| seen (the fp64
  * cross-check of the defined fp32 sequence). */
+double oracle_compress_ex(const uint16_t* x, const uint16_t* gate, int64_t x_seq_stride,
+                          const float* bias, int m, int B, int64_t n_blocks,
+                          int d, int d_rope, int g,
+                          uint8_t* codes, float* scales, uint16_t* rope,
+                          int64_t cap, int64_t entry_begin,
+                          const float* norm_w, float eps, const float* inv_freq);
+
 double oracle_compress(const uint16_t* x, const uint16_t* gate, int64_t x_seq_stride,
                        const float* bias, int m, int B, int64_t n_blocks,
                        int d, int d_rope, int g,
                        uint8_t* codes, float* scales, uint16_t* rope,
                        int64_t cap, int64_t entry_begin)
+{
+    return oracle_compress_ex(x, gate, x_seq_stride, bias, m, B, n_blocks, d, d_rope, g, codes, scales, rope,
+                              cap, entry_begin, NULL, 0.0f, NULL);
+}
+
+/* oracle_compress with the [N9] extras: each pooled entry is RMS-normalised
+ * (norm_w [d], eps) before storage and its RoPE dims rotated to the entry's
+ * position, taken as the position of its block's first token, e * m
+ * (inv_freq [d_rope/2]); either may be NULL. */
+double oracle_compress_ex(const uint16_t* x, const uint16_t* gate, int64_t x_seq_stride,
+                          const float* bias, int m, int B, int64_t n_blocks,
+                          int d, int d_rope, int g,
+                          uint8_t* codes, float* scales, uint16_t* rope,
+                          int64_t cap, int64_t entry_begin,
+                          const float* norm_w, float eps, const float* inv_freq)
 {
     int dn = d - d_rope, ng = dn / g;
     double worst = 0.0;
@@ -304,10 +412,10 @@ double oracle_compress(const uint16_t* x, const uint16_t* gate, int64_t x_seq_st
                 if (dev > worst) worst = dev;
             }
             int64_t e = entry_begin + jj;
-            oracle_quant_entry(y, d, d_rope, g,
-                               codes + ((size_t)b * cap + e) * dn,
-                               scales + ((size_t)b * cap + e) * ng,
-                               rope + ((size_t)b * cap + e) * d_rope);
+            quant_entry_ex(y, d, d_rope, g, norm_w, eps, inv_freq, e * m,
+                           codes + ((size_t)b * cap + e) * dn,
+                           scales + ((size_t)b * cap + e) * ng,
+                           rope + ((size_t)b * cap + e) * d_rope);
         }
         free(y); free(y64); free(mag);
     }
@@ -464,11 +572,42 @@ void oracle_topk(const float* scores, const int32_t* q_pos, int R, int64_t Nc_ca
  * All in fp64.  out [H][d] fp64, lse [H] fp64 (natural-log log-sum-exp of
  * the scaled logits), either may be NULL.  With no keys at all, o = 0 and
  * lse = -inf. */
+void oracle_attend_ex(const uint16_t* q, int H, int d, int d_rope, int g,
+                      const uint8_t* codes, const float* scales, const uint16_t* rope,
+                      const int64_t* ent, int64_t n_ent,
+                      const uint16_t* win, int64_t n_win,
+                      float softmax_scale, const float* q_norm_w, float eps, const float* sink,
+                      const float* inv_freq, int64_t q_pos, double* out, double* lse);
+
 void oracle_attend(const uint16_t* q, int H, int d, int d_rope, int g,
                    const uint8_t* codes, const float* scales, const uint16_t* rope,
                    const int64_t* ent, int64_t n_ent,
                    const uint16_t* win, int64_t n_win,
                    float softmax_scale, double* out, double* lse)
+{
+    oracle_attend_ex(q, H, d, d_rope, g, codes, scales, rope, ent, n_ent, win, n_win, softmax_scale,
+                     NULL, 0.0f, NULL, NULL, 0, out, lse);
+}
+
+/* oracle_attend with the [N9] extras, all in fp64 (each may be NULL):
+ *   q_norm_w [d]  : each query head is RMS-normalised, q / sqrt(mean(q^2) +
+ *                   eps) * w, before the logits;
+ *   inv_freq      : the query's RoPE dims are rotated to its position q_pos
+ *                   (the keys carry their own positions already, as stored),
+ *                   and the output's RoPE dims are rotated back by -q_pos, so
+ *                   that the output, a mix of position-rotated values, carries
+ *                   relative positions;
+ *   sink [H]      : a per-head logit in the softmax denominator with no value:
+ *                   p_j = exp(l_j) / (sum_i exp(l_i) + exp(sink_h)), so the
+ *                   attention mass can be below 1.
+ * lse includes the sink; with no keys the output is 0 and lse = sink (or
+ * -inf without one). */
+void oracle_attend_ex(const uint16_t* q, int H, int d, int d_rope, int g,
+                      const uint8_t* codes, const float* scales, const uint16_t* rope,
+                      const int64_t* ent, int64_t n_ent,
+                      const uint16_t* win, int64_t n_win,
+                      float softmax_scale, const float* q_norm_w, float eps, const float* sink,
+                      const float* inv_freq, int64_t q_pos, double* out, double* lse)
 {
     const int dn = d - d_rope, ng = dn / g;
     const int64_t n = n_ent + n_win;
@@ -488,28 +627,38 @@ void oracle_attend(const uint16_t* q, int H, int d, int d_rope, int g,
     #pragma omp parallel
     {
     double* logit = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    double* qv = (double*)malloc(sizeof(double) * (size_t)d);
+    double* ov = (double*)malloc(sizeof(double) * (size_t)d);
     #pragma omp for schedule(static)
     for (int h = 0; h < H; ++h) {
         const uint16_t* qh = q + (size_t)h * d;
-        double mx = -INFINITY;
+        for (int c = 0; c < d; ++c) qv[c] = (double)oracle_bf16_to_f32(qh[c]);
+        if (q_norm_w) {
+            double ss = 0.0;
+            for (int c = 0; c < d; ++c) ss += qv[c] * qv[c];
+            const double r = sqrt(ss / d + (double)eps);
+            for (int c = 0; c < d; ++c) qv[c] = qv[c] / r * (double)q_norm_w[c];
+        }
+        if (inv_freq) oracle_rope_f64(qv + dn, d_rope, q_pos, inv_freq, +1, qv + dn);
+        double mx = sink ? (double)sink[h] : -INFINITY;
         for (int64_t j = 0; j < n; ++j) {
             double s = 0.0;
-            for (int c = 0; c < d; ++c) s += (double)oracle_bf16_to_f32(qh[c]) * K[(size_t)j * d + c];
+            for (int c = 0; c < d; ++c) s += qv[c] * K[(size_t)j * d + c];
             logit[j] = (double)softmax_scale * s;
             if (logit[j] > mx) mx = logit[j];
         }
-        double den = 0.0;
+        double den = sink ? exp((double)sink[h] - mx) : 0.0;
         for (int64_t j = 0; j < n; ++j) { logit[j] = exp(logit[j] - mx); den += logit[j]; }
-        if (out) {
-            for (int c = 0; c < d; ++c) {
-                double o = 0.0;
-                for (int64_t j = 0; j < n; ++j) o += logit[j] * K[(size_t)j * d + c];
-                out[(size_t)h * d + c] = n > 0 ? o / den : 0.0;
-            }
+        for (int c = 0; c < d; ++c) {
+            double o = 0.0;
+            for (int64_t j = 0; j < n; ++j) o += logit[j] * K[(size_t)j * d + c];
+            ov[c] = n > 0 ? o / den : 0.0;
         }
-        if (lse) lse[h] = n > 0 ? mx + log(den) : -INFINITY;
+        if (inv_freq) oracle_rope_f64(ov + dn, d_rope, q_pos, inv_freq, -1, ov + dn);
+        if (out) for (int c = 0; c < d; ++c) out[(size_t)h * d + c] = ov[c];
+        if (lse) lse[h] = (n > 0 || sink) ? mx + log(den) : -INFINITY;
     }
-    free(logit);
+    free(logit); free(qv); free(ov);
     }
     free(K);
 }
