@@ -121,8 +121,21 @@ def lib():
             L.oracle_token_prep.restype = None
             L.oracle_compress_ex.argtypes = [u16p, u16p, ctypes.c_int64, fp, ctypes.c_int, ctypes.c_int,
                                              ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, u8p, fp, u16p,
-                                             ctypes.c_int64, ctypes.c_int64, fp, ctypes.c_float, fp]
+                                             ctypes.c_int64, ctypes.c_int64, fp, ctypes.c_float, fp, ctypes.c_int64]
             L.oracle_compress_ex.restype = ctypes.c_double
+            L.oracle_f32_to_e2m1.argtypes = [ctypes.c_float]
+            L.oracle_f32_to_e2m1.restype = ctypes.c_uint8
+            L.oracle_fp4_quant_block.argtypes = [fp, u8p, u8p]
+            L.oracle_fp4_quant_block.restype = None
+            L.oracle_compress_overlap.argtypes = [u16p, u16p, u16p, u16p, u16p, u16p, ctypes.c_int64, fp,
+                                                  ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int,
+                                                  ctypes.c_int, ctypes.c_int, u8p, fp, u16p, ctypes.c_int64,
+                                                  ctypes.c_int64]
+            L.oracle_compress_overlap.restype = ctypes.c_double
+            L.oracle_index_key_compress.argtypes = [u16p, u16p, u16p, u16p, u16p, u16p, ctypes.c_int64, fp,
+                                                    ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int, u8p,
+                                                    u8p, ctypes.c_int64, ctypes.c_int64]
+            L.oracle_index_key_compress.restype = None
             _lib = L
     return _lib
 
@@ -218,12 +231,13 @@ def _opt(a, dtype, ct):
 
 
 def compress(x_bits, gate_bits, bias, m, n_blocks, d_rope, g, cap=None, entry_begin=0,
-             norm_w=None, eps=1e-6, inv_freq=None):
+             norm_w=None, eps=1e-6, inv_freq=None, pos_entry0=-1):
     """Pool + quantise n_blocks entries for each sequence.
     x_bits, gate_bits: [B][T][d] bf16 bits whose row 0 is the first token of
     block ``entry_begin``.  norm_w [d] / inv_freq [d_rope/2] (optional): the
     note's section 9 entry RMSNorm and partial RoPE (entry e at position e*m)
-    before storage.  Returns (codes [B][cap][dn], scales [B][cap][dn/g],
+    before storage; pos_entry0 >= 0 places the first pooled block at entry
+    index pos_entry0 for RoPE.  Returns (codes [B][cap][dn], scales [B][cap][dn/g],
     rope [B][cap][d_rope], worst fp32-vs-fp64 relative deviation)."""
     x_bits, gate_bits, bias = _c(x_bits, np.uint16), _c(gate_bits, np.uint16), _c(bias, np.float32)
     nw, nw_p = _opt(norm_w, np.float32, ctypes.c_float)
@@ -238,7 +252,8 @@ def compress(x_bits, gate_bits, bias, m, n_blocks, d_rope, g, cap=None, entry_be
     worst = lib().oracle_compress_ex(_ptr(x_bits, ctypes.c_uint16), _ptr(gate_bits, ctypes.c_uint16), T,
                                      _ptr(bias, ctypes.c_float), m, B, n_blocks, d, d_rope, g,
                                      _ptr(codes, ctypes.c_uint8), _ptr(scales, ctypes.c_float),
-                                     _ptr(rope, ctypes.c_uint16), cap, entry_begin, nw_p, float(eps), fq_p)
+                                     _ptr(rope, ctypes.c_uint16), cap, entry_begin, nw_p, float(eps), fq_p,
+                                     int(pos_entry0))
     return codes, scales, rope, worst
 
 
@@ -373,4 +388,73 @@ def causal_keys(p: int, m: int, W: int, n_cap: int = None):
         e = 0
     first = max(0, p - W + 1)
     return np.arange(max(e, 0)), first, p + 1
+
+
+# ---------------------------------------------------------------- overlapped compressor (section 7)
+def f32_to_e2m1(v) -> int:
+    """e2m1 code of one fp32 value: nearest-even, saturating at +-6, sign kept."""
+    return int(lib().oracle_f32_to_e2m1(float(np.float32(v))))
+
+
+def fp4_quant_block(v):
+    """One 32-element block -> (16 code bytes, ue8m0 byte): the OCP MX rule
+    X = floor(log2 amax) - 2, codes e2m1(v / 2^X)."""
+    v = _c(v, np.float32)
+    assert v.shape == (32,)
+    codes = np.empty(16, np.uint8)
+    sf = np.empty(1, np.uint8)
+    lib().oracle_fp4_quant_block(_ptr(v, ctypes.c_float), _ptr(codes, ctypes.c_uint8), _ptr(sf, ctypes.c_uint8))
+    return codes, int(sf[0])
+
+
+def _overlap_args(xa, za, xb, zb, a_prev, za_prev):
+    xa, za, xb, zb = (_c(a, np.uint16) for a in (xa, za, xb, zb))
+    ap = zp = None
+    if a_prev is not None:
+        ap, zp = _c(a_prev, np.uint16), _c(za_prev, np.uint16)
+    return xa, za, xb, zb, ap, zp
+
+
+def compress_overlap(xa, za, xb, zb, bias, m, n_blocks, d_rope, g, a_prev=None, za_prev=None, cap=None,
+                     entry_begin=0):
+    """The note's overlapped CSA compressor (section 7, two streams, 2m-token
+    windows; reading in oracle.c): entry entry_begin+j pools block j-1 of
+    stream a and block j of stream b (rows from row 0 = block entry_begin;
+    a_prev / za_prev [B][>=m][d]: stream a's block before it, or None).
+    bias [2m][d].  Returns (codes, scales, rope, worst fp32-vs-fp64 deviation)."""
+    xa, za, xb, zb, ap, zp = _overlap_args(xa, za, xb, zb, a_prev, za_prev)
+    bias = _c(bias, np.float32)
+    B, T, d = xb.shape
+    assert xa.shape == xb.shape and n_blocks * m <= T and bias.shape == (2 * m, d)
+    assert ap is None or ap.shape[1] == T
+    cap = entry_begin + n_blocks if cap is None else cap
+    dn = d - d_rope
+    codes = np.zeros((B, cap, dn), np.uint8)
+    scales = np.zeros((B, cap, dn // g), np.float32)
+    rope = np.zeros((B, cap, d_rope), np.uint16)
+    u16 = lambda a: None if a is None else _ptr(a, ctypes.c_uint16)
+    worst = lib().oracle_compress_overlap(u16(xa), u16(za), u16(xb), u16(zb), u16(ap), u16(zp), T,
+                                          _ptr(bias, ctypes.c_float), m, B, n_blocks, d, d_rope, g,
+                                          _ptr(codes, ctypes.c_uint8), _ptr(scales, ctypes.c_float),
+                                          _ptr(rope, ctypes.c_uint16), cap, entry_begin)
+    return codes, scales, rope, worst
+
+
+def index_key_compress(xa, za, xb, zb, bias, m, n_blocks, a_prev=None, za_prev=None, cap=None, entry_begin=0):
+    """Indexer keys K^IComp (note section 7): the overlapped compressor over
+    c-channel indexer-key streams, stored FP4 (e2m1 + ue8m0 per 32).
+    Returns (k_codes [B][cap][c/2], k_sf [B][cap][c/32])."""
+    xa, za, xb, zb, ap, zp = _overlap_args(xa, za, xb, zb, a_prev, za_prev)
+    bias = _c(bias, np.float32)
+    B, T, c = xb.shape
+    assert n_blocks * m <= T and bias.shape == (2 * m, c) and c % 32 == 0
+    assert ap is None or ap.shape[1] == T
+    cap = entry_begin + n_blocks if cap is None else cap
+    kc = np.zeros((B, cap, c // 2), np.uint8)
+    ks = np.zeros((B, cap, c // 32), np.uint8)
+    u16 = lambda a: None if a is None else _ptr(a, ctypes.c_uint16)
+    lib().oracle_index_key_compress(u16(xa), u16(za), u16(xb), u16(zb), u16(ap), u16(zp), T,
+                                    _ptr(bias, ctypes.c_float), m, B, n_blocks, c, _ptr(kc, ctypes.c_uint8),
+                                    _ptr(ks, ctypes.c_uint8), cap, entry_begin)
+    return kc, ks
 

@@ -370,7 +370,7 @@ double oracle_compress_ex(const uint16_t* x, const uint16_t* gate, int64_t x_seq
                           int d, int d_rope, int g,
                           uint8_t* codes, float* scales, uint16_t* rope,
                           int64_t cap, int64_t entry_begin,
-                          const float* norm_w, float eps, const float* inv_freq);
+                          const float* norm_w, float eps, const float* inv_freq, int64_t pos_entry0);
 
 double oracle_compress(const uint16_t* x, const uint16_t* gate, int64_t x_seq_stride,
                        const float* bias, int m, int B, int64_t n_blocks,
@@ -379,20 +379,24 @@ double oracle_compress(const uint16_t* x, const uint16_t* gate, int64_t x_seq_st
                        int64_t cap, int64_t entry_begin)
 {
     return oracle_compress_ex(x, gate, x_seq_stride, bias, m, B, n_blocks, d, d_rope, g, codes, scales, rope,
-                              cap, entry_begin, NULL, 0.0f, NULL);
+                              cap, entry_begin, NULL, 0.0f, NULL, -1);
 }
 
 /* oracle_compress with the [N9] extras: each pooled entry is RMS-normalised
  * (norm_w [d], eps) before storage and its RoPE dims rotated to the entry's
  * position, taken as the position of its block's first token, e * m
- * (inv_freq [d_rope/2]); either may be NULL. */
+ * (inv_freq [d_rope/2]); either may be NULL.  pos_entry0: the entry index
+ * whose position the first pooled block takes (-1: entry_begin; a test that
+ * pools one block of a long sequence into a one-entry buffer passes the
+ * block's real index). */
 double oracle_compress_ex(const uint16_t* x, const uint16_t* gate, int64_t x_seq_stride,
                           const float* bias, int m, int B, int64_t n_blocks,
                           int d, int d_rope, int g,
                           uint8_t* codes, float* scales, uint16_t* rope,
                           int64_t cap, int64_t entry_begin,
-                          const float* norm_w, float eps, const float* inv_freq)
+                          const float* norm_w, float eps, const float* inv_freq, int64_t pos_entry0)
 {
+    const int64_t e_pos0 = pos_entry0 >= 0 ? pos_entry0 : entry_begin;
     int dn = d - d_rope, ng = dn / g;
     double worst = 0.0;
     #pragma omp parallel reduction(max:worst)
@@ -412,7 +416,7 @@ double oracle_compress_ex(const uint16_t* x, const uint16_t* gate, int64_t x_seq
                 if (dev > worst) worst = dev;
             }
             int64_t e = entry_begin + jj;
-            quant_entry_ex(y, d, d_rope, g, norm_w, eps, inv_freq, e * m,
+            quant_entry_ex(y, d, d_rope, g, norm_w, eps, inv_freq, (e_pos0 + jj) * m,
                            codes + ((size_t)b * cap + e) * dn,
                            scales + ((size_t)b * cap + e) * ng,
                            rope + ((size_t)b * cap + e) * d_rope);
@@ -420,6 +424,197 @@ double oracle_compress_ex(const uint16_t* x, const uint16_t* gate, int64_t x_seq
         free(y); free(y64); free(mag);
     }
     return worst;
+}
+
+/* ------------------------------------------------------------------ */
+/* (1b) Overlapped CSA compressor and indexer-key compressor  [N7]      */
+/* ------------------------------------------------------------------ */
+/* [N7] gives CSA two KV streams C_a = H W_a, C_b = H W_b and two gate streams
+ * Z_a, Z_b, and builds each compressed entry from 2m adjacent entries with
+ * row-wise softmax weights, neighbouring entries' sources overlapping.
+ * Reading (the note gives no index formula): entry i pools the m tokens of
+ * block i-1 from stream a and the m tokens of block i from stream b, one
+ * softmax per channel over those 2m tokens, with a positional bias of 2m
+ * rows (rows 0..m-1 for the a-half, m..2m-1 for the b-half).  Each token
+ * thus feeds two entries: entry i through stream b and entry i+1 through
+ * stream a.  Entry 0 has no previous block: its a-half is absent.  The
+ * arithmetic is the fp32 sequence of oracle_pool_block over the 2m tokens in
+ * that order (a-half ascending, then b-half ascending).
+ * The indexer keys K^IComp_s of [N7] come from the same compressor applied to
+ * the indexer-key streams (c channels), then FP4 storage ([N9]: the indexer
+ * is FP4): per 32-element block, the OCP MX rule for e2m1: shared exponent
+ * X = floor(log2 amax) - 2 (2 = the exponent of e2m1's largest value 6),
+ * stored as the ue8m0 byte X + 127 (clamped to 0..254; amax = 0 gives 0),
+ * element codes = e2m1(v / 2^X), round to nearest even, saturating at +-6,
+ * sign kept. */
+
+/* Pool n token rows (xr[i], gr[i]: d bf16 values each; br[i]: d fp32 bias). */
+static void pool_rows(const uint16_t* const* xr, const uint16_t* const* gr, const float* const* br,
+                      int n, int d, float* y, double* y64, double* mag64)
+{
+    for (int c = 0; c < d; ++c) {
+        float zmax = -INFINITY;
+        for (int i = 0; i < n; ++i) {
+            float z = oracle_bf16_to_f32(gr[i][c]) + br[i][c];
+            if (z > zmax) zmax = z;
+        }
+        float S = 0.0f, N = 0.0f;
+        for (int i = 0; i < n; ++i) {
+            float z = oracle_bf16_to_f32(gr[i][c]) + br[i][c];
+            float e = oracle_exp_neg(z - zmax);
+            float xv = oracle_bf16_to_f32(xr[i][c]);
+            S = S + e;
+            float prod = e * xv;
+            N = N + prod;
+        }
+        y[c] = N / S;
+        if (y64) {
+            double zm = -INFINITY, s = 0.0, nn = 0.0, a = 0.0;
+            for (int i = 0; i < n; ++i) {
+                double z = (double)oracle_bf16_to_f32(gr[i][c]) + (double)br[i][c];
+                if (z > zm) zm = z;
+            }
+            for (int i = 0; i < n; ++i) {
+                double z = (double)oracle_bf16_to_f32(gr[i][c]) + (double)br[i][c];
+                double e = exp(z - zm);
+                s += e;
+                nn += e * (double)oracle_bf16_to_f32(xr[i][c]);
+                a += e * fabs((double)oracle_bf16_to_f32(xr[i][c]));
+            }
+            y64[c] = nn / s;
+            if (mag64) mag64[c] = a / s;
+        }
+    }
+}
+
+/* Overlapped pooling of entry jj of sequence b (see above) into y (fp32 d)
+ * and y64 (fp64 cross-check, may be NULL).
+ *   xa, za, xb, zb : [B][x_seq_stride][d] bf16; row 0 = first token of block
+ *                    entry_begin, so the b-half of entry entry_begin+jj is rows
+ *                    jj*m .. jj*m+m-1 of xb/zb and, for jj >= 1, its a-half is
+ *                    rows (jj-1)*m .. jj*m-1 of xa/za
+ *   a_prev, za_prev: [B][x_seq_stride][d], rows 0..m-1 = the a-stream of the
+ *                    block before entry_begin (the first entry's a-half); NULL:
+ *                    the first entry has no a-half (entry_begin = 0) */
+static void pool_overlap_entry(const uint16_t* xa, const uint16_t* za, const uint16_t* xb, const uint16_t* zb,
+                               const uint16_t* a_prev, const uint16_t* za_prev, int64_t x_seq_stride,
+                               const float* bias, int m, int d, int b, int64_t jj, float* y, double* y64,
+                               double* mag64)
+{
+    const uint16_t* xr[512];
+    const uint16_t* gr[512];
+    const float* br[512];
+    int n = 0;
+    const size_t seq = (size_t)b * x_seq_stride;
+    const uint16_t* ax = NULL; const uint16_t* az = NULL;
+    if (jj >= 1) { ax = xa + (seq + (size_t)(jj - 1) * m) * d; az = za + (seq + (size_t)(jj - 1) * m) * d; }
+    else if (a_prev) { ax = a_prev + seq * d; az = za_prev + seq * d; }
+    if (ax)
+        for (int i = 0; i < m; ++i) { xr[n] = ax + (size_t)i * d; gr[n] = az + (size_t)i * d; br[n] = bias + (size_t)i * d; ++n; }
+    for (int i = 0; i < m; ++i) {
+        xr[n] = xb + (seq + (size_t)jj * m + i) * d;
+        gr[n] = zb + (seq + (size_t)jj * m + i) * d;
+        br[n] = bias + (size_t)(m + i) * d;
+        ++n;
+    }
+    pool_rows(xr, gr, br, n, d, y, y64, mag64);
+}
+
+/* fp32 -> e2m1 code (4 bits): round to nearest even, saturating at +-6, the
+ * sign kept (so -0 and small negatives give 0x8). */
+uint8_t oracle_f32_to_e2m1(float v)
+{
+    static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    const uint8_t sign = signbit(v) ? 0x8 : 0x0;
+    double a = fabs((double)v);
+    if (isnan(a)) return 0x7;
+    if (a >= 6.0) return (uint8_t)(sign | 0x7);
+    int best = 0;
+    for (int k = 1; k < 8; ++k) {
+        const double dk = fabs(a - mag[k]), db = fabs(a - mag[best]);
+        if (dk < db || (dk == db && (k & 1) == 0)) best = k;   /* ties: even code (mantissa bit 0) */
+    }
+    return (uint8_t)(sign | best);
+}
+
+/* One 32-element block: the ue8m0 byte and 16 code bytes (element 2i in the
+ * low nibble of byte i). */
+void oracle_fp4_quant_block(const float* v, uint8_t* codes, uint8_t* sf)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < 32; ++i) if (fabsf(v[i]) > amax) amax = fabsf(v[i]);
+    int X = -127;
+    if (amax > 0.0f) {
+        int e;
+        frexp((double)amax, &e);                 /* amax = f 2^e, f in [0.5, 1): floor(log2 amax) = e - 1 */
+        X = (e - 1) - 2;
+        if (X < -127) X = -127;
+        if (X > 127) X = 127;
+    }
+    *sf = (uint8_t)(X + 127);
+    for (int i = 0; i < 16; ++i) {
+        const uint8_t lo = oracle_f32_to_e2m1((float)ldexp((double)v[2 * i], -X));
+        const uint8_t hi = oracle_f32_to_e2m1((float)ldexp((double)v[2 * i + 1], -X));
+        codes[i] = (uint8_t)(lo | (hi << 4));
+    }
+}
+
+/* Overlapped CSA compression of n_blocks entries per sequence (FP8/BF16 entry
+ * storage as oracle_quant_entry); returns the worst fp32-vs-fp64 deviation. */
+double oracle_compress_overlap(const uint16_t* xa, const uint16_t* za, const uint16_t* xb, const uint16_t* zb,
+                               const uint16_t* a_prev, const uint16_t* za_prev, int64_t x_seq_stride,
+                               const float* bias, int m, int B, int64_t n_blocks, int d, int d_rope, int g,
+                               uint8_t* codes, float* scales, uint16_t* rope, int64_t cap, int64_t entry_begin)
+{
+    const int dn = d - d_rope, ng = dn / g;
+    double worst = 0.0;
+    #pragma omp parallel reduction(max:worst)
+    {
+        float* y = (float*)malloc(sizeof(float) * d);
+        double* y64 = (double*)malloc(sizeof(double) * d);
+        double* mag = (double*)malloc(sizeof(double) * d);
+        #pragma omp for schedule(static)
+        for (int64_t be = 0; be < (int64_t)B * n_blocks; ++be) {
+            const int b = (int)(be / n_blocks);
+            const int64_t jj = be % n_blocks;
+            pool_overlap_entry(xa, za, xb, zb, a_prev, za_prev, x_seq_stride, bias, m, d, b, jj, y, y64, mag);
+            for (int c = 0; c < d; ++c) {
+                double den = mag[c] > 1e-30 ? mag[c] : 1e-30;
+                double dev = fabs((double)y[c] - y64[c]) / den;
+                if (dev > worst) worst = dev;
+            }
+            const int64_t e = entry_begin + jj;
+            oracle_quant_entry(y, d, d_rope, g, codes + ((size_t)b * cap + e) * dn,
+                               scales + ((size_t)b * cap + e) * ng, rope + ((size_t)b * cap + e) * d_rope);
+        }
+        free(y); free(y64); free(mag);
+    }
+    return worst;
+}
+
+/* Indexer keys K^IComp: the overlapped compressor over c-channel indexer-key
+ * streams, then FP4 (e2m1 + ue8m0 per 32).  k_codes [B][cap][c/2], k_sf
+ * [B][cap][c/32]. */
+void oracle_index_key_compress(const uint16_t* xa, const uint16_t* za, const uint16_t* xb, const uint16_t* zb,
+                               const uint16_t* a_prev, const uint16_t* za_prev, int64_t x_seq_stride,
+                               const float* bias, int m, int B, int64_t n_blocks, int c,
+                               uint8_t* k_codes, uint8_t* k_sf, int64_t cap, int64_t entry_begin)
+{
+    #pragma omp parallel
+    {
+        float* y = (float*)malloc(sizeof(float) * c);
+        #pragma omp for schedule(static)
+        for (int64_t be = 0; be < (int64_t)B * n_blocks; ++be) {
+            const int b = (int)(be / n_blocks);
+            const int64_t jj = be % n_blocks;
+            pool_overlap_entry(xa, za, xb, zb, a_prev, za_prev, x_seq_stride, bias, m, c, b, jj, y, NULL, NULL);
+            const int64_t e = entry_begin + jj;
+            for (int blk = 0; blk < c / 32; ++blk)
+                oracle_fp4_quant_block(y + blk * 32, k_codes + ((size_t)b * cap + e) * (c / 2) + blk * 16,
+                                       k_sf + ((size_t)b * cap + e) * (c / 32) + blk);
+        }
+        free(y);
+    }
 }
 
 /* ------------------------------------------------------------------ */
