@@ -353,7 +353,8 @@ def bench_decode(args, wl, world, rank, pg):
     for r in range(n_rep):
         dw = build_decode(wl)
         runner = DecodeRunner(dw.layers, wl.B, wl.H, wl.k, wl.t, wl.softmax_scale, schedule=args.schedule,
-                              dense_budget=args.dense_budget)
+                              dense_budget=args.dense_budget, sparse_budget=args.sparse_budget,
+                              index_budget=args.index_budget)
         reps.append((dw, runner))
     main = torch.cuda.current_stream()
 
@@ -471,8 +472,38 @@ def bench_decode(args, wl, world, rank, pg):
     f1.record()
     torch.cuda.synchronize()
     barrier(pg)
-    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / n_e2e, pg)
+    e2e_py_ms = max_over_ranks(f0.elapsed_time(f1) / n_e2e, pg)
     del g_e2e
+
+    # the same step through the C ABI's host-to-host call (hca_decode_step_host:
+    # the library issues the copies and the kernels on two streams), as one graph
+    plan = runner.capi_plan(d_q, d_iq)
+
+    def e2e_step_capi():
+        runner.step_host_capi(plan, h_q, h_iq, h_out)
+
+    s_cap = torch.cuda.Stream()
+    s_cap.wait_stream(main)
+    with torch.cuda.stream(s_cap):
+        e2e_step_capi()
+    main.wait_stream(s_cap)
+    torch.cuda.synchronize()
+    g_capi = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_capi):
+        e2e_step_capi()
+    for _ in range(3):
+        g_capi.replay()
+    torch.cuda.synchronize()
+    barrier(pg)
+    torch.cuda.synchronize()
+    f0.record()
+    for _ in range(n_e2e):
+        g_capi.replay()
+    f1.record()
+    torch.cuda.synchronize()
+    barrier(pg)
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / n_e2e, pg)
+    del g_capi
 
     # ---------------- roofline of the dominant kernel
     # Each candidate kernel alone: one graph launches it once per replica (inputs
@@ -546,8 +577,10 @@ def bench_decode(args, wl, world, rank, pg):
         "roofline": roof,
         "clocks": clocks.summary(t_wall0, t_wall1),
         "e2e": {"value": world * wl.B / (e2e_ms * 1e-3), "unit": "query-tok/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "how": "DecodeRunner.step_host (pinned host inputs in, outputs out, "
-                "copies overlapped with the kernels) captured as one CUDA graph and replayed",
+                "d2h_bytes_per_step": d2h, "how": "hca_decode_step_host (the C ABI's host-to-host decode step: "
+                "pinned host queries in, pinned host outputs out, copies and kernels queued by the library on two "
+                "streams) captured as one CUDA graph and replayed",
+                "python_step_host_value": world * wl.B / (e2e_py_ms * 1e-3),
                 "eager_value": world * wl.B / (e2e_eager_ms * 1e-3)},
         "gpu_launches": reps[0][1].kernels_per_step * args.steps,
     }
@@ -822,6 +855,83 @@ def bench_stack(args, wl, world, rank, pg):
         print(json.dumps(line), flush=True)
 
 
+def bench_select_variants(args, wl, rank):
+    """The note's indexer variants on the decode workload's shapes: 4 or 64
+    indexer heads (section 7 parameters: n_h^I = 64), fp32 or BF16 index
+    scores (section 9: the top-k selector on BF16 scores, reported 2x faster
+    at 99.7% KV recall).  Times the fused index + top-k call alone (one CUDA
+    graph over 4 rotating replicas of the keys and queries, CUDA events), and
+    measures the recall of the BF16 top-k sets against the exact fp32 ones."""
+    import dataclasses
+    import long_context_attention_hca_b200 as hca
+    dev = torch.device("cuda")
+    T = wl.t + 1
+    nc = T // 4
+    n_rep = 4
+    out = {"metric": "decode index + top-k variants", "unit": "us", "config": {"workload": wl.name, "B": wl.B,
+           "entries": nc, "k": wl.k}, "variants": {}, "recall_bf16_vs_fp32": {}}
+    pos = torch.full((wl.B,), wl.t, dtype=torch.int32, device=dev)
+    sets = {}
+    for Hi in (4, 64):
+        w2 = dataclasses.replace(wl, Hi=Hi)
+        reps = []
+        for r in range(n_rep):
+            kc, ks = inp.indexer_keys(w2, wl.B, nc, layer=100 + r, device=dev)
+            qc, qs, w = inp.indexer_queries(w2, wl.B, layer=100 + r, device=dev)
+            reps.append((qc.view(wl.B, 1, Hi, -1), qs.view(wl.B, 1, Hi, -1), w.view(wl.B, 1, Hi), kc, ks))
+        for bf in (False, True):
+            sdt = torch.bfloat16 if bf else torch.float32
+            bufs = []
+            for (qc, qs, w, kc, ks) in reps:
+                need = hca.topk_workspace_size(wl.B, nc, wl.k, bf)
+                bufs.append((torch.empty((wl.B, 1, nc), dtype=sdt, device=dev),
+                             torch.empty((wl.B, wl.k), dtype=torch.int32, device=dev),
+                             torch.empty((wl.B,), dtype=torch.int32, device=dev),
+                             torch.empty(max(need, 16), dtype=torch.uint8, device=dev)))
+
+            def run(st):
+                for (qc, qs, w, kc, ks), (sc, idx, cnt, ws) in zip(reps, bufs):
+                    hca.lightning_index_topk(qc, qs, w, kc, ks, pos, 4, wl.k, scores=sc, idx=idx, count=cnt, ws=ws,
+                                             stream=st, score_bf16=bf)
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(s):
+                run(s)
+                s.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=s):
+                    run(s)
+                for _ in range(3):
+                    g.replay()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                n_it = 20
+                a.record(s)
+                for _ in range(n_it):
+                    g.replay()
+                b.record(s)
+                s.synchronize()
+            us = a.elapsed_time(b) * 1e3 / (n_it * n_rep)
+            key = f"h{Hi}_{'bf16' if bf else 'fp32'}"
+            out["variants"][key] = {"us": us, "key_bytes": wl.B * nc * 68, "gbs": wl.B * nc * 68 / (us * 1e-6) / 1e9}
+            sets[key] = [set_rows(buf[1]) for buf in bufs]
+            del g
+        rec = []
+        for r in range(n_rep):
+            for a_, b_ in zip(sets[f"h{Hi}_fp32"][r], sets[f"h{Hi}_bf16"][r]):
+                rec.append(len(a_ & b_) / max(len(a_), 1))
+        out["recall_bf16_vs_fp32"][f"h{Hi}"] = {"mean": sum(rec) / len(rec), "min": min(rec), "rows": len(rec)}
+        out["variants"][f"h{Hi}_bf16"]["speedup_vs_fp32"] = (out["variants"][f"h{Hi}_fp32"]["us"] /
+                                                             out["variants"][f"h{Hi}_bf16"]["us"])
+    out["pages"] = "BF16 index scores: 2x faster top-k, 99.7% KV recall (note section 9; trained model, no workload given)"
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def set_rows(idx):
+    h = idx.to("cpu").numpy()
+    return [set(int(v) for v in row if v >= 0) for row in h]
+
+
 def cpu_baseline(wl):
     """The oracle on the host cores: one query token of the workload (see
     oracle_decode_sample), at all cores and at one thread."""
@@ -861,6 +971,11 @@ def main():
     ap.add_argument("--schedule", default="after_index", choices=["after_index", "hca_first"],
                     help="decode step: HCA after the indexer, or HCA first on a CTA budget")
     ap.add_argument("--dense-budget", type=int, default=0, help="CTA cap of the dense decode attention (0: none)")
+    ap.add_argument("--sparse-budget", type=int, default=0, help="CTA cap of the sparse decode attention (0: none)")
+    ap.add_argument("--index-budget", type=int, default=0, help="CTA cap of the fused decode indexer (0: none)")
+    ap.add_argument("--select-variants", action="store_true",
+                    help="time the fused index + top-k with 4 / 64 indexer heads and fp32 / BF16 scores, and the "
+                         "recall of BF16 top-k sets (decode workloads)")
     args = ap.parse_args()
     wl = inp.WORKLOADS[args.workload]
     world, rank, local, pg = dist_setup(args.gpus)
@@ -870,7 +985,9 @@ def main():
         if pg is not None:
             pg.destroy_process_group()
         return
-    if wl.prefill:
+    if args.select_variants:
+        bench_select_variants(args, wl, rank)
+    elif wl.prefill:
         bench_prefill(args, wl, world, rank, pg)
     elif wl.layers > 1:
         bench_stack(args, wl, world, rank, pg)

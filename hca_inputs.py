@@ -155,3 +155,28 @@ def indexer_keys(wl: Workload, B: int, n: int, layer=0, device="cpu"):
     kc = uniform_bytes((B, n, wl.c // 2), wl.seed, "ik", layer, device)
     ks = ue8m0_scales((B, n, wl.c // 32), wl.seed, "iks", layer, device)
     return kc, ks
+
+
+# ------------------------------------------------------------------ section 9 extras (parameters, not arithmetic)
+NORM_EPS = 1e-6
+ROPE_BASE = 10000.0
+
+
+def rope_inv_freq(d_rope: int, base: float = ROPE_BASE, device="cpu"):
+    """RoPE frequency table fp32 [d_rope/2]: base^(-2i/d_rope), rounded to fp32
+    (the usual rotary table; the pages fix no base)."""
+    import numpy as np
+    f = (base ** (-np.arange(0, d_rope, 2, dtype=np.float64) / d_rope)).astype(np.float32)
+    return torch.from_numpy(f).to(device)
+
+
+def section9_params(wl: Workload, layer=0, device="cpu"):
+    """Learned-parameter stand-ins for the note's section 9 extras: KV-entry
+    and query RMSNorm weights ~ 1 + N(0, 0.1) fp32 [d], per-head sink logits
+    ~ N(0, 1) fp32 [H], and the RoPE table."""
+    kvw = 1.0 + normal_f32((wl.d,), 0.1, wl.seed, "kv_norm_w", layer, device)
+    qw = 1.0 + normal_f32((wl.d,), 0.1, wl.seed, "q_norm_w", layer, device)
+    sink = normal_f32((wl.H,), 1.0, wl.seed, "sink", layer, device)
+    return {"kv_norm_w": kvw, "q_norm_w": qw, "sink": sink, "inv_freq": rope_inv_freq(wl.d_rope, device=device),
+            "eps": NORM_EPS}
+

@@ -16,7 +16,7 @@ from typing import Callable, List, Optional
 import torch
 
 import hca_inputs as inp
-from long_context_attention_hca_b200 import KVCache, csa_compress, hca_compress
+from long_context_attention_hca_b200 import AttnExtras, EntryExtras, KVCache, csa_compress, hca_compress, kv_token_prep
 from long_context_attention_hca_b200.pipeline import (CSA_RATIO, HCA_RATIO, DecodeLayer, PrefillState,
                                                        pro_layer_ratios)
 
@@ -28,21 +28,29 @@ class DecodeWorkload:
     ratios: List[int]
     q: List[torch.Tensor]                 # per layer [B][H][d] bf16
     iq: List[Optional[tuple]]             # per CSA layer (codes [B][1][Hi][c/2], sf, w [B][1][Hi])
+    extras: Optional[List[AttnExtras]] = None     # per layer, section 9 extras of the attention call
+    s9: Optional[List[dict]] = None               # per layer, the section 9 parameters (hca_inputs)
+    raw_window: Optional[List[torch.Tensor]] = None   # per layer, the window before token preparation
 
 
-def _compress(ratio, x, gate, bias, cache, n_blocks):
-    (csa_compress if ratio == CSA_RATIO else hca_compress)(x, gate, bias, n_blocks, cache)
+def _compress(ratio, x, gate, bias, cache, n_blocks, extras=None):
+    (csa_compress if ratio == CSA_RATIO else hca_compress)(x, gate, bias, n_blocks, cache, extras=extras)
 
 
-def build_decode(wl: inp.Workload, device="cuda", on_raw: Optional[Callable] = None) -> DecodeWorkload:
+def build_decode(wl: inp.Workload, device="cuda", on_raw: Optional[Callable] = None,
+                 section9: bool = False) -> DecodeWorkload:
     """Decode state at position wl.t: every sequence holds tokens 0..t (t+1
     tokens, all blocks complete).  Single-layer workloads pair one CSA and one
     HCA path over the same raw KV (each with its own positional bias); the
-    stack workload has independent inputs per layer."""
+    stack workload has independent inputs per layer.  section9: the note's
+    section 9 extras are on: entries RMS-normalised and rotated when stored,
+    window tokens prepared likewise, and the attention calls take the query
+    RMSNorm, RoPE and sink (parameters from hca_inputs.section9_params)."""
     B, T, layout = wl.B, wl.t + 1, (wl.d, wl.d_rope, wl.g)
     stack = wl.layers > 1
     ratios = pro_layer_ratios(wl.layers) if stack else [CSA_RATIO, HCA_RATIO]
     layers, q, iq = [], [], []
+    extras, s9s, raw_windows = [], [], []
     x = gate = None
     for li, r in enumerate(ratios):
         raw_layer = li if stack else 0
@@ -53,10 +61,19 @@ def build_decode(wl: inp.Workload, device="cuda", on_raw: Optional[Callable] = N
         bias = inp.pos_bias(wl, r, layer=li if stack else 0, device=device)
         n_ent = T // r
         cache = KVCache(B, n_ent, layout, device=device)
-        _compress(r, x, gate, bias, cache, n_ent)
+        s9 = inp.section9_params(wl, layer=li if stack else 0, device=device) if section9 else None
+        ee = EntryExtras(s9["kv_norm_w"], s9["eps"], s9["inv_freq"]) if section9 else None
+        _compress(r, x, gate, bias, cache, n_ent, ee)
         if on_raw is not None:
             on_raw(li, r, x, gate, bias)
         window = x[:, T - wl.W:T].contiguous()
+        if section9:
+            raw_windows.append(window)
+            pos = torch.arange(T - wl.W, T, dtype=torch.int32, device=device).repeat(B)
+            window = kv_token_prep(window.view(B * wl.W, wl.d), pos, layout, ee).view(B, wl.W, wl.d)
+            s9s.append(s9)
+            extras.append(AttnExtras(s9["q_norm_w"], s9["eps"], s9["sink"], s9["inv_freq"],
+                                     torch.full((B,), wl.t, dtype=torch.int32, device=device)))
         kc = ks = None
         if r == CSA_RATIO:
             kc, ks = inp.indexer_keys(wl, B, n_ent, layer=li, device=device)
@@ -72,6 +89,8 @@ def build_decode(wl: inp.Workload, device="cuda", on_raw: Optional[Callable] = N
     x = gate = None
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
+    if section9:
+        return DecodeWorkload(wl, layers, ratios, q, iq, extras, s9s, raw_windows)
     return DecodeWorkload(wl, layers, ratios, q, iq)
 
 
@@ -86,11 +105,15 @@ class PrefillWorkload:
     iq: tuple                             # ([1][Tq][Hi][c/2], sf, [1][Tq][Hi])
     x_all: Optional[torch.Tensor] = None  # kept when keep_raw=True (tests)
     gate_all: Optional[torch.Tensor] = None
+    s9: Optional[dict] = None             # section 9 parameters when on
+    raw_window_unprepared: Optional[torch.Tensor] = None
 
 
-def build_prefill(wl: inp.Workload, device="cuda", keep_raw=False) -> PrefillWorkload:
+def build_prefill(wl: inp.Workload, device="cuda", keep_raw=False, section9: bool = False) -> PrefillWorkload:
     """One sequence with p0 = wl.t cached tokens already compressed into both
-    caches, and the next Tq tokens (the chunk) still raw."""
+    caches, and the next Tq tokens (the chunk) still raw.  section9: entries
+    and window tokens stored with the note's section 9 extras (the state
+    holds the parameters; PrefillRunner takes the attention extras)."""
     p0, Tq, layout = wl.t, wl.Tq, (wl.d, wl.d_rope, wl.g)
     T = p0 + Tq
     x, gate = inp.raw_kv(wl, 1, T, device=device)
@@ -98,17 +121,25 @@ def build_prefill(wl: inp.Workload, device="cuda", keep_raw=False) -> PrefillWor
     b128 = inp.pos_bias(wl, HCA_RATIO, device=device)
     csa = KVCache(1, T // CSA_RATIO, layout, device=device, zero=True)
     hca = KVCache(1, T // HCA_RATIO, layout, device=device, zero=True)
-    csa_compress(x, gate, b4, p0 // CSA_RATIO, csa)
-    hca_compress(x, gate, b128, p0 // HCA_RATIO, hca)
+    s9 = inp.section9_params(wl, device=device) if section9 else None
+    ee = EntryExtras(s9["kv_norm_w"], s9["eps"], s9["inv_freq"]) if section9 else None
+    csa_compress(x, gate, b4, p0 // CSA_RATIO, csa, extras=ee)
+    hca_compress(x, gate, b128, p0 // HCA_RATIO, hca, extras=ee)
     kc, ks = inp.indexer_keys(wl, 1, T // CSA_RATIO, device=device)
-    st = PrefillState(csa, hca, kc, ks, b4, b128)
+    st = PrefillState(csa, hca, kc, ks, b4, b128, ee)
     raw_chunk = x[:, p0:T].contiguous()
     gate_chunk = gate[:, p0:T].contiguous()
     raw_window = x[0, p0 - (wl.W - 1):T].contiguous()
+    raw_unprepared = None
+    if section9:
+        raw_unprepared = raw_window
+        pos = torch.arange(p0 - (wl.W - 1), T, dtype=torch.int32, device=device)
+        raw_window = kv_token_prep(raw_window, pos, layout, ee)
     q = inp.queries(wl, Tq, device=device)
     qc, qs, w = inp.indexer_queries(wl, Tq, device=device)
     iq = (qc.view(1, Tq, wl.Hi, wl.c // 2), qs.view(1, Tq, wl.Hi, wl.c // 32), w.view(1, Tq, wl.Hi))
-    pw = PrefillWorkload(wl, st, raw_chunk, gate_chunk, raw_window, q, iq)
+    pw = PrefillWorkload(wl, st, raw_chunk, gate_chunk, raw_window, q, iq, s9=s9,
+                         raw_window_unprepared=raw_unprepared)
     if keep_raw:
         pw.x_all, pw.gate_all = x, gate
     torch.cuda.synchronize()

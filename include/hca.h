@@ -89,18 +89,21 @@ int hca_last_cuda_error(void);
 int hca_take_device_error(void);
 
 /* Launch budget: a scheduling knob with no counterpart on the pages.  It
- * caps the CTAs (splits x sequences) of one decode attention launch on the
- * tensor-core path (d = 512, H = 64) so that
- * the launch occupies only part of the device and another stream's kernels
- * (the CSA chain: indexer, top-k, sparse attention) run beside it.
- *   op        HCA_BUDGET_DENSE_DECODE or HCA_BUDGET_SPARSE_DECODE
- *   max_ctas  > 0: at most max(max_ctas, B) CTAs; 0: the default (one CTA
- *             per SM at most)
+ * caps the CTAs of one decode launch so that the launch occupies only part
+ * of the device and another stream's kernels run beside it:
+ *   HCA_BUDGET_DENSE_DECODE / HCA_BUDGET_SPARSE_DECODE: the CTAs (splits x
+ *             sequences) of a decode attention launch on the tensor-core path
+ *             (d = 512, H = 64), at most max(max_ctas, B);
+ *   HCA_BUDGET_DECODE_INDEX: the CTAs of the fused decode indexer
+ *             (lightning_index_topk on the tensor pipe), at most
+ *             max(max_ctas, B), two per SM by default.
+ *   max_ctas  > 0: the cap; 0: the default
  * Process-wide; applies to workspace sizing and launches made after the
  * call, so size workspaces after setting it.  Returns the previous value,
  * or -1 for an unknown op or a negative max_ctas. */
 #define HCA_BUDGET_DENSE_DECODE 0
 #define HCA_BUDGET_SPARSE_DECODE 1
+#define HCA_BUDGET_DECODE_INDEX 2
 int hca_set_launch_budget(int op, int max_ctas);
 
 /* ------------------------------------------------------------------ */
@@ -138,6 +141,92 @@ int hca_compress(const uint16_t* x, const uint16_t* gate, int64_t x_seq_stride,
                  void* stream);
 
 /* ------------------------------------------------------------------ */
+/* Section 9 extras of the stored vectors: KV entry RMSNorm and partial  */
+/* RoPE.                                                                 */
+/* ------------------------------------------------------------------ */
+/* "DeepSeek V4 ..." note, section 9: every compressed KV entry (and query
+ * head) is RMS-normalised before core attention, and RoPE is applied to the
+ * last d_rope dims of the query, the KV entry and the attention output.
+ *   norm_w    fp32 [d]: RMSNorm weight, or NULL for no RMSNorm
+ *   norm_eps  RMSNorm epsilon
+ *   inv_freq  fp32 [d_rope/2]: RoPE frequencies (pair i = dims 2i, 2i+1 of
+ *             the RoPE dims, rotated by position * inv_freq[i]), or NULL for
+ *             no RoPE
+ * Arithmetic (fixed so stored codes stay bit-exact): the squares are rounded
+ * and summed as a pairwise tree over consecutive channel pairs, r =
+ * sqrt(sum / d + eps) correctly rounded, y = (y / r) * w in fp32.  RoPE:
+ * the angle position * inv_freq[i] in fp64 (exact), the rotation
+ * (a cos - b sin, a sin + b cos) in fp64 with every product and sum rounded,
+ * then one rounding to bf16.  A compressed entry e of ratio m sits at
+ * position e * m (its block's first token). */
+typedef struct {
+    const float* norm_w;
+    float norm_eps;
+    const float* inv_freq;
+} hca_entry_extras;
+
+/* csa_compress / hca_compress with the extras: the pooled entry is
+ * normalised, then stored (FP8 dims as above; RoPE dims rotated to the
+ * entry's position).  ex == NULL or all-NULL members: identical to the
+ * plain calls. */
+int csa_compress_ex(const uint16_t* x, const uint16_t* gate, int64_t x_seq_stride,
+                    const float* pos_bias, int32_t B, int64_t n_blocks,
+                    hca_kv_layout layout, hca_kv_cache out, int64_t entry_begin,
+                    const hca_entry_extras* ex, void* stream);
+int hca_compress_ex(const uint16_t* x, const uint16_t* gate, int64_t x_seq_stride,
+                    const float* pos_bias, int32_t B, int64_t n_blocks,
+                    hca_kv_layout layout, hca_kv_cache out, int64_t entry_begin,
+                    const hca_entry_extras* ex, void* stream);
+
+/* ------------------------------------------------------------------ */
+/* The note's overlapped CSA compressor and the indexer-key compressor   */
+/* (section 7: two KV streams C_a = H W_a^KV, C_b = H W_b^KV and two gate */
+/* streams Z_a, Z_b; each compressed entry pools 2m adjacent entries     */
+/* with row-wise softmax weights, neighbouring entries overlapping; the  */
+/* indexer keys K^IComp_s come from a compressor too, stored FP4).       */
+/* ------------------------------------------------------------------ */
+/* Reading (the note gives no index formula): entry i pools the m = 4
+ * tokens of block i-1 from stream a and the 4 tokens of block i from stream
+ * b, one softmax per channel over those 8 tokens with a positional bias of
+ * 8 rows (rows 0..3 for the a-half, 4..7 for the b-half); each token feeds
+ * entry i through stream b and entry i+1 through stream a.
+ *   xa, za, xb, zb  bf16 [B][x_seq_stride][d]: row 0 = first token of block
+ *                   entry_begin; the b-half of entry entry_begin+j is rows
+ *                   4j..4j+3 of xb/zb and, for j >= 1, its a-half rows
+ *                   4(j-1)..4j-1 of xa/za
+ *   a_prev, za_prev bf16 [B][x_seq_stride][d], rows 0..3: stream a's block
+ *                   before entry_begin (the first entry's a-half), or both
+ *                   NULL: the first entry has no a-half (entry_begin = 0)
+ *   pos_bias        fp32 [8][d]
+ * Arithmetic: as csa_compress over the 8 tokens in the order a-half
+ * ascending, b-half ascending; storage as csa_compress.  Requires
+ * 4 * n_blocks <= x_seq_stride and entry_begin + n_blocks <= capacity. */
+int csa_compress_overlap(const uint16_t* xa, const uint16_t* za, const uint16_t* xb, const uint16_t* zb,
+                         const uint16_t* a_prev, const uint16_t* za_prev, int64_t x_seq_stride,
+                         const float* pos_bias, int32_t B, int64_t n_blocks, hca_kv_layout layout,
+                         hca_kv_cache out, int64_t entry_begin, void* stream);
+/* Indexer keys: the same overlapped pooling over c-channel indexer-key
+ * streams (c = 64 or 128), stored FP4 as lightning_index reads them:
+ * k_codes uint8 [B][capacity][c/2] (element 2i in the low nibble), k_sf
+ * uint8 [B][capacity][c/32] ue8m0.  Per 32-element block (the OCP MX rule
+ * for e2m1): X = floor(log2 amax) - 2, clamped to [-127, 127] (amax = 0 or
+ * below 2^-126: -127), byte X + 127, codes e2m1(v * 2^-X) rounded to nearest
+ * even, saturating at +-6, the sign kept. */
+int indexer_key_compress(const uint16_t* xa, const uint16_t* za, const uint16_t* xb, const uint16_t* zb,
+                         const uint16_t* a_prev, const uint16_t* za_prev, int64_t x_seq_stride,
+                         const float* pos_bias, int32_t B, int64_t n_blocks, int32_t c,
+                         uint8_t* k_codes, uint8_t* k_sf, int64_t capacity, int64_t entry_begin, void* stream);
+
+/* Raw tokens prepared for the sliding window (the state cache keeps them in
+ * this form): RMSNorm and partial RoPE at each token's position, every
+ * channel stored bf16 (non-RoPE dims rounded from fp32, RoPE dims from fp64).
+ *   x    bf16 [n][d]; pos int32 [n] token positions; out bf16 [n][d] (may
+ *        not overlap x)
+ * Supported layouts: as the cache layouts above. */
+int kv_token_prep(const uint16_t* x, const int32_t* pos, int64_t n, hca_kv_layout layout,
+                  const hca_entry_extras* ex, uint16_t* out, void* stream);
+
+/* ------------------------------------------------------------------ */
 /* Lightning indexer (section 7, eq. I_{t,s}; section 9: FP4).          */
 /* ------------------------------------------------------------------ */
 /*   q_codes  uint8 [B][Tq][Hi][c/2]  FP4 e2m1, element 2i in the low nibble
@@ -155,11 +244,21 @@ int hca_compress(const uint16_t* x, const uint16_t* gate, int64_t x_seq_stride,
  *         exact FP4 dot product.
  * score = fp32, from +0, for h = 0..Hi-1 in order: score += w_h * ReLU(dot_h)
  *         (product rounded, then sum rounded).
- * Supported: c in {64, 128}, 1 <= Hi <= 8, m >= 1. */
+ * Supported: c in {64, 128}, 1 <= Hi <= 8, or Hi = 64 (the note's
+ * n_h^I = 64, section 7 parameters) with c = 128; m >= 1. */
 int lightning_index(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
                     const uint8_t* k_codes, const uint8_t* k_sf, const int32_t* q_pos,
                     int32_t B, int32_t Tq, int64_t Nc_cap, int32_t Hi, int32_t c, int32_t m,
                     float* scores, void* stream);
+/* lightning_index with the note's BF16 index scores (section 9: the top-k
+ * selector's index scores in BF16 instead of FP32): score_bf16 != 0 writes
+ * each score rounded to bf16 (nearest even) into scores as uint16 bit patterns
+ * [B][Tq][Nc_cap] (-inf for ineligible entries); score_bf16 = 0 is
+ * lightning_index (scores fp32).  BF16 scores: c = 128 and Hi in {4, 64}. */
+int lightning_index_ex(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
+                       const uint8_t* k_codes, const uint8_t* k_sf, const int32_t* q_pos,
+                       int32_t B, int32_t Tq, int64_t Nc_cap, int32_t Hi, int32_t c, int32_t m,
+                       int32_t score_bf16, void* scores, void* stream);
 
 /* ------------------------------------------------------------------ */
 /* Top-k selection (section 7: C^SprsComp_t = {C_s | I_{t,s} in Top-k}) */
@@ -178,8 +277,9 @@ int lightning_index(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
  * needs none), 256-byte aligned, owned by the caller, contents need not be
  * initialised and are clobbered.  Few long rows (R * ceil(Nc_cap / 16384)
  * <= the device's SM count, Nc_cap >= 8192) and rows longer than 2^19 scores
- * go through histogram passes
- * spread over the whole device and use it; otherwise a row is split over a
+ * go through histogram passes (the keys above the threshold bin and the
+ * candidates in it gathered by one kernel over the whole device, whose last
+ * CTA per row resolves the exact threshold and writes the row) and use it; otherwise a row is split over a
  * thread-block cluster of up to 16 blocks of at most 32768 scores each
  * (Nc_cap <= 2^19) and the workspace is ignored.  A row longer than 2^19
  * scores without an adequate workspace returns HCA_ERR_WORKSPACE. */
@@ -187,6 +287,15 @@ size_t topk_select_workspace_size(int32_t R, int64_t Nc_cap, int32_t k);
 int topk_select(const float* scores, const int32_t* q_pos, int32_t R, int64_t Nc_cap,
                 int32_t m, int32_t k, int32_t* idx, int32_t* count,
                 void* ws, size_t ws_bytes, void* stream);
+/* topk_select over BF16 scores (score_bf16 != 0: scores are bf16 bit
+ * patterns, uint16 [R][Nc_cap]; values compare as the bf16 values, the same
+ * total order, ties to the lower index), or over fp32 scores (score_bf16 = 0:
+ * topk_select).  BF16 rows always take the histogram passes: a workspace of
+ * topk_select_ex_workspace_size(R, Nc_cap, k, 1) bytes (256-byte aligned) is
+ * required, and Nc_cap >= 1. */
+size_t topk_select_ex_workspace_size(int32_t R, int64_t Nc_cap, int32_t k, int32_t score_bf16);
+int topk_select_ex(const void* scores, int32_t score_bf16, const int32_t* q_pos, int32_t R, int64_t Nc_cap,
+                   int32_t m, int32_t k, int32_t* idx, int32_t* count, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------ */
 /* Fused decode selection: lightning_index (Tq = 1) then topk_select.   */
@@ -207,6 +316,17 @@ int lightning_index_topk(const uint8_t* q_codes, const uint8_t* q_sf, const floa
                          int32_t B, int64_t Nc_cap, int32_t Hi, int32_t c, int32_t m, int32_t k,
                          float* scores, int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
                          void* index_done, void* stream);
+/* lightning_index_topk with BF16 scores (score_bf16 != 0; scores uint16 bf16
+ * bits, see lightning_index_ex and topk_select_ex) or fp32 scores
+ * (score_bf16 = 0).  Hi may be 64 with c = 128 (fused on the tensor pipe).
+ * Workspace: lightning_index_topk_ex_workspace_size(B, Nc_cap, k, score_bf16)
+ * bytes, required with BF16 scores. */
+size_t lightning_index_topk_ex_workspace_size(int32_t B, int64_t Nc_cap, int32_t k, int32_t score_bf16);
+int lightning_index_topk_ex(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
+                            const uint8_t* k_codes, const uint8_t* k_sf, const int32_t* q_pos,
+                            int32_t B, int64_t Nc_cap, int32_t Hi, int32_t c, int32_t m, int32_t k,
+                            int32_t score_bf16, void* scores, int32_t* idx, int32_t* count, void* ws,
+                            size_t ws_bytes, void* index_done, void* stream);
 
 /* ------------------------------------------------------------------ */
 /* Core attention (section 7: shared key-value MQA + sliding window;    */
@@ -294,6 +414,126 @@ int compressed_attn_prefill(const uint16_t* q, int32_t Tq, int32_t H, int32_t p0
                             const uint16_t* raw, int32_t W,
                             float softmax_scale, uint16_t* out,
                             void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ */
+/* Core attention with the section 9 extras.                            */
+/* ------------------------------------------------------------------ */
+/* "DeepSeek V4 ..." note, section 9: query-head RMSNorm, partial RoPE on the
+ * query and the output, and a learnable sink logit per head that lets the
+ * attention mass be below 1.
+ *   q_norm_w  fp32 [d]: RMSNorm weight of every query head (fp32 arithmetic),
+ *             or NULL
+ *   norm_eps  its epsilon
+ *   sink      fp32 [H]: per-head sink logit, on the scale of the scaled
+ *             logits (natural log): p_j = e^{l_j} / (sum_i e^{l_i} + e^{sink}),
+ *             or NULL
+ *   inv_freq  fp32 [d_rope/2] (as hca_entry_extras), or NULL: the query's
+ *             RoPE dims are rotated to its position before the logits and the
+ *             output's RoPE dims rotated back by it (the keys carry their own
+ *             positions, as stored)
+ *   q_pos     int32 [B]: decode only, the position of each sequence's query
+ *             (required with inv_freq); prefill queries sit at p0 + i
+ * lse (decode) includes the sink.  ex == NULL or all-NULL members: identical
+ * to the plain calls. */
+typedef struct {
+    const float* q_norm_w;
+    float norm_eps;
+    const float* sink;
+    const float* inv_freq;
+    const int32_t* q_pos;
+    const int32_t* win_len;  /* decode: [B] valid window rows, each <= W (the
+                                state cache's window before it is full: rows
+                                0 .. win_len-1 hold the tokens); NULL: all W */
+} hca_attn_extras;
+
+int compressed_attn_decode_ex(const uint16_t* q, int32_t B, int32_t H,
+                              hca_kv_layout layout, hca_kv_cache kv,
+                              const int32_t* idx, int32_t idx_stride,
+                              const int32_t* n_comp, int32_t max_comp,
+                              const uint16_t* window, int32_t W,
+                              float softmax_scale, const hca_attn_extras* ex,
+                              uint16_t* out, float* lse,
+                              void* ws, size_t ws_bytes, void* stream);
+int compressed_attn_prefill_ex(const uint16_t* q, int32_t Tq, int32_t H, int32_t p0, int32_t m,
+                               hca_kv_layout layout, hca_kv_cache kv,
+                               const int32_t* idx, int32_t idx_stride, const int32_t* count,
+                               const uint16_t* raw, int32_t W,
+                               float softmax_scale, const hca_attn_extras* ex, uint16_t* out,
+                               void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ */
+/* State cache of the decode loop (section 11: a fixed-size state per     */
+/* sequence holds the recent sliding-window KV entries and the            */
+/* uncompressed tail of the CSA/HCA block not yet complete).             */
+/* ------------------------------------------------------------------ */
+/* Appends one token per sequence at position pos (the same for all B):
+ *   x, gate   bf16 [B][d]: the token's raw KV and gate logits
+ *   window    bf16 [B][W][d]: ring buffer, the token goes to row pos % W
+ *             (win_x, if not NULL, bf16 [B][d], is written there instead of
+ *             x: the token as prepared for attention, see kv_token_prep)
+ *   tail_x, tail_gate  bf16 [B][m][d]: the current block's tokens, row pos % m
+ *             (skipped when m == 0 or tail_x is NULL)
+ * Once the token ends a block ((pos+1) % m == 0), tail_x / tail_gate hold
+ * that block's m tokens in order and csa_compress / hca_compress(tail_x,
+ * tail_gate, m, ..., n_blocks = 1, entry_begin = (pos+1)/m - 1) pools it. */
+int kv_state_append(const uint16_t* x, const uint16_t* gate, const uint16_t* win_x, int32_t B, int32_t d,
+                    int64_t pos, uint16_t* window, int32_t W, uint16_t* tail_x, uint16_t* tail_gate,
+                    int32_t m, void* stream);
+
+/* ------------------------------------------------------------------ */
+/* One decode step from host memory to host memory (sections 7 and 8:    */
+/* the CSA path and the HCA path of one decode position).               */
+/* ------------------------------------------------------------------ */
+/* Device state and buffers of the step, all owned by the caller (device
+ * pointers unless stated): the CSA layer's cache, indexer keys and window,
+ * the HCA layer's cache, entry counts and window, staging buffers for the
+ * queries, the index scores, top-k outputs and workspaces, the outputs; and
+ * for the schedule a second stream and four events (cudaStream_t /
+ * cudaEvent_t as void*, created by the caller). */
+typedef struct {
+    int32_t B, H, Hi, c, k, W;
+    float softmax_scale;
+    hca_kv_layout layout;
+    hca_kv_cache csa_cache;
+    int64_t csa_entries;          /* entries per sequence = indexer keys per sequence    */
+    const uint8_t* k_codes;       /* [B][csa_entries][c/2]                               */
+    const uint8_t* k_sf;          /* [B][csa_entries][c/32]                              */
+    const uint16_t* csa_window;   /* [B][W][d]                                           */
+    hca_kv_cache hca_cache;
+    const int32_t* hca_n;         /* [B] HCA entries per sequence                        */
+    int32_t hca_max;              /* host bound of hca_n                                 */
+    const uint16_t* hca_window;   /* [B][W][d]                                           */
+    const int32_t* q_pos;         /* [B] query position                                  */
+    uint16_t* q_csa;              /* [B][H][d] staging                                   */
+    uint16_t* q_hca;              /* [B][H][d] staging                                   */
+    uint8_t* iq_codes;            /* [B][Hi][c/2] staging                                */
+    uint8_t* iq_sf;               /* [B][Hi][c/32] staging                               */
+    float* iq_w;                  /* [B][Hi] staging                                     */
+    float* scores;                /* [B][csa_entries]                                    */
+    int32_t* idx;                 /* [B][k]                                              */
+    int32_t* count;               /* [B]                                                 */
+    void* topk_ws; size_t topk_ws_bytes;   /* lightning_index_topk_workspace_size        */
+    void* ws_csa; size_t ws_csa_bytes;     /* compressed_attn_decode_workspace_size      */
+    void* ws_hca; size_t ws_hca_bytes;
+    uint16_t* out_csa;            /* [B][H][d]                                           */
+    uint16_t* out_hca;            /* [B][H][d]                                           */
+    void* side_stream;
+    void* ev_fork; void* ev_index; void* ev_q; void* ev_join;
+} hca_decode_step_plan;
+
+/* Host queries in, host outputs out:
+ *   h_q_csa, h_q_hca  bf16 [B][H][d]; h_iq_codes [B][Hi][c/2], h_iq_sf
+ *   [B][Hi][c/32], h_iq_w fp32 [B][Hi]; h_out_csa, h_out_hca bf16 [B][H][d]
+ *   (host memory; pinned for asynchronous copies).
+ * Queues on `stream`: the indexer-query copies, lightning_index_topk, the
+ * CSA attention and its output copy; on the plan's side stream: the
+ * attention-query copies and, once the indexer has run, the HCA attention
+ * and its output copy.  `stream` finally waits for the side stream, so the
+ * outputs are in host memory when `stream` reaches that point.  Nothing is
+ * allocated; errors as the calls it makes. */
+int hca_decode_step_host(const hca_decode_step_plan* plan, const uint16_t* h_q_csa, const uint16_t* h_q_hca,
+                         const uint8_t* h_iq_codes, const uint8_t* h_iq_sf, const float* h_iq_w,
+                         uint16_t* h_out_csa, uint16_t* h_out_hca, void* stream);
 
 #ifdef __cplusplus
 }

@@ -49,7 +49,27 @@ struct Params {
     float* lse;                 // [units][H] or null
     float* part_o;              // [units][splits][HP][D]
     float* part_ml;             // [units][splits][2][HP]
+    // section 9 extras (each null when off)
+    const float* q_norm_w;      // [D] query-head RMSNorm weight
+    float norm_eps;
+    const float* sink;          // [H] sink logit per head (natural log)
+    const float* inv_freq;      // [d_rope/2] RoPE frequencies
+    const int32_t* q_pos;       // decode: [units] query positions
+    const int32_t* win_len;     // decode: [units] valid window rows (<= W), or null: W
 };
+
+constexpr float LOG2E = 1.4426950408889634f;
+
+__device__ __forceinline__ int64_t unit_pos(const Params& p, int64_t u) {
+    return p.prefill ? static_cast<int64_t>(p.p0) + u : (p.q_pos ? static_cast<int64_t>(p.q_pos[u]) : 0);
+}
+
+__device__ __forceinline__ void rope_cs(const float* inv_freq, int i, int64_t t, float& c, float& s) {
+    double sn, cs;
+    sincos(static_cast<double>(t) * static_cast<double>(__ldg(inv_freq + i)), &sn, &cs);
+    c = static_cast<float>(cs);
+    s = static_cast<float>(sn);
+}
 
 template <int D, int HP>
 struct Cfg {
@@ -103,6 +123,10 @@ __device__ __forceinline__ UnitKeys unit_keys(const Params& p, int64_t u, int D)
         k.kv_row0 = u * p.cap;
         k.wrow = p.win + static_cast<size_t>(u) * p.W * D;
         k.n_w = p.W;
+        if (p.win_len) {
+            const int wl = p.win_len[u];
+            k.n_w = wl < 0 ? 0 : (wl > p.W ? p.W : wl);
+        }
     } else {
         const int64_t pos = p.p0 + u;
         if (p.idx) {
@@ -198,6 +222,38 @@ attn_kernel(Params p) {
     const int t_begin = split * p.tiles_per_split;
     const int t_end = min(n_tiles, t_begin + p.tiles_per_split);
 
+    __shared__ float s_qr[HP];
+    __shared__ float s_cos[32], s_sin[32];
+    const bool q_extras = p.q_norm_w != nullptr || p.inv_freq != nullptr;
+    if (q_extras) {
+        // section 9 extras of the query: 1 / rms per head (partial sums of squares
+        // per 16-byte vector in the exchange buffer, free until the first tile),
+        // the RoPE table of the unit's position
+        if (p.inv_freq && tid < p.d_rope / 2) rope_cs(p.inv_freq, tid, unit_pos(p, u), s_cos[tid], s_sin[tid]);
+        if (p.q_norm_w) {
+            for (int w = tid; w < HP * (D / 8); w += C::NTHREADS) {
+                const int r = w / (D / 8), c = w % (D / 8);
+                float ss = 0.0f;
+                if (r < p.H) {
+                    const uint4 b = __ldg(reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(u) * p.H + r) * D + c * 8));
+                    const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float x0 = __uint_as_float(bw[i] << 16), x1 = __uint_as_float(bw[i] & 0xFFFF0000u);
+                        ss += x0 * x0 + x1 * x1;
+                    }
+                }
+                xs[w] = ss;
+            }
+            __syncthreads();
+            if (tid < HP) {
+                float ss = 0.0f;
+                for (int c = 0; c < D / 8; ++c) ss += xs[tid * (D / 8) + c];
+                s_qr[tid] = rsqrtf(ss / static_cast<float>(D) + p.norm_eps);
+            }
+        }
+        __syncthreads();
+    }
     // Q -> fp16 (rows >= H zero)
     for (int w = tid; w < HP * (D / 8); w += C::NTHREADS) {
         const int r = w / (D / 8), c = w % (D / 8);
@@ -205,10 +261,23 @@ attn_kernel(Params p) {
         if (r < p.H) {
             const uint4 b = __ldg(reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(u) * p.H + r) * D + c * 8));
             const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
-            uint32_t hw[4];
+            float f[8];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) hw[i] = pack_half2(__uint_as_float(bw[i] << 16), __uint_as_float(bw[i] & 0xFFFF0000u));
-            v = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            for (int i = 0; i < 4; ++i) { f[2 * i] = __uint_as_float(bw[i] << 16); f[2 * i + 1] = __uint_as_float(bw[i] & 0xFFFF0000u); }
+            if (p.q_norm_w) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) f[i] = f[i] * s_qr[r] * __ldg(p.q_norm_w + c * 8 + i);
+            }
+            if (p.inv_freq && c * 8 >= D - p.d_rope) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int pi = (c * 8 - (D - p.d_rope)) / 2 + i;
+                    const float a = f[2 * i], bb = f[2 * i + 1];
+                    f[2 * i] = a * s_cos[pi] - bb * s_sin[pi];
+                    f[2 * i + 1] = a * s_sin[pi] + bb * s_cos[pi];
+                }
+            }
+            v = make_uint4(pack_half2(f[0], f[1]), pack_half2(f[2], f[3]), pack_half2(f[4], f[5]), pack_half2(f[6], f[7]));
         }
         *reinterpret_cast<uint4*>(qs + swz<D>(r, c)) = v;
     }
@@ -333,24 +402,41 @@ attn_kernel(Params p) {
     const int h0 = hg * 16 + g8, h1 = h0 + 8;
     const size_t ou = static_cast<size_t>(u);
     if (p.n_splits == 1) {
-        const float inv0 = l_r[0] > 0.0f ? 1.0f / l_r[0] : 0.0f;
-        const float inv1 = l_r[1] > 0.0f ? 1.0f / l_r[1] : 0.0f;
+        // the sink joins the denominator (relative to the running max)
+        float lt[2] = {l_r[0], l_r[1]};
+        if (p.sink) {
+            if (lt[0] > 0.0f && h0 < p.H) lt[0] += exp2f(__ldg(p.sink + h0) * LOG2E - m_r[0]);
+            if (lt[1] > 0.0f && h1 < p.H) lt[1] += exp2f(__ldg(p.sink + h1) * LOG2E - m_r[1]);
+        }
+        const float inv0 = lt[0] > 0.0f ? 1.0f / lt[0] : 0.0f;
+        const float inv1 = lt[1] > 0.0f ? 1.0f / lt[1] : 0.0f;
 #pragma unroll
         for (int j = 0; j < C::NT_O; ++j) {
             const int col = half * C::DH + j * 8 + q4 * 2;
+            float v0 = o[j][0] * inv0, v1 = o[j][1] * inv0, v2 = o[j][2] * inv1, v3 = o[j][3] * inv1;
+            if (p.inv_freq && col >= D - p.d_rope) {
+                // RoPE dims: rotate the output back by the query's position
+                const int pi = (col - (D - p.d_rope)) / 2;
+                const float cs = s_cos[pi], sn = s_sin[pi];
+                const float a0 = v0 * cs + v1 * sn, a1 = v1 * cs - v0 * sn;
+                const float b0 = v2 * cs + v3 * sn, b1 = v3 * cs - v2 * sn;
+                v0 = a0; v1 = a1; v2 = b0; v3 = b1;
+            }
             if (h0 < p.H) {
-                __nv_bfloat162 v = __floats2bfloat162_rn(o[j][0] * inv0, o[j][1] * inv0);
+                __nv_bfloat162 v = __floats2bfloat162_rn(v0, v1);
                 *reinterpret_cast<__nv_bfloat162*>(p.out + (ou * p.H + h0) * D + col) = v;
             }
             if (h1 < p.H) {
-                __nv_bfloat162 v = __floats2bfloat162_rn(o[j][2] * inv1, o[j][3] * inv1);
+                __nv_bfloat162 v = __floats2bfloat162_rn(v2, v3);
                 *reinterpret_cast<__nv_bfloat162*>(p.out + (ou * p.H + h1) * D + col) = v;
             }
         }
         if (p.lse && half == 0 && q4 == 0) {
             const float ln2 = 0.69314718055994531f;
-            if (h0 < p.H) p.lse[ou * p.H + h0] = l_r[0] > 0.0f ? (m_r[0] + log2f(l_r[0])) * ln2 : -INFINITY;
-            if (h1 < p.H) p.lse[ou * p.H + h1] = l_r[1] > 0.0f ? (m_r[1] + log2f(l_r[1])) * ln2 : -INFINITY;
+            if (h0 < p.H)
+                p.lse[ou * p.H + h0] = lt[0] > 0.0f ? (m_r[0] + log2f(lt[0])) * ln2 : (p.sink ? __ldg(p.sink + h0) : -INFINITY);
+            if (h1 < p.H)
+                p.lse[ou * p.H + h1] = lt[1] > 0.0f ? (m_r[1] + log2f(lt[1])) * ln2 : (p.sink ? __ldg(p.sink + h1) : -INFINITY);
         }
     } else {
         const size_t ps = ou * p.n_splits + split;
@@ -390,15 +476,30 @@ __global__ void combine_kernel(Params p) {
         const float4 v = *reinterpret_cast<const float4*>(p.part_o + ((u * S + s) * HP + h) * static_cast<size_t>(D) + d0);
         acc[0] += wgt * v.x; acc[1] += wgt * v.y; acc[2] += wgt * v.z; acc[3] += wgt * v.w;
     }
+    const float sink = p.sink ? __ldg(p.sink + h) : -INFINITY;
+    if (p.sink && L > 0.0f) L += exp2f(sink * LOG2E - M);      // the sink joins the denominator
     const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-    __nv_bfloat162 a = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
-    __nv_bfloat162 b = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
+    float o[4] = {acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv};
+    if (p.inv_freq && d0 >= D - p.d_rope) {
+        // RoPE dims: rotate the output back by the query's position
+        const int64_t t = unit_pos(p, u);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            float cs, sn;
+            rope_cs(p.inv_freq, (d0 - (D - p.d_rope)) / 2 + i, t, cs, sn);
+            const float x = o[2 * i], y = o[2 * i + 1];
+            o[2 * i] = x * cs + y * sn;
+            o[2 * i + 1] = y * cs - x * sn;
+        }
+    }
+    __nv_bfloat162 a = __floats2bfloat162_rn(o[0], o[1]);
+    __nv_bfloat162 b = __floats2bfloat162_rn(o[2], o[3]);
     uint2 w;
     w.x = *reinterpret_cast<uint32_t*>(&a);
     w.y = *reinterpret_cast<uint32_t*>(&b);
     *reinterpret_cast<uint2*>(p.out + (static_cast<size_t>(u) * p.H + h) * D + d0) = w;
     if (p.lse && threadIdx.x == 0)
-        p.lse[u * p.H + h] = L > 0.0f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+        p.lse[u * p.H + h] = L > 0.0f ? (M + log2f(L)) * 0.69314718055994531f : sink;
 }
 
 }  // namespace attn
@@ -436,11 +537,21 @@ void tc_decode_plan(int B, int max_comp, int W, bool sparse, int& n_splits, int&
 size_t tc_decode_ws_bytes(int B, int max_comp, int W, bool sparse);
 int tc_attn_decode_launch(const uint16_t* q, int B, int H, const hca_kv_cache& kv, const int32_t* idx,
                           int idx_stride, const int32_t* n_comp, int max_comp, const uint16_t* window, int W,
-                          float softmax_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
-                          cudaStream_t st);
+                          float softmax_scale, const hca_attn_extras* ex, uint16_t* out, float* lse, void* ws,
+                          size_t ws_bytes, cudaStream_t st);
 int tc_attn_prefill_launch(const uint16_t* q, int Tq, int H, int p0, int m, const hca_kv_cache& kv,
                            const int32_t* idx, int idx_stride, const int32_t* count, const uint16_t* raw, int W,
-                           float softmax_scale, uint16_t* out, cudaStream_t st);
+                           float softmax_scale, const hca_attn_extras* ex, uint16_t* out, cudaStream_t st);
+
+static void set_extras(attn::Params& p, const hca_attn_extras* ex, bool decode) {
+    if (!ex) return;
+    p.q_norm_w = ex->q_norm_w;
+    p.norm_eps = ex->norm_eps;
+    p.sink = ex->sink;
+    p.inv_freq = ex->inv_freq;
+    p.q_pos = decode ? ex->q_pos : nullptr;
+    p.win_len = decode ? ex->win_len : nullptr;
+}
 static bool use_tc(int D, int H) { return D == 512 && H == 64; }
 
 // split-K plan shared by the workspace query and the launch
@@ -467,13 +578,14 @@ size_t decode_ws_bytes(int B, int H, int D, int max_comp, int W) {
 
 int attn_decode_launch(const uint16_t* q, int B, int H, const hca_kv_layout& L, const hca_kv_cache& kv,
                        const int32_t* idx, int idx_stride, const int32_t* n_comp, int max_comp,
-                       const uint16_t* window, int W, float softmax_scale, uint16_t* out, float* lse,
-                       void* ws, size_t ws_bytes, cudaStream_t st) {
+                       const uint16_t* window, int W, float softmax_scale, const hca_attn_extras* ex,
+                       uint16_t* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t st) {
     if (B == 0) return HCA_OK;
     if (use_tc(L.d, H))
-        return tc_attn_decode_launch(q, B, H, kv, idx, idx_stride, n_comp, max_comp, window, W, softmax_scale, out,
-                                     lse, ws, ws_bytes, st);
+        return tc_attn_decode_launch(q, B, H, kv, idx, idx_stride, n_comp, max_comp, window, W, softmax_scale, ex,
+                                     out, lse, ws, ws_bytes, st);
     attn::Params p = {};
+    set_extras(p, ex, true);
     p.q = q; p.H = H;
     p.codes = kv.codes; p.scales = kv.scales; p.rope = kv.rope; p.cap = kv.capacity;
     p.d_rope = L.d_rope; p.g = L.scale_group;
@@ -495,11 +607,14 @@ int attn_decode_launch(const uint16_t* q, int B, int H, const hca_kv_layout& L, 
 
 int attn_prefill_launch(const uint16_t* q, int Tq, int H, int p0, int m, const hca_kv_layout& L,
                         const hca_kv_cache& kv, const int32_t* idx, int idx_stride, const int32_t* count,
-                        const uint16_t* raw, int W, float softmax_scale, uint16_t* out, cudaStream_t st) {
+                        const uint16_t* raw, int W, float softmax_scale, const hca_attn_extras* ex, uint16_t* out,
+                        cudaStream_t st) {
     if (Tq == 0) return HCA_OK;
     if (use_tc(L.d, H))
-        return tc_attn_prefill_launch(q, Tq, H, p0, m, kv, idx, idx_stride, count, raw, W, softmax_scale, out, st);
+        return tc_attn_prefill_launch(q, Tq, H, p0, m, kv, idx, idx_stride, count, raw, W, softmax_scale, ex, out,
+                                      st);
     attn::Params p = {};
+    set_extras(p, ex, false);
     p.q = q; p.H = H;
     p.codes = kv.codes; p.scales = kv.scales; p.rope = kv.rope; p.cap = kv.capacity;
     p.d_rope = L.d_rope; p.g = L.scale_group;
@@ -582,5 +697,5 @@ extern "C" int compressed_attn_decode_noalloc(const uint16_t* q, int32_t B, int3
     void* scratch = noalloc_scratch_address(&st);
     if (st != HCA_OK) return st;
     return attn_decode_launch(q, B, H, layout, kv, idx, idx_stride, n_comp, max_comp, window, W, softmax_scale,
-                              out, lse, scratch, HCA_NOALLOC_SCRATCH_BYTES, as_stream(stream));
+                              nullptr, out, lse, scratch, HCA_NOALLOC_SCRATCH_BYTES, as_stream(stream));
 }

@@ -99,7 +99,30 @@ struct Params {
     float* lse;
     float* part_o;              // [units][splits][HP][D]
     float* part_ml;             // [units][splits][2][HP]
+    // section 9 extras (each null when off)
+    const float* q_norm_w;      // [D] query-head RMSNorm weight
+    float norm_eps;
+    const float* sink;          // [HP] sink logit per head (natural log)
+    const float* inv_freq;      // [32] RoPE frequencies of the 64 RoPE dims
+    const int32_t* q_pos;       // decode: [units] query positions
+    const int32_t* win_len;     // decode: [units] valid window rows (<= W), or null: W
 };
+
+constexpr int D_ROPE = 64;
+constexpr float LOG2E = 1.4426950408889634f;
+
+// Position of a unit's query token: its sequence's query (decode), p0 + unit (prefill).
+__device__ __forceinline__ int64_t unit_pos(const Params& p, int64_t u) {
+    return p.prefill ? static_cast<int64_t>(p.p0) + u : (p.q_pos ? static_cast<int64_t>(p.q_pos[u]) : 0);
+}
+
+// cos / sin of RoPE pair i at position t (fp64 angle t * f_i, exact; fp32 out)
+__device__ __forceinline__ void rope_cs(const float* inv_freq, int i, int64_t t, float& c, float& s) {
+    double sn, cs;
+    sincos(static_cast<double>(t) * static_cast<double>(__ldg(inv_freq + i)), &sn, &cs);
+    c = static_cast<float>(cs);
+    s = static_cast<float>(sn);
+}
 
 // ------------------------------------------------------------------ PTX wrappers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
@@ -209,6 +232,10 @@ __device__ __forceinline__ UnitKeys unit_keys(const Params& p, int64_t u) {
         k.kv_row0 = u * p.cap;
         k.wrow = p.win + static_cast<size_t>(u) * p.W * D;
         k.n_w = p.W;
+        if (p.win_len) {
+            const int wl = p.win_len[u];
+            k.n_w = wl < 0 ? 0 : (wl > p.W ? p.W : wl);
+        }
     } else {
         const int64_t pos = p.p0 + u;
         if (p.idx) {
@@ -249,6 +276,9 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     return false;
 }
 
+// EX: the section 9 extras are compiled in (query RMSNorm / RoPE, sink, output
+// RoPE); without them the kernel carries none of that code.
+template <bool EX>
 __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -257,6 +287,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
     __shared__ float s_alpha[HP], s_l[HP];
     __shared__ int s_resc_w[NSOFT];
     __shared__ volatile int s_abort;
+    __shared__ float s_qr[HP];                       // 1 / rms of each query head (query RMSNorm)
+    __shared__ float s_cos[D_ROPE / 2], s_sin[D_ROPE / 2];   // RoPE of the unit's position
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t u = blockIdx.x;
@@ -353,13 +385,79 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
                         ? __ldg(reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(u) * p.H + r) * D + c * 8))
                         : make_uint4(0, 0, 0, 0);
         }
+        if (!EX || (p.q_norm_w == nullptr && p.inv_freq == nullptr)) {
 #pragma unroll
-        for (int k = 0; k < QPT; ++k) {
-            const int w = tid + k * NTHREADS, r = w / (D / 8), c = w % (D / 8);
-            if (w < QV)
-                *reinterpret_cast<uint4*>(smem + Q_OFF + (c >> 3) * QBLK + sw128(r, c & 7)) =
-                    make_uint4(bf16x2_to_f16x2(qv[k].x), bf16x2_to_f16x2(qv[k].y), bf16x2_to_f16x2(qv[k].z),
-                               bf16x2_to_f16x2(qv[k].w));
+            for (int k = 0; k < QPT; ++k) {
+                const int w = tid + k * NTHREADS, r = w / (D / 8), c = w % (D / 8);
+                if (w < QV)
+                    *reinterpret_cast<uint4*>(smem + Q_OFF + (c >> 3) * QBLK + sw128(r, c & 7)) =
+                        make_uint4(bf16x2_to_f16x2(qv[k].x), bf16x2_to_f16x2(qv[k].y), bf16x2_to_f16x2(qv[k].z),
+                                   bf16x2_to_f16x2(qv[k].w));
+            }
+        } else {
+            // section 9 extras of the query, in fp32 before the fp16 store: each head
+            // RMS-normalised (partial sums of squares per 16-byte vector in the P
+            // buffers, free until the softmax), its RoPE dims rotated to the unit's
+            // position
+            const int64_t tpos = unit_pos(p, u);
+            if (p.inv_freq && tid < D_ROPE / 2) rope_cs(p.inv_freq, tid, tpos, s_cos[tid], s_sin[tid]);
+            if (p.q_norm_w) {
+                float* s_qss = reinterpret_cast<float*>(smem + P_OFF);       // [HP][D / 8]
+#pragma unroll
+                for (int k = 0; k < QPT; ++k) {
+                    const int w = tid + k * NTHREADS;
+                    if (w < QV) {
+                        const uint32_t v4[4] = {qv[k].x, qv[k].y, qv[k].z, qv[k].w};
+                        float ss = 0.0f;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float a = __uint_as_float(v4[i] << 16), b = __uint_as_float(v4[i] & 0xFFFF0000u);
+                            ss += a * a + b * b;
+                        }
+                        s_qss[w] = ss;
+                    }
+                }
+                __syncthreads();
+                if (tid < HP) {
+                    float ss = 0.0f;
+                    for (int c = 0; c < D / 8; ++c) ss += s_qss[tid * (D / 8) + c];
+                    s_qr[tid] = rsqrtf(ss / static_cast<float>(D) + p.norm_eps);
+                }
+            }
+            __syncthreads();
+#pragma unroll
+            for (int k = 0; k < QPT; ++k) {
+                const int w = tid + k * NTHREADS, r = w / (D / 8), c = w % (D / 8);
+                if (w < QV) {
+                    const uint32_t v4[4] = {qv[k].x, qv[k].y, qv[k].z, qv[k].w};
+                    float f[8];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        f[2 * i] = __uint_as_float(v4[i] << 16);
+                        f[2 * i + 1] = __uint_as_float(v4[i] & 0xFFFF0000u);
+                    }
+                    if (p.q_norm_w) {
+                        const float4 wa = __ldg(reinterpret_cast<const float4*>(p.q_norm_w + c * 8));
+                        const float4 wb = __ldg(reinterpret_cast<const float4*>(p.q_norm_w + c * 8) + 1);
+                        const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+                        const float rr = s_qr[r];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) f[i] = f[i] * rr * wv[i];
+                    }
+                    if (p.inv_freq && c * 8 >= D - D_ROPE) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int pi = (c * 8 - (D - D_ROPE)) / 2 + i;
+                            const float a = f[2 * i], b = f[2 * i + 1], cs = s_cos[pi], sn = s_sin[pi];
+                            f[2 * i] = a * cs - b * sn;
+                            f[2 * i + 1] = a * sn + b * cs;
+                        }
+                    }
+                    *reinterpret_cast<uint4*>(smem + Q_OFF + (c >> 3) * QBLK + sw128(r, c & 7)) =
+                        make_uint4(pack_half2(f[0], f[1]), pack_half2(f[2], f[3]), pack_half2(f[4], f[5]),
+                                   pack_half2(f[6], f[7]));
+                }
+            }
         }
     }
     fence_async_smem();
@@ -571,7 +669,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
             fence_after();
         }
         const bool hrow = lane < 16;
-        if (hrow) s_l[h] = l_run;
+        // the sink joins the denominator (relative to this split's running max)
+        const float sink_l2 = (EX && p.sink) ? __ldg(p.sink + h) * LOG2E : -INFINITY;
+        const float l_tot = (EX && p.sink && n_tiles > 0) ? l_run + ex2(sink_l2 - m_used) : l_run;
+        if (hrow) s_l[h] = p.n_splits == 1 ? l_tot : l_run;
         named_bar(1, NSOFT * 32);
         const int L = warp * 32 + lane;              // output dim within each M-tile
         const size_t uo = static_cast<size_t>(u);
@@ -587,21 +688,37 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
                         TMEM_LD16(lane_base + O_COL + mt * HP + c0, o, 0);
                         tmem_wait_ld();
                     }
+                    float v[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float l = s_l[c0 + j];
+                        v[j] = (n_tiles > 0 && l > 0.0f) ? __uint_as_float(o[j]) / l : 0.0f;
+                    }
+                    if (EX && p.inv_freq && mt == 3) {
+                        // RoPE dims (448..511, warps 2 and 3): rotate back by the query's position;
+                        // the pair partner is the neighbouring lane
+                        const bool rot = dim >= D - D_ROPE;
+                        const int pi = (dim - (D - D_ROPE)) >> 1;
+                        const float cs = rot ? s_cos[pi] : 1.0f, sn = rot ? s_sin[pi] : 0.0f;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float pv = __shfl_xor_sync(0xffffffffu, v[j], 1);
+                            if (rot) v[j] = (dim & 1) ? v[j] * cs - pv * sn : v[j] * cs + pv * sn;
+                        }
+                    }
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int hh = c0 + j;
-                        if (hh < p.H) {
-                            const float l = s_l[hh];
-                            float v = (n_tiles > 0 && l > 0.0f) ? __uint_as_float(o[j]) / l : 0.0f;
-                            if (!ok) v = qnan;
-                            p.out[(uo * p.H + hh) * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-                        }
+                        if (hh < p.H)
+                            p.out[(uo * p.H + hh) * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(ok ? v[j] : qnan));
                     }
                 }
             }
-            if (p.lse && hrow && h < p.H)
-                p.lse[uo * p.H + h] = (l_run > 0.0f && ok) ? (m_used + log2f(l_run)) * 0.69314718055994531f
-                                                          : (ok ? -INFINITY : qnan);
+            if (p.lse && hrow && h < p.H) {
+                const float none = (EX && p.sink) ? __ldg(p.sink + h) : -INFINITY;    // no keys: the sink alone
+                p.lse[uo * p.H + h] = (l_run > 0.0f && ok) ? (m_used + log2f(l_tot)) * 0.69314718055994531f
+                                                          : (ok ? none : qnan);
+            }
         } else {
             const size_t ps = uo * p.n_splits + split;
             float* po = p.part_o + ps * HP * D;
@@ -675,11 +792,14 @@ __global__ void __launch_bounds__(128) combine_tc_kernel(Params p) {
             bad |= __shfl_xor_sync(0xffffffffu, bad, o);
         }
         if (threadIdx.x == 0) {
+            // the sink joins the denominator relative to the global max M
+            const float sink = p.sink ? __ldg(p.sink + h) : -INFINITY;
+            if (p.sink && L > 0.0f) L += exp2f(sink * LOG2E - M);
             s_L = L;
             s_bad = bad;
             if (p.lse)
                 p.lse[u * p.H + h] = bad ? __int_as_float(0x7fc00000)
-                                         : (L > 0.0f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY);
+                                         : (L > 0.0f ? (M + log2f(L)) * 0.69314718055994531f : sink);
         }
     }
     __syncthreads();
@@ -704,8 +824,21 @@ __global__ void __launch_bounds__(128) combine_tc_kernel(Params p) {
     const float L = s_L;
     const float inv = L > 0.0f ? 1.0f / L : 0.0f;
     const float qnan = __int_as_float(0x7fc00000);
-    __nv_bfloat162 a = __floats2bfloat162_rn(bad ? qnan : acc[0] * inv, bad ? qnan : acc[1] * inv);
-    __nv_bfloat162 b = __floats2bfloat162_rn(bad ? qnan : acc[2] * inv, bad ? qnan : acc[3] * inv);
+    float o[4] = {acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv};
+    if (p.inv_freq && d0 >= D - D_ROPE) {
+        // RoPE dims: rotate the output back by the query's position
+        const int64_t t = unit_pos(p, u);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            float cs, sn;
+            rope_cs(p.inv_freq, (d0 - (D - D_ROPE)) / 2 + i, t, cs, sn);
+            const float x = o[2 * i], y = o[2 * i + 1];
+            o[2 * i] = x * cs + y * sn;
+            o[2 * i + 1] = y * cs - x * sn;
+        }
+    }
+    __nv_bfloat162 a = __floats2bfloat162_rn(bad ? qnan : o[0], bad ? qnan : o[1]);
+    __nv_bfloat162 b = __floats2bfloat162_rn(bad ? qnan : o[2], bad ? qnan : o[3]);
     uint2 w;
     w.x = *reinterpret_cast<uint32_t*>(&a);
     w.y = *reinterpret_cast<uint32_t*>(&b);
@@ -718,10 +851,11 @@ __global__ void __launch_bounds__(128) combine_tc_kernel(Params p) {
 namespace {
 
 int launch_tc(tc::Params& p, int64_t units, cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         tc::SMEM_BYTES);
+    const bool ex = p.q_norm_w || p.sink || p.inv_freq;
+    auto kern = ex ? tc::attn_tc_kernel<true> : tc::attn_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
     if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
-    tc::attn_tc_kernel<<<dim3(static_cast<unsigned>(units), p.n_splits), tc::NTHREADS, tc::SMEM_BYTES, st>>>(p);
+    kern<<<dim3(static_cast<unsigned>(units), p.n_splits), tc::NTHREADS, tc::SMEM_BYTES, st>>>(p);
     HCA_CHECK_LAUNCH();
     if (p.n_splits > 1) {
         tc::combine_tc_kernel<<<dim3(static_cast<unsigned>(units), p.H), tc::D / 4, 0, st>>>(p);
@@ -755,12 +889,23 @@ size_t tc_decode_ws_bytes(int B, int max_comp, int W, bool sparse) {
     return static_cast<size_t>(B) * ns * tc::HP * (static_cast<size_t>(tc::D) + 2) * sizeof(float) + 256;
 }
 
+static void set_extras(tc::Params& p, const hca_attn_extras* ex) {
+    if (!ex) return;
+    p.q_norm_w = ex->q_norm_w;
+    p.norm_eps = ex->norm_eps;
+    p.sink = ex->sink;
+    p.inv_freq = ex->inv_freq;
+    p.q_pos = ex->q_pos;
+    p.win_len = ex->win_len;
+}
+
 int tc_attn_decode_launch(const uint16_t* q, int B, int H, const hca_kv_cache& kv, const int32_t* idx,
                           int idx_stride, const int32_t* n_comp, int max_comp, const uint16_t* window, int W,
-                          float softmax_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
-                          cudaStream_t st) {
+                          float softmax_scale, const hca_attn_extras* ex, uint16_t* out, float* lse, void* ws,
+                          size_t ws_bytes, cudaStream_t st) {
     if (B == 0) return HCA_OK;
     tc::Params p = {};
+    set_extras(p, ex);
     p.q = q; p.H = H;
     p.codes = kv.codes; p.scales = kv.scales; p.rope = kv.rope; p.cap = kv.capacity;
     p.prefill = 0;
@@ -780,9 +925,12 @@ int tc_attn_decode_launch(const uint16_t* q, int B, int H, const hca_kv_cache& k
 
 int tc_attn_prefill_launch(const uint16_t* q, int Tq, int H, int p0, int m, const hca_kv_cache& kv,
                            const int32_t* idx, int idx_stride, const int32_t* count, const uint16_t* raw, int W,
-                           float softmax_scale, uint16_t* out, cudaStream_t st) {
+                           float softmax_scale, const hca_attn_extras* ex, uint16_t* out, cudaStream_t st) {
     if (Tq == 0) return HCA_OK;
     tc::Params p = {};
+    set_extras(p, ex);
+    p.q_pos = nullptr;
+    p.win_len = nullptr;
     p.q = q; p.H = H;
     p.codes = kv.codes; p.scales = kv.scales; p.rope = kv.rope; p.cap = kv.capacity;
     p.prefill = 1;

@@ -407,8 +407,12 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     return false;
 }
 
-// QG queries per CTA (N = 16 QG accumulator columns), NBD accumulator buffers,
-// KS key stages, EG epilogue warps per TMEM lane quarter.
+// QG queries per CTA, HG groups of 4 indexer heads (Hi = 4 HG; N = 16 QG HG
+// accumulator columns: query q, group hg at column 16 (q HG + hg), then block
+// b, head h of the group at + 4 b + h), NBD accumulator buffers, KS key
+// stages, EG epilogue warps per TMEM lane quarter.  bf16: the scores are
+// written rounded to bf16 (nearest even) as uint16 bit patterns, and the
+// histogram counts the rounded values.
 // Larger key = larger score; +0 and -0 map to the same key (the top-k's order).
 __device__ __forceinline__ uint32_t score_key(float f) {
     uint32_t u = __float_as_uint(f);
@@ -419,14 +423,15 @@ __device__ __forceinline__ uint32_t score_key(float f) {
 // hist (optional, one query per CTA): the query row's 2048-bin histogram of the
 // top 11 bits of each eligible score's key, hist + row * hist_stride (u32),
 // accumulated in shared memory and added with global atomics at the end.
-template <int QG, int NBD, int KS, int EG>
+template <int QG, int NBD, int KS, int EG, int HG>
 __global__ void __launch_bounds__(64 + 128 * EG)
 index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
                 const uint8_t* __restrict__ q_codes, const uint8_t* __restrict__ q_sf,
                 const float* __restrict__ w, const int32_t* __restrict__ q_pos,
                 int Tq, int64_t Nc_cap, int m, int64_t chunk, float* __restrict__ scores,
-                uint32_t* __restrict__ hist, int64_t hist_stride) {
-    constexpr int N = 16 * QG;
+                uint32_t* __restrict__ hist, int64_t hist_stride, int bf16) {
+    constexpr int HI = 4 * HG;
+    constexpr int N = 16 * QG * HG;
     constexpr uint32_t NCOLS = (N * NBD) <= 32 ? 32 : (N * NBD <= 64 ? 64 : (N * NBD <= 128 ? 128 : (N * NBD <= 256 ? 256 : 512)));
     constexpr uint32_t IDESC = (1u << 4) | (5u << 7) | (5u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
                                (static_cast<uint32_t>(TILE >> 4) << 24);
@@ -437,9 +442,10 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
     uint32_t* sh_hist = reinterpret_cast<uint32_t*>(sB + N * 128);   // 2048 bins when hist != nullptr
     __shared__ __align__(8) uint64_t bar_full[KS], bar_empty[KS], bar_accf[NBD], bar_acce[NBD], bar_drain;
     __shared__ uint32_t tmem_slot;
-    __shared__ int s_eq[QG][16];                        // (uq - 127) - 127 per (query, block*4+head)
-    __shared__ int s_klo[QG][4], s_khi[QG][4];          // key exponent range of the fast path per block
-    __shared__ float s_w[QG][4];
+    __shared__ int s_eq[QG][16 * HG];                   // (uq - 127) - 127 per (query, group*16 + block*4 + head)
+    __shared__ int s_klo[QG][HG][4], s_khi[QG][HG][4];  // key exponent range of the fast path per (group, block)
+    __shared__ float s_w[QG][HI];
+    uint16_t* scores16 = reinterpret_cast<uint16_t*>(scores);
     __shared__ int64_t s_elig[QG];
     __shared__ int s_abort;
 
@@ -469,31 +475,32 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
         const int st = x / (CODE_BYTES / 16), o = x % (CODE_BYTES / 16);
         *reinterpret_cast<uint4*>(smem + st * STAGE_BYTES + o * 16) = make_uint4(0u, 0u, 0u, 0u);
     }
-    // query operand: row n = q*16 + blk*4 + h; slot j (elements 16j..16j+15) is block j/2
+    // query operand: row n = (q HG + hg) 16 + blk 4 + hh (head h = 4 hg + hh); slot j
+    // (elements 16j..16j+15) is block j/2
     for (int x = tid; x < N * 8; x += blockDim.x) {
         const int n = x >> 3, j = x & 7;
-        const int q = n >> 4, blk = (n >> 2) & 3, h = n & 3;
+        const int q = n / (16 * HG), hg = (n >> 4) % HG, blk = (n >> 2) & 3, h = hg * 4 + (n & 3);
         uint2 v = make_uint2(0, 0);
-        if ((j >> 1) == blk) v = __ldg(reinterpret_cast<const uint2*>(q_codes + ((qrow0 + q) * 4 + h) * 64 + j * 8));
+        if ((j >> 1) == blk) v = __ldg(reinterpret_cast<const uint2*>(q_codes + ((qrow0 + q) * HI + h) * 64 + j * 8));
         *reinterpret_cast<uint4*>(sB + sw128(n, j)) = make_uint4(v.x, v.y, 0u, 0u);
     }
-    for (int x = tid; x < QG * 16; x += blockDim.x) {
-        const int q = x >> 4, blk = (x >> 2) & 3, h = x & 3;
-        s_eq[q][x & 15] = static_cast<int>(__ldg(q_sf + ((qrow0 + q) * 4 + h) * 4 + blk)) - 254;
+    for (int x = tid; x < QG * 16 * HG; x += blockDim.x) {
+        const int q = x / (16 * HG), z = x % (16 * HG), hg = z >> 4, blk = (z >> 2) & 3, h = hg * 4 + (z & 3);
+        s_eq[q][z] = static_cast<int>(__ldg(q_sf + ((qrow0 + q) * HI + h) * 4 + blk)) - 254;
     }
-    for (int x = tid; x < QG * 4; x += blockDim.x) s_w[x >> 2][x & 3] = __ldg(w + (qrow0 + (x >> 2)) * 4 + (x & 3));
-    for (int x = tid; x < QG * 4; x += blockDim.x) {
-        // fast path of a (query, block): every head's 2^(eq + ek) is a normal float and
-        // |block dot| * 2^(eq + ek) < 2^127, i.e. eq + ek in [-126, 116] for all heads
-        const int q = x >> 2, blk = x & 3;
+    for (int x = tid; x < QG * HI; x += blockDim.x) s_w[x / HI][x % HI] = __ldg(w + (qrow0 + x / HI) * HI + x % HI);
+    for (int x = tid; x < QG * HG * 4; x += blockDim.x) {
+        // fast path of a (query, group, block): every head's 2^(eq + ek) is a normal float and
+        // |block dot| * 2^(eq + ek) < 2^127, i.e. eq + ek in [-126, 116] for the group's heads
+        const int q = x / (HG * 4), hg = (x / 4) % HG, blk = x & 3;
         int mn = 1 << 20, mx = -(1 << 20);
-        for (int h = 0; h < 4; ++h) {
-            const int e = static_cast<int>(__ldg(q_sf + ((qrow0 + q) * 4 + h) * 4 + blk)) - 254;
+        for (int hh = 0; hh < 4; ++hh) {
+            const int e = static_cast<int>(__ldg(q_sf + ((qrow0 + q) * HI + hg * 4 + hh) * 4 + blk)) - 254;
             mn = min(mn, e);
             mx = max(mx, e);
         }
-        s_klo[q][blk] = -126 - mn;
-        s_khi[q][blk] = 116 - mx;
+        s_klo[q][hg][blk] = -126 - mn;
+        s_khi[q][hg][blk] = 116 - mx;
     }
     if (tid < QG) {
         int64_t e = (static_cast<int64_t>(q_pos[qrow0 + tid]) + 1) / m;
@@ -511,8 +518,11 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
 
     // ineligible part of the chunk: -inf (per query)
     for (int q = 0; q < QG; ++q) {
-        float* orow = scores + static_cast<size_t>(qrow0 + q) * Nc_cap;
-        for (int64_t s = max(s_begin, s_elig[q]) + tid; s < s_end; s += blockDim.x) orow[s] = -INFINITY;
+        const size_t ro = static_cast<size_t>(qrow0 + q) * Nc_cap;
+        for (int64_t s = max(s_begin, s_elig[q]) + tid; s < s_end; s += blockDim.x) {
+            if (bf16) scores16[ro + s] = 0xFF80u;
+            else scores[ro + s] = -INFINITY;
+        }
     }
     const int row0 = static_cast<int>(b * Nc_cap + s_begin);        // tensor-map row of the chunk's first key
 
@@ -570,18 +580,22 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
         const int n_mine = n_tiles > t0 ? (n_tiles - t0 + TS - 1) / TS : 0;
         const int n_items = n_mine * QPW;
-        int eq1[16], klo1[4], khi1[4];                 // the only query's exponents (QG == 1)
+        // sub-items I = (item i, head group hg): the TMEM load of sub-item I + 1 is in
+        // flight while I is scored; a score is complete after its last group
+        const int n_sub = n_items * HG;
+        int eq1[16], klo1[4], khi1[4];                 // the only query's exponents (QG == 1, HG == 1)
 #pragma unroll
         for (int j = 0; j < 16; ++j) eq1[j] = s_eq[0][j];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) { klo1[j] = s_klo[0][j]; khi1[j] = s_khi[0][j]; }
+        for (int j = 0; j < 4; ++j) { klo1[j] = s_klo[0][0][j]; khi1[j] = s_khi[0][0][j]; }
         uint32_t rn[16];
-        auto tmem_ld = [&](int i) {
+        auto tmem_ld = [&](int I) {
+            const int i = I / HG, hg = I % HG;
             const int t = t0 + TS * (i / QPW), q = q0 + QE * (i % QPW);
             asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
                          : "=r"(rn[0]), "=r"(rn[1]), "=r"(rn[2]), "=r"(rn[3]), "=r"(rn[4]), "=r"(rn[5]), "=r"(rn[6]), "=r"(rn[7]),
                            "=r"(rn[8]), "=r"(rn[9]), "=r"(rn[10]), "=r"(rn[11]), "=r"(rn[12]), "=r"(rn[13]), "=r"(rn[14]), "=r"(rn[15])
-                         : "r"(lane_base + static_cast<uint32_t>((t % NBD) * N + q * 16)));
+                         : "r"(lane_base + static_cast<uint32_t>((t % NBD) * N + (q * HG + hg) * 16)));
         };
         // a tile's accumulators are complete (and its stage's loads visible) after these waits
         auto tile_ready = [&](int t) {
@@ -591,38 +605,41 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
             return true;
         };
         bool ok = true;
-        if (n_items > 0) {
+        if (n_sub > 0) {
             if (tile_ready(t0)) tmem_ld(0); else ok = false;
         }
         uint32_t sw = 0;
-        for (int i = 0; i < n_items && ok; ++i) {
+        float sc = 0.0f;
+        for (int I = 0; I < n_sub && ok; ++I) {
+            const int i = I / HG, hg = I % HG;
             const int t = t0 + TS * (i / QPW), j = i % QPW, q = q0 + QE * j;
             const int st = t % KS, nb = t % NBD;
             asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
             uint32_t r[16];
 #pragma unroll
             for (int z = 0; z < 16; ++z) r[z] = rn[z];
-            if (j == 0) sw = *reinterpret_cast<const uint32_t*>(smem + st * STAGE_BYTES + CODE_BYTES + row * 4);
-            if (j == QPW - 1) {
+            if (j == 0 && hg == 0) sw = *reinterpret_cast<const uint32_t*>(smem + st * STAGE_BYTES + CODE_BYTES + row * 4);
+            if (j == QPW - 1 && hg == HG - 1) {
                 // every load of tile t has completed and its scale word is read: release
                 // the accumulator buffer and the key stage
                 asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) { mbar_arrive(smem_u32(&bar_acce[nb])); mbar_arrive(smem_u32(&bar_empty[st])); }
             }
-            if (i + 1 < n_items) {
-                if ((i + 1) % QPW == 0 && !tile_ready(t + TS)) { ok = false; }
-                else tmem_ld(i + 1);
+            if (I + 1 < n_sub) {
+                if ((I + 1) % (QPW * HG) == 0 && !tile_ready(t + TS)) { ok = false; }
+                else tmem_ld(I + 1);
             }
             int eq[16];
 #pragma unroll
-            for (int z = 0; z < 16; ++z) eq[z] = QG == 1 ? eq1[z] : s_eq[q][z];
+            for (int z = 0; z < 16; ++z) eq[z] = (QG == 1 && HG == 1) ? eq1[z] : s_eq[q][hg * 16 + z];
             int ek[4];
             bool fast = true;
 #pragma unroll
             for (int blk = 0; blk < 4; ++blk) {
                 ek[blk] = static_cast<int>((sw >> (8 * blk)) & 0xFFu);
-                const int lo = QG == 1 ? klo1[blk] : s_klo[q][blk], hi = QG == 1 ? khi1[blk] : s_khi[q][blk];
+                const int lo = (QG == 1 && HG == 1) ? klo1[blk] : s_klo[q][hg][blk];
+                const int hi = (QG == 1 && HG == 1) ? khi1[blk] : s_khi[q][hg][blk];
                 fast &= (ek[blk] >= lo) & (ek[blk] <= hi);
             }
             float dot[4];
@@ -650,14 +667,26 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
                     dot[h] = a;
                 }
             }
-            float sc = 0.0f;
+            // heads 4 hg .. 4 hg + 3, continuing the ordered sum over h = 0 .. Hi - 1
+            if (hg == 0) sc = 0.0f;
 #pragma unroll
-            for (int h = 0; h < 4; ++h) sc = __fadd_rn(sc, __fmul_rn(s_w[q][h], dot[h] > 0.0f ? dot[h] : 0.0f));
-            const int64_t e = s_begin + static_cast<int64_t>(t) * TILE + row;
-            if (e < s_end && e < s_elig[q]) {
-                scores[static_cast<size_t>(qrow0 + q) * Nc_cap + e] = ok ? sc : __int_as_float(0x7fc00000);
-                // a NaN score is not counted: after a device error the top-k is undefined anyway
-                if (QG == 1 && hist && ok) atomicAdd(&sh_hist[score_key(sc) >> 21], 1u);
+            for (int h = 0; h < 4; ++h)
+                sc = __fadd_rn(sc, __fmul_rn(s_w[q][hg * 4 + h], dot[h] > 0.0f ? dot[h] : 0.0f));
+            if (hg == HG - 1) {
+                const int64_t e = s_begin + static_cast<int64_t>(t) * TILE + row;
+                if (e < s_end && e < s_elig[q]) {
+                    const size_t o = static_cast<size_t>(qrow0 + q) * Nc_cap + e;
+                    if (bf16) {
+                        const uint16_t hb = ok ? __bfloat16_as_ushort(__float2bfloat16_rn(sc)) : 0x7FC0u;
+                        scores16[o] = hb;
+                        if (QG == 1 && hist && ok)
+                            atomicAdd(&sh_hist[score_key(__uint_as_float(static_cast<uint32_t>(hb) << 16)) >> 21], 1u);
+                    } else {
+                        scores[o] = ok ? sc : __int_as_float(0x7fc00000);
+                        // a NaN score is not counted: after a device error the top-k is undefined anyway
+                        if (QG == 1 && hist && ok) atomicAdd(&sh_hist[score_key(sc) >> 21], 1u);
+                    }
+                }
             }
         }
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
@@ -665,7 +694,11 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
             // scores of the tiles this warp did not reach: NaN
             for (int q = q0; q < QG; q += QE)
                 for (int64_t e = s_begin + row; e < s_live; e += TILE)
-                    if (e < s_elig[q]) scores[static_cast<size_t>(qrow0 + q) * Nc_cap + e] = __int_as_float(0x7fc00000);
+                    if (e < s_elig[q]) {
+                        const size_t o = static_cast<size_t>(qrow0 + q) * Nc_cap + e;
+                        if (bf16) scores16[o] = 0x7FC0u;
+                        else scores[o] = __int_as_float(0x7fc00000);
+                    }
         }
     }
     __syncthreads();
@@ -734,10 +767,11 @@ bool make_maps(const uint8_t* k_codes, const uint8_t* k_sf, int64_t rows, int64_
 }
 
 // returns HCA_ERR_UNSUPPORTED (nothing launched) when the tensor maps cannot be made
-template <int QG, int NBD, int KS, int EG>
+template <int QG, int NBD, int KS, int EG, int HG = 1>
 int launch_tc(const uint8_t* q_codes, const uint8_t* q_sf, const float* w, const uint8_t* k_codes,
               const uint8_t* k_sf, const int32_t* q_pos, int64_t rows, int B, int Tq, int64_t Nc_cap, int m,
-              float* scores, cudaStream_t st, int64_t want_ctas, uint32_t* hist = nullptr, int64_t hist_stride = 0) {
+              float* scores, cudaStream_t st, int64_t want_ctas, uint32_t* hist = nullptr, int64_t hist_stride = 0,
+              int bf16 = 0) {
     CUtensorMap tm_codes, tm_scales;
     if (!make_maps(k_codes, k_sf, static_cast<int64_t>(B) * Nc_cap, Nc_cap, &tm_codes, &tm_scales)) return HCA_ERR_UNSUPPORTED;
     const int64_t groups = rows / QG;
@@ -745,16 +779,16 @@ int launch_tc(const uint8_t* q_codes, const uint8_t* q_sf, const float* w, const
     chunk = ceil_div(chunk, TILE) * TILE;
     if (chunk < TILE) chunk = TILE;
     if (ceil_div(Nc_cap, chunk) > 65535) chunk = ceil_div(ceil_div(Nc_cap, 65535), TILE) * TILE;
-    size_t smem = static_cast<size_t>(KS) * STAGE_BYTES + 16 * QG * 128 + 1024 + (hist ? 2048 * 4 : 0);
+    size_t smem = static_cast<size_t>(KS) * STAGE_BYTES + 16 * QG * HG * 128 + 1024 + (hist ? 2048 * 4 : 0);
     // a CTA that takes all 512 TMEM columns must be alone on its SM: ask for
     // more than half of the SM's shared memory
-    if (16 * QG * NBD >= 512 && smem < 120 * 1024) smem = 120 * 1024;
-    auto kern = index_tc_kernel<QG, NBD, KS, EG>;
+    if (16 * QG * HG * NBD >= 512 && smem < 120 * 1024) smem = 120 * 1024;
+    auto kern = index_tc_kernel<QG, NBD, KS, EG, HG>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
     const dim3 grid(static_cast<unsigned>(groups), static_cast<unsigned>(ceil_div(Nc_cap, chunk)));
     kern<<<grid, 64 + 128 * EG, smem, st>>>(tm_codes, tm_scales, q_codes, q_sf, w, q_pos, Tq, Nc_cap, m, chunk, scores,
-                                            hist, hist_stride);
+                                            hist, hist_stride, bf16);
     HCA_CHECK_LAUNCH();
     return HCA_OK;
 }
@@ -781,19 +815,33 @@ namespace {
 // nothing was launched.
 int index_launch_hist(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
                       const uint8_t* k_codes, const uint8_t* k_sf, const int32_t* q_pos,
-                      int B, int64_t Nc_cap, int Hi, int c, int m, float* scores, uint32_t* hist,
-                      int64_t hist_stride, cudaStream_t st) {
-    if (c != 128 || Hi != 4 || B <= 0 || Nc_cap <= 0) return HCA_ERR_UNSUPPORTED;
-    return itc::launch_tc<1, 4, 5, 2>(q_codes, q_sf, w, k_codes, k_sf, q_pos, B, B, 1, Nc_cap, m, scores, st,
-                                      2LL * sm_count(), hist, hist_stride);
+                      int B, int64_t Nc_cap, int Hi, int c, int m, void* scores, uint32_t* hist,
+                      int64_t hist_stride, cudaStream_t st, bool bf16) {
+    if (c != 128 || (Hi != 4 && Hi != 64) || B <= 0 || Nc_cap <= 0) return HCA_ERR_UNSUPPORTED;
+    float* sc = static_cast<float*>(scores);
+    const int budget = launch_budget(HCA_BUDGET_DECODE_INDEX);
+    if (Hi == 64)      // 16 head groups: N = 256 columns per buffer, two buffers fill TMEM (one CTA per SM)
+        return itc::launch_tc<1, 2, 5, 2, 16>(q_codes, q_sf, w, k_codes, k_sf, q_pos, B, B, 1, Nc_cap, m, sc, st,
+                                              budget > 0 ? std::min<int64_t>(budget, sm_count()) : sm_count(),
+                                              hist, hist_stride, bf16 ? 1 : 0);
+    return itc::launch_tc<1, 4, 5, 2>(q_codes, q_sf, w, k_codes, k_sf, q_pos, B, B, 1, Nc_cap, m, sc, st,
+                                      budget > 0 ? budget : 2LL * sm_count(), hist, hist_stride, bf16 ? 1 : 0);
 }
 
 int index_launch(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
                  const uint8_t* k_codes, const uint8_t* k_sf, const int32_t* q_pos,
-                 int B, int Tq, int64_t Nc_cap, int Hi, int c, int m, float* scores,
-                 cudaStream_t st) {
+                 int B, int Tq, int64_t Nc_cap, int Hi, int c, int m, void* scores_v,
+                 cudaStream_t st, bool bf16) {
     if (B == 0 || Tq == 0 || Nc_cap == 0) return HCA_OK;
+    float* scores = static_cast<float*>(scores_v);
     const int64_t rows = static_cast<int64_t>(B) * Tq;
+    if (c == 128 && Hi == 64) {
+        // the note's 64 indexer heads: one query per CTA, 16 head groups on the tensor pipe
+        const int rc = itc::launch_tc<1, 2, 5, 2, 16>(q_codes, q_sf, w, k_codes, k_sf, q_pos, rows, B, Tq, Nc_cap, m,
+                                                      scores, st, sm_count(), nullptr, 0, bf16 ? 1 : 0);
+        return rc;   // (unaligned key buffers: HCA_ERR_UNSUPPORTED)
+    }
+    if (bf16 && !(c == 128 && Hi == 4)) return HCA_ERR_UNSUPPORTED;
     // enough blocks to fill the machine several times over for one row, but
     // a chunk of at least one warp step per warp
     int64_t chunk = 4096;
@@ -813,11 +861,11 @@ int index_launch(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
         int rc;
         if (Tq % 16 == 0 && Tq >= 64)
             rc = itc::launch_tc<16, 2, 4, 2>(q_codes, q_sf, w, k_codes, k_sf, q_pos, rows, B, Tq, Nc_cap, m, scores, st,
-                                             2LL * sm_count());
+                                             2LL * sm_count(), nullptr, 0, bf16 ? 1 : 0);
         else
             rc = itc::launch_tc<1, 4, 5, 2>(q_codes, q_sf, w, k_codes, k_sf, q_pos, rows, B, Tq, Nc_cap, m, scores, st,
-                                            2LL * sm_count());
-        if (rc != HCA_ERR_UNSUPPORTED) return rc;
+                                            2LL * sm_count(), nullptr, 0, bf16 ? 1 : 0);
+        if (rc != HCA_ERR_UNSUPPORTED || bf16) return rc;
         // unaligned key buffers: CUDA-core tensor path below
     }
     if (c == 128 && Hi == 4) {

@@ -1,0 +1,83 @@
+// step.cu -- one decode step of a CSA layer and an HCA layer from host
+// memory to host memory through the library alone: the query copies in, the
+// fused index + top-k, both attention calls and the output copies out, with
+// the HCA layer on a second stream ("DeepSeek V4 ..." note, sections 7 and 8:
+// the CSA path -- indexer, top-k, attention over the selected entries and the
+// window -- and the HCA path -- dense attention over every entry and the
+// window -- of one decode position).
+//
+// Schedule (the two paths share no data):
+//   stream: H2D indexer query | index + top-k (records ev_index) | waits ev_q |
+//           CSA attention | D2H CSA output | waits ev_join
+//   side:   waits ev_fork | H2D both attention queries (records ev_q) |
+//           waits ev_index | HCA attention | D2H HCA output (records ev_join)
+// The HCA launch waits for the indexer, which fills every SM anyway.  Every
+// copy is one cudaMemcpyAsync; the host buffers should be pinned so that the
+// copies are asynchronous.
+#include "common.cuh"
+
+using namespace hca;
+
+namespace {
+int rec(void* ev, void* st) {
+    const cudaError_t e = cudaEventRecord(static_cast<cudaEvent_t>(ev), as_stream(st));
+    if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
+    return HCA_OK;
+}
+int wait(void* st, void* ev) {
+    const cudaError_t e = cudaStreamWaitEvent(as_stream(st), static_cast<cudaEvent_t>(ev), 0);
+    if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
+    return HCA_OK;
+}
+int cpy(void* dst, const void* src, size_t n, cudaMemcpyKind kind, void* st) {
+    if (n == 0) return HCA_OK;
+    const cudaError_t e = cudaMemcpyAsync(dst, src, n, kind, as_stream(st));
+    if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
+    return HCA_OK;
+}
+}  // namespace
+
+#define HCA_TRY(x) do { const int _rc = (x); if (_rc != HCA_OK) return _rc; } while (0)
+
+extern "C" int hca_decode_step_host(const hca_decode_step_plan* p, const uint16_t* h_q_csa, const uint16_t* h_q_hca,
+                                    const uint8_t* h_iq_codes, const uint8_t* h_iq_sf, const float* h_iq_w,
+                                    uint16_t* h_out_csa, uint16_t* h_out_hca, void* stream) {
+    if (!p || !h_q_csa || !h_q_hca || !h_iq_codes || !h_iq_sf || !h_iq_w || !h_out_csa || !h_out_hca)
+        return HCA_ERR_INVALID_ARG;
+    if (!p->side_stream || !p->ev_fork || !p->ev_index || !p->ev_q || !p->ev_join) return HCA_ERR_INVALID_ARG;
+    if (p->B <= 0 || p->H <= 0 || p->Hi <= 0 || p->c <= 0 || p->layout.d <= 0) return HCA_ERR_INVALID_ARG;
+    const size_t d = static_cast<size_t>(p->layout.d);
+    const size_t q_bytes = static_cast<size_t>(p->B) * p->H * d * 2;
+    const size_t iqc = static_cast<size_t>(p->B) * p->Hi * (p->c / 2);
+    const size_t iqs = static_cast<size_t>(p->B) * p->Hi * (p->c / 32);
+    const size_t iqw = static_cast<size_t>(p->B) * p->Hi * sizeof(float);
+    void* side = p->side_stream;
+    HCA_TRY(rec(p->ev_fork, stream));
+    // the indexer query first (a few hundred bytes), the attention queries beside the indexer
+    HCA_TRY(cpy(p->iq_codes, h_iq_codes, iqc, cudaMemcpyHostToDevice, stream));
+    HCA_TRY(cpy(p->iq_sf, h_iq_sf, iqs, cudaMemcpyHostToDevice, stream));
+    HCA_TRY(cpy(p->iq_w, h_iq_w, iqw, cudaMemcpyHostToDevice, stream));
+    HCA_TRY(wait(side, p->ev_fork));
+    HCA_TRY(cpy(p->q_csa, h_q_csa, q_bytes, cudaMemcpyHostToDevice, side));
+    HCA_TRY(cpy(p->q_hca, h_q_hca, q_bytes, cudaMemcpyHostToDevice, side));
+    HCA_TRY(rec(p->ev_q, side));
+    // CSA: index + top-k, then attention over the selected entries and the window
+    HCA_TRY(lightning_index_topk(p->iq_codes, p->iq_sf, p->iq_w, p->k_codes, p->k_sf, p->q_pos, p->B,
+                                 p->csa_entries, p->Hi, p->c, 4, p->k, p->scores, p->idx, p->count, p->topk_ws,
+                                 p->topk_ws_bytes, p->ev_index, stream));
+    HCA_TRY(wait(stream, p->ev_q));
+    const int32_t kmax = static_cast<int32_t>(p->csa_entries < p->k ? p->csa_entries : p->k);
+    HCA_TRY(compressed_attn_decode(p->q_csa, p->B, p->H, p->layout, p->csa_cache, p->idx, p->k, p->count, kmax,
+                                   p->csa_window, p->W, p->softmax_scale, p->out_csa, nullptr, p->ws_csa,
+                                   p->ws_csa_bytes, stream));
+    HCA_TRY(cpy(h_out_csa, p->out_csa, q_bytes, cudaMemcpyDeviceToHost, stream));
+    // HCA: dense attention, after the indexer
+    HCA_TRY(wait(side, p->ev_index));
+    HCA_TRY(compressed_attn_decode(p->q_hca, p->B, p->H, p->layout, p->hca_cache, nullptr, 0, p->hca_n, p->hca_max,
+                                   p->hca_window, p->W, p->softmax_scale, p->out_hca, nullptr, p->ws_hca,
+                                   p->ws_hca_bytes, side));
+    HCA_TRY(cpy(h_out_hca, p->out_hca, q_bytes, cudaMemcpyDeviceToHost, side));
+    HCA_TRY(rec(p->ev_join, side));
+    HCA_TRY(wait(stream, p->ev_join));
+    return HCA_OK;
+}

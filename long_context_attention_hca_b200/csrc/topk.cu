@@ -341,31 +341,53 @@ cudaError_t launch_cl(int R, int64_t slice, const float* scores, const int32_t* 
 // The histogram, header and bitmaps are cleared by a memset on the stream.
 namespace wide {
 
+// Few long rows (decode: one row per sequence).  The 11-bit key histogram of
+// each row comes first (built by the indexer's epilogue in the fused decode
+// call, or by hist_kernel); then one select_kernel launch:
+//   every CTA reads the histogram, finds the threshold bin T1 (the highest
+//   bin whose count from the top reaches k), scans its chunk of the row and
+//   appends the keys above bin T1 (all selected, fewer than k of them) and
+//   the keys in bin T1 (the candidates) to the row's two lists, one atomic
+//   per list and CTA;
+//   the CTA that finishes last (a counter per row, behind a memory fence)
+//   resolves the row: a radix select over the candidates' composite keys
+//   (score key, then the complement of the index, so that every composite
+//   is unique and equal scores rank the lower index first) finds the exact
+//   threshold, the selected indices are gathered in shared memory, sorted
+//   ascending by a bitonic network and written out.
+// No CTA waits for another: the last one to arrive does the rest.
 constexpr int kBins = 2048;
-constexpr int kThreads = 256;
-constexpr int kResolveThreads = 1024;
-constexpr int kMaxIt = 64;                 // mark: at most 64 x 256 keys per CTA
+constexpr int kThreads = 256;              // hist_kernel
+constexpr int kSelThreads = 512;           // select_kernel
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kMaxIt = 64;                 // select: at most 64 x 512 scores per CTA
+constexpr int kCandSmem = 4096;            // candidates resolved from shared memory (else from L2)
+constexpr int kMaxK = 4096;
+// dynamic shared memory of select_kernel: the scan's ballot masks, reused by
+// the resolve as the candidate cache, then the selected indices
+constexpr size_t kSelSmem = static_cast<size_t>(kCandSmem) * 8 + static_cast<size_t>(kMaxK) * 4;
+static_assert(2 * kSelWarps * kMaxIt * 4 <= kCandSmem * 8, "masks fit in the candidate cache");
 
 struct Layout {
-    int64_t words;          // bitmap words per row
+    size_t clear_bytes;     // histogram + header, cleared before every call
+    size_t above_off;       // u32 [kMaxK]
+    size_t cand_off;        // u64 [Nc_cap]
     size_t row_bytes;       // per-row stride
-    size_t clear_bytes;     // bytes cleared per row (hist, header, bitmaps)
 };
 
 __host__ __device__ inline Layout layout(int64_t Nc_cap) {
     Layout L;
-    L.words = (Nc_cap + 31) / 32;
-    L.clear_bytes = static_cast<size_t>(kBins) * 4 + 32 + static_cast<size_t>(2 * L.words) * 4;
-    L.clear_bytes = (L.clear_bytes + 255) & ~static_cast<size_t>(255);
-    L.row_bytes = L.clear_bytes + ((static_cast<size_t>(Nc_cap) * 8 + 255) & ~static_cast<size_t>(255));
+    L.clear_bytes = static_cast<size_t>(kBins) * 4 + 256;
+    L.above_off = L.clear_bytes;
+    L.cand_off = L.above_off + static_cast<size_t>(kMaxK) * 4;
+    L.row_bytes = L.cand_off + ((static_cast<size_t>(Nc_cap) * 8 + 255) & ~static_cast<size_t>(255));
     return L;
 }
 
 struct RowWs {
     uint32_t* hist;
-    uint32_t* hdr;          // [0] candidate count, [1] T1, [2] needed from bin T1
-    uint32_t* sel;
-    uint32_t* tie;
+    uint32_t* hdr;          // [0] keys above bin T1, [1] candidates, [2] CTAs done
+    uint32_t* above;
     unsigned long long* cand;
 };
 
@@ -375,9 +397,8 @@ __device__ __forceinline__ RowWs row_ws(uint8_t* ws, int64_t Nc_cap, int64_t r) 
     RowWs w;
     w.hist = reinterpret_cast<uint32_t*>(base);
     w.hdr = w.hist + kBins;
-    w.sel = w.hdr + 8;
-    w.tie = w.sel + L.words;
-    w.cand = reinterpret_cast<unsigned long long*>(base + L.clear_bytes);
+    w.above = reinterpret_cast<uint32_t*>(base + L.above_off);
+    w.cand = reinterpret_cast<unsigned long long*>(base + L.cand_off);
     return w;
 }
 
@@ -386,8 +407,16 @@ __device__ __forceinline__ int64_t n_eligible(const int32_t* q_pos, int64_t r, i
     return e < 0 ? 0 : (e > Nc_cap ? Nc_cap : e);
 }
 
+// Score of entry e as an fp32 value: an fp32 score, or a bf16 score (uint16
+// bits; the note's BF16 index scores) widened exactly.
+__device__ __forceinline__ float score_at(const float* row, int64_t e) { return row[e]; }
+__device__ __forceinline__ float score_at(const uint16_t* row, int64_t e) {
+    return __uint_as_float(static_cast<uint32_t>(row[e]) << 16);
+}
+
+template <typename T>
 __global__ void __launch_bounds__(kThreads)
-hist_kernel(const float* __restrict__ scores, const int32_t* __restrict__ q_pos, int64_t Nc_cap, int m,
+hist_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, int64_t Nc_cap, int m,
             int64_t chunk, uint8_t* __restrict__ ws) {
     __shared__ uint32_t sh[kBins];
     const int64_t r = blockIdx.y;
@@ -397,12 +426,12 @@ hist_kernel(const float* __restrict__ scores, const int32_t* __restrict__ q_pos,
     if (e0 >= e1) return;
     for (int i = threadIdx.x; i < kBins; i += kThreads) sh[i] = 0;
     __syncthreads();
-    const float* row = scores + static_cast<size_t>(r) * Nc_cap;
+    const T* row = scores + static_cast<size_t>(r) * Nc_cap;
     // eight loads in flight per thread before the shared-memory atomics
     for (int64_t e = e0 + threadIdx.x; e < e1; e += kThreads * 8) {
         float v[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = e + j * kThreads < e1 ? row[e + j * kThreads] : 0.0f;
+        for (int j = 0; j < 8; ++j) v[j] = e + j * kThreads < e1 ? score_at(row, e + j * kThreads) : 0.0f;
 #pragma unroll
         for (int j = 0; j < 8; ++j)
             if (e + j * kThreads < e1) atomicAdd(&sh[order_key(v[j]) >> 21], 1u);
@@ -413,108 +442,8 @@ hist_kernel(const float* __restrict__ scores, const int32_t* __restrict__ q_pos,
         if (sh[i]) atomicAdd(&w.hist[i], sh[i]);
 }
 
-// Threshold bin of a row from its histogram (the same result in every CTA):
-// T1 = the highest bin whose suffix count reaches kk; returns the number of
-// keys needed from bin T1 (kk - keys in higher bins).  Block-wide.
-__device__ uint32_t find_t1(const uint32_t* __restrict__ hist, uint32_t kk, uint32_t* sh_cnt, int* t1_out) {
-    // thread t sums bins [2048 - 8 (t + 1), 2048 - 8 t) (thread 0 holds the top bins)
-    const int t = threadIdx.x;
-    uint32_t c[8], tot = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) { c[j] = hist[kBins - 8 * t - 1 - j]; tot += c[j]; }
-    sh_cnt[t] = tot;
-    __syncthreads();
-    // inclusive prefix over threads (from the top bins down), Hillis-Steele in shared memory
-    for (int off = 1; off < kThreads; off <<= 1) {
-        const uint32_t v = t >= off ? sh_cnt[t - off] : 0u;
-        __syncthreads();
-        sh_cnt[t] += v;
-        __syncthreads();
-    }
-    const uint32_t before = t > 0 ? sh_cnt[t - 1] : 0u;   // keys in bins above this thread's range
-    if (before < kk && before + tot >= kk) {
-        uint32_t acc = before;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            if (acc + c[j] >= kk) { *t1_out = kBins - 8 * t - 1 - j; sh_cnt[kThreads] = kk - acc; break; }
-            acc += c[j];
-        }
-    }
-    __syncthreads();
-    return sh_cnt[kThreads];
-}
-
-__global__ void __launch_bounds__(kThreads)
-mark_kernel(const float* __restrict__ scores, const int32_t* __restrict__ q_pos, int64_t Nc_cap, int m, int k,
-            int64_t chunk, uint8_t* __restrict__ ws) {
-    __shared__ uint32_t sh_cnt[kThreads + 1];
-    __shared__ int s_t1;
-    const int64_t r = blockIdx.y;
-    const int64_t n = n_eligible(q_pos, r, m, Nc_cap);
-    const uint32_t kk = static_cast<uint32_t>(min(static_cast<int64_t>(k), n));
-    const int64_t e0 = static_cast<int64_t>(blockIdx.x) * chunk;
-    const int64_t e1 = min(e0 + chunk, n);
-    if (kk == 0 || e0 >= e1) return;
-    RowWs w = row_ws(ws, Nc_cap, r);
-    if (threadIdx.x == 0) s_t1 = -1;
-    const uint32_t need1 = find_t1(w.hist, kk, sh_cnt, &s_t1);
-    const uint32_t t1 = static_cast<uint32_t>(s_t1);
-    if (blockIdx.x == 0 && threadIdx.x == 0) { w.hdr[1] = t1; w.hdr[2] = need1; }
-    const float* row = scores + static_cast<size_t>(r) * Nc_cap;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    // chunk is a multiple of 256 and at most kMaxIt * 256: each warp owns whole bitmap
-    // words.  Pass A marks the keys above bin T1 and keeps the ballot of bin-T1 keys per
-    // (warp, step); one atomic per CTA reserves the candidate slots; pass B writes them.
-    __shared__ uint32_t s_mask[kThreads / 32][kMaxIt];
-    __shared__ uint32_t s_wcnt[kThreads / 32];
-    __shared__ uint32_t s_base;
-    const int n_it = static_cast<int>((e1 - e0 + kThreads - 1) / kThreads);
-    uint32_t cnt = 0;
-    for (int it0 = 0; it0 < n_it; it0 += 8) {
-        float v[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int64_t e = e0 + static_cast<int64_t>(it0 + j) * kThreads + warp * 32 + lane;
-            v[j] = e < e1 ? row[e] : 0.0f;
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int it = it0 + j;
-            if (it >= n_it) break;
-            const int64_t base = e0 + static_cast<int64_t>(it) * kThreads + warp * 32;
-            const bool live = base + lane < e1;
-            const uint32_t bin = order_key(v[j]) >> 21;
-            const unsigned above = __ballot_sync(0xffffffffu, live && bin > t1);
-            const unsigned in_t1 = __ballot_sync(0xffffffffu, live && bin == t1);
-            if (lane == 0) {
-                if (above) w.sel[base >> 5] = above;
-                s_mask[warp][it] = in_t1;
-            }
-            cnt += __popc(in_t1);
-        }
-    }
-    if (lane == 0) s_wcnt[warp] = cnt;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        uint32_t tot = 0;
-        for (int q = 0; q < kThreads / 32; ++q) { const uint32_t c = s_wcnt[q]; s_wcnt[q] = tot; tot += c; }
-        s_base = tot ? atomicAdd(&w.hdr[0], tot) : 0u;
-    }
-    __syncthreads();
-    uint32_t pos = s_base + s_wcnt[warp];
-    for (int it = 0; it < n_it; ++it) {
-        const uint32_t mask = s_mask[warp][it];
-        if (!mask) continue;
-        const int64_t e = e0 + static_cast<int64_t>(it) * kThreads + warp * 32 + lane;
-        if ((mask >> lane) & 1u)
-            w.cand[pos + __popc(mask & ((1u << lane) - 1u))] =
-                (static_cast<unsigned long long>(order_key(row[e])) << 32) | static_cast<uint32_t>(e);
-        pos += __popc(mask);
-    }
-}
-
-// block-wide exclusive prefix sum of one value per thread (kResolveThreads)
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* sh_warp, uint32_t* total) {
+// block-wide inclusive scan of one value per thread (kSelThreads threads)
+__device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t* sh_warp) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t x = v;
 #pragma unroll
@@ -525,180 +454,211 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* sh_war
     if (lane == 31) sh_warp[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        uint32_t s = sh_warp[lane];
+        uint32_t s = lane < kSelWarps ? sh_warp[lane] : 0u;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const uint32_t y = __shfl_up_sync(0xffffffffu, s, o);
             if (lane >= o) s += y;
         }
-        sh_warp[lane] = s;                       // inclusive per warp
+        if (lane < kSelWarps) sh_warp[lane] = s;
     }
     __syncthreads();
-    const uint32_t warp_off = warp > 0 ? sh_warp[warp - 1] : 0u;
-    *total = sh_warp[31];
-    const uint32_t r = warp_off + x - v;
+    const uint32_t r = (warp > 0 ? sh_warp[warp - 1] : 0u) + x;
     __syncthreads();
     return r;
 }
 
-__global__ void __launch_bounds__(kResolveThreads, 1)
-resolve_kernel(const int32_t* __restrict__ q_pos, int64_t Nc_cap, int m, int k, uint8_t* __restrict__ ws,
-               int32_t* __restrict__ idx, int32_t* __restrict__ count) {
-    constexpr int kCandCache = 4096;          // candidates kept in shared memory (else read from L2)
-    constexpr int kRegWords = 8;              // bitmap words a thread keeps in registers
-    __shared__ uint32_t hist2[kBins];
-    __shared__ unsigned long long s_cand[kCandCache];
+// Digit of a histogram h of nb bins (2048 or 1024; the largest digit is nb-1)
+// at which the count from the top reaches `need`.  Block-wide.  s_out[0] =
+// the digit, s_out[1] = need minus the count strictly above it, s_out[2] =
+// the count in it.  (An inconsistent histogram, whose total is below need,
+// leaves digit 0, need and 0: wrong but in bounds.)
+__device__ void find_digit(const uint32_t* h, uint32_t nb, uint32_t need, uint32_t* sh_warp, uint32_t* s_out) {
+    const int t = threadIdx.x;
+    if (t == 0) { s_out[0] = 0u; s_out[1] = need; s_out[2] = 0u; }
+    const uint32_t per = nb / kSelThreads;
+    uint32_t c[4] = {0u, 0u, 0u, 0u}, tot = 0;
+    for (uint32_t j = 0; j < per; ++j) { c[j] = h[nb - 1 - per * t - j]; tot += c[j]; }
+    const uint32_t incl = block_incl_scan(tot, sh_warp);     // (syncs: s_out initialised before any write)
+    const uint32_t before = incl - tot;
+    if (before < need && incl >= need) {
+        uint32_t acc = before;
+        for (uint32_t j = 0; j < per; ++j) {
+            if (acc + c[j] >= need) { s_out[0] = nb - 1 - per * t - j; s_out[1] = need - acc; s_out[2] = c[j]; break; }
+            acc += c[j];
+        }
+    }
+    __syncthreads();
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kSelThreads)
+select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, int64_t Nc_cap, int m, int k,
+              int64_t chunk, uint8_t* __restrict__ ws, int32_t* __restrict__ idx, int32_t* __restrict__ count) {
+    extern __shared__ __align__(16) unsigned long long dyn[];
+    uint32_t* s_ma = reinterpret_cast<uint32_t*>(dyn);                  // [warps][kMaxIt] above masks
+    uint32_t* s_mc = s_ma + kSelWarps * kMaxIt;                          // [warps][kMaxIt] candidate masks
+    unsigned long long* s_cand = dyn;                                    // resolve: candidate cache
+    uint32_t* s_sel = reinterpret_cast<uint32_t*>(dyn + kCandSmem);      // resolve: selected indices
+    __shared__ uint32_t s_hist[kBins];
     __shared__ uint32_t sh_warp[32];
-    __shared__ uint32_t s_digit, s_need;
-    const int64_t r = blockIdx.x;
-    const int tid = threadIdx.x;
+    __shared__ uint32_t s_dig[4];
+    __shared__ uint32_t s_wa[kSelWarps], s_wc[kSelWarps];
+    __shared__ uint32_t s_base[2];
+    __shared__ uint32_t s_nsel;
+    __shared__ int s_last;
+
+    const int64_t r = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t n = n_eligible(q_pos, r, m, Nc_cap);
     const uint32_t kk = static_cast<uint32_t>(min(static_cast<int64_t>(k), n));
     int32_t* orow = idx + static_cast<size_t>(r) * k;
-    if (tid == 0) count[r] = static_cast<int32_t>(kk);
     if (kk == 0) {
-        for (int j = tid; j < k; j += kResolveThreads) orow[j] = -1;
+        if (blockIdx.x == 0) {
+            if (tid == 0) count[r] = 0;
+            for (int j = tid; j < k; j += kSelThreads) orow[j] = -1;
+        }
         return;
     }
     RowWs w = row_ws(ws, Nc_cap, r);
-    const uint32_t n_cand = w.hdr[0], t1 = w.hdr[1], need1 = w.hdr[2];
-    const bool cached = n_cand <= static_cast<uint32_t>(kCandCache);
-    if (cached) {
-        // one round of loads for all candidates
-        unsigned long long v[kCandCache / kResolveThreads];
+    // ---- threshold bin T1 from the row's histogram (the same in every CTA)
+    for (int i = tid; i < kBins; i += kSelThreads) s_hist[i] = __ldcg(w.hist + i);
+    __syncthreads();
+    find_digit(s_hist, kBins, kk, sh_warp, s_dig);
+    const uint32_t t1 = s_dig[0];
+    const T* row = scores + static_cast<size_t>(r) * Nc_cap;
+    // ---- pass A over this CTA's chunk: per (warp, step) ballots of the keys
+    // above bin T1 and in bin T1
+    const int64_t e0 = static_cast<int64_t>(blockIdx.x) * chunk;
+    const int64_t e1 = min(e0 + chunk, n);
+    const int n_it = e1 > e0 ? static_cast<int>((e1 - e0 + kSelThreads - 1) / kSelThreads) : 0;
+    uint32_t ca = 0, cc = 0;
+    for (int it0 = 0; it0 < n_it; it0 += 8) {
+        float v[8];
 #pragma unroll
-        for (int j = 0; j < kCandCache / kResolveThreads; ++j) {
-            const uint32_t c = tid + j * kResolveThreads;
-            v[j] = c < n_cand ? w.cand[c] : 0ull;
+        for (int j = 0; j < 8; ++j) {
+            const int64_t e = e0 + static_cast<int64_t>(it0 + j) * kSelThreads + warp * 32 + lane;
+            v[j] = (it0 + j < n_it && e < e1) ? score_at(row, e) : 0.0f;
         }
 #pragma unroll
-        for (int j = 0; j < kCandCache / kResolveThreads; ++j) s_cand[tid + j * kResolveThreads] = v[j];
-        __syncthreads();
+        for (int j = 0; j < 8; ++j) {
+            const int it = it0 + j;
+            if (it >= n_it) break;
+            const int64_t e = e0 + static_cast<int64_t>(it) * kSelThreads + warp * 32 + lane;
+            const bool live = e < e1;
+            const uint32_t bin = order_key(v[j]) >> 21;
+            const unsigned above = __ballot_sync(0xffffffffu, live && bin > t1);
+            const unsigned in_t1 = __ballot_sync(0xffffffffu, live && bin == t1);
+            if (lane == 0) { s_ma[warp * kMaxIt + it] = above; s_mc[warp * kMaxIt + it] = in_t1; }
+            ca += __popc(above);
+            cc += __popc(in_t1);
+        }
     }
-    auto cand = [&](uint32_t c) { return cached ? s_cand[c] : w.cand[c]; };
-    // exact threshold key T among the candidates (all share the top 11 bits t1)
-    uint32_t prefix = t1 << 21, need = need1;
-    if (need1 < n_cand) {
-        // pass 1: bits 20..10 (2048 bins); pass 2: bits 9..0 (1024 bins) of keys matching the prefix
+    if (lane == 0) { s_wa[warp] = ca; s_wc[warp] = cc; }
+    __syncthreads();
+    if (tid == 0) {
+        uint32_t ta = 0, tc = 0;
+        for (int q = 0; q < kSelWarps; ++q) {
+            const uint32_t a = s_wa[q], c = s_wc[q];
+            s_wa[q] = ta; s_wc[q] = tc;
+            ta += a; tc += c;
+        }
+        s_base[0] = ta ? atomicAdd(&w.hdr[0], ta) : 0u;
+        s_base[1] = tc ? atomicAdd(&w.hdr[1], tc) : 0u;
+    }
+    __syncthreads();
+    // ---- pass B: append (ordered within the CTA; the lists' order is irrelevant)
+    {
+        uint32_t pa = s_base[0] + s_wa[warp], pc = s_base[1] + s_wc[warp];
+        const unsigned lt = (1u << lane) - 1u;
+        for (int it = 0; it < n_it; ++it) {
+            const uint32_t ma = s_ma[warp * kMaxIt + it], mc = s_mc[warp * kMaxIt + it];
+            const int64_t e = e0 + static_cast<int64_t>(it) * kSelThreads + warp * 32 + lane;
+            if ((ma >> lane) & 1u) {
+                const uint32_t at = pa + __popc(ma & lt);
+                if (at < static_cast<uint32_t>(kMaxK)) w.above[at] = static_cast<uint32_t>(e);
+            }
+            if ((mc >> lane) & 1u)
+                w.cand[pc + __popc(mc & lt)] =
+                    (static_cast<unsigned long long>(order_key(score_at(row, e))) << 32) |
+                    static_cast<uint32_t>(~static_cast<uint32_t>(e));
+            pa += __popc(ma);
+            pc += __popc(mc);
+        }
+    }
+    // ---- the last CTA of the row resolves it
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(&w.hdr[2], 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const uint32_t n_above = min(__ldcg(w.hdr + 0), kk);
+    const uint32_t n_cand = __ldcg(w.hdr + 1);
+    const bool cached = n_cand <= static_cast<uint32_t>(kCandSmem);
+    if (cached)
+        for (uint32_t c = tid; c < n_cand; c += kSelThreads) s_cand[c] = __ldcg(w.cand + c);
+    if (tid == 0) s_nsel = n_above;
+    __syncthreads();
+    auto cand = [&](uint32_t c) { return cached ? s_cand[c] : __ldcg(w.cand + c); };
+    uint32_t need = kk - n_above;
+    // threshold: candidates whose composite, on the bits fixed so far, is >= prefix
+    unsigned long long prefix = 0ull, fmask = 0ull;
+    if (need < n_cand) {
+        prefix = static_cast<unsigned long long>(t1) << 53;
+        fmask = 0xFFE0000000000000ull;
+        // digits of the composite below the 11 bits of bin T1: 11, 10 (the rest of
+        // the score key), then 11, 11, 10 (the complemented index)
 #pragma unroll 1
-        for (int pass = 0; pass < 2; ++pass) {
-            const int shift = pass == 0 ? 10 : 0;
-            const uint32_t nb = pass == 0 ? 2048u : 1024u;
-            const uint32_t mask_hi = pass == 0 ? 0xFFE00000u : 0xFFFFFC00u;   // bits already fixed
-            for (uint32_t i = tid; i < nb; i += kResolveThreads) hist2[i] = 0;
+        for (int ps = 0; ps < 5; ++ps) {
+            const int width = (ps == 1 || ps == 4) ? 10 : 11;
+            const int shift = ps == 0 ? 42 : ps == 1 ? 32 : ps == 2 ? 21 : ps == 3 ? 10 : 0;
+            const uint32_t nb = 1u << width;
+            for (uint32_t i = tid; i < nb; i += kSelThreads) s_hist[i] = 0u;
             __syncthreads();
-            for (uint32_t c = tid; c < n_cand; c += kResolveThreads) {
-                const uint32_t key = static_cast<uint32_t>(cand(c) >> 32);
-                if ((key & mask_hi) == prefix) atomicAdd(&hist2[(key >> shift) & (nb - 1)], 1u);
-            }
-            __syncthreads();
-            {
-                // from the top digit down: the digit where the running count reaches need.
-                // Thread t holds digits nb-1-bpt*t .. nb-bpt*(t+1) (top first); a block
-                // scan gives the count above its digits.
-                const uint32_t bpt = nb / kResolveThreads;     // 2 or 1
-                uint32_t cnt[2] = {0u, 0u}, tot = 0;
-                for (uint32_t j = 0; j < bpt; ++j) { cnt[j] = hist2[nb - 1 - bpt * tid - j]; tot += cnt[j]; }
-                uint32_t all;
-                const uint32_t above = block_excl_scan(tot, sh_warp, &all);
-                if (above < need && above + tot >= need) {
-                    uint32_t acc = above;
-                    for (uint32_t j = 0; j < bpt; ++j) {
-                        if (acc + cnt[j] >= need) { s_digit = nb - 1 - bpt * tid - j; s_need = need - acc; break; }
-                        acc += cnt[j];
-                    }
-                }
+            for (uint32_t c = tid; c < n_cand; c += kSelThreads) {
+                const unsigned long long v = cand(c);
+                if ((v & fmask) == prefix) atomicAdd(&s_hist[(v >> shift) & (nb - 1u)], 1u);
             }
             __syncthreads();
-            prefix |= s_digit << shift;
-            need = s_need;
+            find_digit(s_hist, nb, need, sh_warp, s_dig);
+            prefix |= static_cast<unsigned long long>(s_dig[0]) << shift;
+            fmask |= static_cast<unsigned long long>(nb - 1u) << shift;
+            need = s_dig[1];
+            const bool whole = s_dig[2] == need;            // every key of this digit is selected
             __syncthreads();
-        }
-        // keys above T: selected; keys equal to T: ties (need of them, lowest index first)
-        for (uint32_t c = tid; c < n_cand; c += kResolveThreads) {
-            const unsigned long long v = cand(c);
-            const uint32_t key = static_cast<uint32_t>(v >> 32), e = static_cast<uint32_t>(v);
-            if (key > prefix) atomicOr(&w.sel[e >> 5], 1u << (e & 31));
-            else if (key == prefix) atomicOr(&w.tie[e >> 5], 1u << (e & 31));
-        }
-    } else {
-        for (uint32_t c = tid; c < n_cand; c += kResolveThreads) {
-            const uint32_t e = static_cast<uint32_t>(cand(c));
-            atomicOr(&w.sel[e >> 5], 1u << (e & 31));
-        }
-        need = 0;
-    }
-    __syncthreads();       // the bitmap updates above are visible to the whole block
-    // ordered output over the eligible words: thread t owns a contiguous run of words
-    const int64_t words = (n + 31) / 32;
-    const int64_t per = (words + kResolveThreads - 1) / kResolveThreads;
-    const int64_t w0 = min(words, per * tid), w1 = min(words, w0 + per);
-    if (per <= kRegWords) {
-        // the thread's words in registers: one round of loads for both scans and the write
-        uint32_t sl[kRegWords], tw[kRegWords];
-#pragma unroll
-        for (int j = 0; j < kRegWords; ++j) {
-            sl[j] = w0 + j < w1 ? w.sel[w0 + j] : 0u;
-            tw[j] = w0 + j < w1 ? w.tie[w0 + j] : 0u;
-        }
-        uint32_t n_tie = 0;
-#pragma unroll
-        for (int j = 0; j < kRegWords; ++j) n_tie += __popc(tw[j]);
-        uint32_t tie_total;
-        const uint32_t tie_before = block_excl_scan(n_tie, sh_warp, &tie_total);
-        // take the lowest ties while the row still needs them
-        uint32_t tb = tie_before, n_sel = 0;
-#pragma unroll
-        for (int j = 0; j < kRegWords; ++j) {
-            uint32_t t = tw[j];
-            while (t && tb < need) { const uint32_t lo = t & (~t + 1u); sl[j] |= lo; t ^= lo; ++tb; }
-            tb += __popc(t);
-            n_sel += __popc(sl[j]);
-        }
-        uint32_t sel_total;
-        uint32_t out = block_excl_scan(n_sel, sh_warp, &sel_total);
-#pragma unroll
-        for (int j = 0; j < kRegWords; ++j) {
-            uint32_t bits = sl[j];
-            while (bits) {
-                const int b = __ffs(bits) - 1;
-                bits &= bits - 1u;
-                if (out < static_cast<uint32_t>(k)) orow[out] = static_cast<int32_t>((w0 + j) * 32 + b);
-                ++out;
-            }
-        }
-    } else {
-        uint32_t n_tie = 0;
-        for (int64_t q = w0; q < w1; ++q) n_tie += __popc(w.tie[q]);
-        uint32_t tie_total;
-        const uint32_t tie_before = block_excl_scan(n_tie, sh_warp, &tie_total);
-        uint32_t n_sel = 0;
-        {
-            uint32_t tb = tie_before;
-            for (int64_t q = w0; q < w1; ++q) {
-                const uint32_t nt = __popc(w.tie[q]);
-                const uint32_t take = tb >= need ? 0u : min(nt, need - tb);
-                n_sel += __popc(w.sel[q]) + take;
-                tb += nt;
-            }
-        }
-        uint32_t sel_total;
-        uint32_t out = block_excl_scan(n_sel, sh_warp, &sel_total);
-        uint32_t tb = tie_before;
-        for (int64_t q = w0; q < w1; ++q) {
-            uint32_t bits = w.sel[q];
-            uint32_t t = w.tie[q];
-            while (t && tb < need) { const uint32_t lo = t & (~t + 1u); bits |= lo; t ^= lo; ++tb; }
-            tb += __popc(t);
-            while (bits) {
-                const int b = __ffs(bits) - 1;
-                bits &= bits - 1u;
-                if (out < static_cast<uint32_t>(k)) orow[out] = static_cast<int32_t>(q * 32 + b);
-                ++out;
-            }
+            if (whole) break;
         }
     }
-    for (int j = static_cast<int>(kk) + tid; j < k; j += kResolveThreads) orow[j] = -1;
+    // ---- gather: the keys above bin T1, then the candidates at or above the threshold
+    for (uint32_t i = tid; i < n_above; i += kSelThreads) s_sel[i] = __ldcg(w.above + i);
+    for (uint32_t c = tid; c < n_cand; c += kSelThreads) {
+        const unsigned long long v = cand(c);
+        if ((v & fmask) >= prefix) {
+            const uint32_t at = atomicAdd(&s_nsel, 1u);
+            if (at < static_cast<uint32_t>(kMaxK)) s_sel[at] = ~static_cast<uint32_t>(v);
+        }
+    }
+    __syncthreads();
+    // ---- ascending order: bitonic network over the next power of two
+    uint32_t P = 1;
+    while (P < kk) P <<= 1;
+    for (uint32_t i = kk + tid; i < P; i += kSelThreads) s_sel[i] = 0xFFFFFFFFu;
+    __syncthreads();
+    for (uint32_t size = 2; size <= P; size <<= 1) {
+        for (uint32_t stride = size >> 1; stride > 0; stride >>= 1) {
+            for (uint32_t i = tid; i < P / 2; i += kSelThreads) {
+                const uint32_t lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
+                const bool asc = (lo & size) == 0;
+                const uint32_t a = s_sel[lo], b = s_sel[hi];
+                if ((a > b) == asc) { s_sel[lo] = b; s_sel[hi] = a; }
+            }
+            __syncthreads();
+        }
+    }
+    for (uint32_t j = tid; j < static_cast<uint32_t>(k); j += kSelThreads)
+        orow[j] = j < kk ? static_cast<int32_t>(s_sel[j]) : -1;
+    if (tid == 0) count[r] = static_cast<int32_t>(kk);
 }
 
 }  // namespace wide
@@ -715,7 +675,7 @@ size_t topk_wide_ws_bytes(int R, int64_t Nc_cap) {
     return static_cast<size_t>(R) * wide::layout(Nc_cap).row_bytes;
 }
 
-// clear each row's histogram, header and bitmaps
+// clear each row's histogram and header
 int topk_wide_clear(void* ws, int R, int64_t Nc_cap, cudaStream_t st) {
     const wide::Layout L = wide::layout(Nc_cap);
     cudaError_t e = cudaMemset2DAsync(ws, L.row_bytes, 0, L.clear_bytes, static_cast<size_t>(R), st);
@@ -729,35 +689,56 @@ uint32_t* topk_wide_hist(void* ws, int64_t Nc_cap, int64_t* stride_u32) {
     return static_cast<uint32_t*>(ws);
 }
 
-static int64_t wide_chunk(int R, int64_t Nc_cap) {
-    const int64_t ctas_per_row = std::max<int64_t>(1, ceil_div(2LL * sm_count(), R));
+// scores per CTA: about one CTA per SM over all rows, whole 512-score steps
+static int64_t wide_chunk(int R, int64_t Nc_cap, int per_step) {
+    const int64_t ctas_per_row = std::max<int64_t>(1, ceil_div(sm_count(), R));
     int64_t chunk = ceil_div(Nc_cap, ctas_per_row);
-    chunk = std::max<int64_t>(256, ceil_div(chunk, 256) * 256);       // whole bitmap words per warp
-    return std::min<int64_t>(chunk, static_cast<int64_t>(wide::kMaxIt) * wide::kThreads);
+    chunk = std::max<int64_t>(per_step, ceil_div(chunk, per_step) * per_step);
+    return std::min<int64_t>(chunk, static_cast<int64_t>(wide::kMaxIt) * per_step);
 }
 
-// mark + resolve, given the rows' histograms (by hist_kernel or by the indexer)
-int topk_wide_select(const float* scores, const int32_t* q_pos, int R, int64_t Nc_cap, int m, int k,
-                     int32_t* idx, int32_t* count, void* ws, cudaStream_t st) {
-    uint8_t* w = static_cast<uint8_t*>(ws);
-    const int64_t chunk = wide_chunk(R, Nc_cap);
+// select + resolve, given the rows' histograms (by hist_kernel or by the indexer);
+// bf16: the scores are bf16 bit patterns (uint16)
+int topk_wide_select(const void* scores, const int32_t* q_pos, int R, int64_t Nc_cap, int m, int k,
+                     int32_t* idx, int32_t* count, void* ws, cudaStream_t st, bool bf16) {
+    static bool attr_set[2][64] = {{false}, {false}};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[bf16][dev]) {
+        const cudaError_t e =
+            bf16 ? cudaFuncSetAttribute(wide::select_kernel<uint16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(wide::kSelSmem))
+                 : cudaFuncSetAttribute(wide::select_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(wide::kSelSmem));
+        if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
+        attr_set[bf16][dev] = true;
+    }
+    const int64_t chunk = wide_chunk(R, Nc_cap, wide::kSelThreads);
     const dim3 grid(static_cast<unsigned>(ceil_div(Nc_cap, chunk)), static_cast<unsigned>(R));
-    wide::mark_kernel<<<grid, wide::kThreads, 0, st>>>(scores, q_pos, Nc_cap, m, k, chunk, w);
-    HCA_CHECK_LAUNCH();
-    wide::resolve_kernel<<<R, wide::kResolveThreads, 0, st>>>(q_pos, Nc_cap, m, k, w, idx, count);
+    if (bf16)
+        wide::select_kernel<uint16_t><<<grid, wide::kSelThreads, wide::kSelSmem, st>>>(
+            static_cast<const uint16_t*>(scores), q_pos, Nc_cap, m, k, chunk, static_cast<uint8_t*>(ws), idx, count);
+    else
+        wide::select_kernel<float><<<grid, wide::kSelThreads, wide::kSelSmem, st>>>(
+            static_cast<const float*>(scores), q_pos, Nc_cap, m, k, chunk, static_cast<uint8_t*>(ws), idx, count);
     HCA_CHECK_LAUNCH();
     return HCA_OK;
 }
 
-int topk_wide_launch(const float* scores, const int32_t* q_pos, int R, int64_t Nc_cap, int m, int k,
-                     int32_t* idx, int32_t* count, void* ws, cudaStream_t st) {
+int topk_wide_launch(const void* scores, const int32_t* q_pos, int R, int64_t Nc_cap, int m, int k,
+                     int32_t* idx, int32_t* count, void* ws, cudaStream_t st, bool bf16) {
     const int rc = topk_wide_clear(ws, R, Nc_cap, st);
     if (rc != HCA_OK) return rc;
-    const int64_t chunk = wide_chunk(R, Nc_cap);
+    const int64_t chunk = wide_chunk(R, Nc_cap, wide::kThreads * 8);
     const dim3 grid(static_cast<unsigned>(ceil_div(Nc_cap, chunk)), static_cast<unsigned>(R));
-    wide::hist_kernel<<<grid, wide::kThreads, 0, st>>>(scores, q_pos, Nc_cap, m, chunk, static_cast<uint8_t*>(ws));
+    if (bf16)
+        wide::hist_kernel<uint16_t><<<grid, wide::kThreads, 0, st>>>(static_cast<const uint16_t*>(scores), q_pos,
+                                                                    Nc_cap, m, chunk, static_cast<uint8_t*>(ws));
+    else
+        wide::hist_kernel<float><<<grid, wide::kThreads, 0, st>>>(static_cast<const float*>(scores), q_pos, Nc_cap,
+                                                                 m, chunk, static_cast<uint8_t*>(ws));
     HCA_CHECK_LAUNCH();
-    return topk_wide_select(scores, q_pos, R, Nc_cap, m, k, idx, count, ws, st);
+    return topk_wide_select(scores, q_pos, R, Nc_cap, m, k, idx, count, ws, st, bf16);
 }
 
 int topk_launch(const float* scores, const int32_t* q_pos, int R, int64_t Nc_cap, int m, int k,
@@ -765,7 +746,7 @@ int topk_launch(const float* scores, const int32_t* q_pos, int R, int64_t Nc_cap
     if (R == 0) return HCA_OK;
     if (topk_wide_preferred(R, Nc_cap) && ws != nullptr && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0 &&
         ws_bytes >= topk_wide_ws_bytes(R, Nc_cap) && R <= 65535 && Nc_cap <= 0x7FFFFFFFLL)
-        return topk_wide_launch(scores, q_pos, R, Nc_cap, m, k, idx, count, ws, st);
+        return topk_wide_launch(scores, q_pos, R, Nc_cap, m, k, idx, count, ws, st, false);
     if (Nc_cap > 16 * kSliceMax) return HCA_ERR_WORKSPACE;   // only the workspace path takes such rows
     if (g_max_cluster == 0) {
         // probe once whether 16-CTA clusters of this kernel fit the device

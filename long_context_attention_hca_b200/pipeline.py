@@ -20,7 +20,7 @@ import torch
 
 from . import (KVCache, compressed_attn_decode, compressed_attn_prefill, csa_compress, decode_workspace_size,
                hca_compress, lightning_index, lightning_index_topk, topk_select, topk_workspace_size,
-               set_launch_budget, BUDGET_DENSE_DECODE)
+               set_launch_budget, BUDGET_DENSE_DECODE, BUDGET_SPARSE_DECODE, BUDGET_DECODE_INDEX)
 
 CSA_RATIO = 4
 HCA_RATIO = 128
@@ -70,21 +70,27 @@ class DecodeRunner:
     compressed_attn_decode(dense).  CSA chains run on `side`, a stream of
     higher priority, and HCA on the current stream; the step ends with both
     joined.  An HCA launch waits for the indexer queued before it: the
-    indexer fills every SM anyway, and the top-k that follows it needs whole
-    clusters of free SMs, which the HCA CTAs (one per SM) would otherwise
-    hold when the indexer drains."""
+    indexer fills every SM anyway."""
 
     def __init__(self, layers: List[DecodeLayer], B: int, H: int, k: int, pos: int, softmax_scale: float,
-                 device="cuda", schedule: str = "after_index", dense_budget: int = 0, fused_select: bool = True):
+                 device="cuda", schedule: str = "after_index", dense_budget: int = 0, fused_select: bool = True,
+                 sparse_budget: int = 0, extras: Optional[list] = None, index_budget: int = 0):
         """schedule: "after_index" -- an HCA launch waits for the indexer queued
         before it; "hca_first" -- all HCA launches are queued first and start at
         once, with dense_budget (if > 0) capping their CTAs so that the CSA
-        chain runs beside them on the remaining SMs."""
+        chain runs beside them on the remaining SMs.  extras: per layer, an
+        AttnExtras (section 9 query RMSNorm, RoPE, sink) for its attention
+        call, or None."""
+        self.extras = extras if extras is not None else [None] * len(layers)
         if schedule not in ("after_index", "hca_first"):
             raise ValueError(schedule)
         self.schedule = schedule
         if dense_budget:
             set_launch_budget(BUDGET_DENSE_DECODE, dense_budget)
+        if sparse_budget:
+            set_launch_budget(BUDGET_SPARSE_DECODE, sparse_budget)
+        if index_budget:
+            set_launch_budget(BUDGET_DECODE_INDEX, index_budget)
         self.layers, self.B, self.H, self.k, self.pos = layers, B, H, k, pos
         self.scale = softmax_scale
         d = layers[0].cache.layout[0]
@@ -122,8 +128,9 @@ class DecodeRunner:
 
     def _count_kernels(self) -> int:
         """Kernels of this library launched per step: attention (+ split combine) per
-        layer; per CSA layer the indexer and the top-k (three kernels on the
-        histogram path, one on the cluster path)."""
+        layer; per CSA layer the indexer and the top-k (the select kernel, after
+        a histogram kernel unless the indexer built the histogram, on the
+        histogram path; one cluster kernel otherwise)."""
         n = 0
         for li, L in enumerate(self.layers):
             mc = min(self.k, L.n_entries) if L.ratio == CSA_RATIO else L.n_entries
@@ -131,9 +138,58 @@ class DecodeRunner:
             n += 1 + int(split)
             if L.ratio == CSA_RATIO:
                 wide = topk_workspace_size(self.B, L.n_entries, self.k) > 0
-                # indexer + (histogram,) mark, resolve on the histogram path; else the cluster kernel
-                n += 1 + ((2 if self.fused_select[li] else 3) if wide else 1)
+                n += 1 + ((1 if self.fused_select[li] else 2) if wide else 1)
         return n
+
+    def capi_plan(self, d_q: List[torch.Tensor], d_iq: List[Optional[tuple]]):
+        """The hca_decode_step_plan of this runner's two layers (one CSA, one
+        HCA), for hca_decode_step_host: the caches, keys and windows of the
+        layers, d_q / d_iq as the staging buffers of the queries, this runner's
+        scores, top-k and attention buffers, a side stream and four events."""
+        from . import CacheStruct, DecodeStepPlan, Layout
+        ci = [li for li, L in enumerate(self.layers) if L.ratio == CSA_RATIO]
+        hi = [li for li, L in enumerate(self.layers) if L.ratio == HCA_RATIO]
+        if len(ci) != 1 or len(hi) != 1:
+            raise ValueError("capi_plan: one CSA and one HCA layer")
+        c_, h_ = ci[0], hi[0]
+        Lc, Lh = self.layers[c_], self.layers[h_]
+        qc, qs, w = d_iq[c_]
+        lo, hi_prio = torch.cuda.Stream.priority_range()
+        self._capi_side = torch.cuda.Stream(device=d_q[0].device, priority=lo)
+        self._capi_events = [torch.cuda.Event() for _ in range(4)]
+        for e in self._capi_events:
+            e.record(torch.cuda.current_stream())     # creates the CUDA event (outside any capture)
+        torch.cuda.synchronize()
+        ptr = lambda t: t.data_ptr()
+        p = DecodeStepPlan()
+        p.B, p.H, p.Hi, p.c, p.k, p.W = self.B, self.H, qc.shape[2], qc.shape[3] * 2, self.k, Lc.window.shape[1]
+        p.softmax_scale = self.scale
+        p.layout = Layout(*Lc.cache.layout)
+        p.csa_cache = Lc.cache.c_struct
+        p.csa_entries = Lc.n_entries
+        p.k_codes, p.k_sf, p.csa_window = ptr(Lc.k_codes), ptr(Lc.k_sf), ptr(Lc.window)
+        p.hca_cache = Lh.cache.c_struct
+        p.hca_n, p.hca_max, p.hca_window = ptr(self.n_dense[h_]), Lh.n_entries, ptr(Lh.window)
+        p.q_pos = ptr(self.q_pos)
+        p.q_csa, p.q_hca = ptr(d_q[c_]), ptr(d_q[h_])
+        p.iq_codes, p.iq_sf, p.iq_w = ptr(qc), ptr(qs), ptr(w)
+        p.scores, p.idx, p.count = ptr(self.scores[c_]), ptr(self.idx[c_]), ptr(self.count[c_])
+        p.topk_ws, p.topk_ws_bytes = ptr(self.topk_ws[c_]), self.topk_ws[c_].numel()
+        p.ws_csa, p.ws_csa_bytes = ptr(self.ws[c_]), self.ws[c_].numel()
+        p.ws_hca, p.ws_hca_bytes = ptr(self.ws[h_]), self.ws[h_].numel()
+        p.out_csa, p.out_hca = ptr(self.out[c_]), ptr(self.out[h_])
+        p.side_stream = self._capi_side.cuda_stream
+        p.ev_fork, p.ev_index, p.ev_q, p.ev_join = (e.cuda_event for e in self._capi_events)
+        self._capi_layers = (c_, h_)
+        return p
+
+    def step_host_capi(self, plan, h_q: List[torch.Tensor], h_iq: List[Optional[tuple]], h_out: List[torch.Tensor]):
+        """One decode step through hca_decode_step_host (the C ABI's host-to-host
+        call): pinned host queries in, pinned host outputs out."""
+        from . import decode_step_host
+        c_, h_ = self._capi_layers
+        decode_step_host(plan, h_q[c_], h_q[h_], h_iq[c_], h_out[c_], h_out[h_])
+        return h_out
 
     def step_host(self, h_q: List[torch.Tensor], h_iq: List[Optional[tuple]], h_out: List[torch.Tensor],
                   d_q: List[torch.Tensor], d_iq: List[Optional[tuple]]):
@@ -221,7 +277,7 @@ class DecodeRunner:
                         self.side.wait_event(q_ready[li])
                     timed("csa_attn", li, lambda: compressed_attn_decode(
                         q[li], L.cache, self.count[li], min(self.k, L.n_entries), L.window, self.scale,
-                        idx=self.idx[li], out=self.out[li], ws=self.ws[li]))
+                        idx=self.idx[li], out=self.out[li], ws=self.ws[li], extras=self.extras[li]))
                     if on_out is not None:
                         on_out(li, self.side)
             else:
@@ -231,7 +287,7 @@ class DecodeRunner:
                     main.wait_event(q_ready[li])
                 timed("hca_attn", li, lambda: compressed_attn_decode(
                     q[li], L.cache, self.n_dense[li], L.n_entries, L.window, self.scale, out=self.out[li],
-                    ws=self.ws[li]))
+                    ws=self.ws[li], extras=self.extras[li]))
                 if on_out is not None:
                     on_out(li, main)
         main.wait_stream(self.side)
@@ -247,6 +303,7 @@ class PrefillState:
     k_sf: torch.Tensor
     bias4: torch.Tensor                 # [4][d]
     bias128: torch.Tensor               # [128][d]
+    entry_extras: object = None         # EntryExtras used when the chunk's entries are stored (or None)
 
 
 class PrefillRunner:
@@ -256,7 +313,10 @@ class PrefillRunner:
     CSA (sparse) and HCA (dense causal) attention with the causal window."""
 
     def __init__(self, st: PrefillState, p0: int, Tq: int, H: int, k: int, W: int, softmax_scale: float,
-                 device="cuda"):
+                 device="cuda", extras=None):
+        """extras: an AttnExtras (section 9 query RMSNorm, RoPE, sink) for both
+        attention calls, or None."""
+        self.extras = extras
         assert p0 % HCA_RATIO == 0 and Tq % HCA_RATIO == 0
         self.st, self.p0, self.Tq, self.H, self.k, self.W, self.scale = st, p0, Tq, H, k, W, softmax_scale
         dev = torch.device(device)
@@ -285,16 +345,19 @@ class PrefillRunner:
         def timed(name, fn):
             if events is None:
                 return fn()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
+            # external events stay timing events when the step is captured into a graph
+            a = torch.cuda.Event(enable_timing=True, external=True)
+            b = torch.cuda.Event(enable_timing=True, external=True)
             a.record()
             fn()
             b.record()
             events[name] = (a, b)
 
         def compress():
-            csa_compress(raw_chunk, gate_chunk, st.bias4, Tq // CSA_RATIO, st.csa, entry_begin=p0 // CSA_RATIO)
-            hca_compress(raw_chunk, gate_chunk, st.bias128, Tq // HCA_RATIO, st.hca, entry_begin=p0 // HCA_RATIO)
+            csa_compress(raw_chunk, gate_chunk, st.bias4, Tq // CSA_RATIO, st.csa, entry_begin=p0 // CSA_RATIO,
+                         extras=st.entry_extras)
+            hca_compress(raw_chunk, gate_chunk, st.bias128, Tq // HCA_RATIO, st.hca, entry_begin=p0 // HCA_RATIO,
+                         extras=st.entry_extras)
 
         timed("compress", compress)
         self.side.wait_stream(main)
@@ -306,8 +369,156 @@ class PrefillRunner:
                                               idx=self.idx, count=self.count))
             timed("csa_attn", lambda: compressed_attn_prefill(q, p0, CSA_RATIO, st.csa, raw_window, self.W,
                                                               self.scale, idx=self.idx, count=self.count,
-                                                              out=self.out_csa))
+                                                              out=self.out_csa, extras=self.extras))
         timed("hca_attn", lambda: compressed_attn_prefill(q, p0, HCA_RATIO, st.hca, raw_window, self.W, self.scale,
-                                                          out=self.out_hca))
+                                                          out=self.out_hca, extras=self.extras))
         main.wait_stream(self.side)
         return self.out_csa, self.out_hca
+
+
+# ------------------------------------------------------------------ state-cache decode loop
+@dataclasses.dataclass
+class LoopLayer:
+    """One layer of a state-cache decode loop: the classical cache of
+    compressed entries (none for ratio 0), and the per-sequence state cache:
+    the window ring of the last W tokens and the raw tail of the block not yet
+    complete ("DeepSeek V4 ..." note, section 11, KV cache table)."""
+    ratio: int                                  # 0 (window only), 4 (CSA) or 128 (HCA)
+    window: torch.Tensor                        # [B][W][d] ring, token at position p in row p % W
+    cache: Optional[KVCache] = None             # capacity = max_tokens // ratio
+    tail_x: Optional[torch.Tensor] = None       # [B][ratio][d] the current block's raw tokens
+    tail_gate: Optional[torch.Tensor] = None
+    bias: Optional[torch.Tensor] = None         # [ratio][d]
+    k_codes: Optional[torch.Tensor] = None      # CSA: indexer keys of every entry [B][cap][c/2]
+    k_sf: Optional[torch.Tensor] = None
+    entry_extras: object = None                 # EntryExtras (section 9) or None
+    s9: Optional[dict] = None                   # section 9 attention parameters (q_norm_w, sink, inv_freq, eps)
+
+
+class DecodeLoop:
+    """Token-by-token decode over a state cache.  All B sequences advance in
+    lockstep; step(t) takes token t of every sequence, for each layer:
+      1. appends it to the window ring and the block tail (kv_state_append;
+         with the section 9 extras the window keeps the token RMS-normalised
+         and rotated, kv_token_prep);
+      2. pools the block when t is its last token (csa_compress /
+         hca_compress of the tail into entry (t+1)/m - 1);
+      3. runs attention at position t: CSA layers index every eligible entry,
+         select the top-k and attend to them plus the window; HCA layers
+         attend to every complete entry plus the window; ratio-0 layers (the
+         note's section 8 compress_ratio table: compressed branch disabled)
+         attend to the window alone.  Before the window is full only its
+         first t+1 rows hold tokens (win_len)."""
+
+    def __init__(self, B: int, H: int, layout, ratios: List[int], W: int, k: int, max_tokens: int,
+                 softmax_scale: float, Hi: int = 4, c: int = 128, device="cuda", s9: Optional[List[dict]] = None):
+        from . import EntryExtras
+        d, dr, g = layout
+        dev = torch.device(device)
+        self.B, self.H, self.layout, self.W, self.k, self.scale = B, H, tuple(layout), W, k, softmax_scale
+        self.ratios, self.max_tokens, self.Hi, self.c = list(ratios), max_tokens, Hi, c
+        self.layers: List[LoopLayer] = []
+        for li, r in enumerate(ratios):
+            P = s9[li] if s9 is not None else None
+            L = LoopLayer(r, torch.zeros((B, W, d), dtype=torch.bfloat16, device=dev), s9=P)
+            if P is not None:
+                L.entry_extras = EntryExtras(P["kv_norm_w"], P["eps"], P["inv_freq"])
+            if r > 0:
+                L.cache = KVCache(B, max_tokens // r, layout, device=dev, zero=True)
+                L.tail_x = torch.zeros((B, r, d), dtype=torch.bfloat16, device=dev)
+                L.tail_gate = torch.zeros((B, r, d), dtype=torch.bfloat16, device=dev)
+            self.layers.append(L)
+        # a one-entry cache for window-only layers (the attention call takes a cache; it reads no entry)
+        self._empty = KVCache(B, 1, layout, device=dev, zero=True)
+        self.q_pos = torch.zeros((B,), dtype=torch.int32, device=dev)
+        self.win_len = torch.zeros((B,), dtype=torch.int32, device=dev)
+        self.n_ent = {r: torch.zeros((B,), dtype=torch.int32, device=dev) for r in set(ratios)}
+        self.out = [torch.empty((B, H, d), dtype=torch.bfloat16, device=dev) for _ in ratios]
+        self.scores, self.idx, self.count, self.topk_ws, self.ws = {}, {}, {}, {}, {}
+        for li, L in enumerate(self.layers):
+            mc = 0
+            if r_is_csa(L.ratio):
+                cap = L.cache.capacity
+                self.scores[li] = torch.empty((B, 1, cap), dtype=torch.float32, device=dev)
+                self.idx[li] = torch.empty((B, k), dtype=torch.int32, device=dev)
+                self.count[li] = torch.empty((B,), dtype=torch.int32, device=dev)
+                self.topk_ws[li] = torch.empty(max(topk_workspace_size(B, cap, k), 16), dtype=torch.uint8,
+                                               device=dev)
+                mc = min(k, cap)
+            elif L.ratio > 0:
+                mc = L.cache.capacity
+            self.ws[li] = torch.empty(max(decode_workspace_size(B, H, layout, mc, W), 16), dtype=torch.uint8,
+                                      device=dev)
+
+    def set_indexer_keys(self, li: int, k_codes: torch.Tensor, k_sf: torch.Tensor):
+        """CSA layer li: the indexer key of every entry the loop may create
+        ([B][max_tokens/4][c/2], [B][max_tokens/4][c/32]; given inputs)."""
+        self.layers[li].k_codes, self.layers[li].k_sf = k_codes, k_sf
+
+    def load_prefix(self, li: int, x: torch.Tensor, gate: torch.Tensor, bias: torch.Tensor, t0: int):
+        """State of layer li after tokens 0..t0-1 (x, gate: [B][>=t0][d]): every
+        complete block pooled, the tail holding the incomplete block's tokens,
+        the window ring holding the last min(W, t0) tokens."""
+        L = self.layers[li]
+        L.bias = bias
+        r = L.ratio
+        if r > 0:
+            n_blk = t0 // r
+            if n_blk:
+                (csa_compress if r == CSA_RATIO else hca_compress)(x, gate, bias, n_blk, L.cache,
+                                                                   extras=L.entry_extras)
+            for p in range(n_blk * r, t0):
+                L.tail_x[:, p % r].copy_(x[:, p])
+                L.tail_gate[:, p % r].copy_(gate[:, p])
+        from . import kv_token_prep
+        for p in range(max(0, t0 - self.W), t0):
+            tok = x[:, p].contiguous()
+            if L.entry_extras is not None:
+                pos = torch.full((self.B,), p, dtype=torch.int32, device=tok.device)
+                tok = kv_token_prep(tok, pos, self.layout, L.entry_extras)
+            L.window[:, p % self.W].copy_(tok)
+
+    def step(self, t: int, x_new: List[torch.Tensor], gate_new: List[torch.Tensor], q: List[torch.Tensor],
+             iq: List[Optional[tuple]], stream=None):
+        """Token t of every sequence: x_new[li], gate_new[li] [B][d] bf16,
+        q[li] [B][H][d] bf16, iq[li] (codes [B][1][Hi][c/2], sf, w [B][1][Hi])
+        for CSA layers.  Returns the per-layer outputs [B][H][d]."""
+        from . import AttnExtras, kv_state_append, kv_token_prep
+        self.q_pos.fill_(t)
+        self.win_len.fill_(min(self.W, t + 1))
+        for r, n in self.n_ent.items():
+            n.fill_((t + 1) // r if r > 0 else 0)
+        for li, L in enumerate(self.layers):
+            win_x = None
+            if L.entry_extras is not None:
+                win_x = kv_token_prep(x_new[li], self.q_pos, self.layout, L.entry_extras)
+            kv_state_append(x_new[li], gate_new[li], t, L.window, L.tail_x, L.tail_gate, win_x=win_x,
+                            stream=stream)
+            r = L.ratio
+            if r > 0 and (t + 1) % r == 0:
+                (csa_compress if r == CSA_RATIO else hca_compress)(L.tail_x, L.tail_gate, L.bias, 1, L.cache,
+                                                                   entry_begin=(t + 1) // r - 1,
+                                                                   extras=L.entry_extras, stream=stream)
+            P = L.s9
+            ex = AttnExtras(P["q_norm_w"] if P else None, P["eps"] if P else 1e-6, P["sink"] if P else None,
+                            P["inv_freq"] if P else None, self.q_pos, self.win_len)
+            if r == CSA_RATIO:
+                cap = L.cache.capacity
+                qc, qs, w = iq[li]
+                lightning_index(qc, qs, w, L.k_codes, L.k_sf, self.q_pos.view(self.B, 1), CSA_RATIO,
+                                scores=self.scores[li], stream=stream)
+                topk_select(self.scores[li].view(self.B, cap), self.q_pos, CSA_RATIO, self.k, idx=self.idx[li],
+                            count=self.count[li], ws=self.topk_ws[li], stream=stream)
+                compressed_attn_decode(q[li], L.cache, self.count[li], min(self.k, cap), L.window, self.scale,
+                                       idx=self.idx[li], out=self.out[li], ws=self.ws[li], stream=stream, extras=ex)
+            elif r == HCA_RATIO:
+                compressed_attn_decode(q[li], L.cache, self.n_ent[r], L.cache.capacity, L.window, self.scale,
+                                       out=self.out[li], ws=self.ws[li], stream=stream, extras=ex)
+            else:
+                compressed_attn_decode(q[li], self._empty, self.n_ent[0], 0, L.window, self.scale,
+                                       out=self.out[li], ws=self.ws[li], stream=stream, extras=ex)
+        return self.out
+
+
+def r_is_csa(ratio: int) -> bool:
+    return ratio == CSA_RATIO

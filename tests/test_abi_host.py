@@ -132,5 +132,65 @@ def test_fused_selection_and_budget_host_paths(lib):
     assert prev >= 0
     assert lib.hca_set_launch_budget(0, prev) == 60
     assert lib.hca_set_launch_budget(1, 0) >= 0
-    assert lib.hca_set_launch_budget(2, 10) == -1       # unknown op
+    assert lib.hca_set_launch_budget(2, 10) == 0        # the decode indexer's budget
+    assert lib.hca_set_launch_budget(2, 0) == 10
+    assert lib.hca_set_launch_budget(3, 10) == -1       # unknown op
     assert lib.hca_set_launch_budget(0, -1) == -1       # negative budget
+
+
+class EntryEx(ctypes.Structure):
+    _fields_ = [("norm_w", ctypes.c_void_p), ("norm_eps", ctypes.c_float), ("inv_freq", ctypes.c_void_p)]
+
+
+class AttnEx(ctypes.Structure):
+    _fields_ = [("q_norm_w", ctypes.c_void_p), ("norm_eps", ctypes.c_float), ("sink", ctypes.c_void_p),
+                ("inv_freq", ctypes.c_void_p), ("q_pos", ctypes.c_void_p), ("win_len", ctypes.c_void_p)]
+
+
+def test_extension_calls_validate_on_the_host(lib):
+    """The section 9 extras, the overlapped and key compressors, the BF16-score
+    and 64-head indexer calls, the state-cache append and the host-to-host
+    step reject bad arguments before any CUDA call."""
+    V, I32, I64, F, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    P, good = V(0x1000), Layout(512, 64, 64)
+    cache = Cache(0x1000, 0x1000, 0x1000, 10)
+    lib.csa_compress_ex.argtypes = [V, V, I64, V, I32, I64, Layout, Cache, I64, ctypes.POINTER(EntryEx), V]
+    bad_w = EntryEx(0x1004, 1e-6, None)                                  # misaligned weight
+    assert lib.csa_compress_ex(P, P, 8, P, 1, 1, good, cache, 0, ctypes.byref(bad_w), None) == 1
+    neg = EntryEx(None, -1.0, None)                                      # negative epsilon
+    assert lib.csa_compress_ex(P, P, 8, P, 1, 1, good, cache, 0, ctypes.byref(neg), None) == 1
+    lib.kv_token_prep.argtypes = [V, V, I64, Layout, ctypes.POINTER(EntryEx), V, V]
+    assert lib.kv_token_prep(P, P, 4, Layout(256, 64, 64), None, P, None) == 2
+    assert lib.kv_token_prep(None, P, 4, good, None, P, None) == 1
+    assert lib.kv_token_prep(None, None, 0, good, None, None, None) == 0
+    lib.compressed_attn_decode_ex.argtypes = [V, I32, I32, Layout, Cache, V, I32, V, I32, V, I32, F,
+                                              ctypes.POINTER(AttnEx), V, V, V, SZ, V]
+    no_pos = AttnEx(None, 1e-6, None, 0x1000, None, None)                # RoPE without query positions
+    assert lib.compressed_attn_decode_ex(P, 1, 64, good, cache, None, 0, P, 10, P, 128, 0.1, ctypes.byref(no_pos),
+                                         P, None, None, 0, None) == 1
+    lib.compressed_attn_prefill_ex.argtypes = [V, I32, I32, I32, I32, Layout, Cache, V, I32, V, V, I32, F,
+                                               ctypes.POINTER(AttnEx), V, V, SZ, V]
+    win_pf = AttnEx(None, 1e-6, None, None, None, 0x1000)                # window lengths are a decode input
+    assert lib.compressed_attn_prefill_ex(P, 4, 64, 100, 4, good, cache, None, 0, None, P, 128, 0.1,
+                                          ctypes.byref(win_pf), P, None, 0, None) == 1
+    lib.csa_compress_overlap.argtypes = [V, V, V, V, V, V, I64, V, I32, I64, Layout, Cache, I64, V]
+    assert lib.csa_compress_overlap(P, P, P, P, P, None, 8, P, 1, 2, good, cache, 1, None) == 1    # a_prev alone
+    assert lib.csa_compress_overlap(P, P, P, P, None, None, 7, P, 1, 2, good, cache, 0, None) == 1  # 8 rows needed
+    lib.indexer_key_compress.argtypes = [V, V, V, V, V, V, I64, V, I32, I64, I32, V, V, I64, I64, V]
+    assert lib.indexer_key_compress(P, P, P, P, None, None, 8, P, 1, 2, 96, P, P, 10, 0, None) == 2  # c = 96
+    assert lib.indexer_key_compress(P, P, P, P, None, None, 8, P, 1, 2, 128, P, P, 1, 0, None) == 1  # capacity
+    lib.lightning_index_ex.argtypes = [V, V, V, V, V, V, I32, I32, I64, I32, I32, I32, I32, V, V]
+    assert lib.lightning_index_ex(P, P, P, P, P, P, 1, 1, 10, 4, 64, 4, 1, P, None) == 2     # BF16 needs c = 128
+    assert lib.lightning_index_ex(P, P, P, P, P, P, 1, 1, 10, 64, 64, 4, 0, P, None) == 2    # 64 heads: c = 128
+    assert lib.lightning_index_ex(P, P, P, P, P, P, 1, 1, 10, 16, 128, 4, 0, P, None) == 2   # 16 heads
+    lib.topk_select_ex.argtypes = [V, I32, V, I32, I64, I32, I32, V, V, V, SZ, V]
+    assert lib.topk_select_ex(P, 1, P, 2, 1000, 4, 8, P, P, None, 0, None) == 4              # BF16: workspace
+    lib.topk_select_ex_workspace_size.argtypes = [I32, I64, I32, I32]
+    lib.topk_select_ex_workspace_size.restype = SZ
+    assert lib.topk_select_ex_workspace_size(2, 1000, 8, 1) > 0                               # any row length
+    assert lib.topk_select_ex_workspace_size(2, 1000, 8, 0) == 0
+    lib.kv_state_append.argtypes = [V, V, V, I32, I32, I64, V, I32, V, V, I32, V]
+    assert lib.kv_state_append(P, P, None, 2, 100, 5, P, 128, P, P, 4, None) == 1            # d % 8 != 0
+    assert lib.kv_state_append(P, P, None, 2, 128, -1, P, 128, P, P, 4, None) == 1           # negative position
+    lib.hca_decode_step_host.argtypes = [V, V, V, V, V, V, V, V, V]
+    assert lib.hca_decode_step_host(None, P, P, P, P, P, P, P, None) == 1
