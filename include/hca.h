@@ -245,7 +245,9 @@ int kv_token_prep(const uint16_t* x, const int32_t* pos, int64_t n, hca_kv_layou
  * score = fp32, from +0, for h = 0..Hi-1 in order: score += w_h * ReLU(dot_h)
  *         (product rounded, then sum rounded).
  * Supported: c in {64, 128}, 1 <= Hi <= 8, or Hi = 64 (the note's
- * n_h^I = 64, section 7 parameters) with c = 128; m >= 1. */
+ * n_h^I = 64, section 7 parameters) with c = 128 on the tensor pipe (key
+ * code buffer 32-byte and scale buffer 16-byte aligned, Nc_cap a multiple of
+ * 4); m >= 1. */
 int lightning_index(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
                     const uint8_t* k_codes, const uint8_t* k_sf, const int32_t* q_pos,
                     int32_t B, int32_t Tq, int64_t Nc_cap, int32_t Hi, int32_t c, int32_t m,
@@ -254,7 +256,9 @@ int lightning_index(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
  * selector's index scores in BF16 instead of FP32): score_bf16 != 0 writes
  * each score rounded to bf16 (nearest even) into scores as uint16 bit patterns
  * [B][Tq][Nc_cap] (-inf for ineligible entries); score_bf16 = 0 is
- * lightning_index (scores fp32).  BF16 scores: c = 128 and Hi in {4, 64}. */
+ * lightning_index (scores fp32).  BF16 scores and Hi = 64 run on the tensor
+ * pipe only: c = 128, Hi in {4, 64}, key code buffer 32-byte and scale buffer
+ * 16-byte aligned, Nc_cap a multiple of 4 (HCA_ERR_UNSUPPORTED otherwise). */
 int lightning_index_ex(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
                        const uint8_t* k_codes, const uint8_t* k_sf, const int32_t* q_pos,
                        int32_t B, int32_t Tq, int64_t Nc_cap, int32_t Hi, int32_t c, int32_t m,
@@ -525,12 +529,13 @@ typedef struct {
  *   h_q_csa, h_q_hca  bf16 [B][H][d]; h_iq_codes [B][Hi][c/2], h_iq_sf
  *   [B][Hi][c/32], h_iq_w fp32 [B][Hi]; h_out_csa, h_out_hca bf16 [B][H][d]
  *   (host memory; pinned for asynchronous copies).
- * Queues on `stream`: the indexer-query copies, lightning_index_topk, the
- * CSA attention and its output copy; on the plan's side stream: the
- * attention-query copies and, once the indexer has run, the HCA attention
- * and its output copy.  `stream` finally waits for the side stream, so the
- * outputs are in host memory when `stream` reaches that point.  Nothing is
- * allocated; errors as the calls it makes. */
+ * Queues on the plan's side stream (give it the higher priority: it carries
+ * the critical path): the indexer-query copies, lightning_index_topk, the CSA
+ * attention and its output copy; on `stream`: the attention-query copies and,
+ * once the indexer has run, the HCA attention and its output copy.  `stream`
+ * finally waits for the side stream, so both outputs are in host memory when
+ * `stream` reaches that point.  Nothing is allocated; errors as the calls it
+ * makes. */
 int hca_decode_step_host(const hca_decode_step_plan* plan, const uint16_t* h_q_csa, const uint16_t* h_q_hca,
                          const uint8_t* h_iq_codes, const uint8_t* h_iq_sf, const float* h_iq_w,
                          uint16_t* h_out_csa, uint16_t* h_out_hca, void* stream);

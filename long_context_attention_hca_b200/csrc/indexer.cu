@@ -580,22 +580,28 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
         const int n_mine = n_tiles > t0 ? (n_tiles - t0 + TS - 1) / TS : 0;
         const int n_items = n_mine * QPW;
-        // sub-items I = (item i, head group hg): the TMEM load of sub-item I + 1 is in
-        // flight while I is scored; a score is complete after its last group
-        const int n_sub = n_items * HG;
+        // sub-items I = (item i, chunk ch of GPC head groups): the TMEM loads of sub-item
+        // I + 1 are in flight while I is scored; a score is complete after its last chunk
+        constexpr int GPC = HG >= 4 ? 4 : HG;          // head groups per chunk (16 columns each)
+        constexpr int NCH = HG / GPC;                   // chunks per item
+        const int n_sub = n_items * NCH;
         int eq1[16], klo1[4], khi1[4];                 // the only query's exponents (QG == 1, HG == 1)
 #pragma unroll
         for (int j = 0; j < 16; ++j) eq1[j] = s_eq[0][j];
 #pragma unroll
         for (int j = 0; j < 4; ++j) { klo1[j] = s_klo[0][0][j]; khi1[j] = s_khi[0][0][j]; }
-        uint32_t rn[16];
+        uint32_t rn[16 * GPC];
         auto tmem_ld = [&](int I) {
-            const int i = I / HG, hg = I % HG;
+            const int i = I / NCH, ch = I % NCH;
             const int t = t0 + TS * (i / QPW), q = q0 + QE * (i % QPW);
-            asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-                         : "=r"(rn[0]), "=r"(rn[1]), "=r"(rn[2]), "=r"(rn[3]), "=r"(rn[4]), "=r"(rn[5]), "=r"(rn[6]), "=r"(rn[7]),
-                           "=r"(rn[8]), "=r"(rn[9]), "=r"(rn[10]), "=r"(rn[11]), "=r"(rn[12]), "=r"(rn[13]), "=r"(rn[14]), "=r"(rn[15])
-                         : "r"(lane_base + static_cast<uint32_t>((t % NBD) * N + (q * HG + hg) * 16)));
+#pragma unroll
+            for (int g = 0; g < GPC; ++g) {
+                uint32_t* d = rn + 16 * g;
+                asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                             : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]), "=r"(d[4]), "=r"(d[5]), "=r"(d[6]), "=r"(d[7]),
+                               "=r"(d[8]), "=r"(d[9]), "=r"(d[10]), "=r"(d[11]), "=r"(d[12]), "=r"(d[13]), "=r"(d[14]), "=r"(d[15])
+                             : "r"(lane_base + static_cast<uint32_t>((t % NBD) * N + (q * HG + ch * GPC + g) * 16)));
+            }
         };
         // a tile's accumulators are complete (and its stage's loads visible) after these waits
         auto tile_ready = [&](int t) {
@@ -611,15 +617,15 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
         uint32_t sw = 0;
         float sc = 0.0f;
         for (int I = 0; I < n_sub && ok; ++I) {
-            const int i = I / HG, hg = I % HG;
+            const int i = I / NCH, ch = I % NCH;
             const int t = t0 + TS * (i / QPW), j = i % QPW, q = q0 + QE * j;
             const int st = t % KS, nb = t % NBD;
             asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-            uint32_t r[16];
+            uint32_t rc[16 * GPC];
 #pragma unroll
-            for (int z = 0; z < 16; ++z) r[z] = rn[z];
-            if (j == 0 && hg == 0) sw = *reinterpret_cast<const uint32_t*>(smem + st * STAGE_BYTES + CODE_BYTES + row * 4);
-            if (j == QPW - 1 && hg == HG - 1) {
+            for (int z = 0; z < 16 * GPC; ++z) rc[z] = rn[z];
+            if (j == 0 && ch == 0) sw = *reinterpret_cast<const uint32_t*>(smem + st * STAGE_BYTES + CODE_BYTES + row * 4);
+            if (j == QPW - 1 && ch == NCH - 1) {
                 // every load of tile t has completed and its scale word is read: release
                 // the accumulator buffer and the key stage
                 asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -627,9 +633,13 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
                 if (lane == 0) { mbar_arrive(smem_u32(&bar_acce[nb])); mbar_arrive(smem_u32(&bar_empty[st])); }
             }
             if (I + 1 < n_sub) {
-                if ((I + 1) % (QPW * HG) == 0 && !tile_ready(t + TS)) { ok = false; }
+                if ((I + 1) % (QPW * NCH) == 0 && !tile_ready(t + TS)) { ok = false; }
                 else tmem_ld(I + 1);
             }
+#pragma unroll
+            for (int g = 0; g < GPC; ++g) {
+            const int hg = ch * GPC + g;
+            const uint32_t* r = rc + 16 * g;
             int eq[16];
 #pragma unroll
             for (int z = 0; z < 16; ++z) eq[z] = (QG == 1 && HG == 1) ? eq1[z] : s_eq[q][hg * 16 + z];
@@ -688,6 +698,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
                     }
                 }
             }
+            }   // head groups of the chunk
         }
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
         if (!ok) {

@@ -1,19 +1,21 @@
 // step.cu -- one decode step of a CSA layer and an HCA layer from host
 // memory to host memory through the library alone: the query copies in, the
-// fused index + top-k, both attention calls and the output copies out, with
-// the HCA layer on a second stream ("DeepSeek V4 ..." note, sections 7 and 8:
-// the CSA path -- indexer, top-k, attention over the selected entries and the
-// window -- and the HCA path -- dense attention over every entry and the
-// window -- of one decode position).
+// fused index + top-k, both attention calls and the output copies out, on two
+// streams ("DeepSeek V4 ..." note, sections 7 and 8: the CSA path -- indexer,
+// top-k, attention over the selected entries and the window -- and the HCA
+// path -- dense attention over every entry and the window -- of one decode
+// position).
 //
 // Schedule (the two paths share no data):
-//   stream: H2D indexer query | index + top-k (records ev_index) | waits ev_q |
-//           CSA attention | D2H CSA output | waits ev_join
-//   side:   waits ev_fork | H2D both attention queries (records ev_q) |
-//           waits ev_index | HCA attention | D2H HCA output (records ev_join)
-// The HCA launch waits for the indexer, which fills every SM anyway.  Every
-// copy is one cudaMemcpyAsync; the host buffers should be pinned so that the
-// copies are asynchronous.
+//   side:   waits ev_fork | H2D indexer query | index + top-k (records
+//           ev_index) | waits ev_q | CSA attention | D2H CSA output (records
+//           ev_join)
+//   stream: records ev_fork | H2D CSA query (records ev_q) | H2D HCA query |
+//           waits ev_index | HCA attention | D2H HCA output | waits ev_join
+// The CSA chain is the critical path, so the side stream should have the
+// higher priority; the HCA launch waits for the indexer, which fills every SM
+// anyway.  Every copy is one cudaMemcpyAsync; the host buffers should be
+// pinned so that the copies are asynchronous.
 #include "common.cuh"
 
 using namespace hca;
@@ -53,31 +55,32 @@ extern "C" int hca_decode_step_host(const hca_decode_step_plan* p, const uint16_
     const size_t iqw = static_cast<size_t>(p->B) * p->Hi * sizeof(float);
     void* side = p->side_stream;
     HCA_TRY(rec(p->ev_fork, stream));
-    // the indexer query first (a few hundred bytes), the attention queries beside the indexer
-    HCA_TRY(cpy(p->iq_codes, h_iq_codes, iqc, cudaMemcpyHostToDevice, stream));
-    HCA_TRY(cpy(p->iq_sf, h_iq_sf, iqs, cudaMemcpyHostToDevice, stream));
-    HCA_TRY(cpy(p->iq_w, h_iq_w, iqw, cudaMemcpyHostToDevice, stream));
     HCA_TRY(wait(side, p->ev_fork));
-    HCA_TRY(cpy(p->q_csa, h_q_csa, q_bytes, cudaMemcpyHostToDevice, side));
-    HCA_TRY(cpy(p->q_hca, h_q_hca, q_bytes, cudaMemcpyHostToDevice, side));
-    HCA_TRY(rec(p->ev_q, side));
-    // CSA: index + top-k, then attention over the selected entries and the window
+    // CSA chain on the side stream: the indexer query (a few hundred bytes), index + top-k
+    HCA_TRY(cpy(p->iq_codes, h_iq_codes, iqc, cudaMemcpyHostToDevice, side));
+    HCA_TRY(cpy(p->iq_sf, h_iq_sf, iqs, cudaMemcpyHostToDevice, side));
+    HCA_TRY(cpy(p->iq_w, h_iq_w, iqw, cudaMemcpyHostToDevice, side));
     HCA_TRY(lightning_index_topk(p->iq_codes, p->iq_sf, p->iq_w, p->k_codes, p->k_sf, p->q_pos, p->B,
                                  p->csa_entries, p->Hi, p->c, 4, p->k, p->scores, p->idx, p->count, p->topk_ws,
-                                 p->topk_ws_bytes, p->ev_index, stream));
-    HCA_TRY(wait(stream, p->ev_q));
+                                 p->topk_ws_bytes, p->ev_index, side));
+    // the attention queries cross while the indexer runs
+    HCA_TRY(cpy(p->q_csa, h_q_csa, q_bytes, cudaMemcpyHostToDevice, stream));
+    HCA_TRY(rec(p->ev_q, stream));
+    HCA_TRY(cpy(p->q_hca, h_q_hca, q_bytes, cudaMemcpyHostToDevice, stream));
+    // CSA attention over the selected entries and the window, then its output
+    HCA_TRY(wait(side, p->ev_q));
     const int32_t kmax = static_cast<int32_t>(p->csa_entries < p->k ? p->csa_entries : p->k);
     HCA_TRY(compressed_attn_decode(p->q_csa, p->B, p->H, p->layout, p->csa_cache, p->idx, p->k, p->count, kmax,
                                    p->csa_window, p->W, p->softmax_scale, p->out_csa, nullptr, p->ws_csa,
-                                   p->ws_csa_bytes, stream));
-    HCA_TRY(cpy(h_out_csa, p->out_csa, q_bytes, cudaMemcpyDeviceToHost, stream));
-    // HCA: dense attention, after the indexer
-    HCA_TRY(wait(side, p->ev_index));
+                                   p->ws_csa_bytes, side));
+    HCA_TRY(cpy(h_out_csa, p->out_csa, q_bytes, cudaMemcpyDeviceToHost, side));
+    HCA_TRY(rec(p->ev_join, side));
+    // HCA: dense attention once the indexer has run, then its output
+    HCA_TRY(wait(stream, p->ev_index));
     HCA_TRY(compressed_attn_decode(p->q_hca, p->B, p->H, p->layout, p->hca_cache, nullptr, 0, p->hca_n, p->hca_max,
                                    p->hca_window, p->W, p->softmax_scale, p->out_hca, nullptr, p->ws_hca,
-                                   p->ws_hca_bytes, side));
-    HCA_TRY(cpy(h_out_hca, p->out_hca, q_bytes, cudaMemcpyDeviceToHost, side));
-    HCA_TRY(rec(p->ev_join, side));
+                                   p->ws_hca_bytes, stream));
+    HCA_TRY(cpy(h_out_hca, p->out_hca, q_bytes, cudaMemcpyDeviceToHost, stream));
     HCA_TRY(wait(stream, p->ev_join));
     return HCA_OK;
 }

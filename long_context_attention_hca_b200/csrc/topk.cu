@@ -346,9 +346,9 @@ namespace wide {
 // call, or by hist_kernel); then one select_kernel launch:
 //   every CTA reads the histogram, finds the threshold bin T1 (the highest
 //   bin whose count from the top reaches k), scans its chunk of the row and
-//   appends the keys above bin T1 (all selected, fewer than k of them) and
-//   the keys in bin T1 (the candidates) to the row's two lists, one atomic
-//   per list and CTA;
+//   appends the indices of the keys above bin T1 (all selected, fewer than k
+//   of them) and of the keys in bin T1 (the candidates) to the row's two
+//   lists, one atomic per list and CTA;
 //   the CTA that finishes last (a counter per row, behind a memory fence)
 //   resolves the row: a radix select over the candidates' composite keys
 //   (score key, then the complement of the index, so that every composite
@@ -371,7 +371,7 @@ static_assert(2 * kSelWarps * kMaxIt * 4 <= kCandSmem * 8, "masks fit in the can
 struct Layout {
     size_t clear_bytes;     // histogram + header, cleared before every call
     size_t above_off;       // u32 [kMaxK]
-    size_t cand_off;        // u64 [Nc_cap]
+    size_t cand_off;        // u32 [Nc_cap] (8 bytes per entry reserved)
     size_t row_bytes;       // per-row stride
 };
 
@@ -388,7 +388,7 @@ struct RowWs {
     uint32_t* hist;
     uint32_t* hdr;          // [0] keys above bin T1, [1] candidates, [2] CTAs done
     uint32_t* above;
-    unsigned long long* cand;
+    uint32_t* cand;
 };
 
 __device__ __forceinline__ RowWs row_ws(uint8_t* ws, int64_t Nc_cap, int64_t r) {
@@ -398,7 +398,7 @@ __device__ __forceinline__ RowWs row_ws(uint8_t* ws, int64_t Nc_cap, int64_t r) 
     w.hist = reinterpret_cast<uint32_t*>(base);
     w.hdr = w.hist + kBins;
     w.above = reinterpret_cast<uint32_t*>(base + L.above_off);
-    w.cand = reinterpret_cast<unsigned long long*>(base + L.cand_off);
+    w.cand = reinterpret_cast<uint32_t*>(base + L.cand_off);
     return w;
 }
 
@@ -522,7 +522,13 @@ select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, i
     }
     RowWs w = row_ws(ws, Nc_cap, r);
     // ---- threshold bin T1 from the row's histogram (the same in every CTA)
-    for (int i = tid; i < kBins; i += kSelThreads) s_hist[i] = __ldcg(w.hist + i);
+    {
+        uint32_t hv[kBins / kSelThreads];                  // all loads in flight, then the stores
+#pragma unroll
+        for (int j = 0; j < kBins / kSelThreads; ++j) hv[j] = __ldcg(w.hist + tid + j * kSelThreads);
+#pragma unroll
+        for (int j = 0; j < kBins / kSelThreads; ++j) s_hist[tid + j * kSelThreads] = hv[j];
+    }
     __syncthreads();
     find_digit(s_hist, kBins, kk, sh_warp, s_dig);
     const uint32_t t1 = s_dig[0];
@@ -533,15 +539,16 @@ select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, i
     const int64_t e1 = min(e0 + chunk, n);
     const int n_it = e1 > e0 ? static_cast<int>((e1 - e0 + kSelThreads - 1) / kSelThreads) : 0;
     uint32_t ca = 0, cc = 0;
-    for (int it0 = 0; it0 < n_it; it0 += 8) {
-        float v[8];
+    constexpr int kBatch = 16;                         // loads in flight per thread
+    for (int it0 = 0; it0 < n_it; it0 += kBatch) {
+        float v[kBatch];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < kBatch; ++j) {
             const int64_t e = e0 + static_cast<int64_t>(it0 + j) * kSelThreads + warp * 32 + lane;
             v[j] = (it0 + j < n_it && e < e1) ? score_at(row, e) : 0.0f;
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < kBatch; ++j) {
             const int it = it0 + j;
             if (it >= n_it) break;
             const int64_t e = e0 + static_cast<int64_t>(it) * kSelThreads + warp * 32 + lane;
@@ -567,21 +574,19 @@ select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, i
         s_base[1] = tc ? atomicAdd(&w.hdr[1], tc) : 0u;
     }
     __syncthreads();
-    // ---- pass B: append (ordered within the CTA; the lists' order is irrelevant)
+    // ---- pass B: append the indices (ordered within the CTA; the lists' order is
+    // irrelevant): shared-memory masks in, global stores out, no reads of the row
     {
         uint32_t pa = s_base[0] + s_wa[warp], pc = s_base[1] + s_wc[warp];
         const unsigned lt = (1u << lane) - 1u;
         for (int it = 0; it < n_it; ++it) {
             const uint32_t ma = s_ma[warp * kMaxIt + it], mc = s_mc[warp * kMaxIt + it];
-            const int64_t e = e0 + static_cast<int64_t>(it) * kSelThreads + warp * 32 + lane;
+            const uint32_t e = static_cast<uint32_t>(e0 + static_cast<int64_t>(it) * kSelThreads + warp * 32 + lane);
             if ((ma >> lane) & 1u) {
                 const uint32_t at = pa + __popc(ma & lt);
-                if (at < static_cast<uint32_t>(kMaxK)) w.above[at] = static_cast<uint32_t>(e);
+                if (at < static_cast<uint32_t>(kMaxK)) w.above[at] = e;
             }
-            if ((mc >> lane) & 1u)
-                w.cand[pc + __popc(mc & lt)] =
-                    (static_cast<unsigned long long>(order_key(score_at(row, e))) << 32) |
-                    static_cast<uint32_t>(~static_cast<uint32_t>(e));
+            if ((mc >> lane) & 1u) w.cand[pc + __popc(mc & lt)] = e;
             pa += __popc(ma);
             pc += __popc(mc);
         }
@@ -596,11 +601,31 @@ select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, i
     const uint32_t n_above = min(__ldcg(w.hdr + 0), kk);
     const uint32_t n_cand = __ldcg(w.hdr + 1);
     const bool cached = n_cand <= static_cast<uint32_t>(kCandSmem);
-    if (cached)
-        for (uint32_t c = tid; c < n_cand; c += kSelThreads) s_cand[c] = __ldcg(w.cand + c);
+    // a candidate's composite key: its score key, then the complement of its index
+    // (unique; equal scores rank the lower index first)
+    auto composite = [&](uint32_t e) {
+        return (static_cast<unsigned long long>(order_key(score_at(row, e))) << 32) | static_cast<uint32_t>(~e);
+    };
+    if (cached) {
+        // one round of index loads, one round of score loads, for all candidates
+        uint32_t ci[kCandSmem / kSelThreads];
+#pragma unroll
+        for (int j = 0; j < kCandSmem / kSelThreads; ++j) {
+            const uint32_t c = tid + j * kSelThreads;
+            ci[j] = c < n_cand ? __ldcg(w.cand + c) : 0u;
+        }
+        float cs[kCandSmem / kSelThreads];
+#pragma unroll
+        for (int j = 0; j < kCandSmem / kSelThreads; ++j)
+            cs[j] = tid + j * kSelThreads < n_cand ? score_at(row, ci[j]) : 0.0f;
+#pragma unroll
+        for (int j = 0; j < kCandSmem / kSelThreads; ++j)
+            s_cand[tid + j * kSelThreads] =
+                (static_cast<unsigned long long>(order_key(cs[j])) << 32) | static_cast<uint32_t>(~ci[j]);
+    }
     if (tid == 0) s_nsel = n_above;
     __syncthreads();
-    auto cand = [&](uint32_t c) { return cached ? s_cand[c] : __ldcg(w.cand + c); };
+    auto cand = [&](uint32_t c) { return cached ? s_cand[c] : composite(__ldcg(w.cand + c)); };
     uint32_t need = kk - n_above;
     // threshold: candidates whose composite, on the bits fixed so far, is >= prefix
     unsigned long long prefix = 0ull, fmask = 0ull;
@@ -631,7 +656,17 @@ select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, i
         }
     }
     // ---- gather: the keys above bin T1, then the candidates at or above the threshold
-    for (uint32_t i = tid; i < n_above; i += kSelThreads) s_sel[i] = __ldcg(w.above + i);
+    {
+        uint32_t av[kMaxK / kSelThreads];
+#pragma unroll
+        for (int j = 0; j < kMaxK / kSelThreads; ++j) {
+            const uint32_t i = tid + j * kSelThreads;
+            av[j] = i < n_above ? __ldcg(w.above + i) : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxK / kSelThreads; ++j)
+            if (tid + j * kSelThreads < n_above) s_sel[tid + j * kSelThreads] = av[j];
+    }
     for (uint32_t c = tid; c < n_cand; c += kSelThreads) {
         const unsigned long long v = cand(c);
         if ((v & fmask) >= prefix) {
@@ -689,9 +724,11 @@ uint32_t* topk_wide_hist(void* ws, int64_t Nc_cap, int64_t* stride_u32) {
     return static_cast<uint32_t*>(ws);
 }
 
-// scores per CTA: about one CTA per SM over all rows, whole 512-score steps
-static int64_t wide_chunk(int R, int64_t Nc_cap, int per_step) {
-    const int64_t ctas_per_row = std::max<int64_t>(1, ceil_div(sm_count(), R));
+// scores per CTA: about one CTA per SM over all rows (hist_kernel), or per two
+// SMs (select_kernel: its CTAs then fit in one wave on the SMs that a
+// concurrent attention launch leaves free), whole steps
+static int64_t wide_chunk(int R, int64_t Nc_cap, int per_step, int sms_per_cta = 1) {
+    const int64_t ctas_per_row = std::max<int64_t>(1, ceil_div(ceil_div(sm_count(), sms_per_cta), R));
     int64_t chunk = ceil_div(Nc_cap, ctas_per_row);
     chunk = std::max<int64_t>(per_step, ceil_div(chunk, per_step) * per_step);
     return std::min<int64_t>(chunk, static_cast<int64_t>(wide::kMaxIt) * per_step);
@@ -713,7 +750,7 @@ int topk_wide_select(const void* scores, const int32_t* q_pos, int R, int64_t Nc
         if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
         attr_set[bf16][dev] = true;
     }
-    const int64_t chunk = wide_chunk(R, Nc_cap, wide::kSelThreads);
+    const int64_t chunk = wide_chunk(R, Nc_cap, wide::kSelThreads, 2);
     const dim3 grid(static_cast<unsigned>(ceil_div(Nc_cap, chunk)), static_cast<unsigned>(R));
     if (bf16)
         wide::select_kernel<uint16_t><<<grid, wide::kSelThreads, wide::kSelSmem, st>>>(

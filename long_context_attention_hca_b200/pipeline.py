@@ -155,7 +155,7 @@ class DecodeRunner:
         Lc, Lh = self.layers[c_], self.layers[h_]
         qc, qs, w = d_iq[c_]
         lo, hi_prio = torch.cuda.Stream.priority_range()
-        self._capi_side = torch.cuda.Stream(device=d_q[0].device, priority=lo)
+        self._capi_side = torch.cuda.Stream(device=d_q[0].device, priority=hi_prio)   # the CSA chain
         self._capi_events = [torch.cuda.Event() for _ in range(4)]
         for e in self._capi_events:
             e.record(torch.cuda.current_stream())     # creates the CUDA event (outside any capture)

@@ -41,9 +41,9 @@ def _bf16_bits(scores_f32):
 
 @pytest.mark.parametrize("Hi,score_bf16", [(64, False), (64, True), (4, True)])
 def test_index_scores_variants(Hi, score_bf16):
-    B, Tq, Nc, m = 2, 3, 3001, 4
+    B, Tq, Nc, m = 2, 3, 3000, 4          # the tensor-map path: Nc a multiple of 4
     qc, qs, w, kc, ks = _inputs(B, Tq, Hi, Nc, 300 + Hi)
-    pos = torch.tensor([[4 * Nc, 77, 4 * (Nc // 2) - 1], [3, 4 * Nc - 2, 1 << 30]], dtype=torch.int32, device=DEV)
+    pos = torch.tensor([[4 * Nc, 77, 4 * (Nc // 2) - 1], [3, 4 * Nc - 5, 1 << 30]], dtype=torch.int32, device=DEV)
     s = hca.lightning_index(qc, qs, w, kc, ks, pos, m, score_bf16=score_bf16)
     torch.cuda.synchronize()
     want, n_inexact = oracle.index_scores(host(qc), host(qs), host(w), host(kc), host(ks), host(pos), m)

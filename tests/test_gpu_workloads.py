@@ -245,3 +245,32 @@ def test_prefill_4096_131k_sampled(section9):
         assert_attn_close(oc[i], ref, f"CSA pos {p}")
         ref, _ = oracle.attend(qh[i], codes128, scales128, rope128, ent128, win, wl.softmax_scale, wl.g, **akw(p))
         assert_attn_close(oh[i], ref, f"HCA pos {p}")
+
+
+def test_decode_b4_1m_and_prefill_run_twice_identical():
+    """Determinism (no floating-point atomics, the same reduction order on
+    every run): the 1M-context decode step and the prefill chunk give the
+    same bytes when run again (outputs, index scores, top-k sets)."""
+    wl = inp.WORKLOADS["decode_b4_1m"]
+    dw = build_decode(wl)
+    runner = DecodeRunner(dw.layers, wl.B, wl.H, wl.k, wl.t, wl.softmax_scale)
+    first = [o.clone() for o in runner.step(dw.q, dw.iq)]
+    sc1 = {li: t.clone() for li, t in runner.scores.items()}
+    idx1 = {li: t.clone() for li, t in runner.idx.items()}
+    second = runner.step(dw.q, dw.iq)
+    torch.cuda.synchronize()
+    for a, b in zip(first, second):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    for li in sc1:
+        assert torch.equal(sc1[li].view(torch.int32), runner.scores[li].view(torch.int32))
+        assert torch.equal(idx1[li], runner.idx[li])
+    del dw, runner
+    torch.cuda.empty_cache()
+    wl = inp.WORKLOADS["prefill_4096_131k"]
+    pw = build_prefill(wl)
+    pr = PrefillRunner(pw.state, wl.t, wl.Tq, wl.H, wl.k, wl.W, wl.softmax_scale)
+    a = [t.clone() for t in pr.step(pw.raw_chunk, pw.gate_chunk, pw.raw_window, pw.q, pw.iq)]
+    b = pr.step(pw.raw_chunk, pw.gate_chunk, pw.raw_window, pw.q, pw.iq)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert torch.equal(x.view(torch.int16), y.view(torch.int16))
