@@ -347,6 +347,7 @@ int lightning_index_topk_ex(const uint8_t* q_codes, const uint8_t* q_sf, const f
  *   window   bf16 [B][W][d]: the last W raw tokens, oldest first; key =
  *            value = token (all W rows are used)
  *   out      bf16 [B][H][d];  lse fp32 [B][H] (natural log) or NULL
+ * softmax_scale must be positive and finite (else HCA_ERR_INVALID_ARG).
  * Per head: o = sum_j softmax_j(scale * q.k_j) k_j over the compressed keys
  * (dequantised: code * scale, bf16 RoPE dims) and the window tokens, one
  * joint softmax.  Split-K over the keys with a log-sum-exp combine; the
@@ -410,7 +411,7 @@ int compressed_attn_decode_noalloc(const uint16_t* q, int32_t B, int32_t H,
  *   raw     bf16 [W-1+Tq][d]: raw tokens from position p0-(W-1) on; the
  *           window of position p is tokens max(0, p-W+1) .. p
  *   out     bf16 [Tq][H][d]
- * Same attention rule as decode. */
+ * Same attention rule (and softmax_scale rule) as decode. */
 size_t compressed_attn_prefill_workspace_size(int32_t Tq, int32_t H, hca_kv_layout layout);
 int compressed_attn_prefill(const uint16_t* q, int32_t Tq, int32_t H, int32_t p0, int32_t m,
                             hca_kv_layout layout, hca_kv_cache kv,

@@ -580,6 +580,7 @@ int attn_decode_launch(const uint16_t* q, int B, int H, const hca_kv_layout& L, 
                        const int32_t* idx, int idx_stride, const int32_t* n_comp, int max_comp,
                        const uint16_t* window, int W, float softmax_scale, const hca_attn_extras* ex,
                        uint16_t* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t st) {
+    if (!(softmax_scale > 0.0f) || !isfinite(softmax_scale)) return HCA_ERR_INVALID_ARG;
     if (B == 0) return HCA_OK;
     if (use_tc(L.d, H))
         return tc_attn_decode_launch(q, B, H, kv, idx, idx_stride, n_comp, max_comp, window, W, softmax_scale, ex,
@@ -609,6 +610,7 @@ int attn_prefill_launch(const uint16_t* q, int Tq, int H, int p0, int m, const h
                         const hca_kv_cache& kv, const int32_t* idx, int idx_stride, const int32_t* count,
                         const uint16_t* raw, int W, float softmax_scale, const hca_attn_extras* ex, uint16_t* out,
                         cudaStream_t st) {
+    if (!(softmax_scale > 0.0f) || !isfinite(softmax_scale)) return HCA_ERR_INVALID_ARG;
     if (Tq == 0) return HCA_OK;
     if (use_tc(L.d, H))
         return tc_attn_prefill_launch(q, Tq, H, p0, m, kv, idx, idx_stride, count, raw, W, softmax_scale, ex, out,

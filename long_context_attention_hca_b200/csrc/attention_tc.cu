@@ -15,7 +15,8 @@
 //   O^T += V^T . P^T    M = 128 output dims (4 M-tiles), N = 64 heads,
 //                       K = 64 keys; V^T is the key tile itself read MN-major,
 //                       P^T the softmax probabilities stored K-major.
-// TMEM: S in NBUF buffers of 64 columns + O^T (4 x 64 columns).
+// TMEM: S in NBUF buffers, each two 64-column partial sums (K halves), + O^T
+// (4 x 64 columns): all 512 columns.
 // Warp roles (704 threads):
 //   warps 0-3   softmax: head h = 16 w + (lane & 15); lanes 0-15 take keys
 //               0..31 of the tile, lanes 16-31 keys 32..63; online softmax
@@ -73,8 +74,8 @@ constexpr int K_OFF = 8 * QBLK;              // NBUF buffers x 8 column blocks (
 constexpr int P_OFF = K_OFF + NBUF * 8 * KBLK;   // 2 P^T buffers
 constexpr int SMEM_BYTES = P_OFF + 2 * PBLK + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t S_COL = 0;                // S buffer b at columns 64 b
-constexpr uint32_t O_COL = NBUF * TK;        // O^T M-tile mt at 128 + 64 mt
+constexpr uint32_t S_COL = 0;                // S buffer b, half c (of K = 512) at columns 64 (2 b + c)
+constexpr uint32_t O_COL = NBUF * 2 * TK;    // O^T M-tile mt at 256 + 64 mt
 constexpr float RESCALE_THRESHOLD = 8.0f;    // log2 units
 constexpr long long WAIT_LIMIT = 1ll << 24;  // polls before a wait is declared stuck
 
@@ -97,8 +98,8 @@ struct Params {
     int n_splits, tiles_per_split;
     uint16_t* out;
     float* lse;
-    float* part_o;              // [units][splits][HP][D]
-    float* part_ml;             // [units][splits][2][HP]
+    uint16_t* part_o;           // [units][splits][HP/4][D][4] fp16: the split's O / l, heads in fours
+    float* part_ml;             // [units][splits][2][HP]: running max (base 2), l
     // section 9 extras (each null when off)
     const float* q_norm_w;      // [D] query-head RMSNorm weight
     float norm_eps;
@@ -192,6 +193,13 @@ __device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.syn
                    "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),          \
                    "=r"(r[30]), "=r"(r[31])                                                                         \
                  : "r"(taddr))
+// the same with 16 columns per half: threads 0-15 columns c .. c + 15, threads
+// 16-31 columns c + 32 .. c + 47
+#define TMEM_LD_16X32BX2_16(taddr, r)                                                                              \
+    asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], 32;" \
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),      \
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]) \
+                 : "r"(taddr))
 // 2^x with the special-function unit (approximate; x = -inf gives +0)
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -284,7 +292,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ __align__(8) uint64_t bar_kempty[NBUF], bar_kfull[NBUF], bar_sfull[NBUF], bar_pempty[2], bar_drain;
     __shared__ uint32_t tmem_base_slot;
-    __shared__ float s_alpha[HP], s_l[HP];
+    __shared__ float s_alpha[HP], s_l[HP], s_rl[HP];
     __shared__ int s_resc_w[NSOFT];
     __shared__ volatile int s_abort;
     __shared__ float s_qr[HP];                       // 1 / rms of each query head (query RMSNorm)
@@ -293,6 +301,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t u = blockIdx.x;
     const int split = blockIdx.y;
+    pdl_wait();                                    // everything earlier in the stream is visible
     const UnitKeys uk = unit_keys(p, u);
     const int n_tot = uk.n_c + uk.n_w;
     const int n_tiles_all = (n_tot + TK - 1) / TK;
@@ -305,7 +314,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
         for (int i = 0; i < NBUF; ++i) {
             mbar_init(smem_u32(&bar_kempty[i]), 4);  // freed by the four PV issuers
             mbar_init(smem_u32(&bar_kfull[i]), NPROD);  // one arrival per producer warp
-            mbar_init(smem_u32(&bar_sfull[i]), 1);
+            mbar_init(smem_u32(&bar_sfull[i]), NISSUE);   // both QK issuers
         }
         mbar_init(smem_u32(&bar_pempty[0]), 4);      // the four PV issuers
         mbar_init(smem_u32(&bar_pempty[1]), 4);
@@ -470,20 +479,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
     constexpr uint32_t id_pv = idesc_f16(128, HP, 1, 0);
     if (warp >= NSOFT + NPROD) {
         // ------------------------------------------------------------ QK issue
-        const int b = warp - (NSOFT + NPROD);             // this warp's key buffer
+        // Warp 20 + c issues half c of every tile's QK (dims 256 c .. 256 c + 255) into
+        // its own accumulator: one thread issues an MMA every ~70 clocks whatever its
+        // shape, so two issuers on two sub-partitions halve the QK time.
+        const int c = warp - (NSOFT + NPROD);
         if (lane == 0) {
             const uint64_t qd = sdesc(sbase + Q_OFF, 16, 1024);
-            const uint64_t kd = sdesc(sbase + K_OFF + b * 8 * KBLK, 16, 1024);
-            const uint32_t dst = tmem + S_COL + b * TK;
-            for (int i = b; i < n_tiles; i += NBUF) {
+            for (int i = 0; i < n_tiles; ++i) {
+                const int b = i % NBUF;
                 if (!wait_bar(smem_u32(&bar_kfull[b]), (i / NBUF) & 1, &s_abort)) break;
                 fence_after();
+                const uint64_t kd = sdesc(sbase + K_OFF + b * 8 * KBLK, 16, 1024);
+                const uint32_t dst = tmem + S_COL + (2 * b + c) * TK;
                 // descriptors differ per k-step only in the start address (bits 0..13, units of 16 B)
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
+                for (int k2 = 0; k2 < D / 32; ++k2) {
+                    const int kk = c * (D / 32) + k2;
                     const uint32_t qo = static_cast<uint32_t>(((kk >> 2) * QBLK + (kk & 3) * 32) >> 4);
                     const uint32_t ko = static_cast<uint32_t>(((kk >> 2) * KBLK + (kk & 3) * 32) >> 4);
-                    mma_f16(dst, qd + qo, kd + ko, id_qk, kk > 0);
+                    mma_f16(dst, qd + qo, kd + ko, id_qk, k2 > 0);
                 }
                 mma_commit(smem_u32(&bar_sfull[b]));
             }
@@ -560,13 +574,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
             float v[32];
             float tmax = -INFINITY;
             {
-                // row h, keys 32 kh .. 32 kh + 31
-                uint32_t sr[32];
-                TMEM_LD_16X32BX2_32(lane_base + S_COL + b * TK, sr);
+                // row h, keys 32 kh .. 32 kh + 31: the sum of the two K-half accumulators
+                uint32_t sr[32], s2[16];
+                const uint32_t sa = lane_base + S_COL + (2 * b) * TK;
+                TMEM_LD_16X32BX2_32(sa, sr);
+                TMEM_LD_16X32BX2_16(sa + TK, s2);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    v[j] = (kh * 32 + j < nvalid) ? __uint_as_float(sr[j]) * p.scale_log2 : -INFINITY;
+                for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(sr[j]) + __uint_as_float(s2[j]);
+                TMEM_LD_16X32BX2_16(sa + TK + 16, s2);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[16 + j] = __uint_as_float(sr[16 + j]) + __uint_as_float(s2[j]);
+                if (nvalid < TK) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (kh * 32 + j >= nvalid) v[j] = -INFINITY;
+                }
                 // maximum as a tree (depth 5 instead of a 32-long chain)
                 float mx[16];
 #pragma unroll
@@ -575,7 +599,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
                 for (int w2 = 8; w2 >= 1; w2 >>= 1)
 #pragma unroll
                     for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
-                tmax = mx[0];
+                // the scale is positive (checked on the host): the maximum of the raw logits
+                // times the scale is the maximum of the scaled ones
+                tmax = mx[0] * p.scale_log2;
             }
             tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
             bool resc = false;
@@ -594,7 +620,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
             float ps[16];
 #pragma unroll
             for (int z = 0; z < 16; ++z) {
-                pk[z] = pack_half2(ex2(v[2 * z] - m_used), ex2(v[2 * z + 1] - m_used));
+                pk[z] = pack_half2(ex2(fmaf(v[2 * z], p.scale_log2, -m_used)), ex2(fmaf(v[2 * z + 1], p.scale_log2, -m_used)));
                 const float2 f = unpack_half2(pk[z]);
                 ps[z] = f.x + f.y;
             }
@@ -681,13 +707,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
 #pragma unroll 1
             for (int mt = 0; mt < 4; ++mt) {
                 const int dim = mt * 128 + L;
+#pragma unroll 1
+                for (int c1 = 0; c1 < HP; c1 += 32) {
+                // 32 head columns in flight at once, one wait
+                uint32_t oa[32];
+                if (n_tiles > 0) {
+                    TMEM_LD16(lane_base + O_COL + mt * HP + c1, oa, 0);
+                    TMEM_LD16(lane_base + O_COL + mt * HP + c1 + 16, oa, 16);
+                    tmem_wait_ld();
+                }
 #pragma unroll
-                for (int c0 = 0; c0 < HP; c0 += 16) {
-                    uint32_t o[16];
-                    if (n_tiles > 0) {
-                        TMEM_LD16(lane_base + O_COL + mt * HP + c0, o, 0);
-                        tmem_wait_ld();
-                    }
+                for (int c0 = c1; c0 < c1 + 32; c0 += 16) {
+                    const uint32_t* o = oa + (c0 - c1);
                     float v[16];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
@@ -713,38 +744,59 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
                             p.out[(uo * p.H + hh) * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(ok ? v[j] : qnan));
                     }
                 }
+                }
             }
             if (p.lse && hrow && h < p.H) {
                 const float none = (EX && p.sink) ? __ldg(p.sink + h) : -INFINITY;    // no keys: the sink alone
                 p.lse[uo * p.H + h] = (l_run > 0.0f && ok) ? (m_used + log2f(l_tot)) * 0.69314718055994531f
                                                           : (ok ? none : qnan);
             }
-        } else {
+        } else if (hrow) {
             const size_t ps = uo * p.n_splits + split;
-            float* po = p.part_o + ps * HP * D;
-            if (n_tiles > 0) {
+            float* ml = p.part_ml + ps * 2 * HP;
+            ml[h] = m_used;
+            ml[HP + h] = ok ? l_run : qnan;
+            s_rl[h] = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+        }
+    }
+    if (p.n_splits > 1 && warp < 16) {
+        // ---- split partials by warps 0-15: warp w reads TMEM lane quarter w % 4 (the
+        // lanes it may access) of M-tile w / 4, i.e. one output dim per thread, and
+        // stores that dim's 64 heads of O / l as fp16, four heads (8 bytes) per store:
+        // the 32 lanes (consecutive dims) of a warp write 256 contiguous bytes
+        // the softmax warps have seen the last PV complete (their own wait, one phase
+        // at a time); the barrier hands that on
+        fence_before();
+        named_bar(2, 16 * 32);                       // s_rl published, the last PV complete
+        fence_after();
+        if (n_tiles > 0) {
+            const int qd = warp & 3, mt = warp >> 2;
+            const int dim = mt * 128 + qd * 32 + lane;
+            const uint32_t lb = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+            const bool good = s_abort == 0;
+            uint16_t* po = p.part_o + (static_cast<size_t>(u) * p.n_splits + split) * HP * D + static_cast<size_t>(dim) * 4;
 #pragma unroll 1
-                for (int mt = 0; mt < 4; ++mt) {
-                    const int dim = mt * 128 + L;
+            for (int c1 = 0; c1 < HP; c1 += 32) {
+                uint32_t oa[32];
+                TMEM_LD16(lb + O_COL + mt * HP + c1, oa, 0);
+                TMEM_LD16(lb + O_COL + mt * HP + c1 + 16, oa, 16);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int c0 = 0; c0 < HP; c0 += 16) {
-                        uint32_t o[16];
-                        TMEM_LD16(lane_base + O_COL + mt * HP + c0, o, 0);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) po[static_cast<size_t>(c0 + j) * D + dim] = ok ? __uint_as_float(o[j]) : qnan;
-                    }
+                for (int j = 0; j < 8; ++j) {
+                    const int hq = c1 + 4 * j;         // heads hq .. hq + 3
+                    uint2 hv;
+                    hv.x = good ? pack_half2(__uint_as_float(oa[4 * j]) * s_rl[hq], __uint_as_float(oa[4 * j + 1]) * s_rl[hq + 1])
+                                : 0x7E007E00u;
+                    hv.y = good ? pack_half2(__uint_as_float(oa[4 * j + 2]) * s_rl[hq + 2], __uint_as_float(oa[4 * j + 3]) * s_rl[hq + 3])
+                                : 0x7E007E00u;
+                    *reinterpret_cast<uint2*>(po + static_cast<size_t>(hq / 4) * D * 4) = hv;
                 }
-            }
-            if (hrow) {
-                float* ml = p.part_ml + ps * 2 * HP;
-                ml[h] = m_used;
-                ml[HP + h] = ok ? l_run : qnan;
             }
         }
     }
     fence_before();
     __syncthreads();
+    pdl_trigger();                                 // outputs stored: the combine may be scheduled
     if (warp == 0) {
         // every issued MMA has completed before TMEM is freed
         if (lane == 0)
@@ -756,93 +808,128 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
     }
 }
 
-// Log-sum-exp combine of split partials (base-2 maxima): grid (unit, head),
-// 128 threads x 4 dims.  All (m, l) pairs are read first, then the partial
-// outputs 8 splits at a time, so the L2 reads are in flight together.
-__global__ void __launch_bounds__(128) combine_tc_kernel(Params p) {
-    constexpr int MAXS = 256;
-    __shared__ float s_w[MAXS];
-    __shared__ float s_L;
-    __shared__ int s_bad;
+// Log-sum-exp combine of split partials (base-2 maxima): grid (unit, 16-dim
+// block), 128 threads.  Per head: M = max of the live splits' maxima, split
+// weight 2^(m_s - M) l_s (the partials are O_s / l_s), L = their sum (+ the
+// sink); out = sum_s weight_s o_s / L.  Thread t sums heads 4 (t / 8) .. + 3
+// at dims 16 b + 2 (t % 8) and the next one: one 16-byte fp16 load per split
+// (the partials keep heads in fours, dims consecutive), 32 splits in flight.
+// The (m, l) pairs are staged in shared memory first, every load in flight.
+constexpr int COMB_DIMS = 16;
+constexpr int COMB_THREADS = 128;
+constexpr int MAX_SPLITS = 64;
+
+__global__ void __launch_bounds__(COMB_THREADS) combine_tc_kernel(Params p) {
+    __shared__ __align__(16) float s_w[MAX_SPLITS][HP];    // maxima, then the split weights
+    __shared__ __align__(16) float s_lv[MAX_SPLITS][HP];   // l
+    __shared__ int s_live[MAX_SPLITS];
+    __shared__ float s_inv[HP];
+    __shared__ int s_bad[HP];
     const int64_t u = blockIdx.x;
-    const int h = blockIdx.y;
+    const int dblk = blockIdx.y;
     const int S = p.n_splits;
-    const float* ml0 = p.part_ml + static_cast<size_t>(u) * S * 2 * HP;
-    if (threadIdx.x < 32) {
-        // split weights 2^(m_s - M) (0 for empty splits), their l-weighted sum, NaN flag
-        float M = -INFINITY;
-        for (int s = threadIdx.x; s < S; s += 32) {
-            const float ls = ml0[s * 2 * HP + HP + h];
-            if (ls > 0.0f) M = fmaxf(M, ml0[s * 2 * HP + h]);
+    const int t = threadIdx.x;
+    pdl_wait();                                    // the split partials are complete
+    {
+        // (m, l) of every split ([S][2][HP] floats, contiguous) -> shared memory
+        const float4* src = reinterpret_cast<const float4*>(p.part_ml + static_cast<size_t>(u) * S * 2 * HP);
+        constexpr int kPer = MAX_SPLITS * 2 * HP / 4 / COMB_THREADS;
+        const int n4 = S * 2 * HP / 4;
+        float4 buf[kPer];
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int i = t + j * COMB_THREADS;
+            buf[j] = i < n4 ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        for (int j = 0; j < kPer; ++j) {
+            const int i = t + j * COMB_THREADS;
+            if (i < n4) {
+                const int s = (4 * i) / (2 * HP), r = (4 * i) % (2 * HP);
+                float* dst = r < HP ? &s_w[s][r] : &s_lv[s][r - HP];
+                *reinterpret_cast<float4*>(dst) = buf[j];
+            }
+        }
+        for (int s = t; s < S; s += COMB_THREADS) s_live[s] = 0;
+    }
+    __syncthreads();
+    {
+        // two threads per head (neighbouring lanes): maxima, weights, sums
+        const int h = t >> 1, sub = t & 1;
+        float M = -INFINITY;
+        for (int s = sub; s < S; s += 2)
+            if (s_lv[s][h] > 0.0f) M = fmaxf(M, s_w[s][h]);
+        M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 1));
         float L = 0.0f;
         int bad = 0;
-        for (int s = threadIdx.x; s < S; s += 32) {
-            const float ms = ml0[s * 2 * HP + h], ls = ml0[s * 2 * HP + HP + h];
+        for (int s = sub; s < S; s += 2) {
+            const float ms = s_w[s][h], ls = s_lv[s][h];
             if (ls != ls) bad = 1;
-            const float wgt = ls > 0.0f ? exp2f(ms - M) : 0.0f;
-            if (s < MAXS) s_w[s] = wgt;
-            L += wgt * (ls > 0.0f ? ls : 0.0f);
+            if (ls > 0.0f) s_live[s] = 1;               // a split with keys wrote a partial
+            const float wgt = ls > 0.0f ? exp2f(ms - M) * ls : 0.0f;
+            s_w[s][h] = wgt;
+            L += wgt;
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            L += __shfl_xor_sync(0xffffffffu, L, o);
-            bad |= __shfl_xor_sync(0xffffffffu, bad, o);
-        }
-        if (threadIdx.x == 0) {
+        L += __shfl_xor_sync(0xffffffffu, L, 1);
+        bad |= __shfl_xor_sync(0xffffffffu, bad, 1);
+        if (sub == 0) {
             // the sink joins the denominator relative to the global max M
             const float sink = p.sink ? __ldg(p.sink + h) : -INFINITY;
             if (p.sink && L > 0.0f) L += exp2f(sink * LOG2E - M);
-            s_L = L;
-            s_bad = bad;
-            if (p.lse)
+            s_inv[h] = L > 0.0f ? 1.0f / L : 0.0f;
+            s_bad[h] = bad;
+            if (p.lse && dblk == 0 && h < p.H)
                 p.lse[u * p.H + h] = bad ? __int_as_float(0x7fc00000)
                                          : (L > 0.0f ? (M + log2f(L)) * 0.69314718055994531f : sink);
         }
     }
     __syncthreads();
-    const int d0 = threadIdx.x * 4;
-    const float* po = p.part_o + (static_cast<size_t>(u) * S * HP + h) * D + d0;
+    const int hq = t >> 3;                           // heads 4 hq .. 4 hq + 3
+    const int dim = dblk * COMB_DIMS + 2 * (t & 7);  // dims dim, dim + 1
+    const uint16_t* po = p.part_o + (static_cast<size_t>(u) * S * HP + 4 * hq) * D + static_cast<size_t>(dim) * 4;
     const size_t split_stride = static_cast<size_t>(HP) * D;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int s0 = 0; s0 < S; s0 += 8) {
-        float4 v[8];
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // [dim offset][head offset]
+    constexpr int kBatch = 32;                       // partial loads in flight per thread
+    for (int s0 = 0; s0 < S; s0 += kBatch) {
+        uint4 v[kBatch];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            v[j] = (s0 + j < S && s_w[s0 + j] != 0.0f)
-                       ? *reinterpret_cast<const float4*>(po + static_cast<size_t>(s0 + j) * split_stride)
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < kBatch; ++j) {
+            const int s = s0 + j;
+            // an empty split wrote no partial
+            v[j] = (s < S && s_live[s]) ? *reinterpret_cast<const uint4*>(po + s * split_stride)
+                                        : make_uint4(0u, 0u, 0u, 0u);
+        }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float wgt = s0 + j < S ? s_w[s0 + j] : 0.0f;
-            acc[0] += wgt * v[j].x; acc[1] += wgt * v[j].y; acc[2] += wgt * v[j].z; acc[3] += wgt * v[j].w;
+        for (int j = 0; j < kBatch; ++j) {
+            const int s = s0 + j;
+            if (s < S && s_live[s]) {
+                const float4 w4 = *reinterpret_cast<const float4*>(&s_w[s][4 * hq]);
+                const float2 a0 = unpack_half2(v[j].x), a1 = unpack_half2(v[j].y);   // dim: heads 0-1, 2-3
+                const float2 b0 = unpack_half2(v[j].z), b1 = unpack_half2(v[j].w);   // dim + 1
+                acc[0] += w4.x * a0.x; acc[1] += w4.y * a0.y; acc[2] += w4.z * a1.x; acc[3] += w4.w * a1.y;
+                acc[4] += w4.x * b0.x; acc[5] += w4.y * b0.y; acc[6] += w4.z * b1.x; acc[7] += w4.w * b1.y;
+            }
         }
     }
-    const bool bad = s_bad != 0;
-    const float L = s_L;
-    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
     const float qnan = __int_as_float(0x7fc00000);
-    float o[4] = {acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv};
-    if (p.inv_freq && d0 >= D - D_ROPE) {
-        // RoPE dims: rotate the output back by the query's position
-        const int64_t t = unit_pos(p, u);
+    float cs = 1.0f, sn = 0.0f;
+    const bool rot = p.inv_freq && dim >= D - D_ROPE;
+    if (rot) rope_cs(p.inv_freq, (dim - (D - D_ROPE)) / 2, unit_pos(p, u), cs, sn);
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            float cs, sn;
-            rope_cs(p.inv_freq, (d0 - (D - D_ROPE)) / 2 + i, t, cs, sn);
-            const float x = o[2 * i], y = o[2 * i + 1];
-            o[2 * i] = x * cs + y * sn;
-            o[2 * i + 1] = y * cs - x * sn;
+    for (int i = 0; i < 4; ++i) {
+        const int h = 4 * hq + i;
+        float x = acc[i] * s_inv[h], y = acc[4 + i] * s_inv[h];
+        if (rot) {
+            // RoPE pair (dim, dim + 1): rotate back by the query's position
+            const float x2 = x * cs + y * sn, y2 = y * cs - x * sn;
+            x = x2; y = y2;
+        }
+        if (s_bad[h]) { x = qnan; y = qnan; }
+        if (h < p.H) {
+            const __nv_bfloat162 o2 = __floats2bfloat162_rn(x, y);
+            *reinterpret_cast<__nv_bfloat162*>(p.out + (static_cast<size_t>(u) * p.H + h) * D + dim) = o2;
         }
     }
-    __nv_bfloat162 a = __floats2bfloat162_rn(bad ? qnan : o[0], bad ? qnan : o[1]);
-    __nv_bfloat162 b = __floats2bfloat162_rn(bad ? qnan : o[2], bad ? qnan : o[3]);
-    uint2 w;
-    w.x = *reinterpret_cast<uint32_t*>(&a);
-    w.y = *reinterpret_cast<uint32_t*>(&b);
-    *reinterpret_cast<uint2*>(p.out + (static_cast<size_t>(u) * p.H + h) * D + d0) = w;
 }
 
 }  // namespace tc
@@ -855,10 +942,14 @@ int launch_tc(tc::Params& p, int64_t units, cudaStream_t st) {
     auto kern = ex ? tc::attn_tc_kernel<true> : tc::attn_tc_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
     if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
-    kern<<<dim3(static_cast<unsigned>(units), p.n_splits), tc::NTHREADS, tc::SMEM_BYTES, st>>>(p);
+    // programmatic launches: each kernel waits for its predecessor before any read
+    e = launch_pdl(kern, dim3(static_cast<unsigned>(units), p.n_splits), dim3(tc::NTHREADS), tc::SMEM_BYTES, st, p);
+    if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
     HCA_CHECK_LAUNCH();
     if (p.n_splits > 1) {
-        tc::combine_tc_kernel<<<dim3(static_cast<unsigned>(units), p.H), tc::D / 4, 0, st>>>(p);
+        e = launch_pdl(tc::combine_tc_kernel, dim3(static_cast<unsigned>(units), tc::D / tc::COMB_DIMS),
+                       dim3(tc::COMB_THREADS), 0, st, p);
+        if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
         HCA_CHECK_LAUNCH();
     }
     return HCA_OK;
@@ -876,7 +967,7 @@ void tc_decode_plan(int B, int max_comp, int W, bool sparse, int& n_splits, int&
     int splits = (budget > 0 ? budget : sm_count()) / (B > 0 ? B : 1);
     const int cap_by_len = static_cast<int>(ceil_div(n_tiles > 0 ? n_tiles : 1, min_tps));
     if (splits > cap_by_len) splits = cap_by_len;
-    if (splits > 256) splits = 256;           // the combine keeps one weight per split in shared memory
+    if (splits > tc::MAX_SPLITS) splits = tc::MAX_SPLITS;   // the combine keeps the split weights in shared memory
     if (splits < 1) splits = 1;
     tiles_per_split = static_cast<int>(ceil_div(n_tiles > 0 ? n_tiles : 1, splits));
     n_splits = static_cast<int>(ceil_div(n_tiles > 0 ? n_tiles : 1, tiles_per_split));
@@ -886,7 +977,8 @@ size_t tc_decode_ws_bytes(int B, int max_comp, int W, bool sparse) {
     int ns, tps;
     tc_decode_plan(B, max_comp, W, sparse, ns, tps);
     if (ns <= 1) return 0;
-    return static_cast<size_t>(B) * ns * tc::HP * (static_cast<size_t>(tc::D) + 2) * sizeof(float) + 256;
+    // fp16 partial outputs, then fp32 (max, l) pairs
+    return static_cast<size_t>(B) * ns * tc::HP * (static_cast<size_t>(tc::D) * 2 + 2 * sizeof(float)) + 256;
 }
 
 static void set_extras(tc::Params& p, const hca_attn_extras* ex) {
@@ -917,8 +1009,8 @@ int tc_attn_decode_launch(const uint16_t* q, int B, int H, const hca_kv_cache& k
     if (p.n_splits > 1) {
         const size_t need = tc_decode_ws_bytes(B, max_comp, W, idx != nullptr);
         if (ws == nullptr || ws_bytes < need) return HCA_ERR_WORKSPACE;
-        p.part_o = reinterpret_cast<float*>(ws);
-        p.part_ml = p.part_o + static_cast<size_t>(B) * p.n_splits * tc::HP * tc::D;
+        p.part_o = reinterpret_cast<uint16_t*>(ws);
+        p.part_ml = reinterpret_cast<float*>(p.part_o + static_cast<size_t>(B) * p.n_splits * tc::HP * tc::D);
     }
     return launch_tc(p, B, st);
 }

@@ -33,7 +33,32 @@ int sm_count();
 // process-wide CTA cap of a decode attention launch (0: none); see hca_set_launch_budget
 int launch_budget(int op);
 
+// Programmatic dependent launch.  A kernel launched by launch_pdl may be
+// scheduled while the previous kernel of its stream is still running; it calls
+// pdl_wait() before it reads anything that kernel (or any earlier work) wrote:
+// the wait returns once the previous kernel has completed and its stores are
+// visible (for a normal launch it returns at once).  pdl_trigger() in the
+// previous kernel lets the dependent one be scheduled before its own CTAs exit.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // ---------------------------------------------------------------- device
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) {
     return __uint_as_float(static_cast<uint32_t>(h) << 16);
 }

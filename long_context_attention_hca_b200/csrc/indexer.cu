@@ -436,6 +436,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
     constexpr uint32_t IDESC = (1u << 4) | (5u << 7) | (5u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
                                (static_cast<uint32_t>(TILE >> 4) << 24);
     constexpr int EPI = 4 * EG;                         // epilogue warps
+    pdl_trigger();                                      // the top-k select may be placed early (it waits)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sB = smem + KS * STAGE_BYTES;              // N rows x 128 B (query operand)

@@ -345,16 +345,18 @@ namespace wide {
 // each row comes first (built by the indexer's epilogue in the fused decode
 // call, or by hist_kernel); then one select_kernel launch:
 //   every CTA reads the histogram, finds the threshold bin T1 (the highest
-//   bin whose count from the top reaches k), scans its chunk of the row and
-//   appends the indices of the keys above bin T1 (all selected, fewer than k
-//   of them) and of the keys in bin T1 (the candidates) to the row's two
-//   lists, one atomic per list and CTA;
+//   bin whose count from the top reaches k) and scans its chunk of the row
+//   once: the indices of the keys above bin T1 (all selected, fewer than k of
+//   them) and the composite keys of the keys in bin T1 (the candidates) are
+//   staged per warp in shared memory and appended to the row's two lists, one
+//   atomic claim per warp and list (the order inside a list is irrelevant);
 //   the CTA that finishes last (a counter per row, behind a memory fence)
 //   resolves the row: a radix select over the candidates' composite keys
-//   (score key, then the complement of the index, so that every composite
-//   is unique and equal scores rank the lower index first) finds the exact
-//   threshold, the selected indices are gathered in shared memory, sorted
-//   ascending by a bitonic network and written out.
+//   (score key, then the complement of the index, so that every composite is
+//   unique and equal scores rank the lower index first) finds the exact
+//   threshold; the above keys and the selected candidates set their bits in a
+//   shared-memory bitmap of the row, whose block-wide scan places every
+//   selected index at its rank, i.e. in ascending order, without a sort.
 // No CTA waits for another: the last one to arrive does the rest.
 constexpr int kBins = 2048;
 constexpr int kThreads = 256;              // hist_kernel
@@ -363,15 +365,21 @@ constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kMaxIt = 64;                 // select: at most 64 x 512 scores per CTA
 constexpr int kCandSmem = 4096;            // candidates resolved from shared memory (else from L2)
 constexpr int kMaxK = 4096;
-// dynamic shared memory of select_kernel: the scan's ballot masks, reused by
-// the resolve as the candidate cache, then the selected indices
-constexpr size_t kSelSmem = static_cast<size_t>(kCandSmem) * 8 + static_cast<size_t>(kMaxK) * 4;
-static_assert(2 * kSelWarps * kMaxIt * 4 <= kCandSmem * 8, "masks fit in the candidate cache");
+constexpr int kWpt = 16;                   // bitmap words per thread
+constexpr int kSegWords = kSelThreads * kWpt;   // 8192 words = 262144 entries per bitmap segment
+constexpr int kWBuf = 64;                  // per-warp staging entries per list
+// dynamic shared memory of select_kernel: the candidates (resolve), one bitmap
+// segment (resolve; the per-warp staging during the scan), the output
+constexpr size_t kSelSmem = static_cast<size_t>(kCandSmem) * 8 + static_cast<size_t>(kSegWords) * 4 +
+                            static_cast<size_t>(kMaxK) * 4;
+static_assert(kSelWarps * kWBuf * 12 <= kSegWords * 4, "staging fits in the bitmap segment");
+
+__host__ __device__ inline size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct Layout {
     size_t clear_bytes;     // histogram + header, cleared before every call
-    size_t above_off;       // u32 [kMaxK]
-    size_t cand_off;        // u32 [Nc_cap] (8 bytes per entry reserved)
+    size_t above_off;       // u32 [kMaxK]: indices of the keys above bin T1
+    size_t cand_off;        // u64 [Nc_cap]: composite keys of the candidates
     size_t row_bytes;       // per-row stride
 };
 
@@ -380,7 +388,7 @@ __host__ __device__ inline Layout layout(int64_t Nc_cap) {
     L.clear_bytes = static_cast<size_t>(kBins) * 4 + 256;
     L.above_off = L.clear_bytes;
     L.cand_off = L.above_off + static_cast<size_t>(kMaxK) * 4;
-    L.row_bytes = L.cand_off + ((static_cast<size_t>(Nc_cap) * 8 + 255) & ~static_cast<size_t>(255));
+    L.row_bytes = L.cand_off + round256(static_cast<size_t>(Nc_cap) * 8);
     return L;
 }
 
@@ -388,7 +396,7 @@ struct RowWs {
     uint32_t* hist;
     uint32_t* hdr;          // [0] keys above bin T1, [1] candidates, [2] CTAs done
     uint32_t* above;
-    uint32_t* cand;
+    unsigned long long* cand;
 };
 
 __device__ __forceinline__ RowWs row_ws(uint8_t* ws, int64_t Nc_cap, int64_t r) {
@@ -398,7 +406,7 @@ __device__ __forceinline__ RowWs row_ws(uint8_t* ws, int64_t Nc_cap, int64_t r) 
     w.hist = reinterpret_cast<uint32_t*>(base);
     w.hdr = w.hist + kBins;
     w.above = reinterpret_cast<uint32_t*>(base + L.above_off);
-    w.cand = reinterpret_cast<uint32_t*>(base + L.cand_off);
+    w.cand = reinterpret_cast<unsigned long long*>(base + L.cand_off);
     return w;
 }
 
@@ -491,25 +499,68 @@ __device__ void find_digit(const uint32_t* h, uint32_t nb, uint32_t need, uint32
     __syncthreads();
 }
 
+// The bitmap segment in shared memory: thread t's kWpt = 16 words (entries
+// 512 t .. 512 t + 511 of the segment) sit in four 16-byte slots, rotated by
+// t / 2 so that the eight lanes of a 16-byte access phase hit eight
+// different bank groups.
+__device__ __forceinline__ uint32_t slot_of(uint32_t t, uint32_t j) { return 4 * t + ((j + (t >> 1)) & 3u); }
+// shared-memory word index of segment word wd
+__device__ __forceinline__ uint32_t word_at(uint32_t wd) {
+    return 4 * slot_of(wd >> 4, (wd >> 2) & 3u) + (wd & 3u);
+}
+
+// Warp-uniform append of the lanes of mask (one value each) to a list: staged
+// in the warp's shared buffer while it has room (count in *n), else claimed
+// in the row's list at once.
+template <typename V>
+__device__ __forceinline__ void append(unsigned mask, V val, V* stage, uint32_t& n, uint32_t* counter, V* list,
+                                       uint32_t cap) {
+    const int lane = threadIdx.x & 31;
+    const unsigned lt = (1u << lane) - 1u;
+    const uint32_t c = __popc(mask);
+    if (n + c <= static_cast<uint32_t>(kWBuf)) {
+        if ((mask >> lane) & 1u) stage[n + __popc(mask & lt)] = val;
+        n += c;
+    } else {
+        uint32_t b = 0;
+        if (lane == 0) b = atomicAdd(counter, c);
+        b = __shfl_sync(0xffffffffu, b, 0);
+        if ((mask >> lane) & 1u) {
+            const uint32_t at = b + __popc(mask & lt);
+            if (at < cap) list[at] = val;
+        }
+    }
+}
+
+// Flush a warp's staged entries: one claim, then coalesced stores.
+template <typename V>
+__device__ __forceinline__ void flush(const V* stage, uint32_t n, uint32_t* counter, V* list, uint32_t cap) {
+    const int lane = threadIdx.x & 31;
+    __syncwarp();
+    uint32_t b = 0;
+    if (lane == 0 && n) b = atomicAdd(counter, n);
+    b = __shfl_sync(0xffffffffu, b, 0);
+    for (uint32_t i = lane; i < n; i += 32)
+        if (b + i < cap) list[b + i] = stage[i];
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kSelThreads)
 select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, int64_t Nc_cap, int m, int k,
               int64_t chunk, uint8_t* __restrict__ ws, int32_t* __restrict__ idx, int32_t* __restrict__ count) {
     extern __shared__ __align__(16) unsigned long long dyn[];
-    uint32_t* s_ma = reinterpret_cast<uint32_t*>(dyn);                  // [warps][kMaxIt] above masks
-    uint32_t* s_mc = s_ma + kSelWarps * kMaxIt;                          // [warps][kMaxIt] candidate masks
-    unsigned long long* s_cand = dyn;                                    // resolve: candidate cache
-    uint32_t* s_sel = reinterpret_cast<uint32_t*>(dyn + kCandSmem);      // resolve: selected indices
+    unsigned long long* s_cand = dyn;                                          // [kCandSmem]
+    uint32_t* s_bits = reinterpret_cast<uint32_t*>(dyn + kCandSmem);           // [kSegWords]
+    int32_t* s_out = reinterpret_cast<int32_t*>(s_bits + kSegWords);           // [kMaxK]
     __shared__ uint32_t s_hist[kBins];
     __shared__ uint32_t sh_warp[32];
     __shared__ uint32_t s_dig[4];
-    __shared__ uint32_t s_wa[kSelWarps], s_wc[kSelWarps];
-    __shared__ uint32_t s_base[2];
-    __shared__ uint32_t s_nsel;
+    __shared__ uint32_t s_tot;
     __shared__ int s_last;
 
     const int64_t r = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_wait();                                    // the scores and histograms are complete
     const int64_t n = n_eligible(q_pos, r, m, Nc_cap);
     const uint32_t kk = static_cast<uint32_t>(min(static_cast<int64_t>(k), n));
     int32_t* orow = idx + static_cast<size_t>(r) * k;
@@ -533,99 +584,92 @@ select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, i
     find_digit(s_hist, kBins, kk, sh_warp, s_dig);
     const uint32_t t1 = s_dig[0];
     const T* row = scores + static_cast<size_t>(r) * Nc_cap;
-    // ---- pass A over this CTA's chunk: per (warp, step) ballots of the keys
-    // above bin T1 and in bin T1
-    const int64_t e0 = static_cast<int64_t>(blockIdx.x) * chunk;
-    const int64_t e1 = min(e0 + chunk, n);
-    const int n_it = e1 > e0 ? static_cast<int>((e1 - e0 + kSelThreads - 1) / kSelThreads) : 0;
-    uint32_t ca = 0, cc = 0;
-    constexpr int kBatch = 16;                         // loads in flight per thread
-    for (int it0 = 0; it0 < n_it; it0 += kBatch) {
-        float v[kBatch];
+    // ---- one pass over this CTA's chunk: the above keys' indices and the
+    // candidates' composite keys, staged per warp, appended to the row's lists
+    {
+        uint32_t* s_wa = s_bits + warp * kWBuf;
+        unsigned long long* s_wc = reinterpret_cast<unsigned long long*>(s_bits + kSelWarps * kWBuf) + warp * kWBuf;
+        const int64_t e0 = static_cast<int64_t>(blockIdx.x) * chunk;
+        const int64_t e1 = min(e0 + chunk, n);
+        const int n_it = e1 > e0 ? static_cast<int>((e1 - e0 + kSelThreads - 1) / kSelThreads) : 0;
+        uint32_t na = 0, nc = 0;
+        constexpr int kBatch = 32;                         // loads in flight per thread
+        for (int it0 = 0; it0 < n_it; it0 += kBatch) {
+            float v[kBatch];
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
-            const int64_t e = e0 + static_cast<int64_t>(it0 + j) * kSelThreads + warp * 32 + lane;
-            v[j] = (it0 + j < n_it && e < e1) ? score_at(row, e) : 0.0f;
-        }
+            for (int j = 0; j < kBatch; ++j) {
+                const int64_t e = e0 + static_cast<int64_t>(it0 + j) * kSelThreads + warp * 32 + lane;
+                v[j] = (it0 + j < n_it && e < e1) ? score_at(row, e) : 0.0f;
+            }
+            // lane j keeps the two ballot words of step it0 + j (small unrolled body)
+            uint32_t my_a = 0u, my_c = 0u;
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
-            const int it = it0 + j;
-            if (it >= n_it) break;
-            const int64_t e = e0 + static_cast<int64_t>(it) * kSelThreads + warp * 32 + lane;
-            const bool live = e < e1;
-            const uint32_t bin = order_key(v[j]) >> 21;
-            const unsigned above = __ballot_sync(0xffffffffu, live && bin > t1);
-            const unsigned in_t1 = __ballot_sync(0xffffffffu, live && bin == t1);
-            if (lane == 0) { s_ma[warp * kMaxIt + it] = above; s_mc[warp * kMaxIt + it] = in_t1; }
-            ca += __popc(above);
-            cc += __popc(in_t1);
+            for (int j = 0; j < kBatch; ++j) {
+                if (it0 + j >= n_it) break;
+                const bool live = e0 + static_cast<int64_t>(it0 + j) * kSelThreads + warp * 32 + lane < e1;
+                const uint32_t bin = order_key(v[j]) >> 21;
+                const unsigned above = __ballot_sync(0xffffffffu, live && bin > t1);
+                const unsigned in_t1 = __ballot_sync(0xffffffffu, live && bin == t1);
+                if (lane == j) { my_a = above; my_c = in_t1; }
+            }
+            // the steps with keys to append (rare), one at a time; a candidate's score is
+            // read again (an L1 hit: this lane loaded it above)
+            unsigned todo = __ballot_sync(0xffffffffu, (my_a | my_c) != 0u);
+#pragma unroll 1
+            while (todo) {
+                const int j = __ffs(todo) - 1;
+                todo &= todo - 1u;
+                const unsigned am = __shfl_sync(0xffffffffu, my_a, j), cm = __shfl_sync(0xffffffffu, my_c, j);
+                const int64_t e = e0 + static_cast<int64_t>(it0 + j) * kSelThreads + warp * 32 + lane;
+                if (am) append<uint32_t>(am, static_cast<uint32_t>(e), s_wa, na, w.hdr + 0, w.above, kMaxK);
+                if (cm) {
+                    const uint32_t key = ((cm >> lane) & 1u) ? order_key(score_at(row, e)) : 0u;
+                    append<unsigned long long>(cm, (static_cast<unsigned long long>(key) << 32) | static_cast<uint32_t>(~e),
+                                               s_wc, nc, w.hdr + 1, w.cand, static_cast<uint32_t>(Nc_cap));
+                }
+            }
         }
+        flush<uint32_t>(s_wa, na, w.hdr + 0, w.above, kMaxK);
+        flush<unsigned long long>(s_wc, nc, w.hdr + 1, w.cand, static_cast<uint32_t>(Nc_cap));
     }
-    if (lane == 0) { s_wa[warp] = ca; s_wc[warp] = cc; }
+    pdl_trigger();                                 // most CTAs end here: let the next kernel be scheduled
+    // ---- the last CTA of the row resolves it.  The barrier orders every thread's
+    // list stores before thread 0's fence, which (being cumulative) releases them
+    // all before the count; the last CTA's thread 0 fences again before its
+    // threads read the other CTAs' stores.
     __syncthreads();
     if (tid == 0) {
-        uint32_t ta = 0, tc = 0;
-        for (int q = 0; q < kSelWarps; ++q) {
-            const uint32_t a = s_wa[q], c = s_wc[q];
-            s_wa[q] = ta; s_wc[q] = tc;
-            ta += a; tc += c;
-        }
-        s_base[0] = ta ? atomicAdd(&w.hdr[0], ta) : 0u;
-        s_base[1] = tc ? atomicAdd(&w.hdr[1], tc) : 0u;
+        __threadfence();
+        const bool last = atomicAdd(&w.hdr[2], 1u) == gridDim.x - 1;
+        if (last) __threadfence();
+        s_last = last;
     }
-    __syncthreads();
-    // ---- pass B: append the indices (ordered within the CTA; the lists' order is
-    // irrelevant): shared-memory masks in, global stores out, no reads of the row
-    {
-        uint32_t pa = s_base[0] + s_wa[warp], pc = s_base[1] + s_wc[warp];
-        const unsigned lt = (1u << lane) - 1u;
-        for (int it = 0; it < n_it; ++it) {
-            const uint32_t ma = s_ma[warp * kMaxIt + it], mc = s_mc[warp * kMaxIt + it];
-            const uint32_t e = static_cast<uint32_t>(e0 + static_cast<int64_t>(it) * kSelThreads + warp * 32 + lane);
-            if ((ma >> lane) & 1u) {
-                const uint32_t at = pa + __popc(ma & lt);
-                if (at < static_cast<uint32_t>(kMaxK)) w.above[at] = e;
-            }
-            if ((mc >> lane) & 1u) w.cand[pc + __popc(mc & lt)] = e;
-            pa += __popc(ma);
-            pc += __popc(mc);
-        }
-    }
-    // ---- the last CTA of the row resolves it
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(&w.hdr[2], 1u) == gridDim.x - 1;
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
-    const uint32_t n_above = min(__ldcg(w.hdr + 0), kk);
-    const uint32_t n_cand = __ldcg(w.hdr + 1);
+    const uint32_t n_above = min(min(__ldcg(w.hdr + 0), kk), static_cast<uint32_t>(kMaxK));
+    const uint32_t n_cand = min(__ldcg(w.hdr + 1), static_cast<uint32_t>(Nc_cap));
     const bool cached = n_cand <= static_cast<uint32_t>(kCandSmem);
-    // a candidate's composite key: its score key, then the complement of its index
-    // (unique; equal scores rank the lower index first)
-    auto composite = [&](uint32_t e) {
-        return (static_cast<unsigned long long>(order_key(score_at(row, e))) << 32) | static_cast<uint32_t>(~e);
-    };
-    if (cached) {
-        // one round of index loads, one round of score loads, for all candidates
-        uint32_t ci[kCandSmem / kSelThreads];
+    // the above indices stay in registers; cached candidates go to shared memory
+    // (both lists in one round of loads)
+    constexpr int kPer = kMaxK / kSelThreads;
+    static_assert(kCandSmem / kSelThreads == kPer, "one round covers both lists");
+    uint32_t av[kPer];
+    {
+        unsigned long long cv[kPer];
 #pragma unroll
-        for (int j = 0; j < kCandSmem / kSelThreads; ++j) {
-            const uint32_t c = tid + j * kSelThreads;
-            ci[j] = c < n_cand ? __ldcg(w.cand + c) : 0u;
+        for (int j = 0; j < kPer; ++j) {
+            const uint32_t i = tid + j * kSelThreads;
+            av[j] = i < n_above ? __ldcg(w.above + i) : 0u;
+            cv[j] = (cached && i < n_cand) ? __ldcg(w.cand + i) : 0ull;
         }
-        float cs[kCandSmem / kSelThreads];
 #pragma unroll
-        for (int j = 0; j < kCandSmem / kSelThreads; ++j)
-            cs[j] = tid + j * kSelThreads < n_cand ? score_at(row, ci[j]) : 0.0f;
-#pragma unroll
-        for (int j = 0; j < kCandSmem / kSelThreads; ++j)
-            s_cand[tid + j * kSelThreads] =
-                (static_cast<unsigned long long>(order_key(cs[j])) << 32) | static_cast<uint32_t>(~ci[j]);
+        for (int j = 0; j < kPer; ++j) {
+            const uint32_t i = tid + j * kSelThreads;
+            if (cached && i < n_cand) s_cand[i] = cv[j];
+        }
     }
-    if (tid == 0) s_nsel = n_above;
     __syncthreads();
-    auto cand = [&](uint32_t c) { return cached ? s_cand[c] : composite(__ldcg(w.cand + c)); };
+    auto cand = [&](uint32_t c) { return cached ? s_cand[c] : __ldcg(w.cand + c); };
     uint32_t need = kk - n_above;
     // threshold: candidates whose composite, on the bits fixed so far, is >= prefix
     unsigned long long prefix = 0ull, fmask = 0ull;
@@ -655,45 +699,88 @@ select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, i
             if (whole) break;
         }
     }
-    // ---- gather: the keys above bin T1, then the candidates at or above the threshold
-    {
-        uint32_t av[kMaxK / kSelThreads];
+    // ---- output, per bitmap segment: the above keys and the selected candidates
+    // set their bits; a block-wide scan gives every set bit its rank, and the
+    // indices are placed in the output staging at those ranks
+    const size_t nw = static_cast<size_t>((n + 31) / 32);
+    uint32_t written = 0;
+    for (size_t seg = 0; seg < nw; seg += kSegWords) {
 #pragma unroll
-        for (int j = 0; j < kMaxK / kSelThreads; ++j) {
-            const uint32_t i = tid + j * kSelThreads;
-            av[j] = i < n_above ? __ldcg(w.above + i) : 0u;
-        }
+        for (int j = 0; j < kWpt; ++j) s_bits[tid + j * kSelThreads] = 0u;
+        __syncthreads();
+        const uint32_t e_lo = static_cast<uint32_t>(seg * 32);
+        auto mark = [&](uint32_t e) {
+            const uint32_t wd = (e - e_lo) >> 5;
+            if (e >= e_lo && wd < static_cast<uint32_t>(kSegWords)) atomicOr(&s_bits[word_at(wd)], 1u << (e & 31u));
+        };
 #pragma unroll
-        for (int j = 0; j < kMaxK / kSelThreads; ++j)
-            if (tid + j * kSelThreads < n_above) s_sel[tid + j * kSelThreads] = av[j];
-    }
-    for (uint32_t c = tid; c < n_cand; c += kSelThreads) {
-        const unsigned long long v = cand(c);
-        if ((v & fmask) >= prefix) {
-            const uint32_t at = atomicAdd(&s_nsel, 1u);
-            if (at < static_cast<uint32_t>(kMaxK)) s_sel[at] = ~static_cast<uint32_t>(v);
-        }
-    }
-    __syncthreads();
-    // ---- ascending order: bitonic network over the next power of two
-    uint32_t P = 1;
-    while (P < kk) P <<= 1;
-    for (uint32_t i = kk + tid; i < P; i += kSelThreads) s_sel[i] = 0xFFFFFFFFu;
-    __syncthreads();
-    for (uint32_t size = 2; size <= P; size <<= 1) {
-        for (uint32_t stride = size >> 1; stride > 0; stride >>= 1) {
-            for (uint32_t i = tid; i < P / 2; i += kSelThreads) {
-                const uint32_t lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
-                const bool asc = (lo & size) == 0;
-                const uint32_t a = s_sel[lo], b = s_sel[hi];
-                if ((a > b) == asc) { s_sel[lo] = b; s_sel[hi] = a; }
+        for (int j = 0; j < kPer; ++j)
+            if (tid + j * kSelThreads < n_above) mark(av[j]);
+        if (cached) {
+#pragma unroll 1
+            for (uint32_t c = tid; c < n_cand; c += kSelThreads) {
+                const unsigned long long v = s_cand[c];
+                if ((v & fmask) >= prefix) mark(~static_cast<uint32_t>(v));
             }
-            __syncthreads();
+        } else {
+            constexpr int kB = 8;                       // candidate loads in flight per thread
+#pragma unroll 1
+            for (uint32_t c0 = tid; c0 < n_cand; c0 += kSelThreads * kB) {
+                unsigned long long cv[kB];
+#pragma unroll
+                for (int j = 0; j < kB; ++j) {
+                    const uint32_t c = c0 + j * kSelThreads;
+                    cv[j] = c < n_cand ? __ldcg(w.cand + c) : 0ull;
+                }
+#pragma unroll
+                for (int j = 0; j < kB; ++j)
+                    if (c0 + j * kSelThreads < n_cand && (cv[j] & fmask) >= prefix) mark(~static_cast<uint32_t>(cv[j]));
+            }
         }
+        __syncthreads();
+        const uint4* s_b4 = reinterpret_cast<const uint4*>(s_bits);
+        uint32_t cnt = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint4 v4 = s_b4[slot_of(tid, j)];
+            cnt += __popc(v4.x) + __popc(v4.y) + __popc(v4.z) + __popc(v4.w);
+        }
+        const uint32_t incl = block_incl_scan(cnt, sh_warp);
+        if (tid == kSelThreads - 1) s_tot = incl;
+        uint32_t pos = written + incl - cnt;
+        {
+            // one loop iteration per set bit of this thread (not per word and bit, which
+            // would make a warp run the sum over words of its lanes' maxima)
+            uint32_t nz = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint4 v4 = s_b4[slot_of(tid, j)];
+                nz |= (v4.x ? 1u : 0u) << (4 * j) | (v4.y ? 2u : 0u) << (4 * j) | (v4.z ? 4u : 0u) << (4 * j) |
+                      (v4.w ? 8u : 0u) << (4 * j);
+            }
+            uint32_t bits = 0u, eb = 0u;
+#pragma unroll 1
+            for (;;) {
+                if (bits == 0u) {
+                    if (nz == 0u) break;
+                    const uint32_t q = static_cast<uint32_t>(__ffs(nz) - 1);
+                    nz &= nz - 1u;
+                    bits = s_bits[4 * slot_of(tid, q >> 2) + (q & 3u)];
+                    eb = static_cast<uint32_t>((seg + static_cast<size_t>(tid) * kWpt + q) * 32);
+                }
+                const uint32_t e = eb + static_cast<uint32_t>(__ffs(bits) - 1);
+                bits &= bits - 1u;
+                if (pos < static_cast<uint32_t>(kMaxK)) s_out[pos] = static_cast<int32_t>(e);
+                ++pos;
+            }
+        }
+        __syncthreads();
+        written += s_tot;
+        __syncthreads();
     }
-    for (uint32_t j = tid; j < static_cast<uint32_t>(k); j += kSelThreads)
-        orow[j] = j < kk ? static_cast<int32_t>(s_sel[j]) : -1;
-    if (tid == 0) count[r] = static_cast<int32_t>(kk);
+    const uint32_t cnt_out = min(written, kk);
+    for (uint32_t j = tid; j < static_cast<uint32_t>(k); j += kSelThreads) orow[j] = j < cnt_out ? s_out[j] : -1;
+    if (tid == 0) count[r] = static_cast<int32_t>(cnt_out);
 }
 
 }  // namespace wide
@@ -752,12 +839,15 @@ int topk_wide_select(const void* scores, const int32_t* q_pos, int R, int64_t Nc
     }
     const int64_t chunk = wide_chunk(R, Nc_cap, wide::kSelThreads, 2);
     const dim3 grid(static_cast<unsigned>(ceil_div(Nc_cap, chunk)), static_cast<unsigned>(R));
-    if (bf16)
-        wide::select_kernel<uint16_t><<<grid, wide::kSelThreads, wide::kSelSmem, st>>>(
-            static_cast<const uint16_t*>(scores), q_pos, Nc_cap, m, k, chunk, static_cast<uint8_t*>(ws), idx, count);
-    else
-        wide::select_kernel<float><<<grid, wide::kSelThreads, wide::kSelSmem, st>>>(
-            static_cast<const float*>(scores), q_pos, Nc_cap, m, k, chunk, static_cast<uint8_t*>(ws), idx, count);
+    // programmatic launch: the CTAs are placed while the histogram producer finishes
+    const cudaError_t le =
+        bf16 ? launch_pdl(wide::select_kernel<uint16_t>, grid, dim3(wide::kSelThreads), wide::kSelSmem, st,
+                          static_cast<const uint16_t*>(scores), q_pos, Nc_cap, m, k, chunk, static_cast<uint8_t*>(ws),
+                          idx, count)
+             : launch_pdl(wide::select_kernel<float>, grid, dim3(wide::kSelThreads), wide::kSelSmem, st,
+                          static_cast<const float*>(scores), q_pos, Nc_cap, m, k, chunk, static_cast<uint8_t*>(ws),
+                          idx, count);
+    if (le != cudaSuccess) { set_last_cuda_error(static_cast<int>(le)); return HCA_ERR_CUDA; }
     HCA_CHECK_LAUNCH();
     return HCA_OK;
 }

@@ -94,16 +94,23 @@ def test_noalloc_matches_regular_entry_point_twice():
 
 
 def test_noalloc_refuses_requests_beyond_its_scratch():
+    """Under the default launch budget (one split per SM) the split-K scratch of
+    any request stays below the 16 MiB array, so the budget is raised first to
+    make a request that needs more."""
     f = _fn()
-    B, cap, W, H, d = 4, 20000, 128, 64, 512
-    assert hca.decode_workspace_size(B, H, hca.LAYOUT_512, cap, W) > (16 << 20)
-    cache, g = _cache(B, 8, 9)                       # pointers only; nothing may be launched
-    q = torch.zeros((B, H, d), dtype=torch.bfloat16, device=DEV)
-    win = torch.zeros((B, W, d), dtype=torch.bfloat16, device=DEV)
-    n = torch.zeros((B,), dtype=torch.int32, device=DEV)
-    out = torch.full((B, H, d), 7.0, dtype=torch.bfloat16, device=DEV)
-    st = f(_p(q), B, H, cache.c_layout, cache.c_struct, None, 0, _p(n), cap, _p(win), W, d ** -0.5, _p(out),
-           None, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    B, cap, W, H, d = 8, 20000, 128, 64, 512
+    prev = hca.set_launch_budget(hca.BUDGET_DENSE_DECODE, 1024)
+    try:
+        assert hca.decode_workspace_size(B, H, hca.LAYOUT_512, cap, W) > (16 << 20)
+        cache, g = _cache(B, 8, 9)                       # pointers only; nothing may be launched
+        q = torch.zeros((B, H, d), dtype=torch.bfloat16, device=DEV)
+        win = torch.zeros((B, W, d), dtype=torch.bfloat16, device=DEV)
+        n = torch.zeros((B,), dtype=torch.int32, device=DEV)
+        out = torch.full((B, H, d), 7.0, dtype=torch.bfloat16, device=DEV)
+        st = f(_p(q), B, H, cache.c_layout, cache.c_struct, None, 0, _p(n), cap, _p(win), W, d ** -0.5, _p(out),
+               None, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    finally:
+        hca.set_launch_budget(hca.BUDGET_DENSE_DECODE, prev)
     assert st == hca.HCA_ERR_SCRATCH_LIMIT
     torch.cuda.synchronize()
     assert torch.all(out == 7.0)
