@@ -524,9 +524,14 @@ def bench_decode(args, wl, world, rank, pg):
                         dw.q[li], L.cache, runner.count[li], min(runner.k, L.n_entries), L.window, runner.scale,
                         idx=runner.idx[li], out=runner.out[li], ws=runner.ws[li]))
                 elif name == "hca_attn" and L.ratio == 128:
-                    calls.append(lambda dw=dw, runner=runner, li=li, L=L: hca.compressed_attn_decode(
+                    # the kernel alone takes every SM (the library default split plan), with a
+                    # workspace sized for that plan
+                    ws_solo = torch.empty(max(hca.decode_workspace_size(wl.B, wl.H, L.cache.layout, L.n_entries,
+                                                                        L.window.shape[1]), 16),
+                                          dtype=torch.uint8, device=dev)
+                    calls.append(lambda dw=dw, runner=runner, li=li, L=L, ws_solo=ws_solo: hca.compressed_attn_decode(
                         dw.q[li], L.cache, runner.n_dense[li], L.n_entries, L.window, runner.scale,
-                        out=runner.out[li], ws=runner.ws[li]))
+                        out=runner.out[li], ws=ws_solo))
         if not calls:
             continue
         s = torch.cuda.Stream()
@@ -970,7 +975,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--schedule", default="after_index", choices=["after_index", "hca_first"],
                     help="decode step: HCA after the indexer, or HCA first on a CTA budget")
-    ap.add_argument("--dense-budget", type=int, default=0, help="CTA cap of the dense decode attention (0: none)")
+    ap.add_argument("--dense-budget", type=int, default=None,
+                    help="CTA cap of the step's dense (HCA) attention (default: half the SMs beside the CSA chain; "
+                         "0: the library default, every SM)")
     ap.add_argument("--sparse-budget", type=int, default=0, help="CTA cap of the sparse decode attention (0: none)")
     ap.add_argument("--index-budget", type=int, default=0, help="CTA cap of the fused decode indexer (0: none)")
     ap.add_argument("--select-variants", action="store_true",

@@ -524,6 +524,8 @@ typedef struct {
     uint16_t* out_hca;            /* [B][H][d]                                           */
     void* side_stream;
     void* ev_fork; void* ev_index; void* ev_q; void* ev_join;
+    int32_t hca_ctas;             /* CTAs of the HCA attention (its split-K plan); 0: half */
+                                  /* the SMs, the rest left to the concurrent CSA chain    */
 } hca_decode_step_plan;
 
 /* Host queries in, host outputs out:

@@ -117,7 +117,18 @@ int compress_common(int m, const uint16_t* x, const uint16_t* gate, int64_t x_se
 }  // namespace
 
 static std::atomic<int> g_launch_budget[3] = {{0}, {0}, {0}};
-int launch_budget(int op) { return (op >= 0 && op <= 2) ? g_launch_budget[op].load() : 0; }
+// a budget set by a library entry for the calls it makes itself (this thread only)
+static thread_local int t_budget[3] = {0, 0, 0};
+int launch_budget(int op) {
+    if (op < 0 || op > 2) return 0;
+    return t_budget[op] > 0 ? t_budget[op] : g_launch_budget[op].load();
+}
+int thread_budget_swap(int op, int max_ctas) {
+    if (op < 0 || op > 2) return 0;
+    const int prev = t_budget[op];
+    t_budget[op] = max_ctas;
+    return prev;
+}
 
 }  // namespace hca
 

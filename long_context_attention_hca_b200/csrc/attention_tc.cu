@@ -62,9 +62,9 @@ constexpr int D = 512;
 constexpr int HP = 64;
 constexpr int TK = 64;                       // keys per tile
 constexpr int NBUF = 2;                      // key tiles (and S tiles) in flight
-constexpr int NSOFT = 4, NPROD = 16, NISSUE = NBUF;
-constexpr int NWARPS = NSOFT + NPROD + NISSUE;
-constexpr int NTHREADS = NWARPS * 32;        // 704
+constexpr int NSOFT = 4, NPROD = 16, NISSUE = 2, NPV = 2;
+constexpr int NWARPS = NSOFT + NPROD + NISSUE + NPV;
+constexpr int NTHREADS = NWARPS * 32;        // 768
 constexpr int ROWS_PER_THREAD = TK / NPROD;  // key rows a producer thread converts (4)
 constexpr int QBLK = 8192;                   // Q column block: 64 head rows x 128 B (SW128)
 constexpr int KBLK = TK * 128;               // key column block: 64 key rows x 128 B
@@ -290,10 +290,13 @@ template <bool EX>
 __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t bar_kempty[NBUF], bar_kfull[NBUF], bar_sfull[NBUF], bar_pempty[2], bar_drain;
+    __shared__ __align__(8) uint64_t bar_kempty[NBUF], bar_kfull[NBUF], bar_sfull[NBUF], bar_pready[2], bar_pempty[2],
+        bar_drain;
     __shared__ uint32_t tmem_base_slot;
-    __shared__ float s_alpha[HP], s_l[HP], s_rl[HP];
-    __shared__ int s_resc_w[NSOFT];
+    // rescale factors and flags, double-buffered by tile parity: with no barrier
+    // after the P stores a warp may run one tile ahead of the others
+    __shared__ float s_alpha[2][HP], s_l[HP], s_rl[HP];
+    __shared__ int s_resc_w[2][NSOFT];
     __shared__ volatile int s_abort;
     __shared__ float s_qr[HP];                       // 1 / rms of each query head (query RMSNorm)
     __shared__ float s_cos[D_ROPE / 2], s_sin[D_ROPE / 2];   // RoPE of the unit's position
@@ -312,13 +315,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
 
     if (tid == 0) {
         for (int i = 0; i < NBUF; ++i) {
-            mbar_init(smem_u32(&bar_kempty[i]), 4);  // freed by the four PV issuers
+            mbar_init(smem_u32(&bar_kempty[i]), NPV);  // freed by the PV issuers
             mbar_init(smem_u32(&bar_kfull[i]), NPROD);  // one arrival per producer warp
             mbar_init(smem_u32(&bar_sfull[i]), NISSUE);   // both QK issuers
         }
-        mbar_init(smem_u32(&bar_pempty[0]), 4);      // the four PV issuers
-        mbar_init(smem_u32(&bar_pempty[1]), 4);
-        mbar_init(smem_u32(&bar_drain), NISSUE + 4);   // the MMA-issuing threads
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&bar_pready[i]), NSOFT);  // the softmax warps stored P
+            mbar_init(smem_u32(&bar_pempty[i]), NPV);    // the PV issuers' MMAs completed
+        }
+        mbar_init(smem_u32(&bar_drain), NISSUE + NPV);   // the MMA-issuing threads
         s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -477,7 +482,34 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
 
     constexpr uint32_t id_qk = idesc_f16(64, TK, 0, 0);   // S[64 heads x 64 keys]
     constexpr uint32_t id_pv = idesc_f16(128, HP, 1, 0);
-    if (warp >= NSOFT + NPROD) {
+    if (warp >= NSOFT + NPROD + NISSUE) {
+        // ------------------------------------------------------------ PV issue
+        // O^T += V^T . P^T, V^T read MN-major from the key tile: dims in atoms of 64
+        // (column blocks, KBLK apart), keys in atoms of 8 rows (1024 B apart).  Lane 0
+        // of warp 22 + c issues M-tiles 2 c and 2 c + 1 (output dims 256 c .. + 255),
+        // off the softmax warps' path.
+        const int c = warp - (NSOFT + NPROD + NISSUE);
+        if (lane == 0) {
+            for (int i = 0; i < n_tiles; ++i) {
+                const int b = i % NBUF, pb = i & 1;
+                if (!wait_bar(smem_u32(&bar_pready[pb]), (i >> 1) & 1, &s_abort)) break;
+                fence_after();
+                const uint64_t vd = sdesc(sbase + K_OFF + b * 8 * KBLK, KBLK, 1024);
+                const uint64_t pd = sdesc(sbase + P_OFF + pb * PBLK, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < TK / 16; ++kk)
+#pragma unroll
+                    for (int m2 = 0; m2 < 2; ++m2) {
+                        const int mt = 2 * c + m2;
+                        mma_f16(tmem + O_COL + mt * HP, vd + static_cast<uint32_t>((2 * mt * KBLK + kk * 2048) >> 4),
+                                pd + static_cast<uint32_t>((kk * 32) >> 4), id_pv, (i > 0 || kk > 0) ? 1u : 0u);
+                    }
+                mma_commit(smem_u32(&bar_pempty[pb]));
+                mma_commit(smem_u32(&bar_kempty[b]));
+            }
+            mma_commit(smem_u32(&bar_drain));
+        }
+    } else if (warp >= NSOFT + NPROD) {
         // ------------------------------------------------------------ QK issue
         // Warp 20 + c issues half c of every tile's QK (dims 256 c .. 256 c + 255) into
         // its own accumulator: one thread issues an MMA every ~70 clocks whatever its
@@ -632,15 +664,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
             float rs = ps[0];
             rs += __shfl_xor_sync(0xffffffffu, rs, 16);
             l_run += rs;
-            if (lane < 16) s_alpha[h] = alpha;
+            if (lane < 16) s_alpha[i & 1][h] = alpha;
             const unsigned wr = __ballot_sync(0xffffffffu, resc);
-            if (lane == 0) s_resc_w[warp] = wr != 0u;
+            if (lane == 0) s_resc_w[i & 1][warp] = wr != 0u;
             // P buffer pb is free once PV(i-2) has completed
             if (i >= 2) {
                 if (!wait_bar(smem_u32(&bar_pempty[pb]), ((i - 2) >> 1) & 1, &s_abort)) { ok = false; break; }
             }
             named_bar(1, NSOFT * 32);
-            if (s_resc_w[0] | s_resc_w[1] | s_resc_w[2] | s_resc_w[3]) {
+            if (s_resc_w[i & 1][0] | s_resc_w[i & 1][1] | s_resc_w[i & 1][2] | s_resc_w[i & 1][3]) {
                 // O^T must be stable: PV(i-1) complete
                 if (i >= 1 && !wait_bar(smem_u32(&bar_pempty[(i - 1) & 1]), ((i - 1) >> 1) & 1, &s_abort)) { ok = false; break; }
                 fence_after();
@@ -650,7 +682,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
                 for (int c0 = 0; c0 < HP; c0 += 16) {
                     float al[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) al[j] = s_alpha[c0 + j];
+                    for (int j = 0; j < 16; ++j) al[j] = s_alpha[i & 1][c0 + j];
 #pragma unroll 1
                     for (int mt = 0; mt < 4; ++mt) {
                         uint32_t o[16];
@@ -669,26 +701,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
             for (int c = 0; c < 4; ++c)
                 *reinterpret_cast<uint4*>(pbuf + sw128(h, 4 * kh + c)) =
                     make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            // hand P(i) (and any rescale of O^T) to the PV issuers
             fence_async_smem();
             fence_before();
-            named_bar(1, NSOFT * 32);
-            if (lane == 0) {
-                fence_after();
-                // V^T read MN-major from the key tile: dims in atoms of 64 (column blocks,
-                // KBLK apart), keys in atoms of 8 rows (1024 B apart).  Lane 0 of warp w
-                // issues M-tile w (output dims 128 w .. 128 w + 127).
-                const uint64_t vd = sdesc(sbase + K_OFF + b * 8 * KBLK, KBLK, 1024);
-                const uint64_t pd = sdesc(sbase + P_OFF + pb * PBLK, 16, 1024);
-                const int mt = warp;
-#pragma unroll
-                for (int kk = 0; kk < TK / 16; ++kk)
-                    mma_f16(tmem + O_COL + mt * HP, vd + static_cast<uint32_t>((2 * mt * KBLK + kk * 2048) >> 4),
-                            pd + static_cast<uint32_t>((kk * 32) >> 4), id_pv, (i > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(smem_u32(&bar_pempty[pb]));
-                mma_commit(smem_u32(&bar_kempty[b]));
-            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bar_pready[pb]));
         }
-        if (lane == 0) mma_commit(smem_u32(&bar_drain));
         // ---- epilogue: wait for the last PV, then O^T / l -> out (or the split partials)
         if (ok && n_tiles > 0) {
             ok = wait_bar(smem_u32(&bar_pempty[(n_tiles - 1) & 1]), ((n_tiles - 1) >> 1) & 1, &s_abort);

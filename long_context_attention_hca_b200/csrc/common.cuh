@@ -32,6 +32,8 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 int sm_count();
 // process-wide CTA cap of a decode attention launch (0: none); see hca_set_launch_budget
 int launch_budget(int op);
+// Sets this thread's override of a launch budget (0: none); returns the previous one.
+int thread_budget_swap(int op, int max_ctas);
 
 // Programmatic dependent launch.  A kernel launched by launch_pdl may be
 // scheduled while the previous kernel of its stream is still running; it calls

@@ -47,7 +47,8 @@ extern "C" int hca_decode_step_host(const hca_decode_step_plan* p, const uint16_
     if (!p || !h_q_csa || !h_q_hca || !h_iq_codes || !h_iq_sf || !h_iq_w || !h_out_csa || !h_out_hca)
         return HCA_ERR_INVALID_ARG;
     if (!p->side_stream || !p->ev_fork || !p->ev_index || !p->ev_q || !p->ev_join) return HCA_ERR_INVALID_ARG;
-    if (p->B <= 0 || p->H <= 0 || p->Hi <= 0 || p->c <= 0 || p->layout.d <= 0) return HCA_ERR_INVALID_ARG;
+    if (p->B <= 0 || p->H <= 0 || p->Hi <= 0 || p->c <= 0 || p->layout.d <= 0 || p->hca_ctas < 0)
+        return HCA_ERR_INVALID_ARG;
     const size_t d = static_cast<size_t>(p->layout.d);
     const size_t q_bytes = static_cast<size_t>(p->B) * p->H * d * 2;
     const size_t iqc = static_cast<size_t>(p->B) * p->Hi * (p->c / 2);
@@ -75,11 +76,16 @@ extern "C" int hca_decode_step_host(const hca_decode_step_plan* p, const uint16_
                                    p->ws_csa_bytes, side));
     HCA_TRY(cpy(h_out_csa, p->out_csa, q_bytes, cudaMemcpyDeviceToHost, side));
     HCA_TRY(rec(p->ev_join, side));
-    // HCA: dense attention once the indexer has run, then its output
+    // HCA: dense attention once the indexer has run, on at most hca_ctas CTAs (by
+    // default half the SMs) so that the CSA chain's select and attention keep
+    // the rest; then its output
     HCA_TRY(wait(stream, p->ev_index));
-    HCA_TRY(compressed_attn_decode(p->q_hca, p->B, p->H, p->layout, p->hca_cache, nullptr, 0, p->hca_n, p->hca_max,
-                                   p->hca_window, p->W, p->softmax_scale, p->out_hca, nullptr, p->ws_hca,
-                                   p->ws_hca_bytes, stream));
+    const int prev = thread_budget_swap(HCA_BUDGET_DENSE_DECODE, p->hca_ctas > 0 ? p->hca_ctas : sm_count() / 2);
+    const int rc = compressed_attn_decode(p->q_hca, p->B, p->H, p->layout, p->hca_cache, nullptr, 0, p->hca_n,
+                                          p->hca_max, p->hca_window, p->W, p->softmax_scale, p->out_hca, nullptr,
+                                          p->ws_hca, p->ws_hca_bytes, stream);
+    thread_budget_swap(HCA_BUDGET_DENSE_DECODE, prev);
+    HCA_TRY(rc);
     HCA_TRY(cpy(h_out_hca, p->out_hca, q_bytes, cudaMemcpyDeviceToHost, stream));
     HCA_TRY(wait(stream, p->ev_join));
     return HCA_OK;

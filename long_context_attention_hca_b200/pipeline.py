@@ -13,6 +13,7 @@ are CSA (4x) and odd layers HCA.
 """
 from __future__ import annotations
 
+import contextlib
 import dataclasses
 from typing import List, Optional
 
@@ -73,20 +74,26 @@ class DecodeRunner:
     indexer fills every SM anyway."""
 
     def __init__(self, layers: List[DecodeLayer], B: int, H: int, k: int, pos: int, softmax_scale: float,
-                 device="cuda", schedule: str = "after_index", dense_budget: int = 0, fused_select: bool = True,
-                 sparse_budget: int = 0, extras: Optional[list] = None, index_budget: int = 0):
+                 device="cuda", schedule: str = "after_index", dense_budget: Optional[int] = None,
+                 fused_select: bool = True, sparse_budget: int = 0, extras: Optional[list] = None,
+                 index_budget: int = 0):
         """schedule: "after_index" -- an HCA launch waits for the indexer queued
         before it; "hca_first" -- all HCA launches are queued first and start at
-        once, with dense_budget (if > 0) capping their CTAs so that the CSA
-        chain runs beside them on the remaining SMs.  extras: per layer, an
-        AttnExtras (section 9 query RMSNorm, RoPE, sink) for its attention
+        once.  dense_budget caps the CTAs of this runner's HCA launches (applied
+        around its own calls only): None -- half the SMs when CSA and HCA layers
+        run side by side (the select and the CSA attention keep the other half),
+        else the library default; 0 -- the library default.  extras: per layer,
+        an AttnExtras (section 9 query RMSNorm, RoPE, sink) for its attention
         call, or None."""
         self.extras = extras if extras is not None else [None] * len(layers)
         if schedule not in ("after_index", "hca_first"):
             raise ValueError(schedule)
         self.schedule = schedule
-        if dense_budget:
-            set_launch_budget(BUDGET_DENSE_DECODE, dense_budget)
+        dev = torch.device(device)
+        if dense_budget is None:
+            both = any(L.ratio == CSA_RATIO for L in layers) and any(L.ratio != CSA_RATIO for L in layers)
+            dense_budget = torch.cuda.get_device_properties(dev).multi_processor_count // 2 if both else 0
+        self.dense_budget = dense_budget
         if sparse_budget:
             set_launch_budget(BUDGET_SPARSE_DECODE, sparse_budget)
         if index_budget:
@@ -95,7 +102,6 @@ class DecodeRunner:
         self.scale = softmax_scale
         d = layers[0].cache.layout[0]
         self.d = d
-        dev = torch.device(device)
         self.q_pos = torch.full((B, 1), pos, dtype=torch.int32, device=dev)
         self.out = [torch.empty((B, H, d), dtype=torch.bfloat16, device=dev) for _ in layers]
         self.n_dense = {}
@@ -118,13 +124,26 @@ class DecodeRunner:
             else:
                 self.n_dense[li] = torch.full((B,), L.n_entries, dtype=torch.int32, device=dev)
                 mc = L.n_entries
-            nbytes = decode_workspace_size(B, H, L.cache.layout, mc, W)
+            with self._dense_scope(L.ratio != CSA_RATIO):
+                nbytes = decode_workspace_size(B, H, L.cache.layout, mc, W)
             self.ws[li] = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
         lo, hi = torch.cuda.Stream.priority_range()
         self.side = torch.cuda.Stream(device=dev, priority=hi)
         self.copy_in = torch.cuda.Stream(device=dev)     # step_host: attention queries in
         self.copy_out = torch.cuda.Stream(device=dev)    # step_host: outputs out
         self.kernels_per_step = self._count_kernels()
+
+    @contextlib.contextmanager
+    def _dense_scope(self, on: bool):
+        """This runner's HCA CTA budget, around its own dense calls only."""
+        if not on or not self.dense_budget:
+            yield
+            return
+        prev = set_launch_budget(BUDGET_DENSE_DECODE, self.dense_budget)
+        try:
+            yield
+        finally:
+            set_launch_budget(BUDGET_DENSE_DECODE, prev)
 
     def _count_kernels(self) -> int:
         """Kernels of this library launched per step: attention (+ split combine) per
@@ -134,7 +153,8 @@ class DecodeRunner:
         n = 0
         for li, L in enumerate(self.layers):
             mc = min(self.k, L.n_entries) if L.ratio == CSA_RATIO else L.n_entries
-            split = decode_workspace_size(self.B, self.H, L.cache.layout, mc, L.window.shape[1]) > 0
+            with self._dense_scope(L.ratio != CSA_RATIO):
+                split = decode_workspace_size(self.B, self.H, L.cache.layout, mc, L.window.shape[1]) > 0
             n += 1 + int(split)
             if L.ratio == CSA_RATIO:
                 wide = topk_workspace_size(self.B, L.n_entries, self.k) > 0
@@ -180,6 +200,7 @@ class DecodeRunner:
         p.out_csa, p.out_hca = ptr(self.out[c_]), ptr(self.out[h_])
         p.side_stream = self._capi_side.cuda_stream
         p.ev_fork, p.ev_index, p.ev_q, p.ev_join = (e.cuda_event for e in self._capi_events)
+        p.hca_ctas = self.dense_budget
         self._capi_layers = (c_, h_)
         return p
 
@@ -285,9 +306,10 @@ class DecodeRunner:
                     main.wait_event(after_index)
                 if q_ready is not None:
                     main.wait_event(q_ready[li])
-                timed("hca_attn", li, lambda: compressed_attn_decode(
-                    q[li], L.cache, self.n_dense[li], L.n_entries, L.window, self.scale, out=self.out[li],
-                    ws=self.ws[li], extras=self.extras[li]))
+                with self._dense_scope(True):
+                    timed("hca_attn", li, lambda: compressed_attn_decode(
+                        q[li], L.cache, self.n_dense[li], L.n_entries, L.window, self.scale, out=self.out[li],
+                        ws=self.ws[li], extras=self.extras[li]))
                 if on_out is not None:
                     on_out(li, main)
         main.wait_stream(self.side)
