@@ -358,8 +358,11 @@ def bench_decode(args, wl, world, rank, pg):
         reps.append((dw, runner))
     main = torch.cuda.current_stream()
 
-    # one graph per replica, with external timing events around each kernel class
-    graphs, evs = [], []
+    # per replica: the step as one graph (timed), and a second graph with external
+    # timing events around each kernel class (replayed once, untimed, for the
+    # per-kernel breakdown: event nodes between kernels would cost time and break
+    # the programmatic launch edges of the timed graph)
+    graphs, graphs_ev, evs = [], [], []
     for dw, runner in reps:
         s = torch.cuda.Stream()
         s.wait_stream(main)
@@ -369,11 +372,14 @@ def bench_decode(args, wl, world, rank, pg):
         main.wait_stream(s)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
-        ev = {}
-        runner.timing_events = ev
         with torch.cuda.graph(g):
-            runner.step(dw.q, dw.iq, events=ev)
+            runner.step(dw.q, dw.iq)
         graphs.append(g)
+        g2 = torch.cuda.CUDAGraph()
+        ev = {}
+        with torch.cuda.graph(g2):
+            runner.step(dw.q, dw.iq, events=ev)
+        graphs_ev.append(g2)
         evs.append(ev)
     torch.cuda.synchronize()
 
@@ -399,8 +405,8 @@ def bench_decode(args, wl, world, rank, pg):
     ms = e0.elapsed_time(e1) / args.steps
     ms_max = max_over_ranks(ms, pg)
 
-    # per-kernel durations from one more (untimed) replay of each replica graph
-    for g in graphs:
+    # per-kernel durations from one (untimed) replay of each replica's evented graph
+    for g in graphs_ev:
         g.replay()
     torch.cuda.synchronize()
     kern = {}
@@ -679,9 +685,14 @@ def bench_prefill(args, wl, world, rank, pg):
         runner.step(*args_step)
     main.wait_stream(s)
     torch.cuda.synchronize()
+    # the timed graph has no timing events; a second one with them gives the
+    # per-kernel breakdown (replayed once, untimed)
     g = torch.cuda.CUDAGraph()
-    ev = {}
     with torch.cuda.graph(g):
+        runner.step(*args_step)
+    g_ev = torch.cuda.CUDAGraph()
+    ev = {}
+    with torch.cuda.graph(g_ev):
         runner.step(*args_step, events=ev)
     for _ in range(max(3, args.warmup)):
         g.replay()
@@ -701,8 +712,10 @@ def bench_prefill(args, wl, world, rank, pg):
     barrier(pg)
     clocks.stop()
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, pg)
+    g_ev.replay()
+    torch.cuda.synchronize()
     kern_ms = {k: a.elapsed_time(b) for k, (a, b) in ev.items()}
-    del g
+    del g, g_ev
 
     # each attention launch alone (CUDA events on the launching stream)
     st = pw.state
@@ -825,8 +838,11 @@ def bench_stack(args, wl, world, rank, pg):
     main.wait_stream(s)
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
-    ev = {}
     with torch.cuda.graph(g):
+        runner.step(dw.q, dw.iq)
+    g_ev = torch.cuda.CUDAGraph()        # with per-kernel timing events, replayed once untimed
+    ev = {}
+    with torch.cuda.graph(g_ev):
         runner.step(dw.q, dw.iq, events=ev)
     for _ in range(max(1, args.warmup)):
         g.replay()
@@ -845,6 +861,8 @@ def bench_stack(args, wl, world, rank, pg):
     barrier(pg)
     clocks.stop()
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, pg)
+    g_ev.replay()
+    torch.cuda.synchronize()
     per = {k: a.elapsed_time(b) * 1e3 for k, (a, b) in ev.items()}
     ratios = pro_layer_ratios(wl.layers)
     resident = kv_resident_bytes(wl.B, wl.t + 1, ratios)
@@ -855,7 +873,7 @@ def bench_stack(args, wl, world, rank, pg):
             "data": "synthetic", "config": {"workload": wl.name, "global_batch": wl.B, "seq_len": wl.t + 1,
                                             "layers": wl.layers, "parallelism": "single GPU"},
             "kv_resident_bytes": resident, "gqa8_bf16_bytes": gqa, "kv_ratio": resident / gqa,
-            "kernels_us_last_replay": per, "clocks": clocks.summary(t0, t1)}
+            "kernels_us_untimed_replay": per, "clocks": clocks.summary(t0, t1)}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
