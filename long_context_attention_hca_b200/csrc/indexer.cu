@@ -407,6 +407,20 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     return false;
 }
 
+// The same wait for the single-thread roles (loads, MMA issue), with a short
+// sleep between polls: their spinning would otherwise take issue slots from the
+// epilogue warps that share their sub-partitions.
+__device__ __forceinline__ bool wait_bar_idle(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    for (long long it = 0; it < kWaitLimit; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        __nanosleep(32);
+        if ((it & 1023) == 1023 && *abort_flag) return false;
+    }
+    *abort_flag = 1;
+    atomicExch(&g_index_device_error, 1);
+    return false;
+}
+
 // QG queries per CTA, HG groups of 4 indexer heads (Hi = 4 HG; N = 16 QG HG
 // accumulator columns: query q, group hg at column 16 (q HG + hg), then block
 // b, head h of the group at + 4 b + h), NBD accumulator buffers, KS key
@@ -469,6 +483,31 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" :: "r"(smem_u32(&tmem_slot)), "r"(NCOLS) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
+    // the query's operands and exponents: every global load of the prologue is issued
+    // before any of them is used (one round trip, not one per table)
+    constexpr int NQV = N * 8;                          // 16-byte slots of the query operand
+    constexpr int QV_PT = (NQV + (64 + 128 * EG) - 1) / (64 + 128 * EG);
+    uint2 qv[QV_PT];
+#pragma unroll
+    for (int k2 = 0; k2 < QV_PT; ++k2) {
+        const int x = tid + k2 * blockDim.x;
+        qv[k2] = make_uint2(0u, 0u);
+        if (x < NQV) {
+            const int n = x >> 3, j = x & 7;
+            const int q = n / (16 * HG), blk = (n >> 2) & 3, h = ((n >> 4) % HG) * 4 + (n & 3);
+            if ((j >> 1) == blk) qv[k2] = __ldg(reinterpret_cast<const uint2*>(q_codes + ((qrow0 + q) * HI + h) * 64 + j * 8));
+        }
+    }
+    // exponents of (query, group hg, block blk, head hh) at z = hg 16 + blk 4 + hh
+    static_assert(QG * 16 * HG <= 64 + 128 * EG && QG * HI <= 64 + 128 * EG, "one exponent and weight per thread");
+    const bool has_e = tid < QG * 16 * HG;
+    int e_raw = 0;
+    if (has_e) {
+        const int q = tid / (16 * HG), z = tid % (16 * HG), hg = z >> 4, blk = (z >> 2) & 3, h = hg * 4 + (z & 3);
+        e_raw = static_cast<int>(__ldg(q_sf + ((qrow0 + q) * HI + h) * 4 + blk)) - 254;
+    }
+    const float w_raw = tid < QG * HI ? __ldg(w + (qrow0 + tid / HI) * HI + tid % HI) : 0.0f;
+    const int32_t pos_raw = tid < QG ? q_pos[qrow0 + tid] : 0;
     if (QG == 1 && hist)
         for (int x = tid; x < 2048; x += blockDim.x) sh_hist[x] = 0u;
     // the loads write only the 8 data bytes of each 16-byte slot: zero the padding once
@@ -478,34 +517,30 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
     }
     // query operand: row n = (q HG + hg) 16 + blk 4 + hh (head h = 4 hg + hh); slot j
     // (elements 16j..16j+15) is block j/2
-    for (int x = tid; x < N * 8; x += blockDim.x) {
-        const int n = x >> 3, j = x & 7;
-        const int q = n / (16 * HG), hg = (n >> 4) % HG, blk = (n >> 2) & 3, h = hg * 4 + (n & 3);
-        uint2 v = make_uint2(0, 0);
-        if ((j >> 1) == blk) v = __ldg(reinterpret_cast<const uint2*>(q_codes + ((qrow0 + q) * HI + h) * 64 + j * 8));
-        *reinterpret_cast<uint4*>(sB + sw128(n, j)) = make_uint4(v.x, v.y, 0u, 0u);
+#pragma unroll
+    for (int k2 = 0; k2 < QV_PT; ++k2) {
+        const int x = tid + k2 * blockDim.x;
+        if (x < NQV) *reinterpret_cast<uint4*>(sB + sw128(x >> 3, x & 7)) = make_uint4(qv[k2].x, qv[k2].y, 0u, 0u);
     }
-    for (int x = tid; x < QG * 16 * HG; x += blockDim.x) {
-        const int q = x / (16 * HG), z = x % (16 * HG), hg = z >> 4, blk = (z >> 2) & 3, h = hg * 4 + (z & 3);
-        s_eq[q][z] = static_cast<int>(__ldg(q_sf + ((qrow0 + q) * HI + h) * 4 + blk)) - 254;
+    if (has_e) s_eq[tid / (16 * HG)][tid % (16 * HG)] = e_raw;
+    if (tid < QG * HI) s_w[tid / HI][tid % HI] = w_raw;
+    if (tid < QG) {
+        const int64_t e = (static_cast<int64_t>(pos_raw) + 1) / m;
+        s_elig[tid] = e < 0 ? 0 : (e > Nc_cap ? Nc_cap : e);
     }
-    for (int x = tid; x < QG * HI; x += blockDim.x) s_w[x / HI][x % HI] = __ldg(w + (qrow0 + x / HI) * HI + x % HI);
+    __syncthreads();
     for (int x = tid; x < QG * HG * 4; x += blockDim.x) {
         // fast path of a (query, group, block): every head's 2^(eq + ek) is a normal float and
         // |block dot| * 2^(eq + ek) < 2^127, i.e. eq + ek in [-126, 116] for the group's heads
         const int q = x / (HG * 4), hg = (x / 4) % HG, blk = x & 3;
         int mn = 1 << 20, mx = -(1 << 20);
         for (int hh = 0; hh < 4; ++hh) {
-            const int e = static_cast<int>(__ldg(q_sf + ((qrow0 + q) * HI + hg * 4 + hh) * 4 + blk)) - 254;
+            const int e = s_eq[q][hg * 16 + blk * 4 + hh];
             mn = min(mn, e);
             mx = max(mx, e);
         }
         s_klo[q][hg][blk] = -126 - mn;
         s_khi[q][hg][blk] = 116 - mx;
-    }
-    if (tid < QG) {
-        int64_t e = (static_cast<int64_t>(q_pos[qrow0 + tid]) + 1) / m;
-        s_elig[tid] = e < 0 ? 0 : (e > Nc_cap ? Nc_cap : e);
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -532,7 +567,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
         if (lane == 0) {
             for (int t = 0; t < n_tiles; ++t) {
                 const int st = t % KS;
-                if (t >= KS && !wait_bar(smem_u32(&bar_empty[st]), ((t / KS) - 1) & 1, &s_abort)) break;
+                if (t >= KS && !wait_bar_idle(smem_u32(&bar_empty[st]), ((t / KS) - 1) & 1, &s_abort)) break;
                 const uint32_t full = smem_u32(&bar_full[st]);
                 uint8_t* stage = smem + st * STAGE_BYTES;
                 mbar_expect_tx(full, CODE_TX_BYTES + SCALE_BYTES);
@@ -546,8 +581,8 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
             const uint32_t bbase = smem_u32(sB);
             for (int t = 0; t < n_tiles; ++t) {
                 const int st = t % KS, nb = t % NBD;
-                if (!wait_bar(smem_u32(&bar_full[st]), (t / KS) & 1, &s_abort)) break;
-                if (t >= NBD && !wait_bar(smem_u32(&bar_acce[nb]), ((t / NBD) - 1) & 1, &s_abort)) break;
+                if (!wait_bar_idle(smem_u32(&bar_full[st]), (t / KS) & 1, &s_abort)) break;
+                if (t >= NBD && !wait_bar_idle(smem_u32(&bar_acce[nb]), ((t / NBD) - 1) & 1, &s_abort)) break;
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                 const uint32_t abase = smem_u32(smem + st * STAGE_BYTES);
                 const uint32_t d = tmem + static_cast<uint32_t>(nb * N);
