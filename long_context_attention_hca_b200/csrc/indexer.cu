@@ -871,7 +871,7 @@ int index_launch_hist(const uint8_t* q_codes, const uint8_t* q_sf, const float* 
         return itc::launch_tc<1, 2, 5, 2, 16>(q_codes, q_sf, w, k_codes, k_sf, q_pos, B, B, 1, Nc_cap, m, sc, st,
                                               budget > 0 ? std::min<int64_t>(budget, sm_count()) : sm_count(),
                                               hist, hist_stride, bf16 ? 1 : 0);
-    return itc::launch_tc<1, 4, 5, 2>(q_codes, q_sf, w, k_codes, k_sf, q_pos, B, B, 1, Nc_cap, m, sc, st,
+    return itc::launch_tc<1, 8, 5, 2>(q_codes, q_sf, w, k_codes, k_sf, q_pos, B, B, 1, Nc_cap, m, sc, st,
                                       budget > 0 ? budget : 2LL * sm_count(), hist, hist_stride, bf16 ? 1 : 0);
 }
 
@@ -910,7 +910,7 @@ int index_launch(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
             rc = itc::launch_tc<16, 2, 4, 2>(q_codes, q_sf, w, k_codes, k_sf, q_pos, rows, B, Tq, Nc_cap, m, scores, st,
                                              2LL * sm_count(), nullptr, 0, bf16 ? 1 : 0);
         else
-            rc = itc::launch_tc<1, 4, 5, 2>(q_codes, q_sf, w, k_codes, k_sf, q_pos, rows, B, Tq, Nc_cap, m, scores, st,
+            rc = itc::launch_tc<1, 8, 5, 2>(q_codes, q_sf, w, k_codes, k_sf, q_pos, rows, B, Tq, Nc_cap, m, scores, st,
                                             2LL * sm_count(), nullptr, 0, bf16 ? 1 : 0);
         if (rc != HCA_ERR_UNSUPPORTED || bf16) return rc;
         // unaligned key buffers: CUDA-core tensor path below
