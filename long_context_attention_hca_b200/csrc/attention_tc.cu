@@ -831,16 +831,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
 // weight 2^(m_s - M) l_s (the partials are O_s / l_s), L = their sum (+ the
 // sink); out = sum_s weight_s o_s / L.  Thread t sums heads 4 (t / 8) .. + 3
 // at dims 16 b + 2 (t % 8) and the next one: one 16-byte fp16 load per split
-// (the partials keep heads in fours, dims consecutive), 32 splits in flight.
-// The (m, l) pairs are staged in shared memory first, every load in flight.
+// (the partials keep heads in fours, dims consecutive).  Thread t also owns
+// head t / 2's (m, l) of every other split, loaded into registers in the same
+// round as the partials; the weights then come from independent operations,
+// not loops over shared memory (one warp per sub-partition: every latency
+// shows).
 constexpr int COMB_DIMS = 16;
 constexpr int COMB_THREADS = 128;
 constexpr int MAX_SPLITS = 64;
 
 __global__ void __launch_bounds__(COMB_THREADS) combine_tc_kernel(Params p) {
-    __shared__ __align__(16) float s_w[MAX_SPLITS][HP];    // maxima, then the split weights
-    __shared__ __align__(16) float s_lv[MAX_SPLITS][HP];   // l
-    __shared__ int s_live[MAX_SPLITS];
+    __shared__ __align__(16) float s_w[MAX_SPLITS][HP];    // split weights
+    __shared__ unsigned long long s_live;                  // splits with keys (they wrote a partial)
     __shared__ float s_inv[HP];
     __shared__ int s_bad[HP];
     const int64_t u = blockIdx.x;
@@ -848,48 +850,50 @@ __global__ void __launch_bounds__(COMB_THREADS) combine_tc_kernel(Params p) {
     const int S = p.n_splits;
     const int t = threadIdx.x;
     pdl_wait();                                    // the split partials are complete
-    {
-        // (m, l) of every split ([S][2][HP] floats, contiguous) -> shared memory
-        const float4* src = reinterpret_cast<const float4*>(p.part_ml + static_cast<size_t>(u) * S * 2 * HP);
-        constexpr int kPer = MAX_SPLITS * 2 * HP / 4 / COMB_THREADS;
-        const int n4 = S * 2 * HP / 4;
-        float4 buf[kPer];
+    // the first 32 splits' partial rows and this thread's (m, l) pairs cross from L2
+    // in one round (an empty split's row holds stale data: it is loaded, never used)
+    const int hq = t >> 3;                           // heads 4 hq .. 4 hq + 3
+    const int dim = dblk * COMB_DIMS + 2 * (t & 7);  // dims dim, dim + 1
+    const uint16_t* po = p.part_o + (static_cast<size_t>(u) * S * HP + 4 * hq) * D + static_cast<size_t>(dim) * 4;
+    const size_t split_stride = static_cast<size_t>(HP) * D;
+    constexpr int kBatch = 32;                       // partial loads in flight per thread
+    uint4 v[kBatch];
 #pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-            const int i = t + j * COMB_THREADS;
-            buf[j] = i < n4 ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+    for (int j = 0; j < kBatch; ++j)
+        v[j] = j < S ? *reinterpret_cast<const uint4*>(po + j * split_stride) : make_uint4(0u, 0u, 0u, 0u);
+    const int h = t >> 1, sub = t & 1;               // head h, splits sub, sub + 2, ...
+    constexpr int kMl = MAX_SPLITS / 2;
+    const float* ml0 = p.part_ml + static_cast<size_t>(u) * S * 2 * HP;
+    float mr[kMl], lr[kMl];
 #pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-            const int i = t + j * COMB_THREADS;
-            if (i < n4) {
-                const int s = (4 * i) / (2 * HP), r = (4 * i) % (2 * HP);
-                float* dst = r < HP ? &s_w[s][r] : &s_lv[s][r - HP];
-                *reinterpret_cast<float4*>(dst) = buf[j];
-            }
-        }
-        for (int s = t; s < S; s += COMB_THREADS) s_live[s] = 0;
+    for (int j = 0; j < kMl; ++j) {
+        const int sj = sub + 2 * j;
+        mr[j] = sj < S ? ml0[sj * 2 * HP + h] : -INFINITY;
+        lr[j] = sj < S ? ml0[sj * 2 * HP + HP + h] : 0.0f;
     }
-    __syncthreads();
     {
-        // two threads per head (neighbouring lanes): maxima, weights, sums
-        const int h = t >> 1, sub = t & 1;
         float M = -INFINITY;
-        for (int s = sub; s < S; s += 2)
-            if (s_lv[s][h] > 0.0f) M = fmaxf(M, s_w[s][h]);
+#pragma unroll
+        for (int j = 0; j < kMl; ++j)
+            if (lr[j] > 0.0f) M = fmaxf(M, mr[j]);
         M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 1));
         float L = 0.0f;
         int bad = 0;
-        for (int s = sub; s < S; s += 2) {
-            const float ms = s_w[s][h], ls = s_lv[s][h];
-            if (ls != ls) bad = 1;
-            if (ls > 0.0f) s_live[s] = 1;               // a split with keys wrote a partial
-            const float wgt = ls > 0.0f ? exp2f(ms - M) * ls : 0.0f;
-            s_w[s][h] = wgt;
+        unsigned long long live = 0ull;
+#pragma unroll
+        for (int j = 0; j < kMl; ++j) {
+            const int sj = sub + 2 * j;
+            if (lr[j] != lr[j]) bad = 1;
+            const float wgt = lr[j] > 0.0f ? exp2f(mr[j] - M) * lr[j] : 0.0f;
+            if (sj < S) s_w[sj][h] = wgt;
             L += wgt;
+            if (lr[j] > 0.0f) live |= 1ull << sj;
         }
         L += __shfl_xor_sync(0xffffffffu, L, 1);
         bad |= __shfl_xor_sync(0xffffffffu, bad, 1);
+        // a split holds keys for every head or for none: head 0's view decides
+        live |= __shfl_xor_sync(0xffffffffu, live, 1);
+        if (t == 0) s_live = live;
         if (sub == 0) {
             // the sink joins the denominator relative to the global max M
             const float sink = p.sink ? __ldg(p.sink + h) : -INFINITY;
@@ -902,25 +906,19 @@ __global__ void __launch_bounds__(COMB_THREADS) combine_tc_kernel(Params p) {
         }
     }
     __syncthreads();
-    const int hq = t >> 3;                           // heads 4 hq .. 4 hq + 3
-    const int dim = dblk * COMB_DIMS + 2 * (t & 7);  // dims dim, dim + 1
-    const uint16_t* po = p.part_o + (static_cast<size_t>(u) * S * HP + 4 * hq) * D + static_cast<size_t>(dim) * 4;
-    const size_t split_stride = static_cast<size_t>(HP) * D;
+    const unsigned long long live = s_live;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // [dim offset][head offset]
-    constexpr int kBatch = 32;                       // partial loads in flight per thread
     for (int s0 = 0; s0 < S; s0 += kBatch) {
-        uint4 v[kBatch];
+        if (s0 > 0) {
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
-            const int s = s0 + j;
-            // an empty split wrote no partial
-            v[j] = (s < S && s_live[s]) ? *reinterpret_cast<const uint4*>(po + s * split_stride)
-                                        : make_uint4(0u, 0u, 0u, 0u);
+            for (int j = 0; j < kBatch; ++j)
+                v[j] = s0 + j < S ? *reinterpret_cast<const uint4*>(po + (s0 + j) * split_stride)
+                                  : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int j = 0; j < kBatch; ++j) {
             const int s = s0 + j;
-            if (s < S && s_live[s]) {
+            if (s < S && ((live >> s) & 1ull)) {
                 const float4 w4 = *reinterpret_cast<const float4*>(&s_w[s][4 * hq]);
                 const float2 a0 = unpack_half2(v[j].x), a1 = unpack_half2(v[j].y);   // dim: heads 0-1, 2-3
                 const float2 b0 = unpack_half2(v[j].z), b1 = unpack_half2(v[j].w);   // dim + 1
