@@ -154,10 +154,12 @@ def barrier(pg):
 # the one that was captured (first 16 hex digits of its sha256); otherwise the
 # bench reports null.
 MEASURED_TRAFFIC = {
-    "hca_attn": {"bytes": 20651776, "source": "long_context_attention_hca_b200/csrc/attention_tc.cu",
-                 "sha256_16": "6cc15c7abc43b18b"},
-    "indexer": {"bytes": 73379328, "source": "long_context_attention_hca_b200/csrc/indexer.cu",
-                "sha256_16": "34c10bfc9059ad78"},
+    # dram__bytes_read.sum + dram__bytes_write.sum of one launch on decode_b4_1m
+    # (1-pass ncu capture, caches flushed): 20.65 MB + 0 B, and 71.37 MB + 1.40 MB
+    "hca_attn": {"bytes": 20650000, "source": "long_context_attention_hca_b200/csrc/attention_tc.cu",
+                 "sha256_16": "4e5d128602cdc992"},
+    "indexer": {"bytes": 72770000, "source": "long_context_attention_hca_b200/csrc/indexer.cu",
+                "sha256_16": "afc2390707e8cf84"},
 }
 
 

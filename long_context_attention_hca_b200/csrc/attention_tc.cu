@@ -17,13 +17,15 @@
 //                       P^T the softmax probabilities stored K-major.
 // TMEM: S in NBUF buffers, each two 64-column partial sums (K halves), + O^T
 // (4 x 64 columns): all 512 columns.
-// Warp roles (704 threads):
+// Warp roles (768 threads):
 //   warps 0-3   softmax: head h = 16 w + (lane & 15); lanes 0-15 take keys
 //               0..31 of the tile, lanes 16-31 keys 32..63; online softmax
 //               in base 2 with a lazy rescale (O^T and l are rescaled only
 //               when a head's running max grows by more than 8, so P <= 2^8
-//               in fp16); all 128 threads (= the 128 TMEM lanes of O^T)
-//               apply a rescale and run the epilogue.
+//               in fp16).  They store P^T and hand it to the PV issuers
+//               through an mbarrier (no barrier among themselves after the
+//               stores, so the rescale state is double-buffered by tile
+//               parity: a warp may run one tile ahead).
 //   warps 4-19  producers: tile i goes to key buffer i % 2 (FP8 code x
 //               scale -> fp16, bf16 -> fp16).  Warp w converts column block
 //               w % 8 (64 dims) of key rows 32 (w / 8) .. + 31: lane l takes
@@ -33,19 +35,25 @@
 //               loads of tile i + 1 as soon as tile i is stored (before it
 //               waits for the buffer), and prefetches the gather indices one
 //               tile ahead.
-//   warps 20-21 QK issue, one warp per key buffer: once the producers have
-//               stored tile i, lane 0 of warp 20 + i % 2 issues its 32 MMAs,
-//               so the QK of consecutive tiles overlaps.
+//   warps 20-21 QK issue: lane 0 of warp 20 + c issues half c of every
+//               tile's QK (dims 256 c .. + 255, 16 MMAs) into its own
+//               accumulator; the softmax adds the two.  One thread issues a
+//               tcgen05.mma about every 70 clocks whatever its shape, so the
+//               issue is spread over warps on different sub-partitions.
+//   warps 22-23 PV issue: lane 0 of warp 22 + c issues M-tiles 2c, 2c + 1 of
+//               O^T += V^T . P^T once the softmax warps have stored P(i),
+//               then commits the P and key buffers' release (tcgen05.commit
+//               tracks the issuing thread's own MMAs: the release barriers
+//               count two arrivals).
 //   All threads load Q (bf16 -> fp16) at the start, every load in flight at once.
+//   Split partials: warps 0-15 (four per TMEM lane quarter, one M-tile
+//   each) store O / l as fp16 with heads in fours ([HP/4][D][4]), so a warp's
+//   32 lanes (consecutive dims) write 256 contiguous bytes per store.
 // Per 64-key tile the MMAs read 128 KB of shared memory (Q and K for QK) and
 // 96 KB (V^T and P, four M-tiles, for PV) and the stores write 72 KB: at
 // 128 B per clock that is ~2300 clocks, the bound of this data flow.
-//   The softmax issues PV(i) from four threads (lane 0 of each warp, one
-//   M-tile each) once all four warps stored P(i): a thread issues
-//   tcgen05.mma one at a time, so four issuers cut the issue latency by
-//   four.  tcgen05.commit tracks the issuing thread's own MMAs, so each
-//   issuer signals the barriers of the work it issued (the PV barriers
-//   count four arrivals).
+// Launches are programmatic (the kernel waits for its stream predecessor
+// before its first read) and trigger the combine once their outputs are stored.
 // Every mbarrier wait is bounded; a timeout sets the device error word,
 // raises the CTA's abort flag, drains the issued MMAs and frees TMEM.
 #include <mutex>
@@ -835,11 +843,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
 // head t / 2's (m, l) of every other split, loaded into registers in the same
 // round as the partials; the weights then come from independent operations,
 // not loops over shared memory (one warp per sub-partition: every latency
-// shows).
+// shows).  NS bounds the launch's split count (the loops are unrolled for it).
 constexpr int COMB_DIMS = 16;
 constexpr int COMB_THREADS = 128;
 constexpr int MAX_SPLITS = 64;
 
+template <int NS>
 __global__ void __launch_bounds__(COMB_THREADS) combine_tc_kernel(Params p) {
     __shared__ __align__(16) float s_w[MAX_SPLITS][HP];    // split weights
     __shared__ unsigned long long s_live;                  // splits with keys (they wrote a partial)
@@ -856,13 +865,13 @@ __global__ void __launch_bounds__(COMB_THREADS) combine_tc_kernel(Params p) {
     const int dim = dblk * COMB_DIMS + 2 * (t & 7);  // dims dim, dim + 1
     const uint16_t* po = p.part_o + (static_cast<size_t>(u) * S * HP + 4 * hq) * D + static_cast<size_t>(dim) * 4;
     const size_t split_stride = static_cast<size_t>(HP) * D;
-    constexpr int kBatch = 32;                       // partial loads in flight per thread
+    constexpr int kBatch = NS < 32 ? NS : 32;        // partial loads in flight per thread
     uint4 v[kBatch];
 #pragma unroll
     for (int j = 0; j < kBatch; ++j)
         v[j] = j < S ? *reinterpret_cast<const uint4*>(po + j * split_stride) : make_uint4(0u, 0u, 0u, 0u);
     const int h = t >> 1, sub = t & 1;               // head h, splits sub, sub + 2, ...
-    constexpr int kMl = MAX_SPLITS / 2;
+    constexpr int kMl = (NS + 1) / 2;
     const float* ml0 = p.part_ml + static_cast<size_t>(u) * S * 2 * HP;
     float mr[kMl], lr[kMl];
 #pragma unroll
@@ -963,8 +972,13 @@ int launch_tc(tc::Params& p, int64_t units, cudaStream_t st) {
     if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
     HCA_CHECK_LAUNCH();
     if (p.n_splits > 1) {
-        e = launch_pdl(tc::combine_tc_kernel, dim3(static_cast<unsigned>(units), tc::D / tc::COMB_DIMS),
-                       dim3(tc::COMB_THREADS), 0, st, p);
+        // the smallest unrolling that covers the split count
+        const int S = p.n_splits;
+        auto comb = S <= 8 ? tc::combine_tc_kernel<8> : S <= 16 ? tc::combine_tc_kernel<16>
+                  : S <= 24 ? tc::combine_tc_kernel<24> : S <= 32 ? tc::combine_tc_kernel<32>
+                  : tc::combine_tc_kernel<64>;
+        e = launch_pdl(comb, dim3(static_cast<unsigned>(units), tc::D / tc::COMB_DIMS), dim3(tc::COMB_THREADS), 0, st,
+                       p);
         if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
         HCA_CHECK_LAUNCH();
     }
