@@ -157,7 +157,7 @@ MEASURED_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch on decode_b4_1m
     # (1-pass ncu capture, caches flushed): 20.65 MB + 0 B, and 71.37 MB + 1.40 MB
     "hca_attn": {"bytes": 20650000, "source": "long_context_attention_hca_b200/csrc/attention_tc.cu",
-                 "sha256_16": "4e5d128602cdc992"},
+                 "sha256_16": "8afb1c32941a19e3"},
     "indexer": {"bytes": 72770000, "source": "long_context_attention_hca_b200/csrc/indexer.cu",
                 "sha256_16": "afc2390707e8cf84"},
 }
