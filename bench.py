@@ -831,7 +831,7 @@ def bench_stack(args, wl, world, rank, pg):
     from long_context_attention_hca_b200.pipeline import (DecodeRunner, gqa_bf16_bytes, kv_resident_bytes,
                                                            pro_layer_ratios)
     dw = build_decode(wl)
-    runner = DecodeRunner(dw.layers, wl.B, wl.H, wl.k, wl.t, wl.softmax_scale)
+    runner = DecodeRunner(dw.layers, wl.B, wl.H, wl.k, wl.t, wl.softmax_scale, dense_budget=args.dense_budget)
     main = torch.cuda.current_stream()
     s = torch.cuda.Stream()
     s.wait_stream(main)
@@ -875,7 +875,8 @@ def bench_stack(args, wl, world, rank, pg):
             "data": "synthetic", "config": {"workload": wl.name, "global_batch": wl.B, "seq_len": wl.t + 1,
                                             "layers": wl.layers, "parallelism": "single GPU"},
             "kv_resident_bytes": resident, "gqa8_bf16_bytes": gqa, "kv_ratio": resident / gqa,
-            "kernels_us_untimed_replay": per, "clocks": clocks.summary(t0, t1)}
+            "kernels_us_untimed_replay": per, "dense_budget_ctas": runner.dense_budget,
+            "clocks": clocks.summary(t0, t1)}
     if rank == 0:
         print(json.dumps(line), flush=True)
 

@@ -320,25 +320,12 @@ cudaError_t launch_cl(int R, int64_t slice, const float* scores, const int32_t* 
 }
 
 // ------------------------------------------------------------------ few long rows
-// Used when there are few rows (decode: one per sequence) of many scores.
-// No clusters: three short kernels, each spread over the whole device.
-//   hist     per row, a 2048-bin histogram of the top 11 bits of the
-//            order-preserving key (shared-memory histogram per CTA, then
-//            global atomics of the non-zero bins).
-//   mark     every CTA of a row finds the same threshold bin T1 (the bin of
-//            the k-th largest key) from the histogram; keys in higher bins
-//            are selected (one bitmap word per warp ballot, no atomics);
-//            keys in bin T1 are appended to the row's candidate list.
-//   resolve  one CTA per row: two histogram passes over the candidates' low
-//            21 bits give the exact key T of the k-th largest score and how
-//            many keys equal to T are still needed; keys above T are marked
-//            selected, keys equal to T are marked in a tie bitmap.  An
-//            ordered scan of both bitmaps then takes the ties lowest index
-//            first and writes the indices ascending.
-// Workspace per row (256-byte aligned): hist u32[2048], header u32[8]
-// (candidate count, T1, keys needed from bin T1), selected and tie bitmaps
-// u32[ceil(Nc_cap / 32)] each, candidates u64[Nc_cap] (key << 32 | index).
-// The histogram, header and bitmaps are cleared by a memset on the stream.
+// Used when there are few rows (decode: one per sequence) of many scores; no
+// clusters (the kernels are described in namespace wide).  Workspace per row
+// (256-byte aligned): the key histogram u32[2048] and a header u32[64] (keys
+// above bin T1, candidates, CTAs done), cleared by a memset on the stream
+// before every call; then the above keys' indices u32[kMaxK] and the
+// candidates' composite keys u64[Nc_cap].
 namespace wide {
 
 // Few long rows (decode: one row per sequence).  The 11-bit key histogram of
