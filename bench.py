@@ -347,7 +347,7 @@ def run_reference(args, wl):
 def bench_decode(args, wl, world, rank, pg):
     import long_context_attention_hca_b200 as hca
     from hca_workloads import build_decode
-    from long_context_attention_hca_b200.pipeline import DecodeRunner
+    from long_context_attention_hca_b200.pipeline import DecodeRunner, packed_indexer_query
 
     dev = torch.device("cuda")
     n_rep = args.replicas
@@ -420,10 +420,11 @@ def bench_decode(args, wl, world, rank, pg):
     # ---------------- end to end through the public API: host q / indexer q in, outputs out
     dw, runner = reps[0]
     h_q = [t.to("cpu").pin_memory() for t in dw.q]
-    h_iq = [None if t is None else tuple(x.to("cpu").pin_memory() for x in t) for t in dw.iq]
+    # each layer's indexer query packed in one buffer, host and device: one copy
+    h_iq = [None if t is None else packed_indexer_query(t, device="cpu", pin=True) for t in dw.iq]
     h_out = [torch.empty_like(o, device="cpu").pin_memory() for o in runner.out]
     d_q = [t.clone() for t in dw.q]
-    d_iq = [None if t is None else tuple(x.clone() for x in t) for t in dw.iq]
+    d_iq = [None if t is None else packed_indexer_query(t) for t in dw.iq]
     h2d = sum(t.numel() * t.element_size() for t in h_q) + sum(
         sum(x.numel() * x.element_size() for x in t) for t in h_iq if t is not None)
     d2h = sum(t.numel() * t.element_size() for t in h_out)

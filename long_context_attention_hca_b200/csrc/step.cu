@@ -7,15 +7,21 @@
 // position).
 //
 // Schedule (the two paths share no data):
-//   side:   waits ev_fork | H2D indexer query | index + top-k (records
-//           ev_index) | waits ev_q | CSA attention | D2H CSA output (records
-//           ev_join)
-//   stream: records ev_fork | H2D CSA query (records ev_q) | H2D HCA query |
-//           waits ev_index | HCA attention | D2H HCA output | waits ev_join
+//   side:   waits ev_fork | H2D indexer query (records ev_iq) | index + top-k
+//           (records ev_index) | waits ev_q | CSA attention | D2H CSA output
+//           (records ev_join)
+//   stream: records ev_fork | waits ev_iq | H2D CSA query (records ev_q) |
+//           H2D HCA query | waits ev_index | HCA attention | D2H HCA output |
+//           waits ev_join
 // The CSA chain is the critical path, so the side stream should have the
 // higher priority; the HCA launch waits for the indexer, which fills every SM
-// anyway.  Every copy is one cudaMemcpyAsync; the host buffers should be
-// pinned so that the copies are asynchronous.
+// anyway.  The indexer query (a few hundred bytes) crosses alone: queued
+// beside the attention queries it would share the link with them and the
+// indexer would start late; those cross while the indexer runs.  Every copy is one cudaMemcpyAsync (the
+// indexer query's three arrays take one when they lie back to back, in that
+// order and each from a 16-byte boundary, in host and in device memory
+// alike); the host buffers should be pinned so that the copies are
+// asynchronous.
 #include "common.cuh"
 
 using namespace hca;
@@ -46,7 +52,8 @@ extern "C" int hca_decode_step_host(const hca_decode_step_plan* p, const uint16_
                                     uint16_t* h_out_csa, uint16_t* h_out_hca, void* stream) {
     if (!p || !h_q_csa || !h_q_hca || !h_iq_codes || !h_iq_sf || !h_iq_w || !h_out_csa || !h_out_hca)
         return HCA_ERR_INVALID_ARG;
-    if (!p->side_stream || !p->ev_fork || !p->ev_index || !p->ev_q || !p->ev_join) return HCA_ERR_INVALID_ARG;
+    if (!p->side_stream || !p->ev_fork || !p->ev_index || !p->ev_q || !p->ev_join || !p->ev_iq)
+        return HCA_ERR_INVALID_ARG;
     if (p->B <= 0 || p->H <= 0 || p->Hi <= 0 || p->c <= 0 || p->layout.d <= 0 || p->hca_ctas < 0)
         return HCA_ERR_INVALID_ARG;
     const size_t d = static_cast<size_t>(p->layout.d);
@@ -57,14 +64,29 @@ extern "C" int hca_decode_step_host(const hca_decode_step_plan* p, const uint16_
     void* side = p->side_stream;
     HCA_TRY(rec(p->ev_fork, stream));
     HCA_TRY(wait(side, p->ev_fork));
-    // CSA chain on the side stream: the indexer query (a few hundred bytes), index + top-k
-    HCA_TRY(cpy(p->iq_codes, h_iq_codes, iqc, cudaMemcpyHostToDevice, side));
-    HCA_TRY(cpy(p->iq_sf, h_iq_sf, iqs, cudaMemcpyHostToDevice, side));
-    HCA_TRY(cpy(p->iq_w, h_iq_w, iqw, cudaMemcpyHostToDevice, side));
+    // CSA chain on the side stream: the indexer query (a few hundred bytes), then
+    // index + top-k, attention and the output
+    const uint8_t* hc = h_iq_codes;
+    const uint8_t* dc = p->iq_codes;
+    // packed: scales and weights follow the codes, each from the next 16-byte boundary
+    const size_t o_sf = (iqc + 15) & ~static_cast<size_t>(15), o_w = o_sf + ((iqs + 15) & ~static_cast<size_t>(15));
+    const bool packed = reinterpret_cast<const uint8_t*>(h_iq_sf) == hc + o_sf &&
+                        reinterpret_cast<const uint8_t*>(h_iq_w) == hc + o_w &&
+                        reinterpret_cast<const uint8_t*>(p->iq_sf) == dc + o_sf &&
+                        reinterpret_cast<const uint8_t*>(p->iq_w) == dc + o_w;
+    if (packed) {
+        HCA_TRY(cpy(p->iq_codes, h_iq_codes, o_w + iqw, cudaMemcpyHostToDevice, side));
+    } else {
+        HCA_TRY(cpy(p->iq_codes, h_iq_codes, iqc, cudaMemcpyHostToDevice, side));
+        HCA_TRY(cpy(p->iq_sf, h_iq_sf, iqs, cudaMemcpyHostToDevice, side));
+        HCA_TRY(cpy(p->iq_w, h_iq_w, iqw, cudaMemcpyHostToDevice, side));
+    }
+    HCA_TRY(rec(p->ev_iq, side));
     HCA_TRY(lightning_index_topk(p->iq_codes, p->iq_sf, p->iq_w, p->k_codes, p->k_sf, p->q_pos, p->B,
                                  p->csa_entries, p->Hi, p->c, 4, p->k, p->scores, p->idx, p->count, p->topk_ws,
                                  p->topk_ws_bytes, p->ev_index, side));
     // the attention queries cross while the indexer runs
+    HCA_TRY(wait(stream, p->ev_iq));
     HCA_TRY(cpy(p->q_csa, h_q_csa, q_bytes, cudaMemcpyHostToDevice, stream));
     HCA_TRY(rec(p->ev_q, stream));
     HCA_TRY(cpy(p->q_hca, h_q_hca, q_bytes, cudaMemcpyHostToDevice, stream));

@@ -65,6 +65,26 @@ class DecodeLayer:
     k_sf: Optional[torch.Tensor] = None      # CSA: [B][Nc][c/32]
 
 
+def packed_indexer_query(iq, device=None, pin: bool = False):
+    """A copy of one layer's indexer query (codes, scales, weights) in one
+    byte buffer, in that order, each part from a 16-byte boundary: views of
+    the same shapes and dtypes.  hca_decode_step_host moves such a query with
+    one copy when its host and device buffers are both packed so."""
+    parts = tuple(iq)
+    sizes = [t.numel() * t.element_size() for t in parts]
+    offs = [0]
+    for n in sizes[:-1]:
+        offs.append(offs[-1] + (n + 15) // 16 * 16)
+    dev = torch.device(device) if device is not None else parts[0].device
+    buf = torch.zeros(offs[-1] + sizes[-1], dtype=torch.uint8, device=dev, pin_memory=pin and dev.type == "cpu")
+    out = []
+    for t, n, off in zip(parts, sizes, offs):
+        v = buf[off:off + n].view(t.dtype).view(t.shape)
+        v.copy_(t)
+        out.append(v)
+    return tuple(out)
+
+
 class DecodeRunner:
     """Queues one decode step over a list of layers.  Per layer: CSA ->
     lightning_index, topk_select, compressed_attn_decode(sparse); HCA ->
@@ -168,7 +188,7 @@ class DecodeRunner:
         """The hca_decode_step_plan of this runner's two layers (one CSA, one
         HCA), for hca_decode_step_host: the caches, keys and windows of the
         layers, d_q / d_iq as the staging buffers of the queries, this runner's
-        scores, top-k and attention buffers, a side stream and four events."""
+        scores, top-k and attention buffers, a side stream and five events."""
         from . import CacheStruct, DecodeStepPlan, Layout
         ci = [li for li, L in enumerate(self.layers) if L.ratio == CSA_RATIO]
         hi = [li for li, L in enumerate(self.layers) if L.ratio == HCA_RATIO]
@@ -179,7 +199,7 @@ class DecodeRunner:
         qc, qs, w = d_iq[c_]
         lo, hi_prio = torch.cuda.Stream.priority_range()
         self._capi_side = torch.cuda.Stream(device=d_q[0].device, priority=hi_prio)   # the CSA chain
-        self._capi_events = [torch.cuda.Event() for _ in range(4)]
+        self._capi_events = [torch.cuda.Event() for _ in range(5)]
         for e in self._capi_events:
             e.record(torch.cuda.current_stream())     # creates the CUDA event (outside any capture)
         torch.cuda.synchronize()
@@ -202,7 +222,7 @@ class DecodeRunner:
         p.ws_hca, p.ws_hca_bytes = ptr(self.ws[h_]), self.ws[h_].numel()
         p.out_csa, p.out_hca = ptr(self.out[c_]), ptr(self.out[h_])
         p.side_stream = self._capi_side.cuda_stream
-        p.ev_fork, p.ev_index, p.ev_q, p.ev_join = (e.cuda_event for e in self._capi_events)
+        p.ev_fork, p.ev_index, p.ev_q, p.ev_join, p.ev_iq = (e.cuda_event for e in self._capi_events)
         p.hca_ctas = self.dense_budget
         self._capi_layers = (c_, h_)
         return p

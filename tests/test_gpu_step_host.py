@@ -1,6 +1,7 @@
 """hca_decode_step_host, the C ABI's host-to-host decode step (one CSA and
 one HCA layer: query copies in, index + top-k, both attention calls, output
-copies out), called through ctypes with pinned host buffers: its outputs are
+copies out), called through ctypes with pinned host buffers (the indexer
+query as three arrays, or packed back to back for one copy): its outputs are
 those of the device-resident step bit for bit, and the oracle's within the
 attention tolerance, on tiny_decode_1k and decode_b16_64k; the step also
 runs captured in a CUDA graph."""
@@ -16,21 +17,28 @@ pytestmark = pytest.mark.gpu
 
 hca = pytest.importorskip("long_context_attention_hca_b200")
 from hca_workloads import build_decode  # noqa: E402
-from long_context_attention_hca_b200.pipeline import DecodeRunner  # noqa: E402
+from long_context_attention_hca_b200.pipeline import DecodeRunner, packed_indexer_query  # noqa: E402
 
 
-@pytest.mark.parametrize("name", ["tiny_decode_1k", "decode_b16_64k"])
-def test_step_host_capi(name):
+@pytest.mark.parametrize("name,packed", [("tiny_decode_1k", False), ("decode_b16_64k", False),
+                                         ("tiny_decode_1k", True)])
+def test_step_host_capi(name, packed):
     wl = inp.WORKLOADS[name]
     dw = build_decode(wl)
     runner = DecodeRunner(dw.layers, wl.B, wl.H, wl.k, wl.t, wl.softmax_scale)
     ref = [o.clone() for o in runner.step(dw.q, dw.iq)]
     torch.cuda.synchronize()
     h_q = [t.to("cpu").pin_memory() for t in dw.q]
-    h_iq = [None if t is None else tuple(x.to("cpu").pin_memory() for x in t) for t in dw.iq]
+    if packed:      # the indexer query's three arrays back to back: one copy
+        h_iq = [None if t is None else packed_indexer_query(t, device="cpu", pin=True) for t in dw.iq]
+    else:
+        h_iq = [None if t is None else tuple(x.to("cpu").pin_memory() for x in t) for t in dw.iq]
     h_out = [torch.zeros_like(o, device="cpu").pin_memory() for o in runner.out]
     d_q = [torch.zeros_like(t) for t in dw.q]
-    d_iq = [None if t is None else tuple(torch.zeros_like(x) for x in t) for t in dw.iq]
+    if packed:
+        d_iq = [None if t is None else tuple(x.zero_() for x in packed_indexer_query(t)) for t in dw.iq]
+    else:
+        d_iq = [None if t is None else tuple(torch.zeros_like(x) for x in t) for t in dw.iq]
     for o in runner.out:
         o.zero_()
     plan = runner.capi_plan(d_q, d_iq)
