@@ -354,9 +354,8 @@ def bench_decode(args, wl, world, rank, pg):
     reps = []
     for r in range(n_rep):
         dw = build_decode(wl)
-        runner = DecodeRunner(dw.layers, wl.B, wl.H, wl.k, wl.t, wl.softmax_scale, schedule=args.schedule,
-                              dense_budget=args.dense_budget, sparse_budget=args.sparse_budget,
-                              index_budget=args.index_budget)
+        runner = DecodeRunner(dw.layers, wl.B, wl.H, wl.k, wl.t, wl.softmax_scale, dense_budget=args.dense_budget,
+                              sparse_budget=args.sparse_budget, index_budget=args.index_budget)
         reps.append((dw, runner))
     main = torch.cuda.current_stream()
 
@@ -995,8 +994,6 @@ def main():
                     choices=["decode_b4_1m", "decode_b16_64k", "prefill_4096_131k", "stack61_b32_256k"])
     ap.add_argument("--replicas", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--schedule", default="after_index", choices=["after_index", "hca_first"],
-                    help="decode step: HCA after the indexer, or HCA first on a CTA budget")
     ap.add_argument("--dense-budget", type=int, default=None,
                     help="CTA cap of the step's dense (HCA) attention (default: half the SMs beside the CSA chain; "
                          "0: the library default, every SM)")

@@ -412,13 +412,11 @@ int compressed_attn_decode_noalloc(const uint16_t* q, int32_t B, int32_t H,
  *           window of position p is tokens max(0, p-W+1) .. p
  *   out     bf16 [Tq][H][d]
  * Same attention rule (and softmax_scale rule) as decode. */
-size_t compressed_attn_prefill_workspace_size(int32_t Tq, int32_t H, hca_kv_layout layout);
 int compressed_attn_prefill(const uint16_t* q, int32_t Tq, int32_t H, int32_t p0, int32_t m,
                             hca_kv_layout layout, hca_kv_cache kv,
                             const int32_t* idx, int32_t idx_stride, const int32_t* count,
                             const uint16_t* raw, int32_t W,
-                            float softmax_scale, uint16_t* out,
-                            void* ws, size_t ws_bytes, void* stream);
+                            float softmax_scale, uint16_t* out, void* stream);
 
 /* ------------------------------------------------------------------ */
 /* Core attention with the section 9 extras.                            */
@@ -464,7 +462,7 @@ int compressed_attn_prefill_ex(const uint16_t* q, int32_t Tq, int32_t H, int32_t
                                const int32_t* idx, int32_t idx_stride, const int32_t* count,
                                const uint16_t* raw, int32_t W,
                                float softmax_scale, const hca_attn_extras* ex, uint16_t* out,
-                               void* ws, size_t ws_bytes, void* stream);
+                               void* stream);
 
 /* ------------------------------------------------------------------ */
 /* State cache of the decode loop (section 11: a fixed-size state per     */

@@ -33,7 +33,7 @@ EXPORTED = (
     "hca_status_string", "hca_last_cuda_error", "csa_compress", "hca_compress", "lightning_index",
     "topk_select_workspace_size", "topk_select", "lightning_index_topk_workspace_size", "lightning_index_topk",
     "compressed_attn_decode_workspace_size",
-    "compressed_attn_decode", "compressed_attn_prefill_workspace_size", "compressed_attn_prefill",
+    "compressed_attn_decode", "compressed_attn_prefill",
     "csa_compress_ex", "hca_compress_ex", "kv_token_prep", "compressed_attn_decode_ex", "compressed_attn_prefill_ex",
     "kv_state_append", "csa_compress_overlap", "indexer_key_compress",
     "lightning_index_ex", "topk_select_ex_workspace_size", "topk_select_ex",
@@ -139,10 +139,8 @@ _lib.compressed_attn_decode_workspace_size.restype = _SZ
 _lib.compressed_attn_decode.argtypes = [_V, _I32, _I32, Layout, CacheStruct, _V, _I32, _V, _I32, _V, _I32, _F,
                                         _V, _V, _V, _SZ, _V]
 _lib.compressed_attn_decode.restype = ctypes.c_int
-_lib.compressed_attn_prefill_workspace_size.argtypes = [_I32, _I32, Layout]
-_lib.compressed_attn_prefill_workspace_size.restype = _SZ
 _lib.compressed_attn_prefill.argtypes = [_V, _I32, _I32, _I32, _I32, Layout, CacheStruct, _V, _I32, _V, _V, _I32,
-                                         _F, _V, _V, _SZ, _V]
+                                         _F, _V, _V]
 _lib.compressed_attn_prefill.restype = ctypes.c_int
 
 
@@ -156,7 +154,7 @@ _lib.compressed_attn_decode_ex.argtypes = [_V, _I32, _I32, Layout, CacheStruct, 
                                            ctypes.POINTER(AttnExtrasStruct), _V, _V, _V, _SZ, _V]
 _lib.compressed_attn_decode_ex.restype = ctypes.c_int
 _lib.compressed_attn_prefill_ex.argtypes = [_V, _I32, _I32, _I32, _I32, Layout, CacheStruct, _V, _I32, _V, _V, _I32,
-                                            _F, ctypes.POINTER(AttnExtrasStruct), _V, _V, _SZ, _V]
+                                            _F, ctypes.POINTER(AttnExtrasStruct), _V, _V]
 _lib.compressed_attn_prefill_ex.restype = ctypes.c_int
 
 
@@ -457,13 +455,13 @@ def compressed_attn_prefill(q, p0, m, cache: KVCache, raw, W, softmax_scale, idx
         stride = idx.shape[-1]
     if extras is None:
         _check(_lib.compressed_attn_prefill(_p(q), Tq, H, p0, m, cache.c_layout, cache.c_struct, _p(idx), stride,
-                                            _p(count), _p(raw), W, float(softmax_scale), _p(out), None, 0,
+                                            _p(count), _p(raw), W, float(softmax_scale), _p(out),
                                             _stream(stream)), "compressed_attn_prefill")
     else:
         ex = extras.c_struct()
         _check(_lib.compressed_attn_prefill_ex(_p(q), Tq, H, p0, m, cache.c_layout, cache.c_struct, _p(idx), stride,
                                                _p(count), _p(raw), W, float(softmax_scale), ctypes.byref(ex), _p(out),
-                                               None, 0, _stream(stream)), "compressed_attn_prefill_ex")
+                                               _stream(stream)), "compressed_attn_prefill_ex")
     return out
 
 

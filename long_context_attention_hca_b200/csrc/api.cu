@@ -414,16 +414,10 @@ int indexer_key_compress(const uint16_t* xa, const uint16_t* za, const uint16_t*
                           nullptr, nullptr, k_sf, capacity, entry_begin, true, as_stream(stream));
 }
 
-size_t compressed_attn_prefill_workspace_size(int32_t Tq, int32_t H, hca_kv_layout layout) {
-    (void)Tq; (void)H; (void)layout;
-    return 0;
-}
-
 int compressed_attn_prefill_ex(const uint16_t* q, int32_t Tq, int32_t H, int32_t p0, int32_t m,
                                hca_kv_layout layout, hca_kv_cache kv, const int32_t* idx, int32_t idx_stride,
                                const int32_t* count, const uint16_t* raw, int32_t W, float softmax_scale,
-                               const hca_attn_extras* ex, uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
-    (void)ws; (void)ws_bytes;
+                               const hca_attn_extras* ex, uint16_t* out, void* stream) {
     REQUIRE(Tq >= 0 && p0 >= 0 && W >= 1);
     if (!layout_ok(layout)) return HCA_ERR_UNSUPPORTED;
     if (!((layout.d == 512 && H == 64) || (layout.d == 128 && (H == 64 || (H >= 1 && H <= 16)))))
@@ -442,9 +436,9 @@ int compressed_attn_prefill_ex(const uint16_t* q, int32_t Tq, int32_t H, int32_t
 int compressed_attn_prefill(const uint16_t* q, int32_t Tq, int32_t H, int32_t p0, int32_t m,
                             hca_kv_layout layout, hca_kv_cache kv, const int32_t* idx, int32_t idx_stride,
                             const int32_t* count, const uint16_t* raw, int32_t W, float softmax_scale,
-                            uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+                            uint16_t* out, void* stream) {
     return compressed_attn_prefill_ex(q, Tq, H, p0, m, layout, kv, idx, idx_stride, count, raw, W, softmax_scale,
-                                      nullptr, out, ws, ws_bytes, stream);
+                                      nullptr, out, stream);
 }
 
 }  // extern "C"

@@ -94,12 +94,12 @@ class DecodeRunner:
     indexer fills every SM anyway."""
 
     def __init__(self, layers: List[DecodeLayer], B: int, H: int, k: int, pos: int, softmax_scale: float,
-                 device="cuda", schedule: str = "after_index", dense_budget: Optional[int] = None,
+                 device="cuda", dense_budget: Optional[int] = None,
                  fused_select: bool = True, sparse_budget: int = 0, extras: Optional[list] = None,
                  index_budget: int = 0):
-        """schedule: "after_index" -- an HCA launch waits for the indexer queued
-        before it; "hca_first" -- all HCA launches are queued first and start at
-        once.  dense_budget caps the CTAs of this runner's HCA launches (applied
+        """An HCA launch waits for the indexer queued before it (queued first, the
+        HCA launches measured no faster).  dense_budget caps the CTAs of this
+        runner's HCA launches (applied
         around its own calls only): None -- half the SMs when the step is one
         CSA layer beside one HCA layer (the select and the CSA attention keep
         the other half), else the library default (in a deep stack both streams
@@ -109,9 +109,6 @@ class DecodeRunner:
         an AttnExtras (section 9 query RMSNorm, RoPE, sink) for its attention
         call, or None."""
         self.extras = extras if extras is not None else [None] * len(layers)
-        if schedule not in ("after_index", "hca_first"):
-            raise ValueError(schedule)
-        self.schedule = schedule
         dev = torch.device(device)
         if dense_budget is None:
             pair = len(layers) == 2 and sorted(L.ratio == CSA_RATIO for L in layers) == [False, True]
@@ -293,11 +290,7 @@ class DecodeRunner:
             events[key] = (a, b)
 
         after_index = None
-        order = list(range(len(self.layers)))
-        if self.schedule == "hca_first":
-            order = [li for li in order if self.layers[li].ratio != CSA_RATIO] + \
-                    [li for li in order if self.layers[li].ratio == CSA_RATIO]
-        for li in order:
+        for li in range(len(self.layers)):
             L = self.layers[li]
             if L.ratio == CSA_RATIO:
                 with torch.cuda.stream(self.side):
@@ -325,7 +318,7 @@ class DecodeRunner:
                     if on_out is not None:
                         on_out(li, self.side)
             else:
-                if after_index is not None and self.schedule == "after_index":
+                if after_index is not None:
                     main.wait_event(after_index)
                 if q_ready is not None:
                     main.wait_event(q_ready[li])

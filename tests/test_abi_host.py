@@ -169,10 +169,10 @@ def test_extension_calls_validate_on_the_host(lib):
     assert lib.compressed_attn_decode_ex(P, 1, 64, good, cache, None, 0, P, 10, P, 128, 0.1, ctypes.byref(no_pos),
                                          P, None, None, 0, None) == 1
     lib.compressed_attn_prefill_ex.argtypes = [V, I32, I32, I32, I32, Layout, Cache, V, I32, V, V, I32, F,
-                                               ctypes.POINTER(AttnEx), V, V, SZ, V]
+                                               ctypes.POINTER(AttnEx), V, V]
     win_pf = AttnEx(None, 1e-6, None, None, None, 0x1000)                # window lengths are a decode input
     assert lib.compressed_attn_prefill_ex(P, 4, 64, 100, 4, good, cache, None, 0, None, P, 128, 0.1,
-                                          ctypes.byref(win_pf), P, None, 0, None) == 1
+                                          ctypes.byref(win_pf), P, None) == 1
     lib.csa_compress_overlap.argtypes = [V, V, V, V, V, V, I64, V, I32, I64, Layout, Cache, I64, V]
     assert lib.csa_compress_overlap(P, P, P, P, P, None, 8, P, 1, 2, good, cache, 1, None) == 1    # a_prev alone
     assert lib.csa_compress_overlap(P, P, P, P, None, None, 7, P, 1, 2, good, cache, 0, None) == 1  # 8 rows needed
