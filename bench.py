@@ -421,7 +421,9 @@ def bench_decode(args, wl, world, rank, pg):
     h_q = [t.to("cpu").pin_memory() for t in dw.q]
     # each layer's indexer query packed in one buffer, host and device: one copy
     h_iq = [None if t is None else packed_indexer_query(t, device="cpu", pin=True) for t in dw.iq]
-    h_out = [torch.empty_like(o, device="cpu").pin_memory() for o in runner.out]
+    # the outputs back to back in pinned memory, as the runner's device outputs are: one copy
+    h_out = list(torch.empty((len(runner.out),) + tuple(runner.out[0].shape), dtype=runner.out[0].dtype,
+                             pin_memory=True).unbind(0))
     d_q = [t.clone() for t in dw.q]
     d_iq = [None if t is None else packed_indexer_query(t) for t in dw.iq]
     h2d = sum(t.numel() * t.element_size() for t in h_q) + sum(
@@ -485,7 +487,7 @@ def bench_decode(args, wl, world, rank, pg):
 
     # the same step through the C ABI's host-to-host call (hca_decode_step_host:
     # the library issues the copies and the kernels on two streams), as one graph
-    plan = runner.capi_plan(d_q, d_iq)
+    plan = runner.capi_plan(d_q, d_iq, packed=3)
 
     def e2e_step_capi():
         runner.step_host_capi(plan, h_q, h_iq, h_out)

@@ -525,6 +525,12 @@ typedef struct {
     int32_t hca_ctas;             /* CTAs of the HCA attention (its split-K plan); 0: half */
                                   /* the SMs, the rest left to the concurrent CSA chain    */
     void* ev_iq;                  /* marks the indexer query's copy                        */
+    int32_t packed;               /* bit 0: the indexer query's codes, scales and weights */
+                                  /* lie in one allocation each (host and device), in that */
+                                  /* order, each from the next 16-byte boundary: one copy; */
+                                  /* bit 1: out_csa and out_hca lie back to back in one    */
+                                  /* allocation, h_out_csa and h_out_hca likewise, in the  */
+                                  /* same order: one copy of both after the join           */
 } hca_decode_step_plan;
 
 /* Host queries in, host outputs out:
@@ -532,17 +538,18 @@ typedef struct {
  *   [B][Hi][c/32], h_iq_w fp32 [B][Hi]; h_out_csa, h_out_hca bf16 [B][H][d]
  *   (host memory; pinned for asynchronous copies).
  * Queues on the plan's side stream (give it the higher priority: it carries
- * the critical path): the indexer-query copy (one copy when codes, scales and
- * weights lie back to back in that order, each from a 16-byte boundary, in
- * host and in device memory alike; else three), lightning_index_topk, the CSA
- * attention (after the CSA-query copy) and its output copy.  On `stream`,
- * once the indexer query has crossed (ev_iq), so that the small copy the
- * indexer waits for does not share the link with the large ones: the
- * attention-query copies and, once the indexer has run, the HCA attention and
- * its output copy.  `stream` finally waits for the side stream, so both
- * outputs are in host memory when `stream` reaches that point.  The five
- * events of the plan are the caller's (created without timing); nothing is
- * allocated; errors as the calls it makes. */
+ * the critical path): the indexer-query copy (one copy with plan->packed
+ * bit 0, else three), lightning_index_topk, the CSA attention (after the
+ * CSA-query copy) and its output copy.  On `stream`, once the indexer query
+ * has crossed (ev_iq), so that the small copy the indexer waits for does not
+ * share the link with the large ones: the attention-query copies and, once
+ * the indexer has run, the HCA attention and its output copy (with
+ * plan->packed bit 1, one copy of both outputs on `stream` after the join
+ * instead).  `stream` finally waits for the side stream, so both outputs are
+ * in host memory when `stream` reaches that point.  The five events of the
+ * plan are the caller's (created without timing); nothing is allocated.
+ * Errors as the calls it makes; HCA_ERR_INVALID_ARG also when a bit of
+ * plan->packed is set but the pointers do not lie as it states. */
 int hca_decode_step_host(const hca_decode_step_plan* plan, const uint16_t* h_q_csa, const uint16_t* h_q_hca,
                          const uint8_t* h_iq_codes, const uint8_t* h_iq_sf, const float* h_iq_w,
                          uint16_t* h_out_csa, uint16_t* h_out_hca, void* stream);

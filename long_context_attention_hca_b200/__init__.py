@@ -193,7 +193,7 @@ class DecodeStepPlan(ctypes.Structure):
                 ("ws_hca_bytes", ctypes.c_size_t), ("out_csa", ctypes.c_void_p), ("out_hca", ctypes.c_void_p),
                 ("side_stream", ctypes.c_void_p), ("ev_fork", ctypes.c_void_p), ("ev_index", ctypes.c_void_p),
                 ("ev_q", ctypes.c_void_p), ("ev_join", ctypes.c_void_p), ("hca_ctas", ctypes.c_int32),
-                ("ev_iq", ctypes.c_void_p)]
+                ("ev_iq", ctypes.c_void_p), ("packed", ctypes.c_int32)]
 
 
 _lib.hca_decode_step_host.argtypes = [ctypes.POINTER(DecodeStepPlan), _V, _V, _V, _V, _V, _V, _V, _V]

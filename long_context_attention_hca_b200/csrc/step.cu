@@ -17,10 +17,13 @@
 // higher priority; the HCA launch waits for the indexer, which fills every SM
 // anyway.  The indexer query (a few hundred bytes) crosses alone: queued
 // beside the attention queries it would share the link with them and the
-// indexer would start late; those cross while the indexer runs.  Every copy is one cudaMemcpyAsync (the
-// indexer query's three arrays take one when they lie back to back, in that
-// order and each from a 16-byte boundary, in host and in device memory
-// alike); the host buffers should be pinned so that the copies are
+// indexer would start late; those cross while the indexer runs.  Every copy
+// is one cudaMemcpyAsync.  When the caller states it (plan->packed), the
+// indexer query's three arrays take one copy, and the two outputs take one,
+// on `stream` after the join (one copy of 512 KB costs about 12.7 us on a
+// PCIe link, two of 256 KB about 8 us each).  Adjacent pointers alone do not
+// prove one allocation, and a copy across two pinned allocations is refused,
+// hence the flag.  The host buffers should be pinned so that the copies are
 // asynchronous.
 #include "common.cuh"
 
@@ -61,20 +64,38 @@ extern "C" int hca_decode_step_host(const hca_decode_step_plan* p, const uint16_
     const size_t iqc = static_cast<size_t>(p->B) * p->Hi * (p->c / 2);
     const size_t iqs = static_cast<size_t>(p->B) * p->Hi * (p->c / 32);
     const size_t iqw = static_cast<size_t>(p->B) * p->Hi * sizeof(float);
+    if (p->packed & ~3) return HCA_ERR_INVALID_ARG;
+    // packed indexer query: scales and weights follow the codes, each from the next
+    // 16-byte boundary, in host and in device memory
+    const uint8_t* hc = h_iq_codes;
+    const uint8_t* dc = p->iq_codes;
+    const size_t o_sf = (iqc + 15) & ~static_cast<size_t>(15), o_w = o_sf + ((iqs + 15) & ~static_cast<size_t>(15));
+    const bool iq_packed = (p->packed & 1) != 0;
+    if (iq_packed && !(reinterpret_cast<const uint8_t*>(h_iq_sf) == hc + o_sf &&
+                       reinterpret_cast<const uint8_t*>(h_iq_w) == hc + o_w &&
+                       reinterpret_cast<const uint8_t*>(p->iq_sf) == dc + o_sf &&
+                       reinterpret_cast<const uint8_t*>(p->iq_w) == dc + o_w))
+        return HCA_ERR_INVALID_ARG;
+    // packed outputs: both back to back (either order) in device and in host memory
+    // alike, one copy of both once the two paths have joined
+    const size_t n_out = q_bytes / 2;
+    const uint16_t* d_first = nullptr;
+    uint16_t* h_first = nullptr;
+    if (p->packed & 2) {
+        if (p->out_hca == p->out_csa + n_out && h_out_hca == h_out_csa + n_out) {
+            d_first = p->out_csa; h_first = h_out_csa;
+        } else if (p->out_csa == p->out_hca + n_out && h_out_csa == h_out_hca + n_out) {
+            d_first = p->out_hca; h_first = h_out_hca;
+        } else {
+            return HCA_ERR_INVALID_ARG;
+        }
+    }
     void* side = p->side_stream;
     HCA_TRY(rec(p->ev_fork, stream));
     HCA_TRY(wait(side, p->ev_fork));
     // CSA chain on the side stream: the indexer query (a few hundred bytes), then
     // index + top-k, attention and the output
-    const uint8_t* hc = h_iq_codes;
-    const uint8_t* dc = p->iq_codes;
-    // packed: scales and weights follow the codes, each from the next 16-byte boundary
-    const size_t o_sf = (iqc + 15) & ~static_cast<size_t>(15), o_w = o_sf + ((iqs + 15) & ~static_cast<size_t>(15));
-    const bool packed = reinterpret_cast<const uint8_t*>(h_iq_sf) == hc + o_sf &&
-                        reinterpret_cast<const uint8_t*>(h_iq_w) == hc + o_w &&
-                        reinterpret_cast<const uint8_t*>(p->iq_sf) == dc + o_sf &&
-                        reinterpret_cast<const uint8_t*>(p->iq_w) == dc + o_w;
-    if (packed) {
+    if (iq_packed) {
         HCA_TRY(cpy(p->iq_codes, h_iq_codes, o_w + iqw, cudaMemcpyHostToDevice, side));
     } else {
         HCA_TRY(cpy(p->iq_codes, h_iq_codes, iqc, cudaMemcpyHostToDevice, side));
@@ -96,7 +117,7 @@ extern "C" int hca_decode_step_host(const hca_decode_step_plan* p, const uint16_
     HCA_TRY(compressed_attn_decode(p->q_csa, p->B, p->H, p->layout, p->csa_cache, p->idx, p->k, p->count, kmax,
                                    p->csa_window, p->W, p->softmax_scale, p->out_csa, nullptr, p->ws_csa,
                                    p->ws_csa_bytes, side));
-    HCA_TRY(cpy(h_out_csa, p->out_csa, q_bytes, cudaMemcpyDeviceToHost, side));
+    if (!d_first) HCA_TRY(cpy(h_out_csa, p->out_csa, q_bytes, cudaMemcpyDeviceToHost, side));
     HCA_TRY(rec(p->ev_join, side));
     // HCA: dense attention once the indexer has run, on at most hca_ctas CTAs (by
     // default half the SMs) so that the CSA chain's select and attention keep
@@ -108,7 +129,8 @@ extern "C" int hca_decode_step_host(const hca_decode_step_plan* p, const uint16_
                                           p->ws_hca, p->ws_hca_bytes, stream);
     thread_budget_swap(HCA_BUDGET_DENSE_DECODE, prev);
     HCA_TRY(rc);
-    HCA_TRY(cpy(h_out_hca, p->out_hca, q_bytes, cudaMemcpyDeviceToHost, stream));
+    if (!d_first) HCA_TRY(cpy(h_out_hca, p->out_hca, q_bytes, cudaMemcpyDeviceToHost, stream));
     HCA_TRY(wait(stream, p->ev_join));
+    if (d_first) HCA_TRY(cpy(h_first, d_first, 2 * q_bytes, cudaMemcpyDeviceToHost, stream));
     return HCA_OK;
 }

@@ -123,7 +123,8 @@ class DecodeRunner:
         d = layers[0].cache.layout[0]
         self.d = d
         self.q_pos = torch.full((B, 1), pos, dtype=torch.int32, device=dev)
-        self.out = [torch.empty((B, H, d), dtype=torch.bfloat16, device=dev) for _ in layers]
+        # the layers' outputs back to back (hca_decode_step_host then copies both at once)
+        self.out = list(torch.empty((len(layers), B, H, d), dtype=torch.bfloat16, device=dev).unbind(0))
         self.n_dense = {}
         self.scores, self.idx, self.count, self.ws, self.topk_ws, self.fused_select = {}, {}, {}, {}, {}, {}
         self.index_done = {}
@@ -181,11 +182,14 @@ class DecodeRunner:
                 n += 1 + ((1 if self.fused_select[li] else 2) if wide else 1)
         return n
 
-    def capi_plan(self, d_q: List[torch.Tensor], d_iq: List[Optional[tuple]]):
+    def capi_plan(self, d_q: List[torch.Tensor], d_iq: List[Optional[tuple]], packed: int = 0):
         """The hca_decode_step_plan of this runner's two layers (one CSA, one
         HCA), for hca_decode_step_host: the caches, keys and windows of the
         layers, d_q / d_iq as the staging buffers of the queries, this runner's
-        scores, top-k and attention buffers, a side stream and five events."""
+        scores, top-k and attention buffers, a side stream and five events.
+        packed: the plan's packing bits (1: the indexer query's arrays, host
+        and device, as packed_indexer_query lays them out; 2: the host outputs
+        back to back in one allocation, as this runner's device outputs are)."""
         from . import CacheStruct, DecodeStepPlan, Layout
         ci = [li for li, L in enumerate(self.layers) if L.ratio == CSA_RATIO]
         hi = [li for li, L in enumerate(self.layers) if L.ratio == HCA_RATIO]
@@ -221,6 +225,7 @@ class DecodeRunner:
         p.side_stream = self._capi_side.cuda_stream
         p.ev_fork, p.ev_index, p.ev_q, p.ev_join, p.ev_iq = (e.cuda_event for e in self._capi_events)
         p.hca_ctas = self.dense_budget
+        p.packed = packed
         self._capi_layers = (c_, h_)
         return p
 

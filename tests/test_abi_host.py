@@ -194,3 +194,24 @@ def test_extension_calls_validate_on_the_host(lib):
     assert lib.kv_state_append(P, P, None, 2, 128, -1, P, 128, P, P, 4, None) == 1           # negative position
     lib.hca_decode_step_host.argtypes = [V, V, V, V, V, V, V, V, V]
     assert lib.hca_decode_step_host(None, P, P, P, P, P, P, P, None) == 1
+
+
+def test_step_host_packing_bits_checked_before_any_queue(lib):
+    """hca_decode_step_host takes one copy for packed buffers only when the plan
+    says so, and then checks the layout it states: a packing bit whose pointers
+    do not lie that way (or an unknown bit) is refused before anything is
+    queued, so this runs without a device."""
+    from long_context_attention_hca_b200 import DecodeStepPlan, Layout
+    V = ctypes.c_void_p
+    lib.hca_decode_step_host.argtypes = [ctypes.POINTER(DecodeStepPlan), V, V, V, V, V, V, V, V]
+    p = DecodeStepPlan()
+    p.B, p.H, p.Hi, p.c, p.k, p.W = 4, 64, 4, 128, 1024, 128
+    p.layout = Layout(512, 64, 64)
+    p.side_stream = p.ev_fork = p.ev_index = p.ev_q = p.ev_join = p.ev_iq = 0x1000
+    p.iq_codes, p.iq_sf, p.iq_w = 0x100000, 0x100400, 0x100440           # packed on the device
+    p.out_csa, p.out_hca = 0x200000, 0x240000                             # packed on the device
+    hq, hc, hs, hw = 0x300000, 0x400000, 0x500000, 0x600000               # host arrays apart
+    ho_c, ho_h = 0x700000, 0x800000
+    for bits in (1, 2, 4):
+        p.packed = bits
+        assert lib.hca_decode_step_host(ctypes.byref(p), hq, hq, hc, hs, hw, ho_c, ho_h, None) == 1, bits

@@ -1,7 +1,8 @@
 """hca_decode_step_host, the C ABI's host-to-host decode step (one CSA and
 one HCA layer: query copies in, index + top-k, both attention calls, output
 copies out), called through ctypes with pinned host buffers (the indexer
-query as three arrays, or packed back to back for one copy): its outputs are
+query as three arrays and the outputs apart, or each packed back to back
+for one copy): its outputs are
 those of the device-resident step bit for bit, and the oracle's within the
 attention tolerance, on tiny_decode_1k and decode_b16_64k; the step also
 runs captured in a CUDA graph."""
@@ -33,7 +34,11 @@ def test_step_host_capi(name, packed):
         h_iq = [None if t is None else packed_indexer_query(t, device="cpu", pin=True) for t in dw.iq]
     else:
         h_iq = [None if t is None else tuple(x.to("cpu").pin_memory() for x in t) for t in dw.iq]
-    h_out = [torch.zeros_like(o, device="cpu").pin_memory() for o in runner.out]
+    if packed:      # and both outputs back to back: one copy
+        h_out = list(torch.zeros((len(runner.out),) + tuple(runner.out[0].shape), dtype=runner.out[0].dtype,
+                                 pin_memory=True).unbind(0))
+    else:
+        h_out = [torch.zeros_like(o, device="cpu").pin_memory() for o in runner.out]
     d_q = [torch.zeros_like(t) for t in dw.q]
     if packed:
         d_iq = [None if t is None else tuple(x.zero_() for x in packed_indexer_query(t)) for t in dw.iq]
@@ -41,7 +46,7 @@ def test_step_host_capi(name, packed):
         d_iq = [None if t is None else tuple(torch.zeros_like(x) for x in t) for t in dw.iq]
     for o in runner.out:
         o.zero_()
-    plan = runner.capi_plan(d_q, d_iq)
+    plan = runner.capi_plan(d_q, d_iq, packed=3 if packed else 0)
     runner.step_host_capi(plan, h_q, h_iq, h_out)
     torch.cuda.synchronize()
     for a, b in zip(h_out, ref):
