@@ -468,7 +468,7 @@ __device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t* sh_war
 // the digit, s_out[1] = need minus the count strictly above it, s_out[2] =
 // the count in it.  (An inconsistent histogram, whose total is below need,
 // leaves digit 0, need and 0: wrong but in bounds.)
-__device__ void find_digit(const uint32_t* h, uint32_t nb, uint32_t need, uint32_t* sh_warp, uint32_t* s_out) {
+__device__ __forceinline__ void find_digit(const uint32_t* h, uint32_t nb, uint32_t need, uint32_t* sh_warp, uint32_t* s_out) {
     const int t = threadIdx.x;
     if (t == 0) { s_out[0] = 0u; s_out[1] = need; s_out[2] = 0u; }
     const uint32_t per = nb / kSelThreads;
@@ -532,7 +532,7 @@ __device__ __forceinline__ void flush(const V* stage, uint32_t n, uint32_t* coun
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kSelThreads)
+__global__ void __launch_bounds__(kSelThreads, 1)
 select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, int64_t Nc_cap, int m, int k,
               int64_t chunk, uint8_t* __restrict__ ws, int32_t* __restrict__ idx, int32_t* __restrict__ count) {
     extern __shared__ __align__(16) unsigned long long dyn[];
@@ -559,6 +559,19 @@ select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, i
         return;
     }
     RowWs w = row_ws(ws, Nc_cap, r);
+    const T* row = scores + static_cast<size_t>(r) * Nc_cap;
+    const int64_t e0 = static_cast<int64_t>(blockIdx.x) * chunk;
+    const int64_t e1 = min(e0 + chunk, n);
+    const int n_it = e1 > e0 ? static_cast<int>((e1 - e0 + kSelThreads - 1) / kSelThreads) : 0;
+    constexpr int kBatch = 32;                             // loads in flight per thread
+    // the chunk's first batch of scores does not depend on the threshold: its loads
+    // fly while the histogram is read and searched
+    float v[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+        const int64_t e = e0 + static_cast<int64_t>(j) * kSelThreads + warp * 32 + lane;
+        v[j] = (j < n_it && e < e1) ? score_at(row, e) : 0.0f;
+    }
     // ---- threshold bin T1 from the row's histogram (the same in every CTA)
     {
         uint32_t hv[kBins / kSelThreads];                  // all loads in flight, then the stores
@@ -570,23 +583,19 @@ select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, i
     __syncthreads();
     find_digit(s_hist, kBins, kk, sh_warp, s_dig);
     const uint32_t t1 = s_dig[0];
-    const T* row = scores + static_cast<size_t>(r) * Nc_cap;
     // ---- one pass over this CTA's chunk: the above keys' indices and the
     // candidates' composite keys, staged per warp, appended to the row's lists
     {
         uint32_t* s_wa = s_bits + warp * kWBuf;
         unsigned long long* s_wc = reinterpret_cast<unsigned long long*>(s_bits + kSelWarps * kWBuf) + warp * kWBuf;
-        const int64_t e0 = static_cast<int64_t>(blockIdx.x) * chunk;
-        const int64_t e1 = min(e0 + chunk, n);
-        const int n_it = e1 > e0 ? static_cast<int>((e1 - e0 + kSelThreads - 1) / kSelThreads) : 0;
         uint32_t na = 0, nc = 0;
-        constexpr int kBatch = 32;                         // loads in flight per thread
         for (int it0 = 0; it0 < n_it; it0 += kBatch) {
-            float v[kBatch];
+            if (it0 > 0) {
 #pragma unroll
-            for (int j = 0; j < kBatch; ++j) {
-                const int64_t e = e0 + static_cast<int64_t>(it0 + j) * kSelThreads + warp * 32 + lane;
-                v[j] = (it0 + j < n_it && e < e1) ? score_at(row, e) : 0.0f;
+                for (int j = 0; j < kBatch; ++j) {
+                    const int64_t e = e0 + static_cast<int64_t>(it0 + j) * kSelThreads + warp * 32 + lane;
+                    v[j] = (it0 + j < n_it && e < e1) ? score_at(row, e) : 0.0f;
+                }
             }
             // lane j keeps the two ballot words of step it0 + j (small unrolled body)
             uint32_t my_a = 0u, my_c = 0u;
