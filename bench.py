@@ -156,17 +156,19 @@ def barrier(pg):
 MEASURED_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch on decode_b4_1m
     # (1-pass ncu capture, caches flushed): 20.65 MB + 0 B, and 71.37 MB + 1.40 MB
-    "hca_attn": {"bytes": 20650000, "source": "long_context_attention_hca_b200/csrc/attention_tc.cu",
-                 "sha256_16": "8afb1c32941a19e3"},
-    "indexer": {"bytes": 72770000, "source": "long_context_attention_hca_b200/csrc/indexer.cu",
-                "sha256_16": "afc2390707e8cf84"},
+    "hca_attn": {"bytes": 20650000, "workload": "decode_b4_1m",
+                 "source": "long_context_attention_hca_b200/csrc/attention_tc.cu", "sha256_16": "8afb1c32941a19e3"},
+    "indexer": {"bytes": 72770000, "workload": "decode_b4_1m",
+                "source": "long_context_attention_hca_b200/csrc/indexer.cu", "sha256_16": "afc2390707e8cf84"},
 }
 
 
-def measured_traffic(kernel: str):
+def measured_traffic(kernel: str, workload: str):
+    """The captured DRAM bytes of one launch, or None: another workload, or the
+    kernel's source changed since the capture."""
     import hashlib
     e = MEASURED_TRAFFIC.get(kernel)
-    if e is None:
+    if e is None or e["workload"] != workload:
         return None
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), e["source"])
     try:
@@ -570,7 +572,7 @@ def bench_decode(args, wl, world, rank, pg):
     if dominant is not None:
         ach = algo[dominant] / (solo_ms[dominant] * 1e-3) / 1e9
         roof = {"bound": "hbm", "kernel": dominant, "achieved": ach, "peak": hbm, "unit": "GB/s",
-                "frac": ach / hbm, "peak_source": f"{src} (burst copy)", "traffic": measured_traffic(dominant),
+                "frac": ach / hbm, "peak_source": f"{src} (burst copy)", "traffic": measured_traffic(dominant, wl.name),
                 "algorithmic_bytes": algo[dominant], "avg_launch_us": solo_ms[dominant] * 1e3,
                 "timing": "the kernel alone, CUDA events, inputs rotating over replicas (L2-cold)",
                 "solo_us": {k: v * 1e3 for k, v in solo_ms.items()}}

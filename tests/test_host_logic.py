@@ -125,3 +125,14 @@ def test_prefill_attention_flops_counts_causal_keys():
     assert fl["hca_attn"] == 4 * 64 * 512 * n_hca
     att, _ = bench.prefill_flops(wl)
     assert att == fl["csa_attn"] + fl["hca_attn"]
+
+
+def test_measured_traffic_only_for_its_workload_and_source():
+    """A captured DRAM byte count is reported for the workload and the kernel
+    source it was taken on, and for nothing else."""
+    import bench
+    assert bench.measured_traffic("hca_attn", "decode_b16_64k") is None
+    assert bench.measured_traffic("csa_attn", "decode_b4_1m") is None
+    for k, e in bench.MEASURED_TRAFFIC.items():
+        got = bench.measured_traffic(k, e["workload"])
+        assert got in (None, e["bytes"])
