@@ -904,10 +904,12 @@ int index_launch(const uint8_t* q_codes, const uint8_t* q_sf, const float* w,
     const bool small = Hi <= 4;
     if (c == 128 && Hi == 4) {
         // tensor cores on FP4 fed by the tensor memory accelerator: 16 queries per
-        // CTA when a sequence has many query rows (prefill), else one
+        // CTA when a sequence has many query rows (prefill), else one.  Prefill: 16
+        // epilogue warps (4 queries each per tile); with 8 the chunk's indexer took
+        // 2.2 ms instead of 1.6 ms at prefill_4096_131k (the epilogue is latency bound)
         int rc;
         if (Tq % 16 == 0 && Tq >= 64)
-            rc = itc::launch_tc<16, 2, 4, 2>(q_codes, q_sf, w, k_codes, k_sf, q_pos, rows, B, Tq, Nc_cap, m, scores, st,
+            rc = itc::launch_tc<16, 2, 4, 4>(q_codes, q_sf, w, k_codes, k_sf, q_pos, rows, B, Tq, Nc_cap, m, scores, st,
                                              2LL * sm_count(), nullptr, 0, bf16 ? 1 : 0);
         else
             rc = itc::launch_tc<1, 8, 5, 2>(q_codes, q_sf, w, k_codes, k_sf, q_pos, rows, B, Tq, Nc_cap, m, scores, st,
