@@ -159,7 +159,7 @@ MEASURED_TRAFFIC = {
     "hca_attn": {"bytes": 20650000, "workload": "decode_b4_1m",
                  "source": "long_context_attention_hca_b200/csrc/attention_tc.cu", "sha256_16": "8afb1c32941a19e3"},
     "indexer": {"bytes": 72770000, "workload": "decode_b4_1m",
-                "source": "long_context_attention_hca_b200/csrc/indexer.cu", "sha256_16": "029946a51c093ea2"},
+                "source": "long_context_attention_hca_b200/csrc/indexer.cu", "sha256_16": "d1a1a7570f1b9597"},
 }
 
 

@@ -458,7 +458,9 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
     __shared__ __align__(8) uint64_t bar_full[KS], bar_empty[KS], bar_accf[NBD], bar_acce[NBD], bar_drain;
     __shared__ uint32_t tmem_slot;
     __shared__ int s_eq[QG][16 * HG];                   // (uq - 127) - 127 per (query, group*16 + block*4 + head)
-    __shared__ int s_klo[QG][HG][4], s_khi[QG][HG][4];  // key exponent range of the fast path per (group, block)
+    __shared__ __align__(16) int s_klo[QG][HG][4];      // key exponent range of the fast path per (group, block)
+    __shared__ __align__(16) int s_khi[QG][HG][4];
+    __shared__ __align__(16) float s_qf[QG][16 * HG];   // 2^(uq - 127) per (query, group*16 + block*4 + head)
     __shared__ float s_w[QG][HI];
     uint16_t* scores16 = reinterpret_cast<uint16_t*>(scores);
     __shared__ int64_t s_elig[QG];
@@ -539,8 +541,21 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
             mn = min(mn, e);
             mx = max(mx, e);
         }
-        s_klo[q][hg][blk] = -126 - mn;
-        s_khi[q][hg][blk] = 116 - mx;
+        int lo = -126 - mn, hi = 116 - mx;
+        if (!(QG == 1 && HG == 1)) {
+            // the fast path of this instantiation takes each term as (D * 2^(uq - 127)) *
+            // 2^(uk - 127): the key factor a normal float (uk in [1, 254]) and the first
+            // product exact for every block dot (|D| in [1/4, 1152] or 0): uq in [3, 244]
+            lo = max(lo, 1);
+            hi = min(hi, 254);
+            if (mn + 254 < 3 || mx + 254 > 244) { lo = 1; hi = 0; }
+        }
+        s_klo[q][hg][blk] = lo;
+        s_khi[q][hg][blk] = hi;
+    }
+    for (int x = tid; x < QG * HG * 16; x += blockDim.x) {
+        const int uq = s_eq[x / (16 * HG)][x % (16 * HG)] + 254;
+        s_qf[x / (16 * HG)][x % (16 * HG)] = (uq >= 1 && uq <= 254) ? __uint_as_float(static_cast<uint32_t>(uq) << 23) : 0.0f;
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -676,33 +691,63 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
             for (int g = 0; g < GPC; ++g) {
             const int hg = ch * GPC + g;
             const uint32_t* r = rc + 16 * g;
-            int eq[16];
-#pragma unroll
-            for (int z = 0; z < 16; ++z) eq[z] = (QG == 1 && HG == 1) ? eq1[z] : s_eq[q][hg * 16 + z];
+            constexpr bool kOne = QG == 1 && HG == 1;
             int ek[4];
             bool fast = true;
+            int4 lo4 = make_int4(0, 0, 0, 0), hi4 = make_int4(0, 0, 0, 0);
+            if (!kOne) {
+                lo4 = *reinterpret_cast<const int4*>(&s_klo[q][hg][0]);
+                hi4 = *reinterpret_cast<const int4*>(&s_khi[q][hg][0]);
+            }
+            const int los[4] = {lo4.x, lo4.y, lo4.z, lo4.w}, his[4] = {hi4.x, hi4.y, hi4.z, hi4.w};
 #pragma unroll
             for (int blk = 0; blk < 4; ++blk) {
                 ek[blk] = static_cast<int>((sw >> (8 * blk)) & 0xFFu);
-                const int lo = (QG == 1 && HG == 1) ? klo1[blk] : s_klo[q][hg][blk];
-                const int hi = (QG == 1 && HG == 1) ? khi1[blk] : s_khi[q][hg][blk];
+                const int lo = kOne ? klo1[blk] : los[blk];
+                const int hi = kOne ? khi1[blk] : his[blk];
                 fast &= (ek[blk] >= lo) & (ek[blk] <= hi);
             }
             float dot[4];
             if (__all_sync(0xffffffffu, fast)) {
                 // every term is an exact product (a normal power of two, no overflow), so
                 // fma(D, 2^e, acc) rounds exactly as the ordered sum acc + D * 2^e does
+                if (kOne) {
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
+                    for (int h = 0; h < 4; ++h) {
 #pragma unroll
-                    for (int blk = 0; blk < 4; ++blk) {
-                        const int z = blk * 4 + h;
-                        const float s2 = __uint_as_float(static_cast<uint32_t>(eq[z] + 127 + ek[blk]) << 23);
-                        dot[h] = blk == 0 ? __fmul_rn(__uint_as_float(r[z]), s2)
-                                          : __fmaf_rn(__uint_as_float(r[z]), s2, dot[h]);
+                        for (int blk = 0; blk < 4; ++blk) {
+                            const int z = blk * 4 + h;
+                            const float s2 = __uint_as_float(static_cast<uint32_t>(eq1[z] + 127 + ek[blk]) << 23);
+                            dot[h] = blk == 0 ? __fmul_rn(__uint_as_float(r[z]), s2)
+                                              : __fmaf_rn(__uint_as_float(r[z]), s2, dot[h]);
+                        }
+                    }
+                } else {
+                    // D * 2^(eq + ek) as (D * 2^(uq - 127)) * 2^(uk - 127): the first product is
+                    // exact (the range above), so the fma's single rounding is the same one
+                    float qf[16];
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        const float4 f = *reinterpret_cast<const float4*>(&s_qf[q][hg * 16 + 4 * v]);
+                        qf[4 * v] = f.x; qf[4 * v + 1] = f.y; qf[4 * v + 2] = f.z; qf[4 * v + 3] = f.w;
+                    }
+                    float kf[4];
+#pragma unroll
+                    for (int blk = 0; blk < 4; ++blk) kf[blk] = __uint_as_float(static_cast<uint32_t>(ek[blk]) << 23);
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+#pragma unroll
+                        for (int blk = 0; blk < 4; ++blk) {
+                            const int z = blk * 4 + h;
+                            const float a = __fmul_rn(__uint_as_float(r[z]), qf[z]);
+                            dot[h] = blk == 0 ? __fmul_rn(a, kf[blk]) : __fmaf_rn(a, kf[blk], dot[h]);
+                        }
                     }
                 }
             } else {
+                int eq[16];
+#pragma unroll
+                for (int z = 0; z < 16; ++z) eq[z] = kOne ? eq1[z] : s_eq[q][hg * 16 + z];
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
                     // column blk*4 + h: ordered block sum ((t0 + t1) + t2) + t3, each term rounded once
