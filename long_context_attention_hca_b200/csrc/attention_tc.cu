@@ -46,9 +46,12 @@
 //               tracks the issuing thread's own MMAs: the release barriers
 //               count two arrivals).
 //   All threads load Q (bf16 -> fp16) at the start, every load in flight at once.
-//   Split partials: warps 0-15 (four per TMEM lane quarter, one M-tile
-//   each) store O / l as fp16 with heads in fours ([HP/4][D][4]), so a warp's
-//   32 lanes (consecutive dims) write 256 contiguous bytes per store.
+//   Output: warps 0-15 (four per TMEM lane quarter, one M-tile each, one
+//   output dim per thread).  One split: O / l as bf16, the RoPE dims rotated
+//   back (about 5x shorter than the softmax warps alone: 32K clocks of a
+//   prefill CTA's 120K were that epilogue).  Several splits: O / l as fp16
+//   with heads in fours ([HP/4][D][4]), so a warp's 32 lanes (consecutive
+//   dims) write 256 contiguous bytes per store.
 // Per 64-key tile the MMAs read 128 KB of shared memory (Q and K for QK) and
 // 96 KB (V^T and P, four M-tiles, for PV) and the stores write 72 KB: at
 // 128 B per clock that is ~2300 clocks, the bound of this data flow.
@@ -303,7 +306,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
     __shared__ uint32_t tmem_base_slot;
     // rescale factors and flags, double-buffered by tile parity: with no barrier
     // after the P stores a warp may run one tile ahead of the others
-    __shared__ float s_alpha[2][HP], s_l[HP], s_rl[HP];
+    __shared__ float s_alpha[2][HP], s_rl[HP];
     __shared__ int s_resc_w[2][NSOFT];
     __shared__ volatile int s_abort;
     __shared__ float s_qr[HP];                       // 1 / rms of each query head (query RMSNorm)
@@ -715,7 +718,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bar_pready[pb]));
         }
-        // ---- epilogue: wait for the last PV, then O^T / l -> out (or the split partials)
+        // ---- epilogue: wait for the last PV, then 1 / l (and the split's (m, l)) for the output
         if (ok && n_tiles > 0) {
             ok = wait_bar(smem_u32(&bar_pempty[(n_tiles - 1) & 1]), ((n_tiles - 1) >> 1) & 1, &s_abort);
             fence_after();
@@ -724,54 +727,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
         // the sink joins the denominator (relative to this split's running max)
         const float sink_l2 = (EX && p.sink) ? __ldg(p.sink + h) * LOG2E : -INFINITY;
         const float l_tot = (EX && p.sink && n_tiles > 0) ? l_run + ex2(sink_l2 - m_used) : l_run;
-        if (hrow) s_l[h] = p.n_splits == 1 ? l_tot : l_run;
-        named_bar(1, NSOFT * 32);
-        const int L = warp * 32 + lane;              // output dim within each M-tile
         const size_t uo = static_cast<size_t>(u);
         const float qnan = __int_as_float(0x7fc00000);
         if (p.n_splits == 1) {
-#pragma unroll 1
-            for (int mt = 0; mt < 4; ++mt) {
-                const int dim = mt * 128 + L;
-#pragma unroll 1
-                for (int c1 = 0; c1 < HP; c1 += 32) {
-                // 32 head columns in flight at once, one wait
-                uint32_t oa[32];
-                if (n_tiles > 0) {
-                    TMEM_LD16(lane_base + O_COL + mt * HP + c1, oa, 0);
-                    TMEM_LD16(lane_base + O_COL + mt * HP + c1 + 16, oa, 16);
-                    tmem_wait_ld();
-                }
-#pragma unroll
-                for (int c0 = c1; c0 < c1 + 32; c0 += 16) {
-                    const uint32_t* o = oa + (c0 - c1);
-                    float v[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float l = s_l[c0 + j];
-                        v[j] = (n_tiles > 0 && l > 0.0f) ? __uint_as_float(o[j]) / l : 0.0f;
-                    }
-                    if (EX && p.inv_freq && mt == 3) {
-                        // RoPE dims (448..511, warps 2 and 3): rotate back by the query's position;
-                        // the pair partner is the neighbouring lane
-                        const bool rot = dim >= D - D_ROPE;
-                        const int pi = (dim - (D - D_ROPE)) >> 1;
-                        const float cs = rot ? s_cos[pi] : 1.0f, sn = rot ? s_sin[pi] : 0.0f;
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const float pv = __shfl_xor_sync(0xffffffffu, v[j], 1);
-                            if (rot) v[j] = (dim & 1) ? v[j] * cs - pv * sn : v[j] * cs + pv * sn;
-                        }
-                    }
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int hh = c0 + j;
-                        if (hh < p.H)
-                            p.out[(uo * p.H + hh) * D + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(ok ? v[j] : qnan));
-                    }
-                }
-                }
-            }
+            // the output itself (below, by warps 0-15): 1 / l of every head
+            if (hrow) s_rl[h] = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
             if (p.lse && hrow && h < p.H) {
                 const float none = (EX && p.sink) ? __ldg(p.sink + h) : -INFINITY;    // no keys: the sink alone
                 p.lse[uo * p.H + h] = (l_run > 0.0f && ok) ? (m_used + log2f(l_tot)) * 0.69314718055994531f
@@ -785,21 +745,49 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
             s_rl[h] = l_run > 0.0f ? 1.0f / l_run : 0.0f;
         }
     }
-    if (p.n_splits > 1 && warp < 16) {
-        // ---- split partials by warps 0-15: warp w reads TMEM lane quarter w % 4 (the
-        // lanes it may access) of M-tile w / 4, i.e. one output dim per thread, and
-        // stores that dim's 64 heads of O / l as fp16, four heads (8 bytes) per store:
-        // the 32 lanes (consecutive dims) of a warp write 256 contiguous bytes
-        // the softmax warps have seen the last PV complete (their own wait, one phase
-        // at a time); the barrier hands that on
+    if (warp < 16) {
+        // ---- output by warps 0-15: warp w reads TMEM lane quarter w % 4 (the lanes it
+        // may access) of M-tile w / 4, i.e. one output dim per thread.  One split: that
+        // dim of every head, O / l as bf16 (the RoPE dims rotated back), the 32 lanes
+        // (consecutive dims) of a warp writing 64 contiguous bytes per head.  Several
+        // splits: O / l as fp16, four heads (8 bytes) per store, 256 contiguous bytes a
+        // warp.  The softmax warps have seen the last PV complete (their own wait, one
+        // phase at a time); the barrier hands that on with 1 / l
         fence_before();
         named_bar(2, 16 * 32);                       // s_rl published, the last PV complete
         fence_after();
-        if (n_tiles > 0) {
-            const int qd = warp & 3, mt = warp >> 2;
-            const int dim = mt * 128 + qd * 32 + lane;
-            const uint32_t lb = tmem + (static_cast<uint32_t>(qd * 32) << 16);
-            const bool good = s_abort == 0;
+        const int qd = warp & 3, mt = warp >> 2;
+        const int dim = mt * 128 + qd * 32 + lane;
+        const uint32_t lb = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+        const bool good = s_abort == 0;
+        if (p.n_splits == 1) {
+            const size_t uo = static_cast<size_t>(u);
+            const bool rot = EX && p.inv_freq && dim >= D - D_ROPE;
+            const int pi = rot ? (dim - (D - D_ROPE)) >> 1 : 0;
+            const float cs = rot ? s_cos[pi] : 1.0f, sn = rot ? s_sin[pi] : 0.0f;
+            const uint16_t qnan16 = 0x7FC0u;
+#pragma unroll 1
+            for (int c1 = 0; c1 < HP; c1 += 32) {
+                uint32_t oa[32];
+                if (n_tiles > 0) {
+                    TMEM_LD16(lb + O_COL + mt * HP + c1, oa, 0);
+                    TMEM_LD16(lb + O_COL + mt * HP + c1 + 16, oa, 16);
+                    tmem_wait_ld();
+                }
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int hh = c1 + j;
+                    float v = n_tiles > 0 ? __uint_as_float(oa[j]) * s_rl[hh] : 0.0f;
+                    if (EX && p.inv_freq && mt == 3) {
+                        // RoPE pair (dim, dim ^ 1) of neighbouring lanes
+                        const float pv = __shfl_xor_sync(0xffffffffu, v, 1);
+                        if (rot) v = (dim & 1) ? v * cs - pv * sn : v * cs + pv * sn;
+                    }
+                    if (hh < p.H)
+                        p.out[(uo * p.H + hh) * D + dim] = good ? __bfloat16_as_ushort(__float2bfloat16_rn(v)) : qnan16;
+                }
+            }
+        } else if (n_tiles > 0) {
             uint16_t* po = p.part_o + (static_cast<size_t>(u) * p.n_splits + split) * HP * D + static_cast<size_t>(dim) * 4;
 #pragma unroll 1
             for (int c1 = 0; c1 < HP; c1 += 32) {
