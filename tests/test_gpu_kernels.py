@@ -199,6 +199,34 @@ def test_topk_crowded_threshold_bin(R, Nc, k):
     assert np.array_equal(host(idx), wi)
 
 
+@pytest.mark.parametrize("R,Nc,k", [(320, 12000, 700), (300, 70001, 1024)])
+def test_topk_many_rows(R, Nc, k):
+    """Many rows (the prefill shape: a cluster of CTAs per row, more rows than
+    SMs): random, few-valued, all-tied, crowded and tie-dominated rows, rows
+    whose eligible prefix is shorter than k or empty; bit-exact against the
+    oracle."""
+    g = _gen(R * 7 + Nc + k)
+    scores = torch.randn((R, Nc), generator=g, device=DEV)
+    vals = torch.tensor([-1.0, -0.0, 0.0, 0.25, 0.5, 1.0, 1.5, 3.0], device=DEV)
+    scores[0:10] = vals[torch.randint(0, 8, (10, Nc), generator=g, device=DEV)]
+    scores[10] = 0.0
+    scores[11] = 1.0 + torch.randint(0, 3000, (Nc,), generator=g, device=DEV).float() * 2.0 ** -13
+    scores[12] = 0.5
+    scores[12, torch.randperm(Nc, generator=g, device=DEV)[: k // 2]] = 2.0 + torch.rand(k // 2, generator=g, device=DEV)
+    scores[13, :] = -0.0
+    scores[13, ::3] = 0.0
+    pos = torch.full((R,), 4 * Nc - 1, dtype=torch.int32, device=DEV)
+    pos[14] = 4 * (k - 1) + 2          # fewer eligible entries than k
+    pos[15] = 4 * k - 1                # exactly k eligible
+    pos[16] = 2                        # none eligible
+    pos[17] = 4 * (Nc // 3) + 1
+    idx, cnt = hca.topk_select(scores, pos, 4, k)
+    torch.cuda.synchronize()
+    wi, wc = oracle.topk(host(scores), host(pos), 4, k)
+    assert np.array_equal(host(cnt), wc)
+    assert np.array_equal(host(idx), wi)
+
+
 @pytest.mark.parametrize("Nc,k,zero_w", [(20000, 512, False), (5000, 64, False), (70001, 1024, False),
                                          (20000, 777, True)])
 def test_lightning_index_topk_fused(Nc, k, zero_w):
