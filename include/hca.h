@@ -491,7 +491,7 @@ int kv_state_append(const uint16_t* x, const uint16_t* gate, const uint16_t* win
  * pointers unless stated): the CSA layer's cache, indexer keys and window,
  * the HCA layer's cache, entry counts and window, staging buffers for the
  * queries, the index scores, top-k outputs and workspaces, the outputs; and
- * for the schedule a second stream and four events (cudaStream_t /
+ * for the schedule a second stream and five events (cudaStream_t /
  * cudaEvent_t as void*, created by the caller). */
 typedef struct {
     int32_t B, H, Hi, c, k, W;
