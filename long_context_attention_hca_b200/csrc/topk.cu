@@ -356,9 +356,8 @@ constexpr int kWpt = 16;                   // bitmap words per thread
 constexpr int kSegWords = kSelThreads * kWpt;   // 8192 words = 262144 entries per bitmap segment
 constexpr int kWBuf = 64;                  // per-warp staging entries per list
 // dynamic shared memory of select_kernel: the candidates (resolve), one bitmap
-// segment (resolve; the per-warp staging during the scan), the output
-constexpr size_t kSelSmem = static_cast<size_t>(kCandSmem) * 8 + static_cast<size_t>(kSegWords) * 4 +
-                            static_cast<size_t>(kMaxK) * 4;
+// segment (resolve; the per-warp staging during the scan)
+constexpr size_t kSelSmem = static_cast<size_t>(kCandSmem) * 8 + static_cast<size_t>(kSegWords) * 4;
 static_assert(kSelWarps * kWBuf * 12 <= kSegWords * 4, "staging fits in the bitmap segment");
 
 __host__ __device__ inline size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -486,10 +485,11 @@ __device__ __forceinline__ void find_digit(const uint32_t* h, uint32_t nb, uint3
     __syncthreads();
 }
 
-// The bitmap segment in shared memory: thread t's kWpt = 16 words (entries
+// A full bitmap segment in shared memory: thread t's kWpt = 16 words (entries
 // 512 t .. 512 t + 511 of the segment) sit in four 16-byte slots, rotated by
 // t / 2 so that the eight lanes of a 16-byte access phase hit eight
-// different bank groups.
+// different bank groups.  (A shorter segment, at fewer words per thread,
+// keeps its words in order.)
 __device__ __forceinline__ uint32_t slot_of(uint32_t t, uint32_t j) { return 4 * t + ((j + (t >> 1)) & 3u); }
 // shared-memory word index of segment word wd
 __device__ __forceinline__ uint32_t word_at(uint32_t wd) {
@@ -538,7 +538,6 @@ select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, i
     extern __shared__ __align__(16) unsigned long long dyn[];
     unsigned long long* s_cand = dyn;                                          // [kCandSmem]
     uint32_t* s_bits = reinterpret_cast<uint32_t*>(dyn + kCandSmem);           // [kSegWords]
-    int32_t* s_out = reinterpret_cast<int32_t*>(s_bits + kSegWords);           // [kMaxK]
     __shared__ uint32_t s_hist[kBins];
     __shared__ uint32_t sh_warp[32];
     __shared__ uint32_t s_dig[4];
@@ -645,8 +644,19 @@ select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, i
     const uint32_t n_above = min(min(__ldcg(w.hdr + 0), kk), static_cast<uint32_t>(kMaxK));
     const uint32_t n_cand = min(__ldcg(w.hdr + 1), static_cast<uint32_t>(Nc_cap));
     const bool cached = n_cand <= static_cast<uint32_t>(kCandSmem);
+    // the row's bitmap, in segments of at most kSegWords words; a segment of nws
+    // words gives every thread wpt words, the least power of two with
+    // wpt * kSelThreads >= nws (a short row still spreads over all threads)
+    const size_t nw = static_cast<size_t>((n + 31) / 32);
+    auto seg_wpt = [&](size_t seg) {
+        const size_t nws = min(nw - seg, static_cast<size_t>(kSegWords));
+        uint32_t x = 1;
+        while (static_cast<size_t>(x) * kSelThreads < nws) x <<= 1;
+        return x;
+    };
+    uint32_t wpt = seg_wpt(0);
     // the above indices stay in registers; cached candidates go to shared memory
-    // (both lists in one round of loads)
+    // (both lists in one round of loads); the first bitmap segment is cleared
     constexpr int kPer = kMaxK / kSelThreads;
     static_assert(kCandSmem / kSelThreads == kPer, "one round covers both lists");
     uint32_t av[kPer];
@@ -658,6 +668,7 @@ select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, i
             av[j] = i < n_above ? __ldcg(w.above + i) : 0u;
             cv[j] = (cached && i < n_cand) ? __ldcg(w.cand + i) : 0ull;
         }
+        for (uint32_t j = 0; j < wpt; ++j) s_bits[tid + j * kSelThreads] = 0u;
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
             const uint32_t i = tid + j * kSelThreads;
@@ -665,6 +676,20 @@ select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, i
         }
     }
     __syncthreads();
+    // entry e sets its bit in the segment starting at word seg: segment word wd sits
+    // at word_at(wd) at 16 words per thread, else at wd (thread t's words t wpt ..
+    // t wpt + wpt - 1, in order)
+    auto mark = [&](uint32_t e, size_t seg) {
+        const uint32_t e_lo = static_cast<uint32_t>(seg * 32);
+        const uint32_t wd = (e - e_lo) >> 5;
+        if (e >= e_lo && wd < wpt * static_cast<uint32_t>(kSelThreads))
+            atomicOr(&s_bits[wpt == static_cast<uint32_t>(kWpt) ? word_at(wd) : wd], 1u << (e & 31u));
+    };
+    // the above keys of the first segment set their bits beside the radix select
+    // (which works on other shared words)
+#pragma unroll
+    for (int j = 0; j < kPer; ++j)
+        if (tid + j * kSelThreads < n_above) mark(av[j], 0);
     auto cand = [&](uint32_t c) { return cached ? s_cand[c] : __ldcg(w.cand + c); };
     uint32_t need = kk - n_above;
     // threshold: candidates whose composite, on the bits fixed so far, is >= prefix
@@ -695,28 +720,25 @@ select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, i
             if (whole) break;
         }
     }
-    // ---- output, per bitmap segment: the above keys and the selected candidates
-    // set their bits; a block-wide scan gives every set bit its rank, and the
-    // indices are placed in the output staging at those ranks
-    const size_t nw = static_cast<size_t>((n + 31) / 32);
+    // ---- output, per bitmap segment: the selected candidates (and, past the first
+    // segment, the above keys) set their bits; a block-wide scan gives every set
+    // bit its rank, and each index is stored at its rank in the output row, i.e.
+    // in ascending order
     uint32_t written = 0;
     for (size_t seg = 0; seg < nw; seg += kSegWords) {
+        if (seg > 0) {
+            wpt = seg_wpt(seg);
+            for (uint32_t j = 0; j < wpt; ++j) s_bits[tid + j * kSelThreads] = 0u;
+            __syncthreads();
 #pragma unroll
-        for (int j = 0; j < kWpt; ++j) s_bits[tid + j * kSelThreads] = 0u;
-        __syncthreads();
-        const uint32_t e_lo = static_cast<uint32_t>(seg * 32);
-        auto mark = [&](uint32_t e) {
-            const uint32_t wd = (e - e_lo) >> 5;
-            if (e >= e_lo && wd < static_cast<uint32_t>(kSegWords)) atomicOr(&s_bits[word_at(wd)], 1u << (e & 31u));
-        };
-#pragma unroll
-        for (int j = 0; j < kPer; ++j)
-            if (tid + j * kSelThreads < n_above) mark(av[j]);
+            for (int j = 0; j < kPer; ++j)
+                if (tid + j * kSelThreads < n_above) mark(av[j], seg);
+        }
         if (cached) {
 #pragma unroll 1
             for (uint32_t c = tid; c < n_cand; c += kSelThreads) {
                 const unsigned long long v = s_cand[c];
-                if ((v & fmask) >= prefix) mark(~static_cast<uint32_t>(v));
+                if ((v & fmask) >= prefix) mark(~static_cast<uint32_t>(v), seg);
             }
         } else {
             constexpr int kB = 8;                       // candidate loads in flight per thread
@@ -730,16 +752,28 @@ select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, i
                 }
 #pragma unroll
                 for (int j = 0; j < kB; ++j)
-                    if (c0 + j * kSelThreads < n_cand && (cv[j] & fmask) >= prefix) mark(~static_cast<uint32_t>(cv[j]));
+                    if (c0 + j * kSelThreads < n_cand && (cv[j] & fmask) >= prefix)
+                        mark(~static_cast<uint32_t>(cv[j]), seg);
             }
         }
         __syncthreads();
+        const bool rotated = wpt == static_cast<uint32_t>(kWpt);
         const uint4* s_b4 = reinterpret_cast<const uint4*>(s_bits);
-        uint32_t cnt = 0;
+        // this thread's words: count and nonzero mask (bit q: word q)
+        uint32_t cnt = 0, nz = 0;
+        if (rotated) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint4 v4 = s_b4[slot_of(tid, j)];
-            cnt += __popc(v4.x) + __popc(v4.y) + __popc(v4.z) + __popc(v4.w);
+            for (int j = 0; j < 4; ++j) {
+                const uint4 v4 = s_b4[slot_of(tid, j)];
+                cnt += __popc(v4.x) + __popc(v4.y) + __popc(v4.z) + __popc(v4.w);
+                nz |= ((v4.x ? 1u : 0u) | (v4.y ? 2u : 0u) | (v4.z ? 4u : 0u) | (v4.w ? 8u : 0u)) << (4 * j);
+            }
+        } else {
+            for (uint32_t q = 0; q < wpt; ++q) {
+                const uint32_t x = s_bits[tid * wpt + q];
+                cnt += __popc(x);
+                nz |= (x ? 1u : 0u) << q;
+            }
         }
         const uint32_t incl = block_incl_scan(cnt, sh_warp);
         if (tid == kSelThreads - 1) s_tot = incl;
@@ -747,13 +781,6 @@ select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, i
         {
             // one loop iteration per set bit of this thread (not per word and bit, which
             // would make a warp run the sum over words of its lanes' maxima)
-            uint32_t nz = 0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint4 v4 = s_b4[slot_of(tid, j)];
-                nz |= (v4.x ? 1u : 0u) << (4 * j) | (v4.y ? 2u : 0u) << (4 * j) | (v4.z ? 4u : 0u) << (4 * j) |
-                      (v4.w ? 8u : 0u) << (4 * j);
-            }
             uint32_t bits = 0u, eb = 0u;
 #pragma unroll 1
             for (;;) {
@@ -761,12 +788,12 @@ select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, i
                     if (nz == 0u) break;
                     const uint32_t q = static_cast<uint32_t>(__ffs(nz) - 1);
                     nz &= nz - 1u;
-                    bits = s_bits[4 * slot_of(tid, q >> 2) + (q & 3u)];
-                    eb = static_cast<uint32_t>((seg + static_cast<size_t>(tid) * kWpt + q) * 32);
+                    bits = rotated ? s_bits[4 * slot_of(tid, q >> 2) + (q & 3u)] : s_bits[tid * wpt + q];
+                    eb = static_cast<uint32_t>((seg + static_cast<size_t>(tid) * wpt + q) * 32);
                 }
                 const uint32_t e = eb + static_cast<uint32_t>(__ffs(bits) - 1);
                 bits &= bits - 1u;
-                if (pos < static_cast<uint32_t>(kMaxK)) s_out[pos] = static_cast<int32_t>(e);
+                if (pos < kk) orow[pos] = static_cast<int32_t>(e);
                 ++pos;
             }
         }
@@ -775,7 +802,7 @@ select_kernel(const T* __restrict__ scores, const int32_t* __restrict__ q_pos, i
         __syncthreads();
     }
     const uint32_t cnt_out = min(written, kk);
-    for (uint32_t j = tid; j < static_cast<uint32_t>(k); j += kSelThreads) orow[j] = j < cnt_out ? s_out[j] : -1;
+    for (uint32_t j = cnt_out + tid; j < static_cast<uint32_t>(k); j += kSelThreads) orow[j] = -1;
     if (tid == 0) count[r] = static_cast<int32_t>(cnt_out);
 }
 
