@@ -106,6 +106,23 @@ int hca_take_device_error(void);
 #define HCA_BUDGET_DECODE_INDEX 2
 int hca_set_launch_budget(int op, int max_ctas);
 
+/* Early query: a scheduling knob with no counterpart on the pages.  Decode
+ * attention launches are programmatic: a launch may start while the kernel
+ * queued just before it on the stream is still running, and waits for that
+ * kernel before it reads anything.  With the knob on, a sparse decode
+ * attention on the tensor-core path (idx != NULL, d = 512, H = 64) loads and
+ * prepares its query (conversion, and with extras the RMSNorm and RoPE)
+ * before that wait, so that this work overlaps the previous kernel (in the
+ * decode step: the top-k select).  The query (and the extras' weights and
+ * q_pos) must then be complete before the previous kernel starts, i.e.
+ * written by work queued before it or on another stream that the caller's
+ * stream waited on; never by the previous kernel itself.  The index list,
+ * its counts and the caches are still read after the wait.
+ *   on  1: on; 0: off (the default)
+ * Process-wide; applies to launches made after the call.  Returns the
+ * previous value, or -1 for a value other than 0 or 1. */
+int hca_set_early_query(int on);
+
 /* ------------------------------------------------------------------ */
 /* Compression: softmax-gated pooling + FP8/BF16 storage.               */
 /* ------------------------------------------------------------------ */

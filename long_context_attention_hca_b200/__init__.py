@@ -122,6 +122,20 @@ def set_launch_budget(op: int, max_ctas: int) -> int:
     return prev
 
 
+_lib.hca_set_early_query.argtypes = [ctypes.c_int]
+_lib.hca_set_early_query.restype = ctypes.c_int
+
+
+def set_early_query(on: bool) -> bool:
+    """Let a sparse decode attention (tensor-core path) load its query before it
+    waits for the kernel queued just before it; the query must then be complete
+    before that kernel starts.  Process-wide; returns the previous setting."""
+    prev = int(_lib.hca_set_early_query(1 if on else 0))
+    if prev < 0:
+        raise ValueError("set_early_query: on must be 0 or 1")
+    return bool(prev)
+
+
 def take_device_error() -> int:
     """Read and clear the device error word (non-zero: a kernel gave up a bounded wait)."""
     return int(_lib.hca_take_device_error())

@@ -129,6 +129,8 @@ int thread_budget_swap(int op, int max_ctas) {
     t_budget[op] = max_ctas;
     return prev;
 }
+static std::atomic<int> g_early_query{0};
+int early_query() { return g_early_query.load(); }
 
 }  // namespace hca
 
@@ -156,6 +158,11 @@ int hca_set_launch_budget(int op, int max_ctas) {
         max_ctas < 0)
         return -1;
     return hca::g_launch_budget[op].exchange(max_ctas);
+}
+
+int hca_set_early_query(int on) {
+    if (on != 0 && on != 1) return -1;
+    return hca::g_early_query.exchange(on);
 }
 
 int hca_take_device_error(void) {

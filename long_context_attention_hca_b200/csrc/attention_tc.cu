@@ -118,6 +118,7 @@ struct Params {
     const float* inv_freq;      // [32] RoPE frequencies of the 64 RoPE dims
     const int32_t* q_pos;       // decode: [units] query positions
     const int32_t* win_len;     // decode: [units] valid window rows (<= W), or null: W
+    int q_early;                // the query may be read before the wait on the previous kernel
 };
 
 constexpr int D_ROPE = 64;
@@ -315,89 +316,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t u = blockIdx.x;
     const int split = blockIdx.y;
-    pdl_wait();                                    // everything earlier in the stream is visible
-    const UnitKeys uk = unit_keys(p, u);
-    const int n_tot = uk.n_c + uk.n_w;
-    const int n_tiles_all = (n_tot + TK - 1) / TK;
-    const int t_begin = split * p.tiles_per_split;
-    const int t_end = min(n_tiles_all, t_begin + p.tiles_per_split);
-    const int n_tiles = t_end > t_begin ? t_end - t_begin : 0;
-    const uint32_t sbase = smem_u32(smem);
-
-    if (tid == 0) {
-        for (int i = 0; i < NBUF; ++i) {
-            mbar_init(smem_u32(&bar_kempty[i]), NPV);  // freed by the PV issuers
-            mbar_init(smem_u32(&bar_kfull[i]), NPROD);  // one arrival per producer warp
-            mbar_init(smem_u32(&bar_sfull[i]), NISSUE);   // both QK issuers
-        }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(smem_u32(&bar_pready[i]), NSOFT);  // the softmax warps stored P
-            mbar_init(smem_u32(&bar_pempty[i]), NPV);    // the PV issuers' MMAs completed
-        }
-        mbar_init(smem_u32(&bar_drain), NISSUE + NPV);   // the MMA-issuing threads
-        s_abort = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    if (warp == 0) { tmem_alloc(smem_u32(&tmem_base_slot), TMEM_COLS); tmem_relinquish(); }
-    // ---- producer state (warps 4-19), declared here so that the first tile's
-    // gathers are in flight while every thread loads Q
-    const bool producer = warp >= NSOFT && warp < NSOFT + NPROD;
-    const int pw = warp - NSOFT;                   // 0..15
-    const int c16 = (pw & 7) * 4 + (lane >> 3);    // this thread's 16-dim unit (same for all its keys)
-    const int row0 = (pw >> 3) * 32 + (lane & 7);  // its rows: row0 + 8 j
-    const int d0 = c16 * 16;
-    const int dn = D - 64;
-    int32_t ent_next[ROWS_PER_THREAD];
-    auto fetch_ent = [&](int i, int32_t (&e)[ROWS_PER_THREAD]) {
-#pragma unroll
-        for (int j = 0; j < ROWS_PER_THREAD; ++j) {
-            const int slot = (t_begin + i) * TK + row0 + 8 * j;
-            e[j] = (i < n_tiles && slot < uk.n_c) ? (uk.ent ? uk.ent[slot] : slot) : -1;
-        }
-    };
-    uint32_t raw[ROWS_PER_THREAD][8];
-    float sc[ROWS_PER_THREAD];
-    // raw loads of tile i (registers only: no buffer needed yet)
-    auto load_tile = [&](int i, const int32_t (&ent)[ROWS_PER_THREAD]) {
-        const int slot0 = (t_begin + i) * TK;
-#pragma unroll
-        for (int j = 0; j < ROWS_PER_THREAD; ++j) {
-            const int r = row0 + 8 * j;
-            const int slot = slot0 + r;
-            sc[j] = 0.0f;
-#pragma unroll
-            for (int z = 0; z < 8; ++z) raw[j][z] = 0;
-            if (i >= n_tiles) continue;
-            if (slot < uk.n_c) {
-                const int64_t e = ent[j];
-                if (e >= 0 && e < p.cap) {
-                    const int64_t er = uk.kv_row0 + e;
-                    if (d0 < dn) {
-                        const uint4 cv = __ldg(reinterpret_cast<const uint4*>(p.codes + er * dn + d0));
-                        raw[j][0] = cv.x; raw[j][1] = cv.y; raw[j][2] = cv.z; raw[j][3] = cv.w;
-                        sc[j] = __ldg(p.scales + er * (dn / 64) + d0 / 64);
-                    } else {
-                        const uint4* rp = reinterpret_cast<const uint4*>(p.rope + er * 64 + (d0 - dn));
-                        const uint4 a = __ldg(rp), bq = __ldg(rp + 1);
-                        raw[j][0] = a.x; raw[j][1] = a.y; raw[j][2] = a.z; raw[j][3] = a.w;
-                        raw[j][4] = bq.x; raw[j][5] = bq.y; raw[j][6] = bq.z; raw[j][7] = bq.w;
-                    }
-                }
-            } else if (slot < n_tot) {
-                const uint4* rp = reinterpret_cast<const uint4*>(uk.wrow + static_cast<size_t>(slot - uk.n_c) * D + d0);
-                const uint4 a = __ldg(rp), bq = __ldg(rp + 1);
-                raw[j][0] = a.x; raw[j][1] = a.y; raw[j][2] = a.z; raw[j][3] = a.w;
-                raw[j][4] = bq.x; raw[j][5] = bq.y; raw[j][6] = bq.z; raw[j][7] = bq.w;
-            }
-        }
-    };
-    if (producer) {
-        int32_t ent0[ROWS_PER_THREAD];
-        fetch_ent(0, ent0);
-        load_tile(0, ent0);
-        fetch_ent(1, ent_next);
-    }
-    {
+    // the query, converted (and, with the extras, normalised and rotated) into its
+    // shared-memory operand; before the wait on the previous kernel when the launch
+    // says that the query was complete before that kernel started (p.q_early)
+    auto load_q = [&]() {
         // Q -> fp16, K-major SW128: column block cb = dims 64cb.., row = head; all of
         // a thread's loads are issued before the first conversion
         constexpr int QV = HP * (D / 8);                      // 16-byte vectors of Q
@@ -484,7 +406,91 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(Params p) {
                 }
             }
         }
+    };
+    if (p.q_early) load_q();
+    pdl_wait();                                    // everything earlier in the stream is visible
+    const UnitKeys uk = unit_keys(p, u);
+    const int n_tot = uk.n_c + uk.n_w;
+    const int n_tiles_all = (n_tot + TK - 1) / TK;
+    const int t_begin = split * p.tiles_per_split;
+    const int t_end = min(n_tiles_all, t_begin + p.tiles_per_split);
+    const int n_tiles = t_end > t_begin ? t_end - t_begin : 0;
+    const uint32_t sbase = smem_u32(smem);
+
+    if (tid == 0) {
+        for (int i = 0; i < NBUF; ++i) {
+            mbar_init(smem_u32(&bar_kempty[i]), NPV);  // freed by the PV issuers
+            mbar_init(smem_u32(&bar_kfull[i]), NPROD);  // one arrival per producer warp
+            mbar_init(smem_u32(&bar_sfull[i]), NISSUE);   // both QK issuers
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&bar_pready[i]), NSOFT);  // the softmax warps stored P
+            mbar_init(smem_u32(&bar_pempty[i]), NPV);    // the PV issuers' MMAs completed
+        }
+        mbar_init(smem_u32(&bar_drain), NISSUE + NPV);   // the MMA-issuing threads
+        s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    if (warp == 0) { tmem_alloc(smem_u32(&tmem_base_slot), TMEM_COLS); tmem_relinquish(); }
+    // ---- producer state (warps 4-19), declared here so that the first tile's
+    // gathers are in flight while every thread loads Q
+    const bool producer = warp >= NSOFT && warp < NSOFT + NPROD;
+    const int pw = warp - NSOFT;                   // 0..15
+    const int c16 = (pw & 7) * 4 + (lane >> 3);    // this thread's 16-dim unit (same for all its keys)
+    const int row0 = (pw >> 3) * 32 + (lane & 7);  // its rows: row0 + 8 j
+    const int d0 = c16 * 16;
+    const int dn = D - 64;
+    int32_t ent_next[ROWS_PER_THREAD];
+    auto fetch_ent = [&](int i, int32_t (&e)[ROWS_PER_THREAD]) {
+#pragma unroll
+        for (int j = 0; j < ROWS_PER_THREAD; ++j) {
+            const int slot = (t_begin + i) * TK + row0 + 8 * j;
+            e[j] = (i < n_tiles && slot < uk.n_c) ? (uk.ent ? uk.ent[slot] : slot) : -1;
+        }
+    };
+    uint32_t raw[ROWS_PER_THREAD][8];
+    float sc[ROWS_PER_THREAD];
+    // raw loads of tile i (registers only: no buffer needed yet)
+    auto load_tile = [&](int i, const int32_t (&ent)[ROWS_PER_THREAD]) {
+        const int slot0 = (t_begin + i) * TK;
+#pragma unroll
+        for (int j = 0; j < ROWS_PER_THREAD; ++j) {
+            const int r = row0 + 8 * j;
+            const int slot = slot0 + r;
+            sc[j] = 0.0f;
+#pragma unroll
+            for (int z = 0; z < 8; ++z) raw[j][z] = 0;
+            if (i >= n_tiles) continue;
+            if (slot < uk.n_c) {
+                const int64_t e = ent[j];
+                if (e >= 0 && e < p.cap) {
+                    const int64_t er = uk.kv_row0 + e;
+                    if (d0 < dn) {
+                        const uint4 cv = __ldg(reinterpret_cast<const uint4*>(p.codes + er * dn + d0));
+                        raw[j][0] = cv.x; raw[j][1] = cv.y; raw[j][2] = cv.z; raw[j][3] = cv.w;
+                        sc[j] = __ldg(p.scales + er * (dn / 64) + d0 / 64);
+                    } else {
+                        const uint4* rp = reinterpret_cast<const uint4*>(p.rope + er * 64 + (d0 - dn));
+                        const uint4 a = __ldg(rp), bq = __ldg(rp + 1);
+                        raw[j][0] = a.x; raw[j][1] = a.y; raw[j][2] = a.z; raw[j][3] = a.w;
+                        raw[j][4] = bq.x; raw[j][5] = bq.y; raw[j][6] = bq.z; raw[j][7] = bq.w;
+                    }
+                }
+            } else if (slot < n_tot) {
+                const uint4* rp = reinterpret_cast<const uint4*>(uk.wrow + static_cast<size_t>(slot - uk.n_c) * D + d0);
+                const uint4 a = __ldg(rp), bq = __ldg(rp + 1);
+                raw[j][0] = a.x; raw[j][1] = a.y; raw[j][2] = a.z; raw[j][3] = a.w;
+                raw[j][4] = bq.x; raw[j][5] = bq.y; raw[j][6] = bq.z; raw[j][7] = bq.w;
+            }
+        }
+    };
+    if (producer) {
+        int32_t ent0[ROWS_PER_THREAD];
+        fetch_ent(0, ent0);
+        load_tile(0, ent0);
+        fetch_ent(1, ent_next);
+    }
+    if (!p.q_early) load_q();
     fence_async_smem();
     fence_before();
     __syncthreads();
@@ -1023,6 +1029,7 @@ int tc_attn_decode_launch(const uint16_t* q, int B, int H, const hca_kv_cache& k
     p.win = window; p.W = W;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
     tc_decode_plan(B, max_comp, W, idx != nullptr, p.n_splits, p.tiles_per_split);
+    p.q_early = (idx != nullptr && early_query()) ? 1 : 0;
     p.out = out; p.lse = lse;
     if (p.n_splits > 1) {
         const size_t need = tc_decode_ws_bytes(B, max_comp, W, idx != nullptr);

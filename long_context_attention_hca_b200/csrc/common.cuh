@@ -34,6 +34,8 @@ int sm_count();
 int launch_budget(int op);
 // Sets this thread's override of a launch budget (0: none); returns the previous one.
 int thread_budget_swap(int op, int max_ctas);
+// process-wide: sparse decode attention reads its query before waiting on the previous kernel; see hca_set_early_query
+int early_query();
 
 // Programmatic dependent launch.  A kernel launched by launch_pdl may be
 // scheduled while the previous kernel of its stream is still running; it calls

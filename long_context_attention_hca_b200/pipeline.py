@@ -21,7 +21,7 @@ import torch
 
 from . import (KVCache, compressed_attn_decode, compressed_attn_prefill, csa_compress, decode_workspace_size,
                hca_compress, lightning_index, lightning_index_topk, topk_select, topk_workspace_size,
-               set_launch_budget, BUDGET_DENSE_DECODE, BUDGET_SPARSE_DECODE, BUDGET_DECODE_INDEX)
+               set_launch_budget, set_early_query, BUDGET_DENSE_DECODE, BUDGET_SPARSE_DECODE, BUDGET_DECODE_INDEX)
 
 CSA_RATIO = 4
 HCA_RATIO = 128
@@ -165,6 +165,18 @@ class DecodeRunner:
             yield
         finally:
             set_launch_budget(BUDGET_DENSE_DECODE, prev)
+
+    @staticmethod
+    @contextlib.contextmanager
+    def _early_query_scope():
+        """The CSA attention may load its query before it waits for the top-k: the
+        side stream waited for the caller's stream before the indexer, so every
+        query passed to step() is complete before the top-k starts."""
+        prev = set_early_query(True)
+        try:
+            yield
+        finally:
+            set_early_query(prev)
 
     def _count_kernels(self) -> int:
         """Kernels of this library launched per step: attention (+ split combine) per
@@ -317,9 +329,10 @@ class DecodeRunner:
                                                               count=self.count[li], ws=self.topk_ws[li]))
                     if q_ready is not None:
                         self.side.wait_event(q_ready[li])
-                    timed("csa_attn", li, lambda: compressed_attn_decode(
-                        q[li], L.cache, self.count[li], min(self.k, L.n_entries), L.window, self.scale,
-                        idx=self.idx[li], out=self.out[li], ws=self.ws[li], extras=self.extras[li]))
+                    with self._early_query_scope():
+                        timed("csa_attn", li, lambda: compressed_attn_decode(
+                            q[li], L.cache, self.count[li], min(self.k, L.n_entries), L.window, self.scale,
+                            idx=self.idx[li], out=self.out[li], ws=self.ws[li], extras=self.extras[li]))
                     if on_out is not None:
                         on_out(li, self.side)
             else:

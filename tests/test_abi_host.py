@@ -136,6 +136,13 @@ def test_fused_selection_and_budget_host_paths(lib):
     assert lib.hca_set_launch_budget(2, 0) == 10
     assert lib.hca_set_launch_budget(3, 10) == -1       # unknown op
     assert lib.hca_set_launch_budget(0, -1) == -1       # negative budget
+    lib.hca_set_early_query.argtypes = [ctypes.c_int]
+    lib.hca_set_early_query.restype = ctypes.c_int
+    prev = lib.hca_set_early_query(1)
+    assert prev in (0, 1)
+    assert lib.hca_set_early_query(prev) == 1
+    assert lib.hca_set_early_query(2) == -1             # only 0 or 1
+    assert lib.hca_set_early_query(-1) == -1
 
 
 class EntryEx(ctypes.Structure):

@@ -146,6 +146,35 @@ def test_decode_extras(layout, H, which):
         assert_attn_close(host(out_s)[b], refs, f"sparse b={b} {which}")
 
 
+@pytest.mark.parametrize("which", [(), ("norm", "sink", "rope")])
+def test_early_query_is_bit_identical(which):
+    """A sparse decode attention that loads its query before waiting on the top-k
+    launched just before it (set_early_query) gives the same bits as one that
+    loads it after the wait.  The top-k on long rows keeps the previous kernel
+    running while the attention's CTAs are placed."""
+    layout, H = (512, 64, 64), 64
+    d, dr, g = layout
+    B, cap, W, k = 3, 70001, 128, 1024
+    cache = _random_cache(B, cap, layout, 141)
+    q = _bf16((B, H, d), 142)
+    win = _bf16((B, W, d), 143)
+    P = _params(d, dr, H, 144)
+    qpos = torch.tensor([4 * cap - 1, 4 * 2000 + 1, 4 * 600 + 3], dtype=torch.int32, device=DEV)
+    ex = _extras(P, which, qpos) if which else None
+    scores = torch.randn((B, cap), generator=_gen(145), device=DEV)
+    outs = []
+    for early in (False, True):
+        prev = hca.set_early_query(early)
+        try:
+            idx, cnt = hca.topk_select(scores, qpos, 4, k)
+            outs.append(hca.compressed_attn_decode(q, cache, cnt, k, win, d ** -0.5, idx=idx, extras=ex))
+        finally:
+            hca.set_early_query(prev)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    assert torch.isfinite(outs[1].float()).all()
+
+
 @pytest.mark.parametrize("layout,H", [((128, 32, 32), 8), ((512, 64, 64), 64)])
 def test_extras_off_is_the_plain_call(layout, H):
     d, dr, g = layout
