@@ -1000,7 +1000,7 @@ def main():
     ap.add_argument("--replicas", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dense-budget", type=int, default=None,
-                    help="CTA cap of the step's dense (HCA) attention (default: half the SMs beside the CSA chain; "
+                    help="CTA cap of the step's dense (HCA) attention (default: the SMs that the top-k select leaves, at least half; "
                          "0: the library default, every SM)")
     ap.add_argument("--sparse-budget", type=int, default=0, help="CTA cap of the sparse decode attention (0: none)")
     ap.add_argument("--index-budget", type=int, default=0, help="CTA cap of the fused decode indexer (0: none)")

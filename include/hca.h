@@ -539,8 +539,10 @@ typedef struct {
     uint16_t* out_hca;            /* [B][H][d]                                           */
     void* side_stream;
     void* ev_fork; void* ev_index; void* ev_q; void* ev_join;
-    int32_t hca_ctas;             /* CTAs of the HCA attention (its split-K plan); 0: half */
-                                  /* the SMs, the rest left to the concurrent CSA chain    */
+    int32_t hca_ctas;             /* CTAs of the HCA attention (its split-K plan); 0: the  */
+                                  /* SMs that the top-k select's B * floor(SMs / 2 / B)    */
+                                  /* CTAs leave (at least half), the rest left to the      */
+                                  /* concurrent CSA chain                                  */
     void* ev_iq;                  /* marks the indexer query's copy                        */
     int32_t packed;               /* bit 0: the indexer query's codes, scales and weights */
                                   /* lie in one allocation each (host and device), in that */

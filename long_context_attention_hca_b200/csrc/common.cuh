@@ -36,6 +36,8 @@ int launch_budget(int op);
 int thread_budget_swap(int op, int max_ctas);
 // process-wide: sparse decode attention reads its query before waiting on the previous kernel; see hca_set_early_query
 int early_query();
+// default CTA cap of the dense decode attention beside the decode select of B rows (topk.cu)
+int dense_beside_select(int B);
 
 // Programmatic dependent launch.  A kernel launched by launch_pdl may be
 // scheduled while the previous kernel of its stream is still running; it calls

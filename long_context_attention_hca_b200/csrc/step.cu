@@ -120,10 +120,10 @@ extern "C" int hca_decode_step_host(const hca_decode_step_plan* p, const uint16_
     if (!d_first) HCA_TRY(cpy(h_out_csa, p->out_csa, q_bytes, cudaMemcpyDeviceToHost, side));
     HCA_TRY(rec(p->ev_join, side));
     // HCA: dense attention once the indexer has run, on at most hca_ctas CTAs (by
-    // default half the SMs) so that the CSA chain's select and attention keep
-    // the rest; then its output
+    // default the SMs that the select's CTAs leave, at least half) so that the CSA
+    // chain's select and attention keep the rest; then its output
     HCA_TRY(wait(stream, p->ev_index));
-    const int prev = thread_budget_swap(HCA_BUDGET_DENSE_DECODE, p->hca_ctas > 0 ? p->hca_ctas : sm_count() / 2);
+    const int prev = thread_budget_swap(HCA_BUDGET_DENSE_DECODE, p->hca_ctas > 0 ? p->hca_ctas : dense_beside_select(p->B));
     const int rc = compressed_attn_decode(p->q_hca, p->B, p->H, p->layout, p->hca_cache, nullptr, 0, p->hca_n,
                                           p->hca_max, p->hca_window, p->W, p->softmax_scale, p->out_hca, nullptr,
                                           p->ws_hca, p->ws_hca_bytes, stream);

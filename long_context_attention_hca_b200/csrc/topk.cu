@@ -834,14 +834,23 @@ uint32_t* topk_wide_hist(void* ws, int64_t Nc_cap, int64_t* stride_u32) {
     return static_cast<uint32_t*>(ws);
 }
 
-// scores per CTA: about one CTA per SM over all rows (hist_kernel), or per two
-// SMs (select_kernel: its CTAs then fit in one wave on the SMs that a
-// concurrent attention launch leaves free), whole steps
+// scores per CTA: about one CTA per SM over all rows (hist_kernel), or at most
+// one per two SMs (select_kernel: R * floor(SMs / 2 / R) CTAs, which fit in one
+// wave beside a concurrent attention launch on the other SMs), whole steps
 static int64_t wide_chunk(int R, int64_t Nc_cap, int per_step, int sms_per_cta = 1) {
-    const int64_t ctas_per_row = std::max<int64_t>(1, ceil_div(ceil_div(sm_count(), sms_per_cta), R));
+    const int64_t ctas_per_row = sms_per_cta > 1 ? std::max<int64_t>(1, (sm_count() / sms_per_cta) / R)
+                                                 : std::max<int64_t>(1, ceil_div(sm_count(), R));
     int64_t chunk = ceil_div(Nc_cap, ctas_per_row);
     chunk = std::max<int64_t>(per_step, ceil_div(chunk, per_step) * per_step);
     return std::min<int64_t>(chunk, static_cast<int64_t>(wide::kMaxIt) * per_step);
+}
+
+// CTAs left for a dense decode attention beside the decode select of B rows: the
+// SMs that the select's B * floor(SMs / 2 / B) CTAs leave, at least half of them
+int dense_beside_select(int B) {
+    const int sm = sm_count();
+    const int sel = B * std::max(1, (sm / 2) / std::max(B, 1));
+    return std::max(sm / 2, sm - sel);
 }
 
 // select + resolve, given the rows' histograms (by hist_kernel or by the indexer);

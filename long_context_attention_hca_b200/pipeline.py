@@ -100,9 +100,10 @@ class DecodeRunner:
         """An HCA launch waits for the indexer queued before it (queued first, the
         HCA launches measured no faster).  dense_budget caps the CTAs of this
         runner's HCA launches (applied
-        around its own calls only): None -- half the SMs when the step is one
-        CSA layer beside one HCA layer (the select and the CSA attention keep
-        the other half), else the library default (in a deep stack both streams
+        around its own calls only): None -- when the step is one CSA layer
+        beside one HCA layer, the SMs that the top-k select's B * floor(SMs / 2
+        / B) CTAs leave, at least half (the select and then the CSA attention
+        keep the rest), else the library default (in a deep stack both streams
         stay busy and the HCA launches do better on every SM: 3.46 against
         3.62 ms per step for 61 layers at 32 x 256K); 0 -- the library default.
         extras: per layer,
@@ -112,7 +113,10 @@ class DecodeRunner:
         dev = torch.device(device)
         if dense_budget is None:
             pair = len(layers) == 2 and sorted(L.ratio == CSA_RATIO for L in layers) == [False, True]
-            dense_budget = torch.cuda.get_device_properties(dev).multi_processor_count // 2 if pair else 0
+            # the SMs that the decode select's B * floor(SMs / 2 / B) CTAs leave, at
+            # least half (the C host step's default for hca_ctas)
+            sm = torch.cuda.get_device_properties(dev).multi_processor_count
+            dense_budget = max(sm // 2, sm - B * max(1, (sm // 2) // max(B, 1))) if pair else 0
         self.dense_budget = dense_budget
         if sparse_budget:
             set_launch_budget(BUDGET_SPARSE_DECODE, sparse_budget)
