@@ -85,6 +85,13 @@ def packed_indexer_query(iq, device=None, pin: bool = False):
     return tuple(out)
 
 
+def dense_beside_select(sm: int, B: int) -> int:
+    """CTA cap of a decode step's dense (HCA) attention beside the top-k select of B
+    rows: the SMs that the select's B * floor(sm / 2 / B) CTAs leave, at least half
+    of them (the C host step's default for hca_ctas)."""
+    return max(sm // 2, sm - B * max(1, (sm // 2) // max(B, 1)))
+
+
 class DecodeRunner:
     """Queues one decode step over a list of layers.  Per layer: CSA ->
     lightning_index, topk_select, compressed_attn_decode(sparse); HCA ->
@@ -113,10 +120,8 @@ class DecodeRunner:
         dev = torch.device(device)
         if dense_budget is None:
             pair = len(layers) == 2 and sorted(L.ratio == CSA_RATIO for L in layers) == [False, True]
-            # the SMs that the decode select's B * floor(SMs / 2 / B) CTAs leave, at
-            # least half (the C host step's default for hca_ctas)
             sm = torch.cuda.get_device_properties(dev).multi_processor_count
-            dense_budget = max(sm // 2, sm - B * max(1, (sm // 2) // max(B, 1))) if pair else 0
+            dense_budget = dense_beside_select(sm, B) if pair else 0
         self.dense_budget = dense_budget
         if sparse_budget:
             set_launch_budget(BUDGET_SPARSE_DECODE, sparse_budget)

@@ -136,3 +136,20 @@ def test_measured_traffic_only_for_its_workload_and_source():
     for k, e in bench.MEASURED_TRAFFIC.items():
         got = bench.measured_traffic(k, e["workload"])
         assert got in (None, e["bytes"])
+
+
+def test_dense_budget_beside_select(pipeline):
+    """The HCA attention's default CTA cap in the decode step: the SMs that the
+    select's B * floor(SMs / 2 / B) CTAs leave, never fewer than half."""
+    dense_beside_select = pipeline.dense_beside_select
+    assert dense_beside_select(148, 4) == 76         # select 4 x 18 = 72 CTAs
+    assert dense_beside_select(148, 16) == 84        # 16 x 4 = 64
+    assert dense_beside_select(148, 32) == 84        # 32 x 2 = 64
+    assert dense_beside_select(148, 1) == 74         # 74 select CTAs: half
+    assert dense_beside_select(148, 100) == 74       # one CTA per row would leave 48: half
+    for sm in (132, 148, 160):
+        for B in range(1, 200):
+            c = dense_beside_select(sm, B)
+            assert sm // 2 <= c <= sm
+            sel = B * max(1, (sm // 2) // B)
+            assert c == sm - sel or sel > sm - sm // 2
