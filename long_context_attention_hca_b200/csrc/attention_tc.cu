@@ -56,7 +56,9 @@
 // 96 KB (V^T and P, four M-tiles, for PV) and the stores write 72 KB: at
 // 128 B per clock that is ~2300 clocks, the bound of this data flow.
 // Launches are programmatic (the kernel waits for its stream predecessor
-// before its first read) and trigger the combine once their outputs are stored.
+// before its first read, except for the query of a sparse launch made with the
+// early-query knob on, which its caller guarantees complete before that
+// predecessor started) and trigger the combine once their outputs are stored.
 // Every mbarrier wait is bounded; a timeout sets the device error word,
 // raises the CTA's abort flag, drains the issued MMAs and frees TMEM.
 #include <mutex>
@@ -962,6 +964,7 @@ int launch_tc(tc::Params& p, int64_t units, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
     if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
     // programmatic launches: each kernel waits for its predecessor before any read
+    // (but the query, with p.q_early)
     e = launch_pdl(kern, dim3(static_cast<unsigned>(units), p.n_splits), dim3(tc::NTHREADS), tc::SMEM_BYTES, st, p);
     if (e != cudaSuccess) { set_last_cuda_error(static_cast<int>(e)); return HCA_ERR_CUDA; }
     HCA_CHECK_LAUNCH();
