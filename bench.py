@@ -158,7 +158,7 @@ MEASURED_TRAFFIC = {
     # (1-pass ncu capture, caches flushed, 4 launches): 20.65 MB + 0 B, and
     # 71.36 MB + 0.04-1.34 MB (the indexer's scores mostly stay in L2; median taken)
     "hca_attn": {"bytes": 20650000, "workload": "decode_b4_1m",
-                 "source": "long_context_attention_hca_b200/csrc/attention_tc.cu", "sha256_16": "820147ef8191ca4c"},
+                 "source": "long_context_attention_hca_b200/csrc/attention_tc.cu", "sha256_16": "060c4543b74c857b"},
     "indexer": {"bytes": 71440000, "workload": "decode_b4_1m",
                 "source": "long_context_attention_hca_b200/csrc/indexer.cu", "sha256_16": "d1a1a7570f1b9597"},
 }
